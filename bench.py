@@ -1,0 +1,427 @@
+#!/usr/bin/env python3
+"""Benchmark of the MXFP4 MoE layer on B200: tokens/s of one layer step.
+
+A step is one ``moe_forward`` over one batch of tokens (RMSNorm, router, top-k,
+grouping, gate_up + SwiGLU, down + weighted combine + residual).  Inputs are
+seeded synthetic tensors of the workload's shapes (``synth``) and are resident
+in HBM before the timed region; the L2 is flushed (256 MiB write) before every
+step, outside the step's events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--path auto|gemv|gemm|simt]
+    python bench.py --impl reference ...   # the CPU oracle on the host cores, same metric
+
+Under torchrun (N > 1) every rank runs its own batch (token data parallel,
+weights replicated, no collective on the data path); the step time is the max
+over ranks and ``value`` counts the tokens of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s on 1 B200; % of FP4 tensor peak (prefill) / HBM BW (decode)"
+DEFAULT_CONFIG = "decode_20b"
+WORKLOAD_TEXT = {
+    "tiny": "tiny MoE layer: T=32, d=128, I=128, E=4, top-2, MXFP4 block 32",
+    "decode_20b": "gpt-oss-20b MoE layer, decode: T=16, d=2880, I=2880, E=32, top-4, MXFP4 experts",
+    "prefill_20b": "gpt-oss-20b MoE layer, prefill: T=4096, d=2880, I=2880, E=32, top-4, MXFP4 experts",
+    "moe_120b": "gpt-oss-120b MoE layer: T=8192, d=2880, I=2880, E=128, top-4, MXFP4 experts",
+    "skew_120b": "skewed routing: T=16384, d=I=2880, E=128, top-4, Zipf(1.2) router bias, MXFP4 experts",
+}
+KERNELS = ["route", "group", "gather", "gate_up", "down", "combine"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_DENSE_NOMINAL_TFLOPS = 9000.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(synth.CONFIGS))
+    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm", "simt"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key, config_name):
+    """Per-launch DRAM bytes from a committed ncu capture, if it still matches the kernel source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        ent = d.get(config_name, {}).get(kernel_key)
+        if not ent:
+            return None
+        src = os.path.join(ROOT, "mxfp4_expert_gemm_b200", "csrc", ent["source"])
+        if file_sha(src) != ent["source_sha"]:
+            return None
+        return ent["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period_s=0.002):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------ inputs
+
+
+def device_inputs(cfg, rank, need_oracle_weights):
+    """Hidden rows (this rank's tokens), router, and MXFP4 weights quantized on the GPU."""
+    import torch
+    import mxfp4_expert_gemm_b200 as moe
+    rows = np.arange(rank * cfg.T, (rank + 1) * cfg.T)
+    x = synth.hidden_rows(cfg, rows) if rank else synth.hidden(cfg)
+    gamma, rw, rb = synth.norm_weight(cfg), synth.router_weight(cfg), synth.router_bias(cfg)
+    E, d, I = cfg.E, cfg.d, cfg.I
+    dev = "cuda"
+    w1c = torch.empty((E, 2 * I, d // 2), dtype=torch.uint8, device=dev)
+    w1s = torch.empty((E, d // 32, 2 * I), dtype=torch.uint8, device=dev)
+    w2c = torch.empty((E, d, I // 2), dtype=torch.uint8, device=dev)
+    w2s = torch.empty((E, I // 32, d), dtype=torch.uint8, device=dev)
+    ow = None
+    if need_oracle_weights:
+        import oracle
+        ow = (np.empty((E, 2 * I, d // 2), np.uint8), np.empty((E, 2 * I, d // 32), np.uint8),
+              np.empty((E, d, I // 2), np.uint8), np.empty((E, d, I // 32), np.uint8))
+    for e in range(E):
+        w1 = synth.w1_expert(cfg, e)
+        moe.moe_mxfp4_quantize(torch.from_numpy(w1).to(dev), w1c[e:e + 1], w1s[e:e + 1])
+        w2 = synth.w2_expert(cfg, e)
+        moe.moe_mxfp4_quantize(torch.from_numpy(w2).to(dev), w2c[e:e + 1], w2s[e:e + 1])
+        if ow is not None:
+            ow[0][e], ow[1][e] = oracle.quantize(w1)
+            ow[2][e], ow[3][e] = oracle.quantize(w2)
+    torch.cuda.synchronize()
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    return dict(x=x, gamma=gamma, rw=rw, rb=rb, x_dev=xt, gamma_dev=torch.from_numpy(gamma).to(dev),
+                rw_dev=torch.from_numpy(rw).to(dev), rb_dev=torch.from_numpy(rb).to(dev),
+                W=(w1c, w1s, w2c, w2s), oracle_W=ow)
+
+
+# ------------------------------------------------------------------------------ CPU oracle timing
+
+
+def time_oracle(cfg, inp, budget_s, tokens_per_step=None, steps=None, warmup=0):
+    """Time the CPU oracle (as it stands) on samples of the workload's tokens.
+
+    Returns (tokens/s, threads, sample description)."""
+    import oracle
+    T = cfg.T
+    n = tokens_per_step or T
+    order = np.arange(T, dtype=np.int32)
+    times, done = [], 0
+    t_start = time.perf_counter()
+    i = 0
+    while True:
+        toks = order[(np.arange(n) + i * n) % T]
+        t0 = time.perf_counter()
+        oracle.moe_forward(inp["x"], inp["gamma"], inp["rw"], inp["rb"], *inp["oracle_W"], I=cfg.I, k=cfg.k,
+                           eps=cfg.rms_eps, limit=cfg.swiglu_limit, tokens=toks)
+        dt = time.perf_counter() - t0
+        if i >= warmup:
+            times.append(dt)
+            done += n
+        i += 1
+        if steps is not None:
+            if i >= warmup + steps:
+                break
+        elif time.perf_counter() - t_start >= budget_s and times:
+            break
+    total = sum(times)
+    sample = f"{len(times)} oracle forward(s) of {n} token(s) each from the {cfg.name} batch ({total:.1f} s)"
+    return done / total, os.cpu_count(), sample
+
+
+# ------------------------------------------------------------------------------ our arm
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import mxfp4_expert_gemm_b200 as moe
+    torch.cuda.set_device(local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    cfg = synth.CONFIGS[args.config]
+    want_cpu = (rank == 0 and world == 1 and not args.no_cpu_baseline)
+    inp = device_inputs(cfg, rank, need_oracle_weights=want_cpu)
+    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, cfg.rms_eps, cfg.swiglu_limit, path=args.path)
+    ws = moe.new_workspace(dims, cfg.T)
+    y = torch.empty_like(inp["x_dev"])
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    nk = len(KERNELS)
+    W = inp["W"]
+
+    def step(events=None):
+        moe.moe_forward_timed(dims, inp["x_dev"], inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws, y=y,
+                              events=events, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st = moe.moe_device_status(ws)
+    if st != moe.MOE_OK:
+        raise moe.MoeError(st, "device status after warm-up")
+    path_used = moe.resolved_path(dims, cfg.T)
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(K)]
+    for e in [*starts, *stops, *[x for row in kev for x in row]]:
+        e.record()  # creates the underlying CUDA events
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(K):
+            flush.zero_()
+            starts[i].record()
+            step(kev[i])
+            stops[i].record()
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    launches = moe.last_launch_count() * K
+    st = moe.moe_device_status(ws)
+    if st != moe.MOE_OK:
+        raise moe.MoeError(st, "device status after the timed steps")
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
+    total_ms = float(sum(step_ms))
+    kern_ms = {name: statistics.mean(kev[i][2 * j].elapsed_time(kev[i][2 * j + 1]) for i in range(K))
+               for j, name in enumerate(KERNELS[:moe.last_launch_count()])}
+    if pg:
+        t = torch.tensor([total_ms], device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    x_host = torch.empty(inp["x_dev"].shape, dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(inp["x_dev"].cpu())
+    y_host = torch.empty_like(x_host, pin_memory=True)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e_stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    x_dev2 = torch.empty_like(inp["x_dev"])
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        e_starts[i].record()
+        x_dev2.copy_(x_host, non_blocking=True)
+        moe.moe_forward(dims, x_dev2, inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws, y=y)
+        y_host.copy_(y, non_blocking=True)
+        e_stops[i].record()
+    torch.cuda.synchronize()
+    e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(e_starts, e_stops)))
+    if pg:
+        t = torch.tensor([e2e_ms], device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    assert moe.moe_device_status(ws) == moe.MOE_OK
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    counts = np.bincount(_routing(moe, dims, inp, ws, cfg).ravel(), minlength=cfg.E)
+    used = int(np.count_nonzero(counts))
+    P = cfg.T * cfg.k
+    d, I = cfg.d, cfg.I
+    w1_bytes = 2 * I * d // 2 + (d // 32) * 2 * I
+    w2_bytes = d * I // 2 + (I // 32) * d
+    decode_like = (P / cfg.E) <= 24
+    gu_ms = kern_ms.get("gate_up")
+    if decode_like:
+        alg = used * w1_bytes + P * d * 2 + P * I * 2   # expert weights streamed once + activations in/out
+        achieved = alg / (gu_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "kernel": "gate_up (tc_expert_kernel<GATE_UP>)", "achieved": round(achieved, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": ncu_traffic("gate_up", cfg.name),
+                "algorithmic_bytes_per_launch": alg, "launch_ms": round(gu_ms, 5), "peak_source": f"hbm_gbs, {peak_src}"}
+        layer_bytes = used * (w1_bytes + w2_bytes)
+        layer_ms = total_ms / K
+        roof["layer"] = {"unique_expert_bytes": layer_bytes, "experts_used": used,
+                         "achieved_GBps": round(layer_bytes / (layer_ms * 1e-3) / 1e9, 1),
+                         "frac_of_measured_hbm": round(layer_bytes / (layer_ms * 1e-3) / 1e9 / peak, 4),
+                         "frac_of_8TBps": round(layer_bytes / (layer_ms * 1e-3) / 8e12, 4)}
+    else:
+        alg = 4 * d * I * P
+        achieved = alg / (gu_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "kernel": "gate_up (tc_expert_kernel<GATE_UP>)", "achieved": round(achieved, 1),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": ncu_traffic("gate_up", cfg.name), "algorithmic_flops_per_launch": alg,
+                "launch_ms": round(gu_ms, 5), "peak_source": f"bf16_tflops burst ({peak_src}); f16 MMA runs at the bf16 rate"}
+        layer_flops = 6 * d * I * P
+        layer_ms = total_ms / K
+        roof["layer"] = {"flops": layer_flops, "achieved_TFLOPs": round(layer_flops / (layer_ms * 1e-3) / 1e12, 1),
+                         "frac_of_fp4_dense_nominal": round(layer_flops / (layer_ms * 1e-3) / 1e12 / FP4_DENSE_NOMINAL_TFLOPS, 4)}
+
+    value = cfg.T * world * K / (total_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": round(total_ms / K, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[cfg.name], "name": cfg.name, "tokens_per_gpu": cfg.T,
+                   "global_batch": cfg.T * world, "path": path_used, "parallelism": f"dp{world}",
+                   "l2": "flushed before every step (256 MiB write, outside the step events)",
+                   "timing": "sum of per-step CUDA events on the launching stream; max over ranks"},
+        "kernel_ms": {k_: round(v, 5) for k_, v in kern_ms.items()},
+        "roofline": roof,
+        "e2e": {"value": round(cfg.T * world * K / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(inp["x_dev"].numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if want_cpu:
+        v, cores, sample = time_oracle(cfg, inp, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def _routing(moe, dims, inp, ws, cfg):
+    out = moe.moe_route(dims, inp["x_dev"], inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], ws)
+    return out["topk_idx"].cpu().numpy()
+
+
+# ------------------------------------------------------------------------------ reference arm
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    cfg = synth.CONFIGS[args.config]
+    import oracle
+    x = synth.hidden(cfg)
+    inp = dict(x=x, gamma=synth.norm_weight(cfg), rw=synth.router_weight(cfg), rb=synth.router_bias(cfg))
+    E, d, I = cfg.E, cfg.d, cfg.I
+    ow = (np.empty((E, 2 * I, d // 2), np.uint8), np.empty((E, 2 * I, d // 32), np.uint8),
+          np.empty((E, d, I // 2), np.uint8), np.empty((E, d, I // 32), np.uint8))
+    for e in range(E):
+        ow[0][e], ow[1][e] = oracle.quantize(synth.w1_expert(cfg, e))
+        ow[2][e], ow[3][e] = oracle.quantize(synth.w2_expert(cfg, e))
+    inp["oracle_W"] = ow
+    # one token per step keeps --steps K --warmup W within minutes on the host cores
+    n = 1
+    t0 = time.perf_counter()
+    v, cores, sample = time_oracle(cfg, inp, 0, tokens_per_step=n, steps=args.steps, warmup=args.warmup)
+    wall = time.perf_counter() - t0
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(n / v * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT[cfg.name], "name": cfg.name, "tokens_per_step": n},
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample, "value": round(v, 4)},
+            "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": round(wall, 1)}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,194 @@
+/*
+ * moe_mxfp4.h -- C ABI of the B200 (sm_100a) MoE feed-forward layer with MXFP4
+ * expert weights (the gpt-oss MoE block).
+ *
+ * What the layer computes (sources: web pages on gpt-oss, cited by page title
+ * and section):
+ *   xn   = RMSNorm(x) * norm_w                         ("From GPT-2 to gpt-oss",
+ *                                                       sec. 7 RMSNorm; eps from the
+ *                                                       llm-atlas GPT-OSS 20B config
+ *                                                       table, rms_norm_eps 1e-5)
+ *   l    = router_w . xn + router_b   (E logits)      (ewbang.com GPT-OSS article,
+ *   top-k experts by logit; w = softmax over the k      section 混合专家模型: a small
+ *   selected logits                                     router network picks several
+ *                                                       experts and weights them;
+ *                                                       top-4 of 32 or 128)
+ *   per selected expert e:                             ("From GPT-2 to gpt-oss",
+ *     g = W1[e][0:I] . xe,  u = W1[e][I:2I] . xe        sec. 3 Swish/SwiGLU: three
+ *     h = silu(min(g, L)) * clamp(u, -L, L)             linears, silu(z)=z*sigmoid(z);
+ *     o = W2[e] . h                                     swiglu_limit L = 7 from the
+ *                                                       llm-atlas config table)
+ *   y    = x + sum_j w_j * o_j                         (ewbang.com article, sections
+ *                                                       混合专家模型 and Transformer 块:
+ *                                                       weighted mix, block maps
+ *                                                       [N x d] to [N x d])
+ * Expert weights are MXFP4: 4-bit E2M1 values with one 8-bit E8M0 scale per
+ * 32 parameters, 4.25 bits per parameter (ewbang.com article, section
+ * 量化 (Quantization)).  xe = bf16(xn); h and y are rounded to bf16.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers unless stated otherwise; the caller
+ *     owns and allocates every buffer.  The library allocates and frees nothing;
+ *     besides a per-host-thread launch counter it keeps no state between calls.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on that stream.  The returned status covers the synchronous
+ *     argument checks and launch errors only; errors the kernels detect (a
+ *     timed-out wait, non-finite input, a value outside the f16 tensor-core
+ *     range) are recorded in the workspace status word: read them with
+ *     moe_device_status().
+ *   - No call throws across the ABI or prints.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Device pointers must be 16-byte aligned.
+ */
+#ifndef MOE_MXFP4_H
+#define MOE_MXFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,       /* null / misaligned pointer, bad size, bad enum */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2, /* block != 32; d or I not a positive multiple of 64;
+                                    E not in [1, 256]; top_k not in [1, min(E, 32)];
+                                    T*top_k above 2^24 */
+  MOE_ERR_WORKSPACE = 3,         /* ws_bytes < moe_workspace_bytes() */
+  MOE_ERR_CUDA = 4,              /* a CUDA runtime error at launch */
+  MOE_ERR_TIMEOUT = 5,           /* (device) a pipeline wait gave up; the kernel exited cleanly */
+  MOE_ERR_NONFINITE = 6,         /* (device) Inf/NaN in the input or the weights */
+  MOE_ERR_RANGE = 7,             /* (device) an MXFP4 scale or activation outside the range the
+                                    f16 tensor-core path represents exactly (see moe_forward) */
+  MOE_ERR_DEVICE = 8             /* the current device is not sm_100 */
+} moe_status;
+
+typedef enum {
+  MOE_PATH_AUTO = 0, /* GEMV when tokens per expert are few, else GEMM */
+  MOE_PATH_GEMV = 1, /* weight-streaming tcgen05 path with 16-token tiles (small batches) */
+  MOE_PATH_GEMM = 2, /* tcgen05 grouped GEMM with 128-token tiles (large batches) */
+  MOE_PATH_SIMT = 3  /* fp32 CUDA-core path (no tensor cores): a cross-check, not for speed */
+} moe_path;
+
+typedef struct {
+  int32_t d;            /* hidden size (gpt-oss: 2880)                                  */
+  int32_t I;            /* expert intermediate size (gpt-oss: 2880)                     */
+  int32_t E;            /* experts (gpt-oss-20b: 32, gpt-oss-120b: 128)                 */
+  int32_t top_k;        /* experts per token (gpt-oss: 4)                               */
+  int32_t block;        /* MXFP4 block size; must be 32                                 */
+  float rms_eps;        /* RMSNorm epsilon (gpt-oss: 1e-5)                              */
+  float swiglu_limit;   /* SwiGLU clamp (gpt-oss: 7)                                    */
+  int32_t path;         /* a moe_path value                                             */
+} moe_dims;
+
+/* ---------------------------------------------------------------- MXFP4 storage
+ * A weight tensor [E][N][K] (K = reduction axis, K % 32 == 0) is stored as
+ *   codes  [E][N][K/2] bytes: two E2M1 codes per byte, the even k in the low nibble;
+ *          code bits: sign (bit 3), exponent (bits 2..1, bias 1), mantissa (bit 0);
+ *   scales [E][K/32][N] bytes: E8M0, value 2^(byte - 127), one per 32 consecutive k of
+ *          a row (K-block-major so that every row stride is N bytes, a TMA-legal stride
+ *          whenever N % 16 == 0).
+ * W1 (gate_up) is [E][2I][d]: rows 0..I-1 are the gate projection, I..2I-1 the up
+ * projection.  W2 (down) is [E][d][I].
+ */
+size_t moe_mxfp4_codes_bytes(int32_t E, int32_t N, int32_t K);  /* E*N*K/2 */
+size_t moe_mxfp4_scales_bytes(int32_t E, int32_t N, int32_t K); /* E*(K/32)*N */
+
+/* Quantize fp32 weights w [E][N][K] (device) to MXFP4 (codes, scales as above).
+ * Per 32-value block: s = clamp(floor(log2(amax)) - 2, -127, 127); each value
+ * x * 2^-s is rounded to the nearest E2M1 value (ties to the even code), saturating
+ * at +-6; the sign bit is set only on non-zero codes; an all-zero block gets s = 0.
+ * (ewbang.com article, section 量化: 4-bit values, one 8-bit scale per 32.)
+ * status_word: optional device int32; MOE_ERR_NONFINITE is OR-ed into it when a
+ * block holds Inf/NaN (that block's scale byte is then 0xFF, the E8M0 NaN).
+ * Errors: MOE_ERR_INVALID_ARG (null/misaligned pointer, E/N/K <= 0),
+ * MOE_ERR_UNSUPPORTED_SHAPE (K % 32 != 0), MOE_ERR_CUDA. */
+moe_status moe_mxfp4_quantize(const float* w, int32_t E, int32_t N, int32_t K, uint8_t* codes,
+                              uint8_t* scales, int32_t* status_word, void* stream);
+
+/* Bytes of device scratch moe_route / moe_forward need for T tokens.  The first 256
+ * bytes hold the device status word; the rest is scratch that the calls overwrite.
+ * Calls that share a workspace must be ordered on one stream. */
+size_t moe_workspace_bytes(const moe_dims* dims, int32_t T);
+
+/* Steps 1-4 of the layer for T tokens: RMSNorm, router logits, top-k + softmax, and
+ * token-to-expert grouping.
+ *   x        [T][d] bf16          norm_w [d] fp32        router_w [E][d] fp32
+ *   router_b [E] fp32 or NULL (zero bias)
+ * Outputs (device; each may be NULL except as noted):
+ *   topk_idx [T][k] int32  expert ids, by logit descending (ties: lower id first)
+ *   topk_w   [T][k] fp32   softmax over the k selected logits (sums to 1 per token)
+ *   counts   [E]    int32  tokens routed to each expert (sum = T*k)
+ *   offsets  [E+1]  int32  exclusive prefix sum of counts
+ *   perm     [T*k]  int32  pair list sorted by (expert asc, token asc); entry = t*k + slot
+ * The router runs in fp32 on the unrounded RMSNorm output.
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_WORKSPACE, MOE_ERR_CUDA;
+ * device side: MOE_ERR_NONFINITE (non-finite logits). */
+moe_status moe_route(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                     const float* router_w, const float* router_b, int32_t* topk_idx, float* topk_w,
+                     int32_t* counts, int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* The whole layer: y [T][d] bf16 = x + MoE(RMSNorm(x)).
+ *   w1_codes / w1_scales: W1 [E][2I][d] in the MXFP4 storage above
+ *   w2_codes / w2_scales: W2 [E][d][I]
+ * Optional outputs (device, NULL to skip): topk_idx_out [T][k], topk_w_out [T][k],
+ * counts_out [E].
+ * y may not alias x.  T >= 1 (T = 0 returns MOE_OK and launches nothing).
+ * Tensor-core paths (GEMV, GEMM) multiply f16 operands with fp32 accumulation:
+ * xe and h are bf16 values, exact in f16 when |v| <= 65504 (|h| <= L^2 always is);
+ * a decoded weight E2M1 * 2^s is exact in f16 for s in [-23, 13] (scale bytes
+ * 104..140).  Outside those ranges the call records MOE_ERR_RANGE instead of
+ * returning a rounded result; MOE_PATH_SIMT has no such limit.
+ * Errors: as moe_route. */
+moe_status moe_forward(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                       const float* router_w, const float* router_b, const uint8_t* w1_codes,
+                       const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                       uint16_t* y, int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* moe_forward plus per-kernel timing: `events` is an array of n_events cudaEvent_t
+ * handles created by the caller (timing enabled).  Event 2i is recorded on `stream`
+ * just before the i-th kernel this call launches and event 2i+1 just after it, until
+ * the array runs out.  Recording adds no synchronization.  The kernels of a call are,
+ * in order: route (RMSNorm + router + top-k), group, gather, gate_up, down, combine.
+ * Errors: as moe_forward; MOE_ERR_INVALID_ARG if n_events < 0 or events is NULL with
+ * n_events > 0. */
+moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                             const float* router_w, const float* router_b, const uint8_t* w1_codes,
+                             const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                             uint16_t* y, int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out,
+                             void* ws, size_t ws_bytes, void* stream, void* const* events, int32_t n_events);
+
+/* The path moe_forward takes for these dims and T: dims->path, or for MOE_PATH_AUTO the
+ * choice it makes (MOE_PATH_GEMV when T*top_k/E <= 24 tokens per expert, else
+ * MOE_PATH_GEMM).  Returns -1 for invalid dims. */
+int32_t moe_resolve_path(const moe_dims* dims, int32_t T);
+
+/* Byte offsets of the workspace's sub-buffers for T tokens, for inspection by tests and
+ * debuggers (layout may change between versions).  offsets[0..13] receive, in order:
+ * status, counts, offsets, ntiles, tiles, topk_idx, topk_w, perm, inv, w_sorted,
+ * xe [T][d] f16, xs [T*k][d] f16 (xe in sorted pair order), h [T*k][I] f16 (SwiGLU
+ * output, sorted order), ys [T*k][d] fp32 (weighted expert outputs, sorted order);
+ * offsets[14] = total bytes.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE. */
+moe_status moe_workspace_layout(const moe_dims* dims, int32_t T, size_t* offsets);
+
+/* Synchronize `stream`, then read and clear the device status word of workspace `ws`
+ * (device pointer).  Returns MOE_OK or the first device-side error recorded since the
+ * last read (MOE_ERR_TIMEOUT, MOE_ERR_NONFINITE, MOE_ERR_RANGE), or MOE_ERR_CUDA. */
+moe_status moe_device_status(void* ws, void* stream);
+
+/* Static description of a status code. */
+const char* moe_status_string(moe_status status);
+
+/* Number of kernels the last successful moe_forward / moe_route call on this host
+ * thread launched (for launch accounting in benchmarks). */
+int32_t moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_MXFP4_H */

@@ -1,0 +1,265 @@
+"""Python binding of ``libmoe_mxfp4.so``: the B200 MoE layer with MXFP4 experts.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current stream.  The C ABI and
+its contract are in ``include/moe_mxfp4.h``; the functions here carry the same
+names.  There is no fallback: if the library is missing or the device is not
+sm_100, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_mxfp4.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "moe_mxfp4.h")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED_SHAPE = 2
+MOE_ERR_WORKSPACE = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_TIMEOUT = 5
+MOE_ERR_NONFINITE = 6
+MOE_ERR_RANGE = 7
+MOE_ERR_DEVICE = 8
+
+MOE_PATH_AUTO = 0
+MOE_PATH_GEMV = 1
+MOE_PATH_GEMM = 2
+MOE_PATH_SIMT = 3
+PATHS = {"auto": MOE_PATH_AUTO, "gemv": MOE_PATH_GEMV, "gemm": MOE_PATH_GEMM, "simt": MOE_PATH_SIMT}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class moe_dims(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("I", ctypes.c_int32), ("E", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("block", ctypes.c_int32), ("rms_eps", ctypes.c_float), ("swiglu_limit", ctypes.c_float),
+                ("path", ctypes.c_int32)]
+
+
+def make_dims(d: int, I: int, E: int, top_k: int, rms_eps: float = 1e-5, swiglu_limit: float = 7.0,
+              path: int | str = MOE_PATH_AUTO, block: int = 32) -> moe_dims:
+    if isinstance(path, str):
+        path = PATHS[path]
+    return moe_dims(d, I, E, top_k, block, rms_eps, swiglu_limit, path)
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m mxfp4_expert_gemm_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+            dp = ctypes.POINTER(moe_dims)
+            L.moe_mxfp4_codes_bytes.argtypes = [i32, i32, i32]
+            L.moe_mxfp4_codes_bytes.restype = sz
+            L.moe_mxfp4_scales_bytes.argtypes = [i32, i32, i32]
+            L.moe_mxfp4_scales_bytes.restype = sz
+            L.moe_mxfp4_quantize.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
+            L.moe_mxfp4_quantize.restype = ctypes.c_int
+            L.moe_workspace_bytes.argtypes = [dp, i32]
+            L.moe_workspace_bytes.restype = sz
+            L.moe_route.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.moe_route.restype = ctypes.c_int
+            L.moe_forward.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.moe_forward.restype = ctypes.c_int
+            L.moe_forward_timed.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                            vp, i32]
+            L.moe_forward_timed.restype = ctypes.c_int
+            L.moe_resolve_path.argtypes = [dp, i32]
+            L.moe_resolve_path.restype = i32
+            L.moe_workspace_layout.argtypes = [dp, i32, vp]
+            L.moe_workspace_layout.restype = ctypes.c_int
+            L.moe_device_status.argtypes = [vp, vp]
+            L.moe_device_status.restype = ctypes.c_int
+            L.moe_status_string.argtypes = [ctypes.c_int]
+            L.moe_status_string.restype = ctypes.c_char_p
+            L.moe_last_launch_count.argtypes = []
+            L.moe_last_launch_count.restype = i32
+            _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/moe_mxfp4.h declares."""
+    txt = open(HEADER_PATH).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_\w+)\s*\(", txt)))
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(st: int, what: str):
+    if st != MOE_OK:
+        raise MoeError(st, what)
+
+
+def _need(t: torch.Tensor, dtype, name, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name}: a CUDA tensor is required")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def moe_mxfp4_codes_bytes(E: int, N: int, K: int) -> int:
+    return lib().moe_mxfp4_codes_bytes(E, N, K)
+
+
+def moe_mxfp4_scales_bytes(E: int, N: int, K: int) -> int:
+    return lib().moe_mxfp4_scales_bytes(E, N, K)
+
+
+def moe_mxfp4_quantize(w: torch.Tensor, codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                       status_word: torch.Tensor | None = None, stream=None):
+    """fp32 weights [E, N, K] -> (codes uint8 [E, N, K/2], scales uint8 [E, K/32, N])."""
+    if w.dim() == 2:
+        w = w.unsqueeze(0)
+    _need(w, torch.float32, "w")
+    E, N, K = w.shape
+    if codes is None:
+        codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty((E, K // 32, N), dtype=torch.uint8, device=w.device)
+    _check(lib().moe_mxfp4_quantize(_ptr(w), E, N, K, _ptr(codes), _ptr(scales), _ptr(status_word), _stream(stream)),
+           "moe_mxfp4_quantize")
+    return codes, scales
+
+
+def moe_workspace_bytes(dims: moe_dims, T: int) -> int:
+    return lib().moe_workspace_bytes(ctypes.byref(dims), T)
+
+
+def new_workspace(dims: moe_dims, T: int, device="cuda") -> torch.Tensor:
+    """A zeroed workspace (its status word starts clear)."""
+    n = moe_workspace_bytes(dims, T)
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def moe_route(dims: moe_dims, x, norm_w, router_w, router_b, ws, stream=None):
+    """-> dict(topk_idx [T,k] int32, topk_w [T,k] f32, counts [E], offsets [E+1], perm [T*k])."""
+    T = x.shape[0]
+    _need(x, torch.bfloat16, "x")
+    dev = x.device
+    k, E = dims.top_k, dims.E
+    out = dict(topk_idx=torch.empty((T, k), dtype=torch.int32, device=dev),
+               topk_w=torch.empty((T, k), dtype=torch.float32, device=dev),
+               counts=torch.empty(E, dtype=torch.int32, device=dev),
+               offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+               perm=torch.empty(T * k, dtype=torch.int32, device=dev))
+    _check(lib().moe_route(ctypes.byref(dims), T, _ptr(x), _ptr(norm_w), _ptr(router_w), _ptr(router_b),
+                           _ptr(out["topk_idx"]), _ptr(out["topk_w"]), _ptr(out["counts"]), _ptr(out["offsets"]),
+                           _ptr(out["perm"]), _ptr(ws), ws.numel(), _stream(stream)), "moe_route")
+    return out
+
+
+def moe_forward(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales, ws,
+                y=None, want_routing=False, stream=None):
+    """y [T, d] bf16 = x + MoE(RMSNorm(x)); with want_routing also (topk_idx, topk_w, counts)."""
+    T = x.shape[0]
+    _need(x, torch.bfloat16, "x")
+    dev = x.device
+    if y is None:
+        y = torch.empty_like(x)
+    r = None
+    if want_routing:
+        r = dict(topk_idx=torch.empty((T, dims.top_k), dtype=torch.int32, device=dev),
+                 topk_w=torch.empty((T, dims.top_k), dtype=torch.float32, device=dev),
+                 counts=torch.empty(dims.E, dtype=torch.int32, device=dev))
+    _check(lib().moe_forward(ctypes.byref(dims), T, _ptr(x), _ptr(norm_w), _ptr(router_w), _ptr(router_b),
+                             _ptr(w1_codes), _ptr(w1_scales), _ptr(w2_codes), _ptr(w2_scales), _ptr(y),
+                             _ptr(r["topk_idx"]) if r else None, _ptr(r["topk_w"]) if r else None,
+                             _ptr(r["counts"]) if r else None, _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_forward")
+    return (y, r) if want_routing else y
+
+
+WS_FIELDS = ("status", "counts", "offsets", "ntiles", "tiles", "topk_idx", "topk_w", "perm", "inv", "w_sorted",
+             "xe", "xs", "h", "ys", "total")
+
+
+def moe_workspace_layout(dims: moe_dims, T: int) -> dict:
+    """Byte offsets of the workspace sub-buffers (for tests and debugging)."""
+    arr = (ctypes.c_size_t * 15)()
+    _check(lib().moe_workspace_layout(ctypes.byref(dims), T, arr), "moe_workspace_layout")
+    return dict(zip(WS_FIELDS, list(arr)))
+
+
+def workspace_view(ws: torch.Tensor, dims: moe_dims, T: int, field: str, dtype, shape) -> torch.Tensor:
+    """A typed view of one workspace sub-buffer."""
+    off = moe_workspace_layout(dims, T)[field]
+    n = 1
+    for s_ in shape:
+        n *= s_
+    nbytes = n * torch.empty((), dtype=dtype).element_size()
+    return ws[off:off + nbytes].view(dtype).view(*shape)
+
+
+def moe_forward_timed(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales, ws,
+                      y=None, events=None, stream=None):
+    """moe_forward that records ``events`` (torch.cuda.Event, timing enabled) around each kernel:
+    event 2i before kernel i and 2i+1 after it (kernels: route, group, gather, gate_up, down, combine)."""
+    _need(x, torch.bfloat16, "x")
+    if y is None:
+        y = torch.empty_like(x)
+    arr, n = None, 0
+    if events:
+        arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        n = len(events)
+    _check(lib().moe_forward_timed(ctypes.byref(dims), x.shape[0], _ptr(x), _ptr(norm_w), _ptr(router_w),
+                                   _ptr(router_b), _ptr(w1_codes), _ptr(w1_scales), _ptr(w2_codes), _ptr(w2_scales),
+                                   _ptr(y), None, None, None, _ptr(ws), ws.numel(), _stream(stream), arr, n),
+           "moe_forward_timed")
+    return y
+
+
+PATH_NAMES = {v: k for k, v in PATHS.items()}
+
+
+def resolved_path(dims: moe_dims, T: int) -> str:
+    """The path moe_forward takes for these dims and T (resolves MOE_PATH_AUTO)."""
+    return PATH_NAMES[lib().moe_resolve_path(ctypes.byref(dims), T)]
+
+
+def moe_device_status(ws: torch.Tensor, stream=None) -> int:
+    return lib().moe_device_status(_ptr(ws), _stream(stream))
+
+
+def last_launch_count() -> int:
+    return lib().moe_last_launch_count()

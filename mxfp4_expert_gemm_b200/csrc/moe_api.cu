@@ -1,0 +1,238 @@
+// C-ABI front end: argument checks, workspace carve-up, path choice, launches.
+// Declarations and the contract of every entry point: include/moe_mxfp4.h.
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstring>
+
+#include "moe_internal.cuh"
+
+namespace {
+
+thread_local int32_t g_last_launches = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  return (major == 10 && minor == 0) ? MOE_OK : MOE_ERR_DEVICE;
+}
+
+moe_status check_dims(const moe_dims* dm, int32_t T) {
+  if (!dm || T < 0) return MOE_ERR_INVALID_ARG;
+  if (dm->path < MOE_PATH_AUTO || dm->path > MOE_PATH_SIMT) return MOE_ERR_INVALID_ARG;
+  if (!(dm->rms_eps >= 0.f) || !std::isfinite(dm->rms_eps)) return MOE_ERR_INVALID_ARG;
+  if (!(dm->swiglu_limit > 0.f) || !std::isfinite(dm->swiglu_limit)) return MOE_ERR_INVALID_ARG;
+  if (dm->block != 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (dm->d <= 0 || dm->I <= 0 || dm->d % 64 || dm->I % 64) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (dm->d > (1 << 16) || dm->I > (1 << 16)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (dm->E < 1 || dm->E > 256) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (dm->top_k < 1 || dm->top_k > dm->E || dm->top_k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)T * dm->top_k > (int64_t(1) << 24)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+int resolve_path(const moe_dims& dm, int32_t T) {
+  if (dm.path != MOE_PATH_AUTO) return dm.path;
+  // Few tokens per expert: stream the weights with narrow token tiles.
+  const double per_expert = (double)T * dm.top_k / dm.E;
+  return per_expert <= 24.0 ? MOE_PATH_GEMV : MOE_PATH_GEMM;
+}
+
+int tile_tokens_of(int path) {
+  return path == MOE_PATH_SIMT ? moe::simt_tile_tokens() : moe::tc_tile_tokens(path);
+}
+
+moe_status prepare(const moe_dims* dm, int32_t T, const uint16_t* x, const float* norm_w, const float* router_w,
+                   const float* router_b, void* ws, size_t ws_bytes, moe::FwdArgs& a, moe::WsLayout& L) {
+  moe_status st = check_dims(dm, T);
+  if (st != MOE_OK) return st;
+  if (!x || !norm_w || !router_w || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(norm_w) || !aligned16(router_w) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (router_b && !aligned16(router_b)) return MOE_ERR_INVALID_ARG;
+  L = moe::ws_layout(*dm, T);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  st = check_device();
+  if (st != MOE_OK) return st;
+  std::memset(&a, 0, sizeof(a));
+  a.T = T;
+  a.d = dm->d;
+  a.I = dm->I;
+  a.E = dm->E;
+  a.k = dm->top_k;
+  a.eps = dm->rms_eps;
+  a.limit = dm->swiglu_limit;
+  a.x = x;
+  a.norm_w = norm_w;
+  a.router_w = router_w;
+  a.router_b = router_b;
+  a.ws = moe::ws_pointers(ws, L);
+  return MOE_OK;
+}
+
+moe_status copy_out(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+  if (!dst) return MOE_OK;
+  return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_mxfp4_codes_bytes(int32_t E, int32_t N, int32_t K) {
+  if (E <= 0 || N <= 0 || K <= 0) return 0;
+  return (size_t)E * N * (K / 2);
+}
+
+size_t moe_mxfp4_scales_bytes(int32_t E, int32_t N, int32_t K) {
+  if (E <= 0 || N <= 0 || K <= 0) return 0;
+  return (size_t)E * (K / 32) * N;
+}
+
+moe_status moe_mxfp4_quantize(const float* w, int32_t E, int32_t N, int32_t K, uint8_t* codes, uint8_t* scales,
+                              int32_t* status_word, void* stream) {
+  g_last_launches = 0;
+  if (!w || !codes || !scales || E <= 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(codes) || !aligned16(scales)) return MOE_ERR_INVALID_ARG;
+  if (K % 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+  moe_status st = check_device();
+  if (st != MOE_OK) return st;
+  const int n = moe::launch_quantize(w, (int64_t)E * N, N, K, E, codes, scales, status_word,
+                                     static_cast<cudaStream_t>(stream));
+  if (n < 0) return MOE_ERR_CUDA;
+  g_last_launches = n;
+  return MOE_OK;
+}
+
+size_t moe_workspace_bytes(const moe_dims* dims, int32_t T) {
+  if (check_dims(dims, T) != MOE_OK) return 0;
+  return moe::ws_layout(*dims, T).total;
+}
+
+moe_status moe_route(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                     const float* router_w, const float* router_b, int32_t* topk_idx, float* topk_w,
+                     int32_t* counts, int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
+  g_last_launches = 0;
+  moe::FwdArgs a;
+  moe::WsLayout L;
+  moe_status st = prepare(dims, T, x, norm_w, router_w, router_b, ws, ws_bytes, a, L);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  a.stream = static_cast<cudaStream_t>(stream);
+  const int path = resolve_path(*dims, T);
+  const int n = moe::launch_route(a, tile_tokens_of(path));
+  if (n < 0) return MOE_ERR_CUDA;
+  const size_t P = (size_t)T * dims->top_k;
+  if ((st = copy_out(topk_idx, a.ws.topk_idx, 4 * P, a.stream)) != MOE_OK) return st;
+  if ((st = copy_out(topk_w, a.ws.topk_w, 4 * P, a.stream)) != MOE_OK) return st;
+  if ((st = copy_out(counts, a.ws.counts, 4 * (size_t)dims->E, a.stream)) != MOE_OK) return st;
+  if ((st = copy_out(offsets, a.ws.offsets, 4 * (size_t)(dims->E + 1), a.stream)) != MOE_OK) return st;
+  if ((st = copy_out(perm, a.ws.perm, 4 * P, a.stream)) != MOE_OK) return st;
+  g_last_launches = n;
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                       const float* router_w, const float* router_b, const uint8_t* w1_codes,
+                       const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales, uint16_t* y,
+                       int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes,
+                       void* stream) {
+  return moe_forward_timed(dims, T, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales, y,
+                           topk_idx_out, topk_w_out, counts_out, ws, ws_bytes, stream, nullptr, 0);
+}
+
+moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                             const float* router_w, const float* router_b, const uint8_t* w1_codes,
+                             const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                             uint16_t* y, int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, void* ws,
+                             size_t ws_bytes, void* stream, void* const* events, int32_t n_events) {
+  g_last_launches = 0;
+  if (n_events < 0 || (n_events > 0 && !events)) return MOE_ERR_INVALID_ARG;
+  moe::FwdArgs a;
+  moe::WsLayout L;
+  moe_status st = prepare(dims, T, x, norm_w, router_w, router_b, ws, ws_bytes, a, L);
+  if (st != MOE_OK) return st;
+  if (!w1_codes || !w1_scales || !w2_codes || !w2_scales || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w1_codes) || !aligned16(w1_scales) || !aligned16(w2_codes) || !aligned16(w2_scales) ||
+      !aligned16(y))
+    return MOE_ERR_INVALID_ARG;
+  if ((const void*)y == (const void*)x) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  a.w1c = w1_codes;
+  a.w1s = w1_scales;
+  a.w2c = w2_codes;
+  a.w2s = w2_scales;
+  a.y = y;
+  a.stream = static_cast<cudaStream_t>(stream);
+  moe::EventRec rec;
+  rec.events = events;
+  rec.n = n_events;
+  a.ev = &rec;
+  const int path = resolve_path(*dims, T);
+  int n = moe::launch_route(a, tile_tokens_of(path));
+  if (n < 0) return MOE_ERR_CUDA;
+  const int ne = (path == MOE_PATH_SIMT) ? moe::launch_experts_simt(a)
+                                         : moe::launch_experts_tc(a, tile_tokens_of(path));
+  if (ne < 0) return MOE_ERR_CUDA;
+  n += ne;
+  const int nc = moe::launch_combine(a);
+  if (nc < 0) return MOE_ERR_CUDA;
+  n += nc;
+  const size_t P = (size_t)T * dims->top_k;
+  if ((st = copy_out(topk_idx_out, a.ws.topk_idx, 4 * P, a.stream)) != MOE_OK) return st;
+  if ((st = copy_out(topk_w_out, a.ws.topk_w, 4 * P, a.stream)) != MOE_OK) return st;
+  if ((st = copy_out(counts_out, a.ws.counts, 4 * (size_t)dims->E, a.stream)) != MOE_OK) return st;
+  g_last_launches = n;
+  return MOE_OK;
+}
+
+int32_t moe_resolve_path(const moe_dims* dims, int32_t T) {
+  if (check_dims(dims, T) != MOE_OK) return -1;
+  return resolve_path(*dims, T);
+}
+
+moe_status moe_workspace_layout(const moe_dims* dims, int32_t T, size_t* offsets) {
+  if (!offsets) return MOE_ERR_INVALID_ARG;
+  const moe_status st = check_dims(dims, T);
+  if (st != MOE_OK) return st;
+  const moe::WsLayout L = moe::ws_layout(*dims, T);
+  const size_t v[15] = {L.status, L.counts, L.offsets, L.ntiles, L.tiles, L.topk_idx, L.topk_w, L.perm,
+                        L.inv, L.w_sorted, L.xe, L.xs, L.h, L.ys, L.total};
+  for (int i = 0; i < 15; ++i) offsets[i] = v[i];
+  return MOE_OK;
+}
+
+moe_status moe_device_status(void* ws, void* stream) {
+  if (!ws || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0) {
+    const int32_t zero = 0;
+    if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return static_cast<moe_status>(v);
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_NONFINITE: return "non-finite value";
+    case MOE_ERR_RANGE: return "value outside the f16 tensor-core range";
+    case MOE_ERR_DEVICE: return "device is not sm_100";
+  }
+  return "unknown status";
+}
+
+int32_t moe_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

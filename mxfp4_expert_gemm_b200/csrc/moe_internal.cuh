@@ -1,0 +1,168 @@
+// Internal declarations shared by the kernels and the C-ABI front end.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "moe_mxfp4.h"
+
+namespace moe {
+
+constexpr int kStatusBytes = 256;
+constexpr int kMinTileTokens = 16;  // smallest token tile of any path (sizes the tile list)
+
+// Token tile of the grouped expert kernels: rows [row0, row0 + rows) of the
+// expert-sorted pair list, all belonging to expert `e`.
+struct Tile {
+  int32_t e;
+  int32_t row0;
+  int32_t rows;
+  int32_t pad;
+};
+
+// Carve-up of the caller's workspace (byte offsets, 256-byte aligned).
+struct WsLayout {
+  size_t status;    // int32 device status word (first device error wins)
+  size_t counts;    // int32 [E]
+  size_t offsets;   // int32 [E+1]
+  size_t ntiles;    // int32 [4]: number of token tiles
+  size_t tiles;     // Tile [max_tiles]
+  size_t topk_idx;  // int32 [T*k]
+  size_t topk_w;    // f32 [T*k]
+  size_t perm;      // int32 [P]   sorted position -> t*k + slot
+  size_t inv;       // int32 [P]   t*k + slot -> sorted position
+  size_t w_sorted;  // f32 [P]     routing weight of each sorted pair
+  size_t xe;        // f16 [T][d]  bf16(RMSNorm(x)) held as f16
+  size_t xs;        // f16 [P][d]  xe gathered in sorted pair order
+  size_t h;         // f16 [P][I]  SwiGLU output (bf16 values) in sorted order
+  size_t ys;        // f32 [P][d]  routing-weighted expert outputs, sorted order
+  size_t total;
+  int64_t max_tiles;
+};
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+inline WsLayout ws_layout(const moe_dims& dm, int64_t T) {
+  WsLayout L{};
+  const int64_t P = T * dm.top_k;
+  L.max_tiles = (P + kMinTileTokens - 1) / kMinTileTokens + dm.E;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.status = take(kStatusBytes);
+  L.counts = take(4 * (size_t)dm.E);
+  L.offsets = take(4 * (size_t)(dm.E + 1));
+  L.ntiles = take(16);
+  L.tiles = take(sizeof(Tile) * (size_t)L.max_tiles);
+  L.topk_idx = take(4 * (size_t)P);
+  L.topk_w = take(4 * (size_t)P);
+  L.perm = take(4 * (size_t)P);
+  L.inv = take(4 * (size_t)P);
+  L.w_sorted = take(4 * (size_t)P);
+  L.xe = take(2 * (size_t)T * dm.d);
+  L.xs = take(2 * (size_t)P * dm.d);
+  L.h = take(2 * (size_t)P * dm.I);
+  L.ys = take(4 * (size_t)P * dm.d);
+  L.total = o;
+  return L;
+}
+
+// Pointers into one workspace.
+struct Ws {
+  int32_t* status;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* ntiles;
+  Tile* tiles;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* perm;
+  int32_t* inv;
+  float* w_sorted;
+  uint16_t* xe;
+  uint16_t* xs;
+  uint16_t* h;
+  float* ys;
+  int64_t max_tiles;
+};
+
+inline Ws ws_pointers(void* base, const WsLayout& L) {
+  char* b = static_cast<char*>(base);
+  Ws w;
+  w.status = reinterpret_cast<int32_t*>(b + L.status);
+  w.counts = reinterpret_cast<int32_t*>(b + L.counts);
+  w.offsets = reinterpret_cast<int32_t*>(b + L.offsets);
+  w.ntiles = reinterpret_cast<int32_t*>(b + L.ntiles);
+  w.tiles = reinterpret_cast<Tile*>(b + L.tiles);
+  w.topk_idx = reinterpret_cast<int32_t*>(b + L.topk_idx);
+  w.topk_w = reinterpret_cast<float*>(b + L.topk_w);
+  w.perm = reinterpret_cast<int32_t*>(b + L.perm);
+  w.inv = reinterpret_cast<int32_t*>(b + L.inv);
+  w.w_sorted = reinterpret_cast<float*>(b + L.w_sorted);
+  w.xe = reinterpret_cast<uint16_t*>(b + L.xe);
+  w.xs = reinterpret_cast<uint16_t*>(b + L.xs);
+  w.h = reinterpret_cast<uint16_t*>(b + L.h);
+  w.ys = reinterpret_cast<float*>(b + L.ys);
+  w.max_tiles = L.max_tiles;
+  return w;
+}
+
+// Optional per-kernel CUDA events supplied by the caller: event 2i is recorded just
+// before the i-th kernel of a call and event 2i+1 just after it.
+struct EventRec {
+  void* const* events = nullptr;
+  int n = 0;
+  int next = 0;
+};
+
+// Everything a forward launch needs.
+struct FwdArgs {
+  int32_t T, d, I, E, k;
+  float eps, limit;
+  const uint16_t* x;
+  const float* norm_w;
+  const float* router_w;
+  const float* router_b;
+  const uint8_t* w1c;
+  const uint8_t* w1s;
+  const uint8_t* w2c;
+  const uint8_t* w2s;
+  uint16_t* y;
+  Ws ws;
+  cudaStream_t stream;
+  EventRec* ev;
+};
+
+inline void ev_before(const FwdArgs& a) {
+  if (a.ev && a.ev->events && a.ev->next + 1 < a.ev->n)
+    cudaEventRecord(static_cast<cudaEvent_t>(a.ev->events[a.ev->next]), a.stream);
+}
+
+inline void ev_after(const FwdArgs& a) {
+  if (a.ev && a.ev->events && a.ev->next + 1 < a.ev->n) {
+    cudaEventRecord(static_cast<cudaEvent_t>(a.ev->events[a.ev->next + 1]), a.stream);
+    a.ev->next += 2;
+  }
+}
+
+// Record the first device-side error in the status word.
+__device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// --------------------------------------------------------------------------- launchers
+// Each returns the number of kernels it launched (>= 0) or -1 on a launch error.
+int launch_quantize(const float* w, int64_t rows, int32_t N, int32_t K, int32_t E, uint8_t* codes,
+                    uint8_t* scales, int32_t* status, cudaStream_t st);
+int launch_route(const FwdArgs& a, int tile_tokens);   // norm + router + top-k + grouping + gather
+int launch_combine(const FwdArgs& a);                  // y = x + sum_j ys[inv]
+int launch_experts_simt(const FwdArgs& a);             // CUDA-core expert MLPs
+int launch_experts_tc(const FwdArgs& a, int tile_tokens);  // tcgen05 expert MLPs
+int tc_tile_tokens(int path);                          // token tile of a tensor-core path
+int simt_tile_tokens();                                // token tile of the CUDA-core path
+
+}  // namespace moe

@@ -1,0 +1,413 @@
+// MXFP4 quantization, RMSNorm + router + top-k, grouping, gather and combine.
+//
+// Layer definition (web pages on gpt-oss):
+//  - RMSNorm: "From GPT-2 to gpt-oss" (新智元 translation), sec. 7: divide by the
+//    RMS, no mean subtraction, no bias; rms_norm_eps 1e-5 (llm-atlas GPT-OSS 20B
+//    config table).
+//  - Router + top-k: ewbang.com GPT-OSS article, section 混合专家模型: a small
+//    network scores the experts, several are chosen per token and weighted
+//    (e.g. 0.7 x NN2 + 0.3 x NN4); top-4 of 32 / 128.
+//  - MXFP4: same article, section 量化: 4-bit values, one 8-bit scale per 32
+//    parameters, 4.25 bits per parameter.
+#include <cuda_fp16.h>
+#include <algorithm>
+#include <cfloat>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// Round fp32 to bf16 (nearest, ties to even); input finite.
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+  uint32_t u = __float_as_uint(f);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+// ----------------------------------------------------------------------------------
+// Quantization: one warp per 32-value block, lane i holds element i.
+// Scale exponent s = floor(log2 amax) - 2 from the exponent bits of amax (exact);
+// the E2M1 code of |x| * 2^-s is the number of rounding thresholds it passes,
+// each threshold taking ties toward the even code.
+// ----------------------------------------------------------------------------------
+__device__ __forceinline__ int e2m1_code_of(float a) {
+  // grid 0 .5 1 1.5 2 3 4 6; thresholds between neighbours, "<" where the tie
+  // belongs to the upper (even) code, "<=" where it belongs to the lower one.
+  int c = 0;
+  c += a > 0.25f;   // tie -> 0
+  c += a >= 0.75f;  // tie -> 1.0
+  c += a > 1.25f;   // tie -> 1.0
+  c += a >= 1.75f;  // tie -> 2.0
+  c += a > 2.5f;    // tie -> 2.0
+  c += a >= 3.5f;   // tie -> 4.0
+  c += a > 5.0f;    // tie -> 4.0
+  return c;
+}
+
+__global__ void quantize_kernel(const float* __restrict__ w, int64_t nblocks, int32_t N, int32_t K,
+                                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int kb_per_row = K / 32;
+  for (int64_t b = warp; b < nblocks; b += nwarps) {
+    const int64_t row = b / kb_per_row;          // row of [E*N]
+    const int kb = (int)(b - row * kb_per_row);
+    const float v = w[b * 32 + lane];
+    const float a = fabsf(v);
+    const bool finite = isfinite(v);
+    float amax = a;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const bool all_finite = __all_sync(0xffffffffu, finite);
+    int s = 0;
+    if (amax > 0.f && all_finite) {
+      const uint32_t bits = __float_as_uint(amax);
+      int e = (int)((bits >> 23) & 0xFF);
+      int fl;
+      if (e != 0) fl = e - 127;                                  // normal: floor(log2) = exponent
+      else fl = (31 - __clz((int)(bits & 0x7FFFFF))) - 149;      // subnormal: m * 2^-149
+      s = max(-127, min(127, fl - 2));
+    }
+    // x * 2^-s exactly (power-of-two scaling; ldexpf is exact when no under/overflow
+    // changes a value that matters: scaled values below 0.25 all round to code 0).
+    const float scaled = ldexpf(a, -s);
+    int c = all_finite ? e2m1_code_of(scaled) : 0;
+    if (v < 0.f && c != 0) c |= 8;
+    const int hi = __shfl_down_sync(0xffffffffu, c, 1);
+    const int64_t e_idx = row / N;
+    const int64_t n = row - e_idx * N;
+    if ((lane & 1) == 0) codes[row * (K / 2) + kb * 16 + (lane >> 1)] = (uint8_t)(c | (hi << 4));
+    if (lane == 0) {
+      scales[(e_idx * kb_per_row + kb) * (int64_t)N + n] = all_finite ? (uint8_t)(s + 127) : (uint8_t)0xFF;
+      if (!all_finite) set_status(status, MOE_ERR_NONFINITE);
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------------
+// Fused RMSNorm + router GEMV + top-k + softmax, 32 tokens per CTA, 256 threads.
+// Outputs: xe (f16 copy of bf16(xn)), topk_idx, topk_w, expert histogram.
+// ----------------------------------------------------------------------------------
+constexpr int RT = 32;   // tokens per CTA
+constexpr int RK = 64;   // d-chunk
+
+template <int NJ>  // experts per lane group: E <= 32*NJ
+__global__ void __launch_bounds__(256) route_kernel(FwdArgs a) {
+  extern __shared__ float smem[];
+  const int E = a.E, d = a.d, k = a.k;
+  const int EP = 32 * NJ;
+  float* s_r = smem;                         // [RT]
+  float* s_x = s_r + RT;                     // [RT][RK+1]
+  float* s_w = s_x + RT * (RK + 1);          // [RK][EP+1]
+  float* s_l = s_w + RK * (EP + 1);          // [RT][EP+1]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = blockIdx.x * RT;
+  const int nt = min(RT, a.T - t0);
+
+  // Phase A: 1/rms per token (warp w: tokens w, w+8, ...).
+  for (int tt = warp; tt < RT; tt += 8) {
+    float ss = 0.f;
+    if (tt < nt) {
+      const uint16_t* xr = a.x + (int64_t)(t0 + tt) * d;
+      for (int i = lane * 8; i < d; i += 256) {
+        const uint4 q = *reinterpret_cast<const uint4*>(xr + i);
+        const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float lo = __uint_as_float(wv[j] << 16), hi = __uint_as_float(wv[j] & 0xFFFF0000u);
+          ss = fmaf(lo, lo, ss);
+          ss = fmaf(hi, hi, ss);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) s_r[tt] = 1.0f / sqrtf(ss / (float)d + a.eps);
+  }
+  __syncthreads();
+
+  // Phase B: router logits, d in chunks of RK.  Thread = (token group tg of 4, lane).
+  const int tg = warp;  // tokens 4*tg .. 4*tg+3
+  float acc[4][NJ];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
+  bool range_bad = false;
+
+  for (int k0 = 0; k0 < d; k0 += RK) {
+    // x chunk -> xn (fp32, smem) and xe (f16 of bf16(xn), global)
+    for (int q = tid; q < RT * (RK / 2); q += 256) {
+      const int tt = q / (RK / 2), c2 = (q % (RK / 2)) * 2;
+      float v0 = 0.f, v1 = 0.f;
+      if (tt < nt) {
+        const int64_t gi = (int64_t)(t0 + tt) * d + k0 + c2;
+        const uint32_t pr = *reinterpret_cast<const uint32_t*>(a.x + gi);
+        const float r = s_r[tt];
+        v0 = __uint_as_float(pr << 16) * r * a.norm_w[k0 + c2];
+        v1 = __uint_as_float(pr & 0xFFFF0000u) * r * a.norm_w[k0 + c2 + 1];
+        const float b0 = bf16_to_f32(f32_to_bf16_rne(v0)), b1 = bf16_to_f32(f32_to_bf16_rne(v1));
+        range_bad |= fabsf(b0) > 65504.f || fabsf(b1) > 65504.f;
+        const __half2 hv = __floats2half2_rn(b0, b1);  // exact for bf16 values in f16 range
+        *reinterpret_cast<__half2*>(a.ws.xe + gi) = hv;
+      }
+      s_x[tt * (RK + 1) + c2] = v0;
+      s_x[tt * (RK + 1) + c2 + 1] = v1;
+    }
+    for (int q = tid; q < RK * EP; q += 256) {  // coalesced along d; padded rows avoid bank conflicts
+      const int e = q / RK, kk = q % RK;
+      s_w[kk * (EP + 1) + e] = (e < E) ? a.router_w[(int64_t)e * d + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < RK; ++kk) {
+      float xv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[i] = s_x[(4 * tg + i) * (RK + 1) + kk];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const float wv = s_w[kk * (EP + 1) + lane + 32 * j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(xv[i], wv, acc[i][j]);
+      }
+    }
+    __syncthreads();
+  }
+  if (range_bad) set_status(a.ws.status, MOE_ERR_RANGE);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const int e = lane + 32 * j;
+      s_l[(4 * tg + i) * (EP + 1) + e] = (e < E) ? acc[i][j] + (a.router_b ? a.router_b[e] : 0.f) : -INFINITY;
+    }
+  __syncthreads();
+
+  // Phase C: top-k + softmax per token (warp w: tokens w, w+8, ...).
+  for (int tt = warp; tt < nt; tt += 8) {
+    float l[NJ];
+    bool bad = false;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      l[j] = s_l[tt * (EP + 1) + lane + 32 * j];
+      if (lane + 32 * j < E && !isfinite(l[j])) {
+        bad = true;
+        l[j] = -INFINITY;
+      }
+    }
+    if (__any_sync(0xffffffffu, bad)) set_status(a.ws.status, MOE_ERR_NONFINITE);
+    const int t = t0 + tt;
+    float lsel = 0.f, lmax = 0.f, z = 0.f;
+    int esel = 0;
+    for (int j = 0; j < k; ++j) {
+      // best (value desc, index asc) over the lane's candidates, then over the warp
+      float bv = -INFINITY;
+      int be = 0x7FFFFFFF;
+#pragma unroll
+      for (int jj = 0; jj < NJ; ++jj) {
+        const int e = lane + 32 * jj;
+        if (e < E && (l[jj] > bv || (l[jj] == bv && e < be))) {
+          bv = l[jj];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if (be >= E) be = j;  // only when every logit was non-finite; the status already says so
+      if (j == 0) lmax = bv;
+      // remove the winner from its owner's candidates
+#pragma unroll
+      for (int jj = 0; jj < NJ; ++jj)
+        if (lane + 32 * jj == be) l[jj] = -INFINITY;
+      const float ex = expf(bv - lmax);
+      z += ex;
+      if (lane == j) {
+        lsel = ex;
+        esel = be;
+      }
+    }
+    if (lane < k) {
+      a.ws.topk_idx[(int64_t)t * k + lane] = esel;
+      a.ws.topk_w[(int64_t)t * k + lane] = lsel / z;
+      atomicAdd(&a.ws.counts[esel], 1);
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------------
+// Grouping: CTA e lists expert e's pairs in token order (exclusive block scan of the
+// per-token match flags), writes perm / inv / w_sorted, its offsets entry and its
+// token tiles.  Deterministic: every position is a count, no order of atomics.
+// ----------------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) group_kernel(FwdArgs a, int tile_tokens) {
+  __shared__ int s_warp[32];
+  __shared__ int s_base, s_tile_base, s_total_tiles, s_off;
+  const int e = blockIdx.x, E = a.E, k = a.k, T = a.T;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    int off = 0, tb = 0, tot = 0;
+    for (int q = 0; q < E; ++q) {
+      const int c = a.ws.counts[q];
+      const int nt = (c + tile_tokens - 1) / tile_tokens;
+      if (q < e) {
+        off += c;
+        tb += nt;
+      }
+      tot += nt;
+    }
+    s_off = off;
+    s_tile_base = tb;
+    s_total_tiles = tot;
+    s_base = 0;
+  }
+  __syncthreads();
+  const int off = s_off;
+  const int cnt = a.ws.counts[e];
+  a.ws.offsets[e] = off;
+  if (e == E - 1) a.ws.offsets[E] = off + cnt;
+  if (e == 0) a.ws.ntiles[0] = s_total_tiles;
+  for (int i = tid; i * tile_tokens < cnt; i += blockDim.x) {
+    Tile tl;
+    tl.e = e;
+    tl.row0 = off + i * tile_tokens;
+    tl.rows = min(tile_tokens, cnt - i * tile_tokens);
+    tl.pad = 0;
+    a.ws.tiles[s_tile_base + i] = tl;
+  }
+  for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+    const int t = t0 + tid;
+    int slot = -1;
+    if (t < T)
+      for (int s = 0; s < k; ++s)
+        if (a.ws.topk_idx[(int64_t)t * k + s] == e) slot = s;
+    const unsigned m = __ballot_sync(0xffffffffu, slot >= 0);
+    if (lane == 0) s_warp[warp] = __popc(m);
+    __syncthreads();
+    if (warp == 0) {
+      int v = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      s_warp[lane] = incl - v;  // exclusive prefix of the warps
+    }
+    __syncthreads();
+    if (slot >= 0) {
+      const int pos = off + s_base + s_warp[warp] + __popc(m & ((1u << lane) - 1u));
+      const int q = t * k + slot;
+      a.ws.perm[pos] = q;
+      a.ws.inv[q] = pos;
+      a.ws.w_sorted[pos] = a.ws.topk_w[q];
+    }
+    __syncthreads();
+    if (tid == blockDim.x - 1) s_base += s_warp[warp] + __popc(m);
+    __syncthreads();
+  }
+}
+
+// xs[p] = xe[perm[p] / k]: 16-byte copies, one warp per row.
+__global__ void gather_kernel(FwdArgs a) {
+  const int P = a.T * a.k;
+  const int lane = threadIdx.x & 31;
+  const int n16 = a.d / 8;
+  for (int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x >> 5)) {
+    const int t = a.ws.perm[p] / a.k;
+    const uint4* src = reinterpret_cast<const uint4*>(a.ws.xe + (int64_t)t * a.d);
+    uint4* dst = reinterpret_cast<uint4*>(a.ws.xs + (int64_t)p * a.d);
+    for (int i = lane; i < n16; i += 32) dst[i] = src[i];
+  }
+}
+
+// y[t] = bf16(x[t] + sum_j ys[inv[t*k + j]]), j in slot order.
+__global__ void combine_kernel(FwdArgs a) {
+  const int i4 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i4 >= a.d) return;
+  for (int t = blockIdx.y; t < a.T; t += gridDim.y) {
+  const uint2 xr = *reinterpret_cast<const uint2*>(a.x + (int64_t)t * a.d + i4);
+  float v[4] = {__uint_as_float(xr.x << 16), __uint_as_float(xr.x & 0xFFFF0000u), __uint_as_float(xr.y << 16),
+                __uint_as_float(xr.y & 0xFFFF0000u)};
+  for (int j = 0; j < a.k; ++j) {
+    const int p = a.ws.inv[(int64_t)t * a.k + j];
+    const float4 o = *reinterpret_cast<const float4*>(a.ws.ys + (int64_t)p * a.d + i4);
+    v[0] += o.x;
+    v[1] += o.y;
+    v[2] += o.z;
+    v[3] += o.w;
+  }
+  uint2 out;
+  out.x = (uint32_t)f32_to_bf16_rne(v[0]) | ((uint32_t)f32_to_bf16_rne(v[1]) << 16);
+  out.y = (uint32_t)f32_to_bf16_rne(v[2]) | ((uint32_t)f32_to_bf16_rne(v[3]) << 16);
+  *reinterpret_cast<uint2*>(a.y + (int64_t)t * a.d + i4) = out;
+  }
+}
+
+template <int NJ>
+int launch_route_nj(const FwdArgs& a) {
+  const int EP = 32 * NJ;
+  const size_t smem = sizeof(float) * (RT + RT * (RK + 1) + RK * (EP + 1) + RT * (EP + 1));
+  if (cudaFuncSetAttribute(route_kernel<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return -1;
+  ev_before(a);
+  route_kernel<NJ><<<(a.T + RT - 1) / RT, 256, smem, a.stream>>>(a);
+  ev_after(a);
+  return 1;
+}
+
+}  // namespace
+
+int launch_quantize(const float* w, int64_t rows, int32_t N, int32_t K, int32_t E, uint8_t* codes,
+                    uint8_t* scales, int32_t* status, cudaStream_t st) {
+  (void)E;
+  const int64_t nblocks = rows * (K / 32);
+  const int64_t want = (nblocks + 7) / 8;
+  const int grid = (int)std::min<int64_t>(want, 148 * 64);
+  quantize_kernel<<<grid, 256, 0, st>>>(w, nblocks, N, K, codes, scales, status);
+  return cudaGetLastError() == cudaSuccess ? 1 : -1;
+}
+
+int launch_route(const FwdArgs& a, int tile_tokens) {
+  int n = 0;
+  if (cudaMemsetAsync(a.ws.counts, 0, sizeof(int32_t) * a.E, a.stream) != cudaSuccess) return -1;
+  int r;
+  if (a.E <= 32) r = launch_route_nj<1>(a);
+  else if (a.E <= 64) r = launch_route_nj<2>(a);
+  else if (a.E <= 128) r = launch_route_nj<4>(a);
+  else r = launch_route_nj<8>(a);
+  if (r < 0) return -1;
+  n += r;
+  ev_before(a);
+  group_kernel<<<a.E, 1024, 0, a.stream>>>(a, tile_tokens);
+  ev_after(a);
+  ++n;
+  const int P = a.T * a.k;
+  ev_before(a);
+  gather_kernel<<<std::min((P + 7) / 8, 148 * 16), 256, 0, a.stream>>>(a);
+  ev_after(a);
+  ++n;
+  return cudaGetLastError() == cudaSuccess ? n : -1;
+}
+
+int launch_combine(const FwdArgs& a) {
+  dim3 grid((a.d / 4 + 127) / 128, std::min(a.T, 65535));
+  ev_before(a);
+  combine_kernel<<<grid, 128, 0, a.stream>>>(a);
+  ev_after(a);
+  return cudaGetLastError() == cudaSuccess ? 1 : -1;
+}
+
+}  // namespace moe

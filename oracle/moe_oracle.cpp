@@ -45,6 +45,7 @@
 // Oracle storage layout (its own, documented here): codes [rows][K/2], two codes
 // per byte, low nibble = even k; scale bytes [rows][K/32].
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -156,9 +157,12 @@ double oracle_e2m1_value(int32_t code) { return e2m1_value(code & 15); }
 // not finite (outputs for such blocks are unspecified).
 int32_t oracle_quantize(const float* w, int64_t rows, int32_t K, uint8_t* codes, uint8_t* scales) {
   if (K % 32 != 0) return 2;
-  int32_t status = 0;
   const int nb = K / 32;
-  for (int64_t r = 0; r < rows; ++r) {
+  std::atomic<int32_t> any_bad{0};
+  // Rows are independent; split them over threads.
+  parallel_chunks(rows, 0, [&](int64_t r0, int64_t r1) {
+  int32_t status = 0;
+  for (int64_t r = r0; r < r1; ++r) {
     for (int b = 0; b < nb; ++b) {
       const float* blk = w + r * K + b * 32;
       double amax = 0.0;
@@ -181,7 +185,9 @@ int32_t oracle_quantize(const float* w, int64_t rows, int32_t K, uint8_t* codes,
       }
     }
   }
-  return status;
+  if (status) any_bad = 1;
+  });
+  return any_bad.load();
 }
 
 // Decode rows to fp64: value = E2M1(code) * 2^(byte - 127).  Returns 1 if a

@@ -1,0 +1,99 @@
+"""GPU-side assembly of parity cases (test infrastructure).
+
+Inputs come from ``synth``; the library quantizes the fp32 weights on the GPU and
+the oracle quantizes the same fp32 weights on the CPU, expert by expert, so the
+two sides share nothing but the generator.  The GPU's codes and scales are
+compared with the oracle's bit for bit as they are produced.
+"""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import torch
+
+import mxfp4_expert_gemm_b200 as moe
+import oracle
+import synth
+from _inputs import routed_inputs
+
+
+def bf16_dev(u16: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def bf16_host(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@functools.lru_cache(maxsize=2)
+def weights(seed: int, E: int, d: int, I: int, w1_mul: float):
+    """GPU MXFP4 weights (library layout) + oracle MXFP4 weights + bit-exactness record."""
+    cfg = synth.MoEConfig("w", T=1, d=d, I=I, E=E, k=1, seed=seed, w1_mul=w1_mul)
+    dev = "cuda"
+    g1c = torch.empty((E, 2 * I, d // 2), dtype=torch.uint8, device=dev)
+    g1s = torch.empty((E, d // 32, 2 * I), dtype=torch.uint8, device=dev)
+    g2c = torch.empty((E, d, I // 2), dtype=torch.uint8, device=dev)
+    g2s = torch.empty((E, I // 32, d), dtype=torch.uint8, device=dev)
+    o1c = np.empty((E, 2 * I, d // 2), np.uint8)
+    o1s = np.empty((E, 2 * I, d // 32), np.uint8)
+    o2c = np.empty((E, d, I // 2), np.uint8)
+    o2s = np.empty((E, d, I // 32), np.uint8)
+    mismatches = 0
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for e in range(E):
+        for w, gc, gs, oc, os_ in ((synth.w1_expert(cfg, e), g1c, g1s, o1c, o1s),
+                                   (synth.w2_expert(cfg, e), g2c, g2s, o2c, o2s)):
+            wt = torch.from_numpy(w).cuda()
+            moe.moe_mxfp4_quantize(wt, gc[e:e + 1], gs[e:e + 1], status_word=status)
+            oc[e], os_[e] = oracle.quantize(w)
+            mismatches += int(np.count_nonzero(gc[e].cpu().numpy() != oc[e]))
+            mismatches += int(np.count_nonzero(gs[e].cpu().numpy().T != os_[e]))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return dict(gpu=(g1c, g1s, g2c, g2s), oracle=(o1c, o1s, o2c, o2s), mismatches=mismatches)
+
+
+def case(cfg: synth.MoEConfig):
+    """Everything a parity test needs for one workload."""
+    x, gamma, rw, rb, attempts, r = routed_inputs(cfg)
+    W = weights(cfg.seed, cfg.E, cfg.d, cfg.I, cfg.w1_mul)
+    return dict(cfg=cfg, x=x, gamma=gamma, rw=rw, rb=rb, route=r, W=W,
+                x_dev=bf16_dev(x), gamma_dev=torch.from_numpy(gamma).cuda(), rw_dev=torch.from_numpy(rw).cuda(),
+                rb_dev=torch.from_numpy(rb).cuda())
+
+
+def run_gpu(c, path, T=None):
+    cfg = c["cfg"]
+    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, cfg.rms_eps, cfg.swiglu_limit, path=path)
+    T = cfg.T
+    ws = moe.new_workspace(dims, T)
+    y, r = moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws,
+                           want_routing=True)
+    st = moe.moe_device_status(ws)
+    return dict(y=y, routing=r, ws=ws, dims=dims, status=st)
+
+
+def oracle_rows(c, tokens=None, want_h=False):
+    cfg = c["cfg"]
+    return oracle.moe_forward(c["x"], c["gamma"], c["rw"], c["rb"], *c["W"]["oracle"], I=cfg.I, k=cfg.k,
+                              eps=cfg.rms_eps, limit=cfg.swiglu_limit, tokens=tokens, want_h=want_h)
+
+
+def parity_stats(y_gpu_u16, y_ref_u16, x_u16) -> dict:
+    f = lambda u: synth.bf16_to_f32(u).astype(np.float64)
+    yg, yr, x = f(y_gpu_u16), f(y_ref_u16), f(x_u16)
+    diff = yg - yr
+    rms = float(np.sqrt(np.mean(yr * yr)))
+    dref = yr - x
+    return dict(rel_fro=float(np.linalg.norm(diff) / np.linalg.norm(yr)),
+                max_abs=float(np.abs(diff).max()),
+                max_abs_over_rms=float(np.abs(diff).max() / rms),
+                delta_rel_fro=float(np.linalg.norm(diff) / max(np.linalg.norm(dref), 1e-30)),
+                exact_frac=float(np.mean(y_gpu_u16 == y_ref_u16)))
+
+
+def assert_parity(st: dict, label: str = ""):
+    """The layer's tolerance: relative Frobenius <= 1e-2 and max-abs <= 5e-2 x RMS(y*)."""
+    assert st["rel_fro"] <= 1e-2, (label, st)
+    assert st["max_abs_over_rms"] <= 5e-2, (label, st)

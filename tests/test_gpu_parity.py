@@ -1,0 +1,229 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle, same seeded inputs.
+
+Bars: expert indices, per-expert counts, offsets and the grouping bit-exact;
+MXFP4 codes and scales bit-exact; outputs within relative Frobenius 1e-2 and
+max-abs 5e-2 x RMS(y*) of the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mxfp4_expert_gemm_b200 as moe
+import oracle
+import synth
+from _gpu_case import assert_parity, bf16_dev, bf16_host, case, oracle_rows, parity_stats, run_gpu, weights
+
+pytestmark = pytest.mark.gpu
+
+C = synth.CONFIGS
+SMALL = {
+    "tiny": C["tiny"],
+    "decode_20b": C["decode_20b"],
+    "odd": synth.MoEConfig("odd", T=37, d=192, I=320, E=5, k=3),
+    "k_eq_E": synth.MoEConfig("k_eq_E", T=24, d=128, I=128, E=4, k=4),
+    "single": synth.MoEConfig("single", T=9, d=128, I=192, E=1, k=1),
+    "wide_E": synth.MoEConfig("wide_E", T=16, d=256, I=128, E=256, k=8),
+    "mid_ragged": synth.MoEConfig("mid_ragged", T=200, d=2880, I=2880, E=8, k=4),
+    "clamp": synth.MoEConfig("clamp", T=32, d=2880, I=2880, E=4, k=2, w1_mul=8.0),
+}
+PATHS = ["simt", "gemv", "gemm"]
+
+
+def _pairs(idx: np.ndarray, perm: np.ndarray, k: int):
+    """(token, expert) pairs in sorted order."""
+    t = perm // k
+    return np.stack([t, idx[t, perm % k]], axis=1)
+
+
+# ------------------------------------------------------------------------------ quantization
+
+
+@pytest.mark.parametrize("name", ["tiny", "odd", "decode_20b"])
+def test_quantize_bit_exact(name):
+    cfg = SMALL[name]
+    W = weights(cfg.seed, cfg.E, cfg.d, cfg.I, cfg.w1_mul)
+    assert W["mismatches"] == 0
+
+
+def test_quantize_special_values_bit_exact():
+    rng = np.random.default_rng(7)
+    rows = []
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0, -0.1, 0.2, 0.3, -2.75, 6.0, -7.9, -0.0, 4.0],
+                    np.float32)
+    rows.append(np.concatenate([ties, ties * -1]))
+    rows.append(np.zeros(32, np.float32))                                   # all-zero block
+    rows.append(np.full(32, 1e-40, np.float32) * np.arange(32))             # subnormal amax
+    rows.append((rng.standard_normal(32) * 3e37).astype(np.float32))        # near the top of fp32
+    rows.append(np.exp2(np.arange(-16, 16)).astype(np.float32))             # powers of two
+    rows.append(np.nextafter(np.exp2(np.arange(-16, 16)), 0).astype(np.float32))
+    w = np.stack(rows).astype(np.float32)
+    w = np.concatenate([w, (rng.standard_normal((58, 32)) * 0.02).astype(np.float32)])  # 64 rows
+    w = np.tile(w, (1, 2))  # K = 64
+    codes, scales = moe.moe_mxfp4_quantize(torch.from_numpy(w).cuda())
+    oc, os_ = oracle.quantize(w)
+    np.testing.assert_array_equal(codes[0].cpu().numpy(), oc)
+    np.testing.assert_array_equal(scales[0].cpu().numpy().T, os_)
+
+
+def test_quantize_non_finite_is_flagged():
+    w = np.ones((16, 64), np.float32)
+    w[3, 40] = np.inf
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    codes, scales = moe.moe_mxfp4_quantize(torch.from_numpy(w).cuda(), status_word=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == moe.MOE_ERR_NONFINITE
+    assert scales[0, 1, 3].item() == 0xFF and scales[0, 0, 3].item() != 0xFF
+
+
+# ------------------------------------------------------------------------------ routing / grouping
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_route_bit_exact(name):
+    c = case(SMALL[name])
+    cfg = c["cfg"]
+    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k)
+    ws = moe.new_workspace(dims, cfg.T)
+    out = moe.moe_route(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], ws)
+    assert moe.moe_device_status(ws) == moe.MOE_OK
+    idx = out["topk_idx"].cpu().numpy()
+    ref = c["route"]
+    np.testing.assert_array_equal(np.sort(idx, 1), np.sort(ref["idx"], 1))
+    gr = oracle.group(ref["idx"], cfg.E)
+    np.testing.assert_array_equal(out["counts"].cpu().numpy(), gr["counts"])
+    np.testing.assert_array_equal(out["offsets"].cpu().numpy(), gr["offsets"])
+    np.testing.assert_array_equal(_pairs(idx, out["perm"].cpu().numpy(), cfg.k),
+                                  _pairs(ref["idx"], gr["perm"], cfg.k))
+    # weights per (token, expert); slot order follows the logits (ties aside)
+    wg = out["topk_w"].cpu().numpy()
+    for t in range(cfg.T):
+        m_g = dict(zip(idx[t].tolist(), wg[t].tolist()))
+        m_o = dict(zip(ref["idx"][t].tolist(), ref["w"][t].tolist()))
+        for e in m_o:
+            assert abs(m_g[e] - m_o[e]) <= 2e-6, (t, e, m_g[e], m_o[e])
+    np.testing.assert_allclose(wg.sum(1), 1.0, atol=2e-6)
+    lg = ref["logits"][np.arange(cfg.T)[:, None], idx]
+    assert np.all(np.diff(lg, axis=1) <= 1e-5)
+
+
+# ------------------------------------------------------------------------------ whole layer
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_parity(name, path):
+    c = case(SMALL[name])
+    cfg = c["cfg"]
+    g = run_gpu(c, path)
+    assert g["status"] == moe.MOE_OK, moe.status_string(g["status"])
+    ref = oracle_rows(c)
+    st = parity_stats(bf16_host(g["y"]), ref["y"], c["x"])
+    assert_parity(st, f"{name}/{path}")
+    assert st["delta_rel_fro"] <= 2.5e-2, st
+    np.testing.assert_array_equal(np.sort(g["routing"]["topk_idx"].cpu().numpy(), 1), np.sort(ref["idx"], 1))
+
+
+@pytest.mark.parametrize("path", ["gemv", "gemm", "simt"])
+def test_swiglu_output_h_matches_oracle(path):
+    """The gate_up stage alone: h (bf16 values) in the workspace vs the oracle's h."""
+    c = case(SMALL["mid_ragged"])
+    cfg = c["cfg"]
+    g = run_gpu(c, path)
+    assert g["status"] == moe.MOE_OK
+    P = cfg.T * cfg.k
+    h = moe.workspace_view(g["ws"], g["dims"], cfg.T, "h", torch.float16, (P, cfg.I)).float().cpu().numpy()
+    inv = moe.workspace_view(g["ws"], g["dims"], cfg.T, "inv", torch.int32, (P,)).cpu().numpy()
+    idx = g["routing"]["topk_idx"].cpu().numpy()
+    ref = oracle_rows(c, want_h=True)
+    href = synth.bf16_to_f32(ref["h"]).astype(np.float64)  # [T, k, I] in the oracle's slot order
+    num = den = 0.0
+    for t in range(cfg.T):
+        for s in range(cfg.k):
+            so = int(np.nonzero(ref["idx"][t] == idx[t, s])[0][0])
+            diff = h[inv[t * cfg.k + s]] - href[t, so]
+            num += float(diff @ diff)
+            den += float(href[t, so] @ href[t, so])
+    assert np.sqrt(num / den) <= 1e-2
+
+
+@pytest.mark.parametrize("name,path,n_sample", [
+    ("prefill_20b", "gemm", 48), ("prefill_20b", "gemv", 16),
+    ("moe_120b", "gemm", 48), ("skew_120b", "gemm", 48), ("skew_120b", "auto", 16),
+])
+def test_full_size_sampled(name, path, n_sample):
+    """Full-size workloads: all routing bit-exact, outputs on a sample of tokens."""
+    c = case(C[name])
+    cfg = c["cfg"]
+    assert c["W"]["mismatches"] == 0
+    g = run_gpu(c, path)
+    assert g["status"] == moe.MOE_OK, moe.status_string(g["status"])
+    idx = g["routing"]["topk_idx"].cpu().numpy()
+    np.testing.assert_array_equal(np.sort(idx, 1), np.sort(c["route"]["idx"], 1))
+    np.testing.assert_array_equal(g["routing"]["counts"].cpu().numpy(),
+                                  np.bincount(c["route"]["idx"].ravel(), minlength=cfg.E))
+    rng = np.random.default_rng(0)
+    toks = np.sort(rng.choice(cfg.T, size=n_sample, replace=False)).astype(np.int32)
+    toks[0], toks[-1] = 0, cfg.T - 1
+    ref = oracle_rows(c, tokens=toks)
+    y = bf16_host(g["y"])[toks]
+    st = parity_stats(y, ref["y"], c["x"][toks])
+    assert_parity(st, f"{name}/{path}")
+
+
+# ------------------------------------------------------------------------------ edge cases
+
+
+def test_T_zero_and_one():
+    c = case(SMALL["tiny"])
+    cfg = c["cfg"]
+    for path in ("gemv", "gemm", "simt"):
+        dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path=path)
+        ws = moe.new_workspace(dims, 1)
+        y = moe.moe_forward(dims, c["x_dev"][:1], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws)
+        assert moe.moe_device_status(ws) == moe.MOE_OK
+        ref = oracle_rows(c, tokens=np.array([0], np.int32))
+        assert_parity(parity_stats(bf16_host(y), ref["y"], c["x"][:1]), path)
+        # T = 0 launches nothing
+        moe.moe_forward(dims, c["x_dev"][:0], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws)
+        assert moe.last_launch_count() == 0
+
+
+def test_deterministic():
+    c = case(SMALL["mid_ragged"])
+    for path in ("gemm", "gemv"):
+        a = bf16_host(run_gpu(c, path)["y"])
+        b = bf16_host(run_gpu(c, path)["y"])
+        np.testing.assert_array_equal(a, b)
+
+
+def test_scale_out_of_f16_range_is_reported():
+    c = case(SMALL["tiny"])
+    cfg = c["cfg"]
+    g1c, g1s, g2c, g2s = (t.clone() for t in c["W"]["gpu"])
+    g1s[0, 0, 0] = 127 + 20   # 2^20: E2M1 * 2^20 is not exact in f16
+    for path, expect in (("gemm", moe.MOE_ERR_RANGE), ("gemv", moe.MOE_ERR_RANGE), ("simt", moe.MOE_OK)):
+        dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path=path)
+        ws = moe.new_workspace(dims, cfg.T)
+        moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], g1c, g1s, g2c, g2s, ws)
+        assert moe.moe_device_status(ws) == expect, path
+
+
+def test_non_finite_input_is_reported():
+    c = case(SMALL["tiny"])
+    cfg = c["cfg"]
+    x = c["x"].copy()
+    x[3, 5] = 0x7F80  # +inf
+    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path="gemm")
+    ws = moe.new_workspace(dims, cfg.T)
+    moe.moe_forward(dims, bf16_dev(x), c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws)
+    assert moe.moe_device_status(ws) == moe.MOE_ERR_NONFINITE
+    assert moe.moe_device_status(ws) == moe.MOE_OK  # reading clears the word
+
+
+def test_launch_count_reported():
+    c = case(SMALL["tiny"])
+    cfg = c["cfg"]
+    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path="gemm")
+    ws = moe.new_workspace(dims, cfg.T)
+    moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws)
+    assert moe.last_launch_count() == 6  # route, group, gather, gate_up, down, combine
