@@ -161,10 +161,12 @@ def device_inputs(cfg, rank, need_oracle_weights):
     gamma, rw, rb = synth.norm_weight(cfg), synth.router_weight(cfg), synth.router_bias(cfg)
     E, d, I = cfg.E, cfg.d, cfg.I
     dev = "cuda"
-    w1c = torch.empty((E, 2 * I, d // 2), dtype=torch.uint8, device=dev)
-    w1s = torch.empty((E, d // 32, 2 * I), dtype=torch.uint8, device=dev)
-    w2c = torch.empty((E, d, I // 2), dtype=torch.uint8, device=dev)
-    w2s = torch.empty((E, I // 32, d), dtype=torch.uint8, device=dev)
+    s1c, s1s = moe.mxfp4_shapes(E, 2 * I, d)
+    s2c, s2s = moe.mxfp4_shapes(E, d, I)
+    w1c = torch.empty(s1c, dtype=torch.uint8, device=dev)
+    w1s = torch.empty(s1s, dtype=torch.uint8, device=dev)
+    w2c = torch.empty(s2c, dtype=torch.uint8, device=dev)
+    w2s = torch.empty(s2s, dtype=torch.uint8, device=dev)
     ow = None
     if need_oracle_weights:
         import oracle

@@ -84,12 +84,17 @@ typedef struct {
 } moe_dims;
 
 /* ---------------------------------------------------------------- MXFP4 storage
- * A weight tensor [E][N][K] (K = reduction axis, K % 32 == 0) is stored as
- *   codes  [E][N][K/2] bytes: two E2M1 codes per byte, the even k in the low nibble;
- *          code bits: sign (bit 3), exponent (bits 2..1, bias 1), mantissa (bit 0);
- *   scales [E][K/32][N] bytes: E8M0, value 2^(byte - 127), one per 32 consecutive k of
- *          a row (K-block-major so that every row stride is N bytes, a TMA-legal stride
- *          whenever N % 16 == 0).
+ * A weight tensor [E][N][K] (K = reduction axis; N and K multiples of 64) is stored in
+ * blocks of 64 rows x 64 k, each block one contiguous run (exactly 4.25 bits/param):
+ *   codes  [E][N/64][K/64][64 rows][32 bytes]: row r of a block keeps its 64 E2M1
+ *          codes as two 16-byte chunks (k 0..31, k 32..63); chunk c is stored at
+ *          chunk position c ^ ((r >> 2) & 1); byte j of a chunk holds k = 2j in the low
+ *          nibble and k = 2j+1 in the high nibble.  Code bits: sign (bit 3), exponent
+ *          (bits 2..1, bias 1), mantissa (bit 0).
+ *   scales [E][N/64][K/64][2][64] bytes: E8M0 scale 2^(byte - 127) of row r for
+ *          k = 32c .. 32c+31 of the block at index [c][r].
+ * One block is what the tensor-core kernels stream per pipeline stage: 2048 contiguous
+ * code bytes and 128 contiguous scale bytes, copied with single bulk copies.
  * W1 (gate_up) is [E][2I][d]: rows 0..I-1 are the gate projection, I..2I-1 the up
  * projection.  W2 (down) is [E][d][I].
  */
@@ -104,7 +109,7 @@ size_t moe_mxfp4_scales_bytes(int32_t E, int32_t N, int32_t K); /* E*(K/32)*N */
  * status_word: optional device int32; MOE_ERR_NONFINITE is OR-ed into it when a
  * block holds Inf/NaN (that block's scale byte is then 0xFF, the E8M0 NaN).
  * Errors: MOE_ERR_INVALID_ARG (null/misaligned pointer, E/N/K <= 0),
- * MOE_ERR_UNSUPPORTED_SHAPE (K % 32 != 0), MOE_ERR_CUDA. */
+ * MOE_ERR_UNSUPPORTED_SHAPE (N or K not a multiple of 64), MOE_ERR_CUDA. */
 moe_status moe_mxfp4_quantize(const float* w, int32_t E, int32_t N, int32_t K, uint8_t* codes,
                               uint8_t* scales, int32_t* status_word, void* stream);
 

@@ -144,17 +144,26 @@ def moe_mxfp4_scales_bytes(E: int, N: int, K: int) -> int:
     return lib().moe_mxfp4_scales_bytes(E, N, K)
 
 
+def mxfp4_shapes(E: int, N: int, K: int):
+    """Tensor shapes of the library's MXFP4 block layout (see include/moe_mxfp4.h):
+    codes [E, N/64, K/64, 64, 32], scales [E, N/64, K/64, 2, 64] (uint8)."""
+    return (E, N // 64, K // 64, 64, 32), (E, N // 64, K // 64, 2, 64)
+
+
 def moe_mxfp4_quantize(w: torch.Tensor, codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
                        status_word: torch.Tensor | None = None, stream=None):
-    """fp32 weights [E, N, K] -> (codes uint8 [E, N, K/2], scales uint8 [E, K/32, N])."""
+    """fp32 weights [E, N, K] -> (codes, scales) in the library's MXFP4 block layout."""
     if w.dim() == 2:
         w = w.unsqueeze(0)
     _need(w, torch.float32, "w")
     E, N, K = w.shape
+    cs, ss = mxfp4_shapes(E, N, K)
     if codes is None:
-        codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=w.device)
+        codes = torch.empty(cs, dtype=torch.uint8, device=w.device)
     if scales is None:
-        scales = torch.empty((E, K // 32, N), dtype=torch.uint8, device=w.device)
+        scales = torch.empty(ss, dtype=torch.uint8, device=w.device)
+    if codes.numel() != E * N * K // 2 or scales.numel() != E * N * K // 32:
+        raise ValueError("codes / scales have the wrong size")
     _check(lib().moe_mxfp4_quantize(_ptr(w), E, N, K, _ptr(codes), _ptr(scales), _ptr(status_word), _stream(stream)),
            "moe_mxfp4_quantize")
     return codes, scales

@@ -50,6 +50,7 @@ moe_status prepare(const moe_dims* dm, int32_t T, const uint16_t* x, const float
                    const float* router_b, void* ws, size_t ws_bytes, moe::FwdArgs& a, moe::WsLayout& L) {
   moe_status st = check_dims(dm, T);
   if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;  // nothing to do; empty tensors may carry null pointers
   if (!x || !norm_w || !router_w || !ws) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(norm_w) || !aligned16(router_w) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
   if (router_b && !aligned16(router_b)) return MOE_ERR_INVALID_ARG;
@@ -97,7 +98,7 @@ moe_status moe_mxfp4_quantize(const float* w, int32_t E, int32_t N, int32_t K, u
   g_last_launches = 0;
   if (!w || !codes || !scales || E <= 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w) || !aligned16(codes) || !aligned16(scales)) return MOE_ERR_INVALID_ARG;
-  if (K % 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (K % 64 || N % 64) return MOE_ERR_UNSUPPORTED_SHAPE;
   moe_status st = check_device();
   if (st != MOE_OK) return st;
   const int n = moe::launch_quantize(w, (int64_t)E * N, N, K, E, codes, scales, status_word,
@@ -155,6 +156,7 @@ moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x,
   moe::WsLayout L;
   moe_status st = prepare(dims, T, x, norm_w, router_w, router_b, ws, ws_bytes, a, L);
   if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
   if (!w1_codes || !w1_scales || !w2_codes || !w2_scales || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w1_codes) || !aligned16(w1_scales) || !aligned16(w2_codes) || !aligned16(w2_scales) ||
       !aligned16(y))

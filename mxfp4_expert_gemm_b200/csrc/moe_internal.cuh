@@ -149,6 +149,35 @@ inline void ev_after(const FwdArgs& a) {
   }
 }
 
+// ------------------------------------------------------------------ MXFP4 storage layout
+// Weights [E][N][K] are stored in blocks of 64 rows x 64 k (N % 64 == 0, K % 64 == 0):
+//   codes  [E][N/64][K/64][64 rows][32 bytes]   (one 2048-byte run per block)
+//   scales [E][N/64][K/64][2][64]               (one 128-byte run per block)
+// Row r of a block keeps its 64 codes as two 16-byte chunks (k 0..31 and k 32..63);
+// chunk c sits at chunk position c ^ ((r >> 2) & 1), so that consecutive rows read by
+// consecutive threads fall in different shared-memory banks.  Byte j of a chunk holds
+// k = 2j (low nibble) and k = 2j + 1 (high nibble).  Scale byte (c, r) is the E8M0
+// scale of row r, k = 32c .. 32c + 31 of the block.
+constexpr int kBlkRows = 64;
+constexpr int kBlkK = 64;
+constexpr int kBlkCodeBytes = kBlkRows * kBlkK / 2;   // 2048
+constexpr int kBlkScaleBytes = kBlkRows * kBlkK / 32; // 128
+
+__host__ __device__ __forceinline__ int64_t mx_block_index(int64_t e, int64_t rb, int64_t ks, int64_t N, int64_t K) {
+  return (e * (N / kBlkRows) + rb) * (K / kBlkK) + ks;
+}
+
+// Byte offset of the 16-byte code chunk holding k = 32*kb .. 32*kb+31 of row n.
+__host__ __device__ __forceinline__ int64_t mx_code_chunk_offset(int64_t e, int64_t n, int64_t kb, int64_t N,
+                                                                  int64_t K) {
+  const int64_t r = n % kBlkRows, c = kb & 1;
+  return mx_block_index(e, n / kBlkRows, kb >> 1, N, K) * kBlkCodeBytes + r * 32 + ((c ^ ((r >> 2) & 1)) << 4);
+}
+
+__host__ __device__ __forceinline__ int64_t mx_scale_offset(int64_t e, int64_t n, int64_t kb, int64_t N, int64_t K) {
+  return mx_block_index(e, n / kBlkRows, kb >> 1, N, K) * kBlkScaleBytes + (kb & 1) * kBlkRows + n % kBlkRows;
+}
+
 // Record the first device-side error in the status word.
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);

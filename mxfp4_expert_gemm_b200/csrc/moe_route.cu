@@ -82,11 +82,142 @@ __global__ void quantize_kernel(const float* __restrict__ w, int64_t nblocks, in
     const int hi = __shfl_down_sync(0xffffffffu, c, 1);
     const int64_t e_idx = row / N;
     const int64_t n = row - e_idx * N;
-    if ((lane & 1) == 0) codes[row * (K / 2) + kb * 16 + (lane >> 1)] = (uint8_t)(c | (hi << 4));
+    if ((lane & 1) == 0)
+      codes[mx_code_chunk_offset(e_idx, n, kb, N, K) + (lane >> 1)] = (uint8_t)(c | (hi << 4));
     if (lane == 0) {
-      scales[(e_idx * kb_per_row + kb) * (int64_t)N + n] = all_finite ? (uint8_t)(s + 127) : (uint8_t)0xFF;
+      scales[mx_scale_offset(e_idx, n, kb, N, K)] = all_finite ? (uint8_t)(s + 127) : (uint8_t)0xFF;
       if (!all_finite) set_status(status, MOE_ERR_NONFINITE);
     }
+  }
+}
+
+// ----------------------------------------------------------------------------------
+// Top-k (value desc, index asc) + softmax over the selected logits for one token, by one
+// warp; the lane holding logit e is lane e % 32.  Writes the outputs and the histogram.
+// ----------------------------------------------------------------------------------
+template <int NJ>
+__device__ __forceinline__ void warp_topk_softmax(float (&l)[NJ], int E, int k, int64_t t, const FwdArgs& a) {
+  const int lane = threadIdx.x & 31;
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    if (lane + 32 * j < E && !isfinite(l[j])) {
+      bad = true;
+      l[j] = -INFINITY;
+    }
+    if (lane + 32 * j >= E) l[j] = -INFINITY;
+  }
+  if (__any_sync(0xffffffffu, bad)) set_status(a.ws.status, MOE_ERR_NONFINITE);
+  float lsel = 0.f, lmax = 0.f, z = 0.f;
+  int esel = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int jj = 0; jj < NJ; ++jj) {
+      const int e = lane + 32 * jj;
+      if (e < E && (l[jj] > bv || (l[jj] == bv && e < be))) {
+        bv = l[jj];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if (be >= E) be = j;  // only when every logit was non-finite; the status already says so
+    if (j == 0) lmax = bv;
+#pragma unroll
+    for (int jj = 0; jj < NJ; ++jj)
+      if (lane + 32 * jj == be) l[jj] = -INFINITY;
+    const float ex = expf(bv - lmax);
+    z += ex;
+    if (lane == j) {
+      lsel = ex;
+      esel = be;
+    }
+  }
+  if (lane < k) {
+    a.ws.topk_idx[t * k + lane] = esel;
+    a.ws.topk_w[t * k + lane] = lsel / z;
+    atomicAdd(&a.ws.counts[esel], 1);
+  }
+}
+
+// ----------------------------------------------------------------------------------
+// Small batches: one CTA per token.  The token's normalized row stays in shared
+// memory (fp32); warp w computes the logits of experts w, w+8, ... with 16-byte loads
+// of the router rows; warp 0 then selects the top-k.
+// ----------------------------------------------------------------------------------
+template <int NJ>
+__global__ void __launch_bounds__(256) route_token_kernel(FwdArgs a) {
+  extern __shared__ float smem[];
+  const int d = a.d, E = a.E;
+  float* s_xn = smem;          // [d]
+  float* s_l = smem + d;       // [32*NJ]
+  __shared__ float s_red[8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t = blockIdx.x;
+  const uint16_t* xr = a.x + t * d;
+  float ss = 0.f;
+  for (int i = tid * 8; i < d; i += 256 * 8) {
+    const uint4 q = *reinterpret_cast<const uint4*>(xr + i);
+    const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = __uint_as_float(wv[j] << 16), hi = __uint_as_float(wv[j] & 0xFFFF0000u);
+      ss = fmaf(lo, lo, ss);
+      ss = fmaf(hi, hi, ss);
+      s_xn[i + 2 * j] = lo;
+      s_xn[i + 2 * j + 1] = hi;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) s_red[warp] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += s_red[w];
+  const float r = 1.0f / sqrtf(tot / (float)d + a.eps);
+  bool range_bad = false;
+  for (int i = tid * 2; i < d; i += 512) {
+    const float v0 = s_xn[i] * r * a.norm_w[i], v1 = s_xn[i + 1] * r * a.norm_w[i + 1];
+    s_xn[i] = v0;
+    s_xn[i + 1] = v1;
+    const float b0 = bf16_to_f32(f32_to_bf16_rne(v0)), b1 = bf16_to_f32(f32_to_bf16_rne(v1));
+    range_bad |= fabsf(b0) > 65504.f || fabsf(b1) > 65504.f;
+    *reinterpret_cast<__half2*>(a.ws.xe + t * d + i) = __floats2half2_rn(b0, b1);
+  }
+  if (range_bad) set_status(a.ws.status, MOE_ERR_RANGE);
+  __syncthreads();
+  for (int e = warp; e < E; e += 8) {
+    const float* wr = a.router_w + (int64_t)e * d;
+    float acc = 0.f;
+#pragma unroll 4
+    for (int i = lane * 4; i < d; i += 128) {
+      const float4 w4 = *reinterpret_cast<const float4*>(wr + i);
+      const float4 x4 = *reinterpret_cast<const float4*>(s_xn + i);
+      acc = fmaf(w4.x, x4.x, acc);
+      acc = fmaf(w4.y, x4.y, acc);
+      acc = fmaf(w4.z, x4.z, acc);
+      acc = fmaf(w4.w, x4.w, acc);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) s_l[e] = acc + (a.router_b ? a.router_b[e] : 0.f);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float l[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) l[j] = (lane + 32 * j < E) ? s_l[lane + 32 * j] : -INFINITY;
+    warp_topk_softmax<NJ>(l, E, a.k, t, a);
   }
 }
 
@@ -94,7 +225,8 @@ __global__ void quantize_kernel(const float* __restrict__ w, int64_t nblocks, in
 // Fused RMSNorm + router GEMV + top-k + softmax, 32 tokens per CTA, 256 threads.
 // Outputs: xe (f16 copy of bf16(xn)), topk_idx, topk_w, expert histogram.
 // ----------------------------------------------------------------------------------
-constexpr int RT = 32;   // tokens per CTA
+constexpr int RT = 32;   // tokens per CTA (tiled kernel)
+constexpr int kTokenKernelMaxT = 1024;  // up to this many tokens: one CTA per token
 constexpr int RK = 64;   // d-chunk
 
 template <int NJ>  // experts per lane group: E <= 32*NJ
@@ -141,30 +273,51 @@ __global__ void __launch_bounds__(256) route_kernel(FwdArgs a) {
     for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
   bool range_bad = false;
 
+  // Register prefetch of the next d-chunk overlaps its global loads with the FMAs.
+  constexpr int XQ = RT * (RK / 2) / 256;   // bf16 pairs of x per thread per chunk
+  constexpr int WQ = RK * 32 * NJ / 256;    // router weights per thread per chunk
+  uint32_t px[XQ];
+  float pw[WQ];
+  auto load_chunk = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < XQ; ++u) {
+      const int q = tid + 256 * u;
+      const int tt = q / (RK / 2), c2 = (q % (RK / 2)) * 2;
+      px[u] = (tt < nt) ? *reinterpret_cast<const uint32_t*>(a.x + (int64_t)(t0 + tt) * d + k0 + c2) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < WQ; ++u) {
+      const int q = tid + 256 * u;
+      const int e = q / RK, kk = q % RK;
+      pw[u] = (e < E) ? a.router_w[(int64_t)e * d + k0 + kk] : 0.f;
+    }
+  };
+  load_chunk(0);
   for (int k0 = 0; k0 < d; k0 += RK) {
-    // x chunk -> xn (fp32, smem) and xe (f16 of bf16(xn), global)
-    for (int q = tid; q < RT * (RK / 2); q += 256) {
+#pragma unroll
+    for (int u = 0; u < XQ; ++u) {
+      const int q = tid + 256 * u;
       const int tt = q / (RK / 2), c2 = (q % (RK / 2)) * 2;
       float v0 = 0.f, v1 = 0.f;
       if (tt < nt) {
-        const int64_t gi = (int64_t)(t0 + tt) * d + k0 + c2;
-        const uint32_t pr = *reinterpret_cast<const uint32_t*>(a.x + gi);
         const float r = s_r[tt];
-        v0 = __uint_as_float(pr << 16) * r * a.norm_w[k0 + c2];
-        v1 = __uint_as_float(pr & 0xFFFF0000u) * r * a.norm_w[k0 + c2 + 1];
+        v0 = __uint_as_float(px[u] << 16) * r * a.norm_w[k0 + c2];
+        v1 = __uint_as_float(px[u] & 0xFFFF0000u) * r * a.norm_w[k0 + c2 + 1];
         const float b0 = bf16_to_f32(f32_to_bf16_rne(v0)), b1 = bf16_to_f32(f32_to_bf16_rne(v1));
         range_bad |= fabsf(b0) > 65504.f || fabsf(b1) > 65504.f;
-        const __half2 hv = __floats2half2_rn(b0, b1);  // exact for bf16 values in f16 range
-        *reinterpret_cast<__half2*>(a.ws.xe + gi) = hv;
+        *reinterpret_cast<__half2*>(a.ws.xe + (int64_t)(t0 + tt) * d + k0 + c2) = __floats2half2_rn(b0, b1);
       }
       s_x[tt * (RK + 1) + c2] = v0;
       s_x[tt * (RK + 1) + c2 + 1] = v1;
     }
-    for (int q = tid; q < RK * EP; q += 256) {  // coalesced along d; padded rows avoid bank conflicts
+#pragma unroll
+    for (int u = 0; u < WQ; ++u) {
+      const int q = tid + 256 * u;
       const int e = q / RK, kk = q % RK;
-      s_w[kk * (EP + 1) + e] = (e < E) ? a.router_w[(int64_t)e * d + k0 + kk] : 0.f;
+      s_w[kk * (EP + 1) + e] = pw[u];
     }
     __syncthreads();
+    if (k0 + RK < d) load_chunk(k0 + RK);
 #pragma unroll 4
     for (int kk = 0; kk < RK; ++kk) {
       float xv[4];
@@ -192,58 +345,9 @@ __global__ void __launch_bounds__(256) route_kernel(FwdArgs a) {
   // Phase C: top-k + softmax per token (warp w: tokens w, w+8, ...).
   for (int tt = warp; tt < nt; tt += 8) {
     float l[NJ];
-    bool bad = false;
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      l[j] = s_l[tt * (EP + 1) + lane + 32 * j];
-      if (lane + 32 * j < E && !isfinite(l[j])) {
-        bad = true;
-        l[j] = -INFINITY;
-      }
-    }
-    if (__any_sync(0xffffffffu, bad)) set_status(a.ws.status, MOE_ERR_NONFINITE);
-    const int t = t0 + tt;
-    float lsel = 0.f, lmax = 0.f, z = 0.f;
-    int esel = 0;
-    for (int j = 0; j < k; ++j) {
-      // best (value desc, index asc) over the lane's candidates, then over the warp
-      float bv = -INFINITY;
-      int be = 0x7FFFFFFF;
-#pragma unroll
-      for (int jj = 0; jj < NJ; ++jj) {
-        const int e = lane + 32 * jj;
-        if (e < E && (l[jj] > bv || (l[jj] == bv && e < be))) {
-          bv = l[jj];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if (be >= E) be = j;  // only when every logit was non-finite; the status already says so
-      if (j == 0) lmax = bv;
-      // remove the winner from its owner's candidates
-#pragma unroll
-      for (int jj = 0; jj < NJ; ++jj)
-        if (lane + 32 * jj == be) l[jj] = -INFINITY;
-      const float ex = expf(bv - lmax);
-      z += ex;
-      if (lane == j) {
-        lsel = ex;
-        esel = be;
-      }
-    }
-    if (lane < k) {
-      a.ws.topk_idx[(int64_t)t * k + lane] = esel;
-      a.ws.topk_w[(int64_t)t * k + lane] = lsel / z;
-      atomicAdd(&a.ws.counts[esel], 1);
-    }
+    for (int j = 0; j < NJ; ++j) l[j] = s_l[tt * (EP + 1) + lane + 32 * j];
+    warp_topk_softmax<NJ>(l, E, k, t0 + tt, a);
   }
 }
 
@@ -358,6 +462,16 @@ __global__ void combine_kernel(FwdArgs a) {
 
 template <int NJ>
 int launch_route_nj(const FwdArgs& a) {
+  if (a.T <= kTokenKernelMaxT) {
+    const size_t smem = sizeof(float) * (a.d + 32 * NJ);
+    if (cudaFuncSetAttribute(route_token_kernel<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return -1;
+    ev_before(a);
+    route_token_kernel<NJ><<<a.T, 256, smem, a.stream>>>(a);
+    ev_after(a);
+    return 1;
+  }
   const int EP = 32 * NJ;
   const size_t smem = sizeof(float) * (RT + RT * (RK + 1) + RK * (EP + 1) + RT * (EP + 1));
   if (cudaFuncSetAttribute(route_kernel<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)

@@ -23,12 +23,12 @@ __device__ __forceinline__ float e2m1_f32(int c) {
   return (c & 8) ? -mag : mag;
 }
 
-// Decode one 32-value block of row `row` (codes: K/2 bytes per row; scales [K/32][N]).
-__device__ __forceinline__ void decode_block(const uint8_t* codes, const uint8_t* scales, int64_t row,
+// Decode one 32-value block of row `row` of expert `e` (library MXFP4 layout).
+__device__ __forceinline__ void decode_block(const uint8_t* codes, const uint8_t* scales, int e, int64_t row,
                                              int64_t N, int K, int kb, float* out, int out_stride,
                                              int32_t* status) {
-  const uint4 q = *reinterpret_cast<const uint4*>(codes + row * (K / 2) + kb * 16);
-  const int sb = scales[(int64_t)kb * N + row];
+  const uint4 q = *reinterpret_cast<const uint4*>(codes + mx_code_chunk_offset(e, row, kb, N, K));
+  const int sb = scales[mx_scale_offset(e, row, kb, N, K)];
   if (sb == 0xFF) set_status(status, MOE_ERR_NONFINITE);
   const float sc = ldexpf(1.0f, sb - 127);
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
@@ -55,8 +55,6 @@ __global__ void __launch_bounds__(256) gate_up_simt(FwdArgs a) {
   const int d = a.d, I = a.I;
   const int j0 = blockIdx.y * SJ;
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
-  const uint8_t* w1c = a.w1c + (int64_t)tl.e * 2 * I * (d / 2);
-  const uint8_t* w1s = a.w1s + (int64_t)tl.e * (d / 32) * 2 * I;
   float ag[4][2] = {}, au[4][2] = {};
   for (int kb = 0; kb < d / SK; ++kb) {
     {  // activations: 64 rows x 32 k (f16), 8 per thread
@@ -78,7 +76,8 @@ __global__ void __launch_bounds__(256) gate_up_simt(FwdArgs a) {
     if (tid < 2 * SJ) {  // weights: 32 gate rows + 32 up rows, one block each
       const int jj = tid % SJ;
       const int64_t row = (tid < SJ) ? (j0 + jj) : (I + j0 + jj);
-      decode_block(w1c, w1s, row, 2 * I, d, kb, (tid < SJ) ? &s_g[0][jj] : &s_u[0][jj], SJ + 1, a.ws.status);
+      decode_block(a.w1c, a.w1s, tl.e, row, 2 * I, d, kb, (tid < SJ) ? &s_g[0][jj] : &s_u[0][jj], SJ + 1,
+                   a.ws.status);
     }
     __syncthreads();
 #pragma unroll 8
@@ -129,8 +128,6 @@ __global__ void __launch_bounds__(256) down_simt(FwdArgs a) {
   const int d = a.d, I = a.I;
   const int m0 = blockIdx.y * SJ;
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
-  const uint8_t* w2c = a.w2c + (int64_t)tl.e * d * (I / 2);
-  const uint8_t* w2s = a.w2s + (int64_t)tl.e * (I / 32) * d;
   float acc[4][2] = {};
   for (int kb = 0; kb < I / SK; ++kb) {
     {
@@ -151,7 +148,7 @@ __global__ void __launch_bounds__(256) down_simt(FwdArgs a) {
     }
     if (tid < SJ) {
       const int m = m0 + tid;
-      if (m < d) decode_block(w2c, w2s, m, d, I, kb, &s_w[0][tid], SJ + 1, a.ws.status);
+      if (m < d) decode_block(a.w2c, a.w2s, tl.e, m, d, I, kb, &s_w[0][tid], SJ + 1, a.ws.status);
       else
         for (int i = 0; i < SK; ++i) s_w[i][tid] = 0.f;
     }

@@ -41,6 +41,9 @@ enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
 struct TcParams {
   const Tile* tiles;
   const int32_t* ntiles;
+  const uint8_t* codes;   // MXFP4 codes of W1 or W2 (library block layout)
+  const uint8_t* scales;
+  int32_t N;              // weight rows per expert (2I or d)
   const float* w_sorted;
   uint16_t* h_out;   // gate_up: [P][I] f16
   float* ys_out;     // down:    [P][d] f32
@@ -60,7 +63,7 @@ struct Cfg {
   static constexpr int COLS_NEEDED = A0 + 32 * STAGES;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 : COLS_NEEDED <= 128 ? 128
                                    : COLS_NEEDED <= 256 ? 256 : 512;
-  static constexpr int TX_BYTES = ACT_BYTES + CODE_BYTES + SCALE_BYTES;
+
   // At most 512 / TMEM_COLS CTAs can hold TMEM on one SM; ask for enough shared memory
   // that no more than that become resident (a third CTA would only wait in tcgen05.alloc).
   static constexpr int SMEM_USED = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
@@ -79,8 +82,7 @@ __device__ __forceinline__ uint32_t f16_pow2_bits(int e) {
 
 template <int MODE, int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_expert_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
-                     const __grid_constant__ CUtensorMap tm_scales, const TcParams p) {
+    tc_expert_kernel(const __grid_constant__ CUtensorMap tm_act, const TcParams p) {
   using C = Cfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   if ((int)blockIdx.x >= *p.ntiles) return;  // uniform: more CTAs are launched than tiles exist
@@ -97,6 +99,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Tile tl = p.tiles[blockIdx.x];
   const int nk = p.K / kBK;
   const int row_tile0 = (MODE == MODE_GATE_UP) ? blockIdx.y * 64 : blockIdx.y * kBM;
+  // The tile's two 64-row halves: gate_up pairs gate rows j0.. with up rows I+j0..;
+  // down takes rows m0..m0+63 and m0+64..m0+127 (the second half may not exist).
+  const int rbA = row_tile0 / kBlkRows;
+  const int rbB = (MODE == MODE_GATE_UP) ? (p.I + row_tile0) / kBlkRows : rbA + 1;
+  const bool halfB = rbB < p.N / kBlkRows;
+  const uint32_t tx_bytes = C::ACT_BYTES + (halfB ? 2 : 1) * (kBlkCodeBytes + kBlkScaleBytes);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -108,8 +116,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     *s_abort = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tm_act);
-    ptx::prefetch_tensormap(&tm_codes);
-    ptx::prefetch_tensormap(&tm_scales);
   }
   if (warp == 1) {
     ptx::tmem_alloc(s_tmem, C::TMEM_COLS);
@@ -132,16 +138,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = kb % STAGES;
         if (kb >= STAGES && !ptx::mbar_wait_bounded(&empty[s], ((kb / STAGES) - 1) & 1, s_abort, kWaitLimitNs))
           break;
-        ptx::mbar_arrive_expect_tx(&full[s], C::TX_BYTES);
+        ptx::mbar_arrive_expect_tx(&full[s], tx_bytes);
         ptx::tma_load_2d(act_s(s), &tm_act, kb * kBK, tl.row0, &full[s]);
-        if (MODE == MODE_GATE_UP) {
-          ptx::tma_load_3d(code_s(s), &tm_codes, kb * (kBK / 2), row_tile0, tl.e, &full[s]);
-          ptx::tma_load_3d(code_s(s) + 64 * 32, &tm_codes, kb * (kBK / 2), p.I + row_tile0, tl.e, &full[s]);
-          ptx::tma_load_3d(scale_s(s), &tm_scales, row_tile0, kb * (kBK / 32), tl.e, &full[s]);
-          ptx::tma_load_3d(scale_s(s) + 128, &tm_scales, p.I + row_tile0, kb * (kBK / 32), tl.e, &full[s]);
-        } else {
-          ptx::tma_load_3d(code_s(s), &tm_codes, kb * (kBK / 2), row_tile0, tl.e, &full[s]);
-          ptx::tma_load_3d(scale_s(s), &tm_scales, row_tile0, kb * (kBK / 32), tl.e, &full[s]);
+        const int64_t bA = mx_block_index(tl.e, rbA, kb, p.N, p.K);
+        ptx::bulk_load(code_s(s), p.codes + bA * kBlkCodeBytes, kBlkCodeBytes, &full[s]);
+        ptx::bulk_load(scale_s(s), p.scales + bA * kBlkScaleBytes, kBlkScaleBytes, &full[s]);
+        if (halfB) {
+          const int64_t bB = mx_block_index(tl.e, rbB, kb, p.N, p.K);
+          ptx::bulk_load(code_s(s) + kBlkCodeBytes, p.codes + bB * kBlkCodeBytes, kBlkCodeBytes, &full[s]);
+          ptx::bulk_load(scale_s(s) + kBlkScaleBytes, p.scales + bB * kBlkScaleBytes, kBlkScaleBytes, &full[s]);
         }
         issued = kb + 1;
       }
@@ -186,15 +191,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;              // TMEM lane quarter this warp may access
     const int row = 32 * q + lane;       // weight row of the tile == TMEM lane
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
-    bool row_valid = true;
-    int scale_off;
-    if (MODE == MODE_GATE_UP) {
-      scale_off = (row < 64) ? row : 128 + (row - 64);
-    } else {
-      scale_off = row;
-      row_valid = row_tile0 + row < p.d;
-    }
-    const int scale_kstride = (MODE == MODE_GATE_UP) ? 64 : 128;
+    const bool row_valid = row < 64 || halfB;
+    const int scale_off = (row < 64) ? row : 128 + (row - 64);   // [half][c][64]
+    constexpr int scale_kstride = 64;
     bool range_bad = false;
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % STAGES;
@@ -216,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 8; ++i) {
         uint32_t o0, o1, o2, o3;
         ptx::e2m1x8_to_f16x8(cw[i], o0, o1, o2, o3);
-        const uint32_t m = (i < 4) ? m0 : m1;
+        const uint32_t m = row_valid ? ((i < 4) ? m0 : m1) : 0u;   // rows past the matrix: zeros
         r[4 * i + 0] = ptx::hmul2_u32(o0, m);
         r[4 * i + 1] = ptx::hmul2_u32(o1, m);
         r[4 * i + 2] = ptx::hmul2_u32(o2, m);
@@ -240,29 +239,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       const int et = threadIdx.x - 64;  // 0..127 over the four epilogue warps
       if (MODE == MODE_GATE_UP) {
-        float* s_u = reinterpret_cast<float*>(smem);                       // [32][64]
+        // Per 32-token chunk the gate thread of column j (lane row j < 64) and the up
+        // thread of the same column (row j + 64) trade halves: the gate side finishes
+        // tokens 0..15 of the chunk, the up side tokens 16..31.
+        float* s_x = reinterpret_cast<float*>(smem);                       // [32][64] exchange
         uint16_t* s_h = reinterpret_cast<uint16_t*>(smem + 32 * 64 * 4);  // [BN][64]
         const float L = p.limit;
+        const bool gate_side = row < 64;
+        const int j = gate_side ? row : row - 64;
+        constexpr int CW = BN < 32 ? BN : 32;   // accumulator columns per chunk
+        constexpr int HW = CW / 2;              // tokens each side finishes
         for (int c0 = 0; c0 < BN; c0 += 32) {
           uint32_t v[32];
           ptx::tmem_ld32(tmem + lane_addr + c0, v);
           ptx::tmem_wait_ld();
-          constexpr int CW = BN < 32 ? BN : 32;  // accumulator columns in this chunk
-          if (row >= 64) {
+          // gate side publishes its g for the upper half, up side its u for the lower half
 #pragma unroll
-            for (int c = 0; c < CW; ++c) s_u[c * 64 + (row - 64)] = __uint_as_float(v[c]);
+          for (int c = 0; c < HW; ++c) {
+            const int cc = gate_side ? HW + c : c;
+            s_x[cc * 64 + j] = __uint_as_float(v[cc]);
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
-          if (row < 64) {
 #pragma unroll
-            for (int c = 0; c < CW; ++c) {
-              const float g = fminf(__uint_as_float(v[c]), L);
-              const float u = fminf(fmaxf(s_u[c * 64 + row], -L), L);
-              const float hval = g / (1.0f + expf(-g)) * u;
-              uint32_t b = __float_as_uint(hval);
-              b = (b + 0x7FFFu + ((b >> 16) & 1u)) & 0xFFFF0000u;  // round to bf16
-              s_h[(c0 + c) * 64 + row] = __half_as_ushort(__float2half_rn(__uint_as_float(b)));
-            }
+          for (int c = 0; c < HW; ++c) {
+            const int cc = gate_side ? c : HW + c;
+            const float mine = __uint_as_float(v[cc]);
+            const float other = s_x[cc * 64 + j];
+            const float g = fminf(gate_side ? mine : other, L);
+            const float u = fminf(fmaxf(gate_side ? other : mine, -L), L);
+            const float hval = g * __frcp_rn(1.0f + __expf(-g)) * u;   // silu(g) * u
+            uint32_t b = __float_as_uint(hval);
+            b = (b + 0x7FFFu + ((b >> 16) & 1u)) & 0xFFFF0000u;       // round to bf16
+            s_h[(c0 + cc) * 64 + j] = __half_as_ushort(__float2half_rn(__uint_as_float(b)));
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
         }
@@ -350,9 +358,8 @@ int launch_one(const FwdArgs& a) {
   const uint8_t* codes = (MODE == MODE_GATE_UP) ? a.w1c : a.w2c;
   const uint8_t* scales = (MODE == MODE_GATE_UP) ? a.w1s : a.w2s;
   const uint16_t* act = (MODE == MODE_GATE_UP) ? a.ws.xs : a.ws.h;
-  const uint32_t rows_box = (MODE == MODE_GATE_UP) ? 64 : kBM;
 
-  CUtensorMap m_act, m_codes, m_scales;
+  CUtensorMap m_act;
   {
     const uint64_t dims[2] = {(uint64_t)K, (uint64_t)P};
     const uint64_t str[1] = {(uint64_t)K * 2};
@@ -360,23 +367,12 @@ int launch_one(const FwdArgs& a) {
     if (!make_map(&m_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, act, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return -1;
   }
-  {
-    const uint64_t dims[3] = {(uint64_t)K / 2, (uint64_t)R, (uint64_t)a.E};
-    const uint64_t str[2] = {(uint64_t)K / 2, (uint64_t)R * (K / 2)};
-    const uint32_t box[3] = {kBK / 2, rows_box, 1};
-    if (!make_map(&m_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, codes, dims, str, box, CU_TENSOR_MAP_SWIZZLE_32B))
-      return -1;
-  }
-  {
-    const uint64_t dims[3] = {(uint64_t)R, (uint64_t)K / 32, (uint64_t)a.E};
-    const uint64_t str[2] = {(uint64_t)R, (uint64_t)R * (K / 32)};
-    const uint32_t box[3] = {rows_box, kBK / 32, 1};
-    if (!make_map(&m_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, scales, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return -1;
-  }
   TcParams prm;
   prm.tiles = a.ws.tiles;
   prm.ntiles = a.ws.ntiles;
+  prm.codes = codes;
+  prm.scales = scales;
+  prm.N = R;
   prm.w_sorted = a.ws.w_sorted;
   prm.h_out = a.ws.h;
   prm.ys_out = a.ws.ys;
@@ -392,7 +388,7 @@ int launch_one(const FwdArgs& a) {
   const int max_tiles = (P + BN - 1) / BN + a.E;
   const int row_tiles = (MODE == MODE_GATE_UP) ? a.I / 64 : (a.d + kBM - 1) / kBM;
   ev_before(a);
-  kern<<<dim3(max_tiles, row_tiles), kThreads, C::SMEM_BYTES, a.stream>>>(m_act, m_codes, m_scales, prm);
+  kern<<<dim3(max_tiles, row_tiles), kThreads, C::SMEM_BYTES, a.stream>>>(m_act, prm);
   ev_after(a);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }

@@ -18,6 +18,22 @@ import synth
 from _inputs import routed_inputs
 
 
+def blocks_to_rowmajor(codes: np.ndarray, scales: np.ndarray, N: int, K: int):
+    """Library MXFP4 block layout -> the oracle's row-major layout.
+
+    codes [E, N/64, K/64, 64, 32] -> [E, N, K/2]; scales [E, N/64, K/64, 2, 64] -> [E, N, K/32].
+    In a block, row r's logical 16-byte chunk c is stored at chunk c ^ ((r >> 2) & 1).
+    """
+    E = codes.shape[0]
+    c = codes.reshape(E, N // 64, K // 64, 64, 2, 16)
+    r = np.arange(64)
+    phys = np.stack([(0 ^ ((r >> 2) & 1)), (1 ^ ((r >> 2) & 1))], axis=1)  # [64, 2] physical chunk of logical c
+    logical = np.take_along_axis(c, phys[None, None, None, :, :, None], axis=4)
+    rows = logical.reshape(E, N // 64, K // 64, 64, 32).transpose(0, 1, 3, 2, 4).reshape(E, N, K // 2)
+    sc = scales.reshape(E, N // 64, K // 64, 2, 64).transpose(0, 1, 4, 2, 3).reshape(E, N, K // 32)
+    return np.ascontiguousarray(rows), np.ascontiguousarray(sc)
+
+
 def bf16_dev(u16: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16).cuda()
 
@@ -31,10 +47,12 @@ def weights(seed: int, E: int, d: int, I: int, w1_mul: float):
     """GPU MXFP4 weights (library layout) + oracle MXFP4 weights + bit-exactness record."""
     cfg = synth.MoEConfig("w", T=1, d=d, I=I, E=E, k=1, seed=seed, w1_mul=w1_mul)
     dev = "cuda"
-    g1c = torch.empty((E, 2 * I, d // 2), dtype=torch.uint8, device=dev)
-    g1s = torch.empty((E, d // 32, 2 * I), dtype=torch.uint8, device=dev)
-    g2c = torch.empty((E, d, I // 2), dtype=torch.uint8, device=dev)
-    g2s = torch.empty((E, I // 32, d), dtype=torch.uint8, device=dev)
+    s1c, s1s = moe.mxfp4_shapes(E, 2 * I, d)
+    s2c, s2s = moe.mxfp4_shapes(E, d, I)
+    g1c = torch.empty(s1c, dtype=torch.uint8, device=dev)
+    g1s = torch.empty(s1s, dtype=torch.uint8, device=dev)
+    g2c = torch.empty(s2c, dtype=torch.uint8, device=dev)
+    g2s = torch.empty(s2s, dtype=torch.uint8, device=dev)
     o1c = np.empty((E, 2 * I, d // 2), np.uint8)
     o1s = np.empty((E, 2 * I, d // 32), np.uint8)
     o2c = np.empty((E, d, I // 2), np.uint8)
@@ -47,8 +65,9 @@ def weights(seed: int, E: int, d: int, I: int, w1_mul: float):
             wt = torch.from_numpy(w).cuda()
             moe.moe_mxfp4_quantize(wt, gc[e:e + 1], gs[e:e + 1], status_word=status)
             oc[e], os_[e] = oracle.quantize(w)
-            mismatches += int(np.count_nonzero(gc[e].cpu().numpy() != oc[e]))
-            mismatches += int(np.count_nonzero(gs[e].cpu().numpy().T != os_[e]))
+            rc, rs = blocks_to_rowmajor(gc[e:e + 1].cpu().numpy(), gs[e:e + 1].cpu().numpy(), *w.shape)
+            mismatches += int(np.count_nonzero(rc[0] != oc[e]))
+            mismatches += int(np.count_nonzero(rs[0] != os_[e]))
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     return dict(gpu=(g1c, g1s, g2c, g2s), oracle=(o1c, o1s, o2c, o2s), mismatches=mismatches)
