@@ -64,6 +64,26 @@ def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
 
+def rank_rows(rank, T):
+    """Token rows of this rank's batch: rank r processes global rows [r*T, (r+1)*T) (weak scaling)."""
+    return np.arange(rank * T, (rank + 1) * T)
+
+
+def max_over_ranks(value, pg, device="cuda"):
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if pg is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, steps, total_ms):
+    """Whole-job tokens/s: the tokens of all ranks over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (total_ms * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -156,7 +176,7 @@ def device_inputs(cfg, rank, need_oracle_weights):
     """Hidden rows (this rank's tokens), router, and MXFP4 weights quantized on the GPU."""
     import torch
     import mxfp4_expert_gemm_b200 as moe
-    rows = np.arange(rank * cfg.T, (rank + 1) * cfg.T)
+    rows = rank_rows(rank, cfg.T)
     x = synth.hidden_rows(cfg, rows) if rank else synth.hidden(cfg)
     gamma, rw, rb = synth.norm_weight(cfg), synth.router_weight(cfg), synth.router_bias(cfg)
     E, d, I = cfg.E, cfg.d, cfg.I
@@ -286,10 +306,7 @@ def run_ours(args, rank, world, local_rank):
     total_ms = float(sum(step_ms))
     kern_ms = {name: statistics.mean(kev[i][2 * j].elapsed_time(kev[i][2 * j + 1]) for i in range(K))
                for j, name in enumerate(KERNELS[:moe.last_launch_count()])}
-    if pg:
-        t = torch.tensor([total_ms], device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, pg)
 
     # ---- end to end through the public API with host buffers
     x_host = torch.empty(inp["x_dev"].shape, dtype=torch.bfloat16, pin_memory=True)
@@ -310,10 +327,7 @@ def run_ours(args, rank, world, local_rank):
         e_stops[i].record()
     torch.cuda.synchronize()
     e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(e_starts, e_stops)))
-    if pg:
-        t = torch.tensor([e2e_ms], device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, pg)
     assert moe.moe_device_status(ws) == moe.MOE_OK
 
     # ---- roofline of the dominant kernel
@@ -352,7 +366,7 @@ def run_ours(args, rank, world, local_rank):
         roof["layer"] = {"flops": layer_flops, "achieved_TFLOPs": round(layer_flops / (layer_ms * 1e-3) / 1e12, 1),
                          "frac_of_fp4_dense_nominal": round(layer_flops / (layer_ms * 1e-3) / 1e12 / FP4_DENSE_NOMINAL_TFLOPS, 4)}
 
-    value = cfg.T * world * K / (total_ms * 1e-3)
+    value = job_throughput(cfg.T, world, K, total_ms)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": max(3, args.warmup), "ms_per_step": round(total_ms / K, 5), "higher_is_better": True,
@@ -363,7 +377,7 @@ def run_ours(args, rank, world, local_rank):
                    "timing": "sum of per-step CUDA events on the launching stream; max over ranks"},
         "kernel_ms": {k_: round(v, 5) for k_, v in kern_ms.items()},
         "roofline": roof,
-        "e2e": {"value": round(cfg.T * world * K / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(job_throughput(cfg.T, world, K, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(inp["x_dev"].numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
         "gpu_launches": launches,
         "clocks": clk.summary(),

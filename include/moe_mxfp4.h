@@ -192,6 +192,14 @@ const char* moe_status_string(moe_status status);
  * thread launched (for launch accounting in benchmarks). */
 int32_t moe_last_launch_count(void);
 
+/* Test hook for the device-side failure path.  With enable != 0, the next moe_forward
+ * (or moe_forward_timed) call on this host thread, if it takes a tensor-core path, launches
+ * its gate_up kernel with one pipeline arrival withheld in its first CTA: that CTA's bounded
+ * wait expires after about 2 s, the CTA drains its copies, frees its tensor memory and
+ * exits, and the workspace status word records MOE_ERR_TIMEOUT (y of that call is then
+ * unspecified).  The hook clears itself after that call; nothing faults or hangs. */
+void moe_debug_inject_timeout(int32_t enable);
+
 #ifdef __cplusplus
 }
 #endif

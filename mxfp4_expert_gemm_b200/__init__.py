@@ -92,6 +92,8 @@ def lib():
             L.moe_device_status.restype = ctypes.c_int
             L.moe_status_string.argtypes = [ctypes.c_int]
             L.moe_status_string.restype = ctypes.c_char_p
+            L.moe_debug_inject_timeout.argtypes = [i32]
+            L.moe_debug_inject_timeout.restype = None
             L.moe_last_launch_count.argtypes = []
             L.moe_last_launch_count.restype = i32
             _lib = L
@@ -272,3 +274,8 @@ def moe_device_status(ws: torch.Tensor, stream=None) -> int:
 
 def last_launch_count() -> int:
     return lib().moe_last_launch_count()
+
+
+def moe_debug_inject_timeout(enable: bool = True) -> None:
+    """Test hook: the next tensor-core forward on this thread times out in one CTA (see the header)."""
+    lib().moe_debug_inject_timeout(1 if enable else 0)

@@ -9,6 +9,7 @@
 namespace {
 
 thread_local int32_t g_last_launches = 0;
+thread_local int32_t g_inject_timeout = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -173,6 +174,8 @@ moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x,
   rec.events = events;
   rec.n = n_events;
   a.ev = &rec;
+  a.inject_timeout = g_inject_timeout;
+  g_inject_timeout = 0;
   const int path = resolve_path(*dims, T);
   int n = moe::launch_route(a, tile_tokens_of(path));
   if (n < 0) return MOE_ERR_CUDA;
@@ -236,5 +239,7 @@ const char* moe_status_string(moe_status s) {
 }
 
 int32_t moe_last_launch_count(void) { return g_last_launches; }
+
+void moe_debug_inject_timeout(int32_t enable) { g_inject_timeout = enable ? 1 : 0; }
 
 }  // extern "C"

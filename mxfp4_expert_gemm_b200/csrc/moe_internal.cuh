@@ -135,6 +135,7 @@ struct FwdArgs {
   Ws ws;
   cudaStream_t stream;
   EventRec* ev;
+  int32_t inject_timeout;  // test hook: withhold one pipeline arrival in the gate_up kernel
 };
 
 inline void ev_before(const FwdArgs& a) {

@@ -150,22 +150,27 @@ __device__ __forceinline__ void warp_topk_softmax(float (&l)[NJ], int E, int k, 
 }
 
 // ----------------------------------------------------------------------------------
-// Small batches: one CTA per token.  The token's normalized row stays in shared
-// memory (fp32); warp w computes the logits of experts w, w+8, ... with 16-byte loads
-// of the router rows; warp 0 then selects the top-k.
+// Small batches: one CTA of 1024 threads per token.  The token's normalized row stays
+// in shared memory (fp32); warp w computes the logits of experts w, w+32, ..., each
+// lane issuing all of its 16-byte loads of the router row before the FMAs; warp 0 then
+// selects the top-k.
 // ----------------------------------------------------------------------------------
+constexpr int kTokThreads = 1024;
+constexpr int kTokWarps = kTokThreads / 32;
+constexpr int kTokBatch = 12;   // router-row loads in flight per lane
+
 template <int NJ>
-__global__ void __launch_bounds__(256) route_token_kernel(FwdArgs a) {
+__global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
   extern __shared__ float smem[];
   const int d = a.d, E = a.E;
   float* s_xn = smem;          // [d]
   float* s_l = smem + d;       // [32*NJ]
-  __shared__ float s_red[8];
+  __shared__ float s_red[kTokWarps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t t = blockIdx.x;
   const uint16_t* xr = a.x + t * d;
   float ss = 0.f;
-  for (int i = tid * 8; i < d; i += 256 * 8) {
+  for (int i = tid * 8; i < d; i += kTokThreads * 8) {
     const uint4 q = *reinterpret_cast<const uint4*>(xr + i);
     const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
@@ -183,10 +188,10 @@ __global__ void __launch_bounds__(256) route_token_kernel(FwdArgs a) {
   __syncthreads();
   float tot = 0.f;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) tot += s_red[w];
+  for (int w = 0; w < kTokWarps; ++w) tot += s_red[w];
   const float r = 1.0f / sqrtf(tot / (float)d + a.eps);
   bool range_bad = false;
-  for (int i = tid * 2; i < d; i += 512) {
+  for (int i = tid * 2; i < d; i += 2 * kTokThreads) {
     const float v0 = s_xn[i] * r * a.norm_w[i], v1 = s_xn[i + 1] * r * a.norm_w[i + 1];
     s_xn[i] = v0;
     s_xn[i + 1] = v1;
@@ -196,17 +201,29 @@ __global__ void __launch_bounds__(256) route_token_kernel(FwdArgs a) {
   }
   if (range_bad) set_status(a.ws.status, MOE_ERR_RANGE);
   __syncthreads();
-  for (int e = warp; e < E; e += 8) {
-    const float* wr = a.router_w + (int64_t)e * d;
+  const int n4 = d / 4;
+  for (int e = warp; e < E; e += kTokWarps) {
+    const float4* wr = reinterpret_cast<const float4*>(a.router_w + (int64_t)e * d);
     float acc = 0.f;
-#pragma unroll 4
-    for (int i = lane * 4; i < d; i += 128) {
-      const float4 w4 = *reinterpret_cast<const float4*>(wr + i);
-      const float4 x4 = *reinterpret_cast<const float4*>(s_xn + i);
-      acc = fmaf(w4.x, x4.x, acc);
-      acc = fmaf(w4.y, x4.y, acc);
-      acc = fmaf(w4.z, x4.z, acc);
-      acc = fmaf(w4.w, x4.w, acc);
+    // batches of kTokBatch 16-byte loads per lane, all issued before their FMAs
+    for (int base = 0; base < n4; base += 32 * kTokBatch) {
+      float4 w4[kTokBatch];
+#pragma unroll
+      for (int j = 0; j < kTokBatch; ++j) {
+        const int i4 = base + lane + 32 * j;
+        w4[j] = (i4 < n4) ? wr[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < kTokBatch; ++j) {
+        const int i4 = base + lane + 32 * j;
+        if (i4 < n4) {
+          const float4 x4 = reinterpret_cast<const float4*>(s_xn)[i4];
+          acc = fmaf(w4[j].x, x4.x, acc);
+          acc = fmaf(w4[j].y, x4.y, acc);
+          acc = fmaf(w4[j].z, x4.z, acc);
+          acc = fmaf(w4[j].w, x4.w, acc);
+        }
+      }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -468,7 +485,7 @@ int launch_route_nj(const FwdArgs& a) {
         cudaSuccess)
       return -1;
     ev_before(a);
-    route_token_kernel<NJ><<<a.T, 256, smem, a.stream>>>(a);
+    route_token_kernel<NJ><<<a.T, kTokThreads, smem, a.stream>>>(a);
     ev_after(a);
     return 1;
   }

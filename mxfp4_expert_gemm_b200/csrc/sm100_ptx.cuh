@@ -67,6 +67,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// OR of `flag` over the `count` threads of named barrier `id` (a barrier of its own:
+// every participant receives the same answer).
+template <int ID, int COUNT>
+__device__ __forceinline__ bool bar_or(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pin, pout;\n\t"
+      "setp.ne.u32 pin, %1, 0;\n\t"
+      "bar.red.or.pred pout, %2, %3, pin;\n\t"
+      "selp.u32 %0, 1, 0, pout;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)flag), "n"(ID), "n"(COUNT)
+      : "memory");
+  return r != 0;
+}
+
 // ----------------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c1,
                                             uint64_t* bar) {
