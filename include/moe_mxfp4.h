@@ -192,6 +192,27 @@ const char* moe_status_string(moe_status status);
  * thread launched (for launch accounting in benchmarks). */
 int32_t moe_last_launch_count(void);
 
+/* moe_forward for callers that cannot allocate device memory: it takes no workspace and
+ * allocates nothing (no cudaMalloc, no library allocator).  The pages have no
+ * counterpart; this is a deployment convenience.  Callers that run where allocation is
+ * not available -- inside an allocator or memory-pool callback, in a plugin host that
+ * lends out only its own tensors, or in a serving loop that forbids cudaMalloc and its
+ * implicit synchronization once it is running -- use it instead of moe_forward.
+ * Scratch: a fixed 16 MiB array in the library's own device memory, present on every GPU
+ * that loads the library until the process exits.  T whose moe_workspace_bytes() exceed
+ * 16 MiB is rejected with MOE_ERR_WORKSPACE (at d = I = 2880, top-4: up to 171 tokens).
+ * The first call on a device looks up the array's device address for that device
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the one array and it keeps the previous call's contents; the device
+ * status word and the expert counters are cleared by every call.  Calls that overlap on
+ * the GPU (unordered streams, or several host threads) race on the array.
+ * Arguments as moe_forward; status_out (device int32, may be NULL) receives the call's
+ * device status word (0 = MOE_OK) on `stream` once the call's kernels have run. */
+moe_status moe_forward_no_alloc(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                                const float* router_w, const float* router_b, const uint8_t* w1_codes,
+                                const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                                uint16_t* y, int32_t* status_out, void* stream);
+
 /* Test hook for the device-side failure path.  With enable != 0, the next moe_forward
  * (or moe_forward_timed) call on this host thread, if it takes a tensor-core path, launches
  * its gate_up kernel with one pipeline arrival withheld in its first CTA: that CTA's bounded

@@ -92,6 +92,8 @@ def lib():
             L.moe_device_status.restype = ctypes.c_int
             L.moe_status_string.argtypes = [ctypes.c_int]
             L.moe_status_string.restype = ctypes.c_char_p
+            L.moe_forward_no_alloc.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            L.moe_forward_no_alloc.restype = ctypes.c_int
             L.moe_debug_inject_timeout.argtypes = [i32]
             L.moe_debug_inject_timeout.restype = None
             L.moe_last_launch_count.argtypes = []
@@ -274,6 +276,22 @@ def moe_device_status(ws: torch.Tensor, stream=None) -> int:
 
 def last_launch_count() -> int:
     return lib().moe_last_launch_count()
+
+
+def moe_forward_no_alloc(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales,
+                         y=None, status_out=None, stream=None):
+    """moe_forward without a workspace, for callers that cannot allocate device memory while
+    they run (the library's fixed 16 MiB device scratch is used instead; see the header).
+    ``y`` and ``status_out`` (int32 [1]) are caller buffers; this wrapper creates ``y`` with
+    torch only when it is not given."""
+    _need(x, torch.bfloat16, "x")
+    if y is None:
+        y = torch.empty_like(x)
+    _check(lib().moe_forward_no_alloc(ctypes.byref(dims), x.shape[0], _ptr(x), _ptr(norm_w), _ptr(router_w),
+                                      _ptr(router_b), _ptr(w1_codes), _ptr(w1_scales), _ptr(w2_codes),
+                                      _ptr(w2_scales), _ptr(y), _ptr(status_out), _stream(stream)),
+           "moe_forward_no_alloc")
+    return y
 
 
 def moe_debug_inject_timeout(enable: bool = True) -> None:
