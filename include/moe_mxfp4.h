@@ -157,7 +157,9 @@ moe_status moe_forward(const moe_dims* dims, int32_t T, const uint16_t* x, const
 /* moe_forward plus per-kernel timing: `events` is an array of n_events cudaEvent_t
  * handles created by the caller (timing enabled).  Event 2i is recorded on `stream`
  * just before the i-th kernel this call launches and event 2i+1 just after it, until
- * the array runs out.  Recording adds no synchronization.  The kernels of a call are,
+ * the array runs out.  Recording adds no synchronization; when `stream` is being captured
+ * into a CUDA graph the events are recorded as external event nodes of the graph, so
+ * that every replay records them.  The kernels of a call are,
  * in order: route (RMSNorm + router + top-k), group, gather, gate_up, down, combine.
  * Errors: as moe_forward; MOE_ERR_INVALID_ARG if n_events < 0 or events is NULL with
  * n_events > 0. */
@@ -174,7 +176,8 @@ int32_t moe_resolve_path(const moe_dims* dims, int32_t T);
 
 /* Byte offsets of the workspace's sub-buffers for T tokens, for inspection by tests and
  * debuggers (layout may change between versions).  offsets[0..13] receive, in order:
- * status, counts, offsets, ntiles, tiles, topk_idx, topk_w, perm, inv, w_sorted,
+ * status, counts (int32 [E], then internal counters), offsets, ntiles, tiles, topk_idx,
+ * topk_w, perm, inv, w_sorted,
  * xe [T][d] f16, xs [T*k][d] f16 (xe in sorted pair order), h [T*k][I] f16 (SwiGLU
  * output, sorted order), ys [T*k][d] fp32 (weighted expert outputs, sorted order);
  * offsets[14] = total bytes.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE. */

@@ -1,6 +1,7 @@
 // C-ABI front end: argument checks, workspace carve-up, path choice, launches.
 // Declarations and the contract of every entry point: include/moe_mxfp4.h.
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -13,13 +14,20 @@ thread_local int32_t g_inject_timeout = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Compute capability check, remembered per device (bit set = checked and sm_100).
+std::atomic<uint64_t> g_device_ok{0};
+
 moe_status check_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (dev < 64 && (g_device_ok.load(std::memory_order_acquire) & bit)) return MOE_OK;
   int major = 0, minor = 0;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return MOE_ERR_CUDA;
-  return (major == 10 && minor == 0) ? MOE_OK : MOE_ERR_DEVICE;
+  if (major != 10 || minor != 0) return MOE_ERR_DEVICE;
+  if (dev < 64) g_device_ok.fetch_or(bit, std::memory_order_release);
+  return MOE_OK;
 }
 
 moe_status check_dims(const moe_dims* dm, int32_t T) {
@@ -71,7 +79,7 @@ moe_status prepare(const moe_dims* dm, int32_t T, const uint16_t* x, const float
   a.norm_w = norm_w;
   a.router_w = router_w;
   a.router_b = router_b;
-  a.ws = moe::ws_pointers(ws, L);
+  a.ws = moe::ws_pointers(ws, L, dm->E);
   return MOE_OK;
 }
 
@@ -173,19 +181,29 @@ moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x,
   moe::EventRec rec;
   rec.events = events;
   rec.n = n_events;
+  if (n_events > 0) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(a.stream, &cs) != cudaSuccess) return MOE_ERR_CUDA;
+    rec.capturing = cs == cudaStreamCaptureStatusActive;
+  }
   a.ev = &rec;
   a.inject_timeout = g_inject_timeout;
   g_inject_timeout = 0;
   const int path = resolve_path(*dims, T);
+  // Small-batch path: fewer, fused kernels (routing + grouping + gather; down + combine).
+  a.fuse_group = (path == MOE_PATH_GEMV && T <= moe::kFusedGroupMaxT) ? 1 : 0;
+  a.fuse_combine = (path == MOE_PATH_GEMV) ? 1 : 0;
   int n = moe::launch_route(a, tile_tokens_of(path));
   if (n < 0) return MOE_ERR_CUDA;
   const int ne = (path == MOE_PATH_SIMT) ? moe::launch_experts_simt(a)
                                          : moe::launch_experts_tc(a, tile_tokens_of(path));
   if (ne < 0) return MOE_ERR_CUDA;
   n += ne;
-  const int nc = moe::launch_combine(a);
-  if (nc < 0) return MOE_ERR_CUDA;
-  n += nc;
+  if (!a.fuse_combine) {
+    const int nc = moe::launch_combine(a);
+    if (nc < 0) return MOE_ERR_CUDA;
+    n += nc;
+  }
   const size_t P = (size_t)T * dims->top_k;
   if ((st = copy_out(topk_idx_out, a.ws.topk_idx, 4 * P, a.stream)) != MOE_OK) return st;
   if ((st = copy_out(topk_w_out, a.ws.topk_w, 4 * P, a.stream)) != MOE_OK) return st;

@@ -24,7 +24,8 @@ struct Tile {
 // Carve-up of the caller's workspace (byte offsets, 256-byte aligned).
 struct WsLayout {
   size_t status;    // int32 device status word (first device error wins)
-  size_t counts;    // int32 [E]
+  size_t counts;    // int32 [E] expert histogram, then int32 [4] (routing ticket), then int32
+                    // [T * ceil(d/128)] combine arrivals; cleared at the start of every call
   size_t offsets;   // int32 [E+1]
   size_t ntiles;    // int32 [4]: number of token tiles
   size_t tiles;     // Tile [max_tiles]
@@ -54,7 +55,7 @@ inline WsLayout ws_layout(const moe_dims& dm, int64_t T) {
     return at;
   };
   L.status = take(kStatusBytes);
-  L.counts = take(4 * (size_t)dm.E);
+  L.counts = take(4 * ((size_t)dm.E + 4 + (size_t)T * ((dm.d + 127) / 128)));
   L.offsets = take(4 * (size_t)(dm.E + 1));
   L.ntiles = take(16);
   L.tiles = take(sizeof(Tile) * (size_t)L.max_tiles);
@@ -75,6 +76,8 @@ inline WsLayout ws_layout(const moe_dims& dm, int64_t T) {
 struct Ws {
   int32_t* status;
   int32_t* counts;
+  int32_t* ticket;     // routing CTAs that finished (the last one builds the grouping)
+  int32_t* arrivals;   // [T][ceil(d/128)] expert outputs written per (token, 128 columns)
   int32_t* offsets;
   int32_t* ntiles;
   Tile* tiles;
@@ -90,7 +93,7 @@ struct Ws {
   int64_t max_tiles;
 };
 
-inline Ws ws_pointers(void* base, const WsLayout& L) {
+inline Ws ws_pointers(void* base, const WsLayout& L, int E) {
   char* b = static_cast<char*>(base);
   Ws w;
   w.status = reinterpret_cast<int32_t*>(b + L.status);
@@ -107,6 +110,8 @@ inline Ws ws_pointers(void* base, const WsLayout& L) {
   w.xs = reinterpret_cast<uint16_t*>(b + L.xs);
   w.h = reinterpret_cast<uint16_t*>(b + L.h);
   w.ys = reinterpret_cast<float*>(b + L.ys);
+  w.ticket = w.counts + E;
+  w.arrivals = w.counts + E + 4;
   w.max_tiles = L.max_tiles;
   return w;
 }
@@ -117,7 +122,14 @@ struct EventRec {
   void* const* events = nullptr;
   int n = 0;
   int next = 0;
+  bool capturing = false;  // the stream is being captured: record as external graph nodes
 };
+
+inline void record_event(const EventRec& r, int i, cudaStream_t st) {
+  cudaEvent_t e = static_cast<cudaEvent_t>(r.events[i]);
+  if (r.capturing) cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+  else cudaEventRecord(e, st);
+}
 
 // Everything a forward launch needs.
 struct FwdArgs {
@@ -136,16 +148,19 @@ struct FwdArgs {
   cudaStream_t stream;
   EventRec* ev;
   int32_t inject_timeout;  // test hook: withhold one pipeline arrival in the gate_up kernel
+  int32_t fuse_group;      // small batches: the routing kernel also groups and gathers
+  int32_t fuse_combine;    // the down kernel also adds the k expert outputs and the residual
 };
 
+constexpr int kFusedGroupMaxT = 64;   // fused grouping: one CTA walks the tokens in order
+
 inline void ev_before(const FwdArgs& a) {
-  if (a.ev && a.ev->events && a.ev->next + 1 < a.ev->n)
-    cudaEventRecord(static_cast<cudaEvent_t>(a.ev->events[a.ev->next]), a.stream);
+  if (a.ev && a.ev->events && a.ev->next + 1 < a.ev->n) record_event(*a.ev, a.ev->next, a.stream);
 }
 
 inline void ev_after(const FwdArgs& a) {
   if (a.ev && a.ev->events && a.ev->next + 1 < a.ev->n) {
-    cudaEventRecord(static_cast<cudaEvent_t>(a.ev->events[a.ev->next + 1]), a.stream);
+    record_event(*a.ev, a.ev->next + 1, a.stream);
     a.ev->next += 2;
   }
 }

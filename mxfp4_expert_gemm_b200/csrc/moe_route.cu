@@ -11,6 +11,7 @@
 //    parameters, 4.25 bits per parameter.
 #include <cuda_fp16.h>
 #include <algorithm>
+#include <atomic>
 #include <cfloat>
 
 #include "moe_internal.cuh"
@@ -150,6 +151,96 @@ __device__ __forceinline__ void warp_topk_softmax(float (&l)[NJ], int E, int k, 
 }
 
 // ----------------------------------------------------------------------------------
+// Grouping and gather for a small batch, run by the routing CTA that finished last
+// (all others have published their top-k, counts and xe rows before taking a ticket).
+// Pairs are listed per expert in token order: one warp walks the tokens in order and
+// hands each of a token's k (distinct) experts the next free position of that expert.
+// Deterministic: positions depend on counts and token order only.
+// ----------------------------------------------------------------------------------
+__device__ void group_and_gather_block(const FwdArgs& a, int tile_tokens) {
+  __shared__ int s_off[257];
+  __shared__ int s_cur[256];
+  __shared__ int s_tb[257];
+  __shared__ int s_perm_tok[kFusedGroupMaxT * 32];
+  const int E = a.E, k = a.k, T = a.T, P = T * k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (warp == 0) {
+    // exclusive scans of counts and of tiles-per-expert over E <= 256 (8 experts per lane)
+    int c[8], nt[8], sc = 0, st = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      c[j] = (e < E) ? __ldcg(a.ws.counts + e) : 0;
+      nt[j] = (c[j] + tile_tokens - 1) / tile_tokens;
+      sc += c[j];
+      st += nt[j];
+    }
+    int ic = sc, it = st;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yc = __shfl_up_sync(0xffffffffu, ic, o), yt = __shfl_up_sync(0xffffffffu, it, o);
+      if (lane >= o) {
+        ic += yc;
+        it += yt;
+      }
+    }
+    int oc = ic - sc, ot = it - st;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      if (e < E) {
+        s_off[e] = oc;
+        s_tb[e] = ot;
+        s_cur[e] = 0;
+        a.ws.offsets[e] = oc;
+      }
+      oc += c[j];
+      ot += nt[j];
+    }
+    if (lane == 31) {
+      a.ws.offsets[E] = oc;
+      a.ws.ntiles[0] = ot;
+    }
+  }
+  __syncthreads();
+  // token tiles of every expert
+  for (int e = warp; e < E; e += 32) {
+    const int base = s_tb[e];
+    const int c_e = (e + 1 < E ? s_off[e + 1] : P) - s_off[e];
+    for (int i = lane; i * tile_tokens < c_e; i += 32) {
+      Tile tl;
+      tl.e = e;
+      tl.row0 = s_off[e] + i * tile_tokens;
+      tl.rows = min(tile_tokens, c_e - i * tile_tokens);
+      tl.pad = 0;
+      a.ws.tiles[base + i] = tl;
+    }
+  }
+  if (warp == 0) {
+    for (int t = 0; t < T; ++t) {
+      if (lane < k) {
+        const int q = t * k + lane;
+        const int e = __ldcg(a.ws.topk_idx + q);
+        const int pos = s_off[e] + s_cur[e]++;
+        a.ws.perm[pos] = q;
+        a.ws.inv[q] = pos;
+        a.ws.w_sorted[pos] = __ldcg(a.ws.topk_w + q);
+        s_perm_tok[pos] = t;
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // xs[p] = xe[token of p]: 16-byte copies over all pairs
+  const int n16 = a.d / 8;
+  for (int idx = tid; idx < P * n16; idx += blockDim.x) {
+    const int p = idx / n16, c = idx - p * n16;
+    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.ws.xe + (int64_t)s_perm_tok[p] * a.d) + c);
+    reinterpret_cast<uint4*>(a.ws.xs + (int64_t)p * a.d)[c] = v;
+  }
+}
+
+// ----------------------------------------------------------------------------------
 // Small batches: one CTA of 1024 threads per token.  The token's normalized row stays
 // in shared memory (fp32); warp w computes the logits of experts w, w+32, ..., each
 // lane issuing all of its 16-byte loads of the router row before the FMAs; warp 0 then
@@ -235,6 +326,18 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
 #pragma unroll
     for (int j = 0; j < NJ; ++j) l[j] = (lane + 32 * j < E) ? s_l[lane + 32 * j] : -INFINITY;
     warp_topk_softmax<NJ>(l, E, a.k, t, a);
+  }
+  if (a.fuse_group) {
+    // Publish this token (top-k, counts, xe row), then take a ticket; the last CTA groups.
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(a.ws.ticket, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      group_and_gather_block(a, a.fuse_group);
+    }
   }
 }
 
@@ -477,13 +580,27 @@ __global__ void combine_kernel(FwdArgs a) {
   }
 }
 
+// Sets a kernel's dynamic shared-memory limit once per device (the largest size asked).
+template <class K>
+bool ensure_smem_limit(K kern, size_t bytes, std::atomic<int>* limits /*[64]*/) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::atomic<int>& lim = limits[dev & 63];
+  if ((int)bytes <= lim.load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+    return false;
+  int cur = lim.load();
+  while ((int)bytes > cur && !lim.compare_exchange_weak(cur, (int)bytes)) {
+  }
+  return true;
+}
+
 template <int NJ>
 int launch_route_nj(const FwdArgs& a) {
+  static std::atomic<int> tok_limits[64], tile_limits[64];
   if (a.T <= kTokenKernelMaxT) {
     const size_t smem = sizeof(float) * (a.d + 32 * NJ);
-    if (cudaFuncSetAttribute(route_token_kernel<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return -1;
+    if (!ensure_smem_limit(route_token_kernel<NJ>, smem, tok_limits)) return -1;
     ev_before(a);
     route_token_kernel<NJ><<<a.T, kTokThreads, smem, a.stream>>>(a);
     ev_after(a);
@@ -491,8 +608,7 @@ int launch_route_nj(const FwdArgs& a) {
   }
   const int EP = 32 * NJ;
   const size_t smem = sizeof(float) * (RT + RT * (RK + 1) + RK * (EP + 1) + RT * (EP + 1));
-  if (cudaFuncSetAttribute(route_kernel<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return -1;
+  if (!ensure_smem_limit(route_kernel<NJ>, smem, tile_limits)) return -1;
   ev_before(a);
   route_kernel<NJ><<<(a.T + RT - 1) / RT, 256, smem, a.stream>>>(a);
   ev_after(a);
@@ -511,9 +627,13 @@ int launch_quantize(const float* w, int64_t rows, int32_t N, int32_t K, int32_t 
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 
-int launch_route(const FwdArgs& a, int tile_tokens) {
+int launch_route(const FwdArgs& a_in, int tile_tokens) {
   int n = 0;
-  if (cudaMemsetAsync(a.ws.counts, 0, sizeof(int32_t) * a.E, a.stream) != cudaSuccess) return -1;
+  FwdArgs a = a_in;
+  // fuse_group carries the token-tile size into the routing kernel (0 = separate kernels)
+  a.fuse_group = a_in.fuse_group ? tile_tokens : 0;
+  const size_t clear_ints = (size_t)a.E + 4 + (a.fuse_combine ? (size_t)a.T * ((a.d + 127) / 128) : 0);
+  if (cudaMemsetAsync(a.ws.counts, 0, sizeof(int32_t) * clear_ints, a.stream) != cudaSuccess) return -1;
   int r;
   if (a.E <= 32) r = launch_route_nj<1>(a);
   else if (a.E <= 64) r = launch_route_nj<2>(a);
@@ -521,6 +641,7 @@ int launch_route(const FwdArgs& a, int tile_tokens) {
   else r = launch_route_nj<8>(a);
   if (r < 0) return -1;
   n += r;
+  if (a.fuse_group) return cudaGetLastError() == cudaSuccess ? n : -1;
   ev_before(a);
   group_kernel<<<a.E, 1024, 0, a.stream>>>(a, tile_tokens);
   ev_after(a);

@@ -6,7 +6,7 @@
 // swiglu_limit 7 from the llm-atlas GPT-OSS 20B config table; MXFP4 weights per the
 // ewbang.com GPT-OSS article, section 量化 (E2M1 values, one E8M0 scale per 32).
 //
-// Persistent kernel, one CTA per SM.  A work item is a 128 (weight rows) x BN (tokens
+// Persistent kernel, CPS CTAs per SM.  A work item is a 128 (weight rows) x BN (tokens
 // of one expert) output tile over the whole reduction axis; CTA b takes items b,
 // b + grid, ...  A pipeline stage covers KS of the reduction axis (KS/64 chunks of 64;
 // the last stage of a row may hold fewer).  The weights are the MMA's A operand and
@@ -36,6 +36,7 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -67,9 +68,18 @@ struct TcParams {
   int32_t n_rt;           // row tiles per token tile
   float limit;
   int32_t inject_timeout; // test hook: CTA 0 withholds its first decode arrival
+  // fused combine (down): y = bf16(x + sum_j ys[inv[t*k + j]]) by the last writer of a
+  // (token, 128-column) block
+  int32_t fuse_combine;
+  int32_t k;
+  const int32_t* perm;
+  const int32_t* inv;
+  const uint16_t* x;
+  uint16_t* y;
+  int32_t* arrivals;
 };
 
-template <int BN, int KS, int S, int SA, int DG>
+template <int BN, int KS, int S, int SA, int DG, int CPS>
 struct Cfg {
   static constexpr int NC = KS / kCK;                          // chunks per stage
   static constexpr int ACT_CHUNK = BN * 128;                   // one 64-wide activation chunk
@@ -86,7 +96,7 @@ struct Cfg {
   static constexpr int TMEM_COLS = COLS_NEEDED <= 64 ? 64 : COLS_NEEDED <= 128 ? 128
                                    : COLS_NEEDED <= 256 ? 256 : 512;
   static constexpr int EPI_GU = 32 * 64 * 4 + BN * 64 * 2;     // exchange + h staging
-  static constexpr int EPI_DN = 32 * 128 * 4;                  // one 32-token chunk of outputs
+  static constexpr int EPI_DN = 32 * 128 * 4 + 32 * 4;         // one 32-token chunk + token ids
   static constexpr int EPI_BYTES = EPI_GU > EPI_DN ? EPI_GU : EPI_DN;
   static constexpr int BAR_BYTES = 8 * (2 * S + 2 * SA + 4 + 1) + 16;
   static constexpr int SMEM_BYTES = S * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024 /*align slack*/;
@@ -94,9 +104,9 @@ struct Cfg {
   static constexpr int THREADS = 32 * WARPS;
   static constexpr int EPI_WARP0 = 2 + 4 * DG;
   static_assert(KS % kCK == 0 && NC >= 1, "stage = whole chunks");
-  static_assert(COLS_NEEDED <= 512, "TMEM budget");
+  static_assert(TMEM_COLS * CPS <= 512, "TMEM budget of CPS co-resident CTAs");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M = 128");
-  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(SMEM_BYTES * CPS <= 226 * 1024, "shared memory budget of CPS co-resident CTAs");
 };
 
 // f16 bit pattern of 2^e, or 0 when E2M1 * 2^e is not exact in f16 (e outside [-23, 13]).
@@ -108,6 +118,7 @@ __device__ __forceinline__ uint32_t f16_pow2_bits(int e) {
 
 struct Item {
   Tile tl;
+  int rt;
   int row_tile0;
   int rbA, rbB;
   bool halfB;
@@ -118,6 +129,7 @@ __device__ __forceinline__ Item item_of(const TcParams& p, int i) {
   Item it;
   const int tt = i / p.n_rt, rt = i - tt * p.n_rt;
   it.tl = p.tiles[tt];
+  it.rt = rt;
   it.row_tile0 = (MODE == MODE_GATE_UP) ? rt * 64 : rt * kBM;
   it.rbA = it.row_tile0 / kBlkRows;
   // gate_up pairs gate rows j0.. with up rows I+j0..; down takes rows m0.. and m0+64..
@@ -126,10 +138,10 @@ __device__ __forceinline__ Item item_of(const TcParams& p, int i) {
   return it;
 }
 
-template <int MODE, int BN, int KS, int S, int SA, int DG>
-__global__ void __launch_bounds__(Cfg<BN, KS, S, SA, DG>::THREADS, 1)
+template <int MODE, int BN, int KS, int S, int SA, int DG, int CPS>
+__global__ void __launch_bounds__(Cfg<BN, KS, S, SA, DG, CPS>::THREADS, CPS)
     tc_expert_kernel(const __grid_constant__ CUtensorMap tm_act, const TcParams p) {
-  using C = Cfg<BN, KS, S, SA, DG>;
+  using C = Cfg<BN, KS, S, SA, DG, CPS>;
   extern __shared__ uint8_t smem_raw[];
   const int n_items = *p.ntiles * p.n_rt;
   if ((int)blockIdx.x >= n_items) return;  // uniform for the CTA
@@ -434,6 +446,35 @@ __global__ void __launch_bounds__(Cfg<BN, KS, S, SA, DG>::THREADS, 1)
             val.w *= wgt;
             *reinterpret_cast<float4*>(p.ys_out + (int64_t)prow * p.d + it.row_tile0 + c4 * 4) = val;
           }
+          if (p.fuse_combine) {
+            // Publish this chunk's outputs, count them per (token, column block); the writer of
+            // a token's k-th contribution adds the k outputs in slot order plus the residual.
+            int* s_tok = reinterpret_cast<int*>(s_y + 32 * 128) - 0;  // reuse past the staging rows
+            __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (et < nt) {
+              const int tok = p.perm[it.tl.row0 + c0 + et] / p.k;
+              const int prev = atomicAdd(p.arrivals + (int64_t)tok * p.n_rt + it.rt, 1);
+              s_tok[et] = (prev == p.k - 1) ? tok : -1;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            __threadfence();
+            for (int t = 0; t < nt; ++t) {
+              const int tok = s_tok[t];
+              if (tok < 0) continue;
+              for (int col = et; col < ncol; col += 128) {
+                const int64_t gc = it.row_tile0 + col;
+                float acc = __uint_as_float((uint32_t)p.x[(int64_t)tok * p.d + gc] << 16);
+                for (int j = 0; j < p.k; ++j) {
+                  const int srow = p.inv[(int64_t)tok * p.k + j];
+                  acc += __ldcg(p.ys_out + (int64_t)srow * p.d + gc);
+                }
+                uint32_t b = __float_as_uint(acc);
+                b = (b + 0x7FFFu + ((b >> 16) & 1u)) >> 16;   // round to bf16
+                p.y[(int64_t)tok * p.d + gc] = (uint16_t)b;
+              }
+            }
+          }
           asm volatile("bar.sync 1, 128;" ::: "memory");
         }
       }
@@ -489,9 +530,9 @@ int sm_count() {
   return n;
 }
 
-template <int MODE, int BN, int KS, int S, int SA, int DG>
+template <int MODE, int BN, int KS, int S, int SA, int DG, int CPS>
 int launch_one(const FwdArgs& a) {
-  using C = Cfg<BN, KS, S, SA, DG>;
+  using C = Cfg<BN, KS, S, SA, DG, CPS>;
   const int P = a.T * a.k;
   const int K = (MODE == MODE_GATE_UP) ? a.d : a.I;
   const int R = (MODE == MODE_GATE_UP) ? 2 * a.I : a.d;  // weight rows per expert
@@ -527,12 +568,26 @@ int launch_one(const FwdArgs& a) {
   prm.n_rt = (MODE == MODE_GATE_UP) ? a.I / 64 : (a.d + kBM - 1) / kBM;
   prm.limit = a.limit;
   prm.inject_timeout = (MODE == MODE_GATE_UP) ? a.inject_timeout : 0;
+  prm.fuse_combine = (MODE == MODE_DOWN) ? a.fuse_combine : 0;
+  prm.k = a.k;
+  prm.perm = a.ws.perm;
+  prm.inv = a.ws.inv;
+  prm.x = a.x;
+  prm.y = a.y;
+  prm.arrivals = a.ws.arrivals;
 
-  auto kern = tc_expert_kernel<MODE, BN, KS, S, SA, DG>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
-    return -1;
+  auto kern = tc_expert_kernel<MODE, BN, KS, S, SA, DG, CPS>;
+  static std::atomic<uint64_t> attr_done{0};   // per-device "attribute set" bits
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return -1;
+    attr_done.fetch_or(bit, std::memory_order_release);
+  }
   const int64_t max_items = (int64_t)((P + BN - 1) / BN + a.E) * prm.n_rt;
-  const int grid = (int)std::min<int64_t>(max_items, sm_count());
+  const int grid = (int)std::min<int64_t>(max_items, (int64_t)sm_count() * CPS);
   ev_before(a);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, a.stream>>>(m_act, prm);
   ev_after(a);
@@ -540,9 +595,10 @@ int launch_one(const FwdArgs& a) {
 }
 
 // Pipeline shapes (compile-time; overridable with -D for tuning builds).
-// Small batches (few tokens per expert): 16-token tiles, 320-wide stages.
+// Small batches (few tokens per expert): 16-token tiles, 192-wide stages, two
+// independent pipelines (CTAs) per SM.
 #ifndef MOE_GEMV_KS
-#define MOE_GEMV_KS 320
+#define MOE_GEMV_KS 192
 #endif
 #ifndef MOE_GEMV_S
 #define MOE_GEMV_S 5
@@ -551,7 +607,10 @@ int launch_one(const FwdArgs& a) {
 #define MOE_GEMV_SA 2
 #endif
 #ifndef MOE_GEMV_DG
-#define MOE_GEMV_DG 2
+#define MOE_GEMV_DG 1
+#endif
+#ifndef MOE_GEMV_CPS
+#define MOE_GEMV_CPS 2
 #endif
 // Large batches: 128-token tiles, 192-wide stages.
 #ifndef MOE_GEMM_KS
@@ -566,10 +625,13 @@ int launch_one(const FwdArgs& a) {
 #ifndef MOE_GEMM_DG
 #define MOE_GEMM_DG 2
 #endif
+#ifndef MOE_GEMM_CPS
+#define MOE_GEMM_CPS 1
+#endif
 constexpr int kGemvBN = 16, kGemvKS = MOE_GEMV_KS, kGemvS = MOE_GEMV_S, kGemvSA = MOE_GEMV_SA,
-              kGemvDG = MOE_GEMV_DG;
+              kGemvDG = MOE_GEMV_DG, kGemvCPS = MOE_GEMV_CPS;
 constexpr int kGemmBN = 128, kGemmKS = MOE_GEMM_KS, kGemmS = MOE_GEMM_S, kGemmSA = MOE_GEMM_SA,
-              kGemmDG = MOE_GEMM_DG;
+              kGemmDG = MOE_GEMM_DG, kGemmCPS = MOE_GEMM_CPS;
 
 }  // namespace
 
@@ -578,13 +640,13 @@ int tc_tile_tokens(int path) { return path == MOE_PATH_GEMV ? kGemvBN : kGemmBN;
 int launch_experts_tc(const FwdArgs& a, int tile_tokens) {
   int n1, n2;
   if (tile_tokens == kGemvBN) {
-    n1 = launch_one<MODE_GATE_UP, kGemvBN, kGemvKS, kGemvS, kGemvSA, kGemvDG>(a);
+    n1 = launch_one<MODE_GATE_UP, kGemvBN, kGemvKS, kGemvS, kGemvSA, kGemvDG, kGemvCPS>(a);
     if (n1 < 0) return -1;
-    n2 = launch_one<MODE_DOWN, kGemvBN, kGemvKS, kGemvS, kGemvSA, kGemvDG>(a);
+    n2 = launch_one<MODE_DOWN, kGemvBN, kGemvKS, kGemvS, kGemvSA, kGemvDG, kGemvCPS>(a);
   } else {
-    n1 = launch_one<MODE_GATE_UP, kGemmBN, kGemmKS, kGemmS, kGemmSA, kGemmDG>(a);
+    n1 = launch_one<MODE_GATE_UP, kGemmBN, kGemmKS, kGemmS, kGemmSA, kGemmDG, kGemmCPS>(a);
     if (n1 < 0) return -1;
-    n2 = launch_one<MODE_DOWN, kGemmBN, kGemmKS, kGemmS, kGemmSA, kGemmDG>(a);
+    n2 = launch_one<MODE_DOWN, kGemmBN, kGemmKS, kGemmS, kGemmSA, kGemmDG, kGemmCPS>(a);
   }
   if (n2 < 0) return -1;
   return n1 + n2;

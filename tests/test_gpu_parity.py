@@ -226,7 +226,10 @@ def test_non_finite_input_is_reported():
 def test_launch_count_reported():
     c = case(SMALL["tiny"])
     cfg = c["cfg"]
-    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path="gemm")
-    ws = moe.new_workspace(dims, cfg.T)
-    moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws)
-    assert moe.last_launch_count() == 6  # route, group, gather, gate_up, down, combine
+    for path, n in (("gemm", 6),   # route, group, gather, gate_up, down, combine
+                    ("gemv", 3),   # route (+ grouping + gather), gate_up, down (+ combine)
+                    ("simt", 6)):
+        dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path=path)
+        ws = moe.new_workspace(dims, cfg.T)
+        moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws)
+        assert moe.last_launch_count() == n, path
