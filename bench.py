@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(synth.CONFIGS))
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm", "simt"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of "
+                    "replaying a captured CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     return ap.parse_args()
 
@@ -266,8 +268,9 @@ def run_ours(args, rank, world, local_rank):
     W = inp["W"]
 
     def step(events=None):
+        # the current stream: inside a graph capture this is the capturing stream
         moe.moe_forward_timed(dims, inp["x_dev"], inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws, y=y,
-                              events=events, stream=stream)
+                              events=events)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -281,31 +284,68 @@ def run_ours(args, rank, world, local_rank):
     K = args.steps
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(K)]
-    for e in [*starts, *stops, *[x for row in kev for x in row]]:
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)]]
+    for e in [*starts, *stops, *kev[0]]:
         e.record()  # creates the underlying CUDA events
     torch.cuda.synchronize()
+
+    def plain_step():
+        moe.moe_forward(dims, inp["x_dev"], inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws, y=y)
+
+    use_graph = not args.no_graph
+    graph = None
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            plain_step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
+    # ---- timed region: the layer as a user runs it (one graph replay per step)
     with ClockSampler(local_rank) as clk:
         for i in range(K):
             flush.zero_()
             starts[i].record()
-            step(kev[i])
+            if use_graph:
+                graph.replay()
+            else:
+                plain_step()
             stops[i].record()
         torch.cuda.synchronize()
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    launches = moe.last_launch_count() * K
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
+    total_ms = float(sum(step_ms))
+    plain_step()
+    launches = moe.last_launch_count() * K   # kernels per forward x timed steps
+    # ---- instrumented pass (outside the timed region): the same steps with a CUDA event
+    # pair around each of the library's launches, replayed from one graph per step
+    kgraph = None
+    if use_graph:
+        kgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(kgraph):
+            step(kev[0])
+    n_timed = moe.last_launch_count()
+    names = KERNELS if n_timed == len(KERNELS) else ["route", "gate_up", "down"]
+    per_kernel = {name: [] for name in names[:n_timed]}
+    for i in range(K):
+        flush.zero_()
+        if use_graph:
+            kgraph.replay()
+        else:
+            step(kev[0])
+        torch.cuda.synchronize()
+        for j, name in enumerate(names[:n_timed]):
+            per_kernel[name].append(kev[0][2 * j].elapsed_time(kev[0][2 * j + 1]))
+    del kgraph
     st = moe.moe_device_status(ws)
     if st != moe.MOE_OK:
         raise moe.MoeError(st, "device status after the timed steps")
-    step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
-    total_ms = float(sum(step_ms))
-    kern_ms = {name: statistics.mean(kev[i][2 * j].elapsed_time(kev[i][2 * j + 1]) for i in range(K))
-               for j, name in enumerate(KERNELS[:moe.last_launch_count()])}
+    kern_ms = {name: statistics.mean(v) for name, v in per_kernel.items()}
     total_ms = max_over_ranks(total_ms, pg)
 
     # ---- end to end through the public API with host buffers
@@ -315,15 +355,28 @@ def run_ours(args, rank, world, local_rank):
     e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     e_stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     x_dev2 = torch.empty_like(inp["x_dev"])
+    def e2e_step():
+        x_dev2.copy_(x_host, non_blocking=True)
+        moe.moe_forward(dims, x_dev2, inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws, y=y)
+        y_host.copy_(y, non_blocking=True)
+
+    e2e_graph = None
+    if use_graph:
+        e2e_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(e2e_graph):
+            e2e_step()
+        e2e_graph.replay()
+        torch.cuda.synchronize()
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
     for i in range(K):
         flush.zero_()
         e_starts[i].record()
-        x_dev2.copy_(x_host, non_blocking=True)
-        moe.moe_forward(dims, x_dev2, inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws, y=y)
-        y_host.copy_(y, non_blocking=True)
+        if use_graph:
+            e2e_graph.replay()
+        else:
+            e2e_step()
         e_stops[i].record()
     torch.cuda.synchronize()
     e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(e_starts, e_stops)))
@@ -374,7 +427,9 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD_TEXT[cfg.name], "name": cfg.name, "tokens_per_gpu": cfg.T,
                    "global_batch": cfg.T * world, "path": path_used, "parallelism": f"dp{world}",
                    "l2": "flushed before every step (256 MiB write, outside the step events)",
-                   "timing": "sum of per-step CUDA events on the launching stream; max over ranks"},
+                   "timing": "sum of per-step CUDA events on the launching stream; max over ranks",
+                   "launch": "CUDA graph replay per step" if use_graph else "host launches per step",
+                   "kernel_timing": "separate pass of the same steps with CUDA events around each kernel"},
         "kernel_ms": {k_: round(v, 5) for k_, v in kern_ms.items()},
         "roofline": roof,
         "e2e": {"value": round(job_throughput(cfg.T, world, K, e2e_ms), 1), "unit": "tokens/s",
@@ -388,6 +443,7 @@ def run_ours(args, rank, world, local_rank):
                                 "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graph, e2e_graph
     if pg:
         pg.barrier()
         pg.destroy_process_group()

@@ -193,6 +193,9 @@ moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x,
   // Small-batch path: fewer, fused kernels (routing + grouping + gather; down + combine).
   a.fuse_group = (path == MOE_PATH_GEMV && T <= moe::kFusedGroupMaxT) ? 1 : 0;
   a.fuse_combine = (path == MOE_PATH_GEMV) ? 1 : 0;
+  // Overlap each kernel's launch and prologue with its predecessor, except when per-kernel
+  // events are recorded between the kernels.
+  a.pdl = (n_events == 0) ? 1 : 0;
   int n = moe::launch_route(a, tile_tokens_of(path));
   if (n < 0) return MOE_ERR_CUDA;
   const int ne = (path == MOE_PATH_SIMT) ? moe::launch_experts_simt(a)

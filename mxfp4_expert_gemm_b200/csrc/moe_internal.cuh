@@ -150,7 +150,31 @@ struct FwdArgs {
   int32_t inject_timeout;  // test hook: withhold one pipeline arrival in the gate_up kernel
   int32_t fuse_group;      // small batches: the routing kernel also groups and gathers
   int32_t fuse_combine;    // the down kernel also adds the k expert outputs and the residual
+  int32_t pdl;             // launch dependent kernels with programmatic stream serialization
 };
+
+// Programmatic dependent launch: a kernel launched with the attribute may start while
+// its predecessor in the stream is still running; it calls pdl_wait() before touching
+// anything the predecessor writes.  pdl_trigger() lets the successor start launching.
+// Both are no-ops for kernels launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                          Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 constexpr int kFusedGroupMaxT = 64;   // fused grouping: one CTA walks the tokens in order
 

@@ -253,6 +253,7 @@ constexpr int kTokBatch = 12;   // router-row loads in flight per lane
 template <int NJ>
 __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
   extern __shared__ float smem[];
+  pdl_trigger();
   const int d = a.d, E = a.E;
   float* s_xn = smem;          // [d]
   float* s_l = smem + d;       // [32*NJ]
@@ -352,6 +353,7 @@ constexpr int RK = 64;   // d-chunk
 template <int NJ>  // experts per lane group: E <= 32*NJ
 __global__ void __launch_bounds__(256) route_kernel(FwdArgs a) {
   extern __shared__ float smem[];
+  pdl_trigger();
   const int E = a.E, d = a.d, k = a.k;
   const int EP = 32 * NJ;
   float* s_r = smem;                         // [RT]
@@ -479,6 +481,8 @@ __global__ void __launch_bounds__(256) route_kernel(FwdArgs a) {
 __global__ void __launch_bounds__(1024) group_kernel(FwdArgs a, int tile_tokens) {
   __shared__ int s_warp[32];
   __shared__ int s_base, s_tile_base, s_total_tiles, s_off;
+  pdl_trigger();
+  pdl_wait();
   const int e = blockIdx.x, E = a.E, k = a.k, T = a.T;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
@@ -546,6 +550,8 @@ __global__ void __launch_bounds__(1024) group_kernel(FwdArgs a, int tile_tokens)
 
 // xs[p] = xe[perm[p] / k]: 16-byte copies, one warp per row.
 __global__ void gather_kernel(FwdArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int P = a.T * a.k;
   const int lane = threadIdx.x & 31;
   const int n16 = a.d / 8;
@@ -559,6 +565,8 @@ __global__ void gather_kernel(FwdArgs a) {
 
 // y[t] = bf16(x[t] + sum_j ys[inv[t*k + j]]), j in slot order.
 __global__ void combine_kernel(FwdArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int i4 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i4 >= a.d) return;
   for (int t = blockIdx.y; t < a.T; t += gridDim.y) {
@@ -643,12 +651,15 @@ int launch_route(const FwdArgs& a_in, int tile_tokens) {
   n += r;
   if (a.fuse_group) return cudaGetLastError() == cudaSuccess ? n : -1;
   ev_before(a);
-  group_kernel<<<a.E, 1024, 0, a.stream>>>(a, tile_tokens);
+  if (launch_kernel(group_kernel, dim3(a.E), dim3(1024), 0, a.stream, a.pdl != 0, a, tile_tokens) != cudaSuccess)
+    return -1;
   ev_after(a);
   ++n;
   const int P = a.T * a.k;
   ev_before(a);
-  gather_kernel<<<std::min((P + 7) / 8, 148 * 16), 256, 0, a.stream>>>(a);
+  if (launch_kernel(gather_kernel, dim3(std::min((P + 7) / 8, 148 * 16)), dim3(256), 0, a.stream, a.pdl != 0, a) !=
+      cudaSuccess)
+    return -1;
   ev_after(a);
   ++n;
   return cudaGetLastError() == cudaSuccess ? n : -1;
@@ -657,7 +668,7 @@ int launch_route(const FwdArgs& a_in, int tile_tokens) {
 int launch_combine(const FwdArgs& a) {
   dim3 grid((a.d / 4 + 127) / 128, std::min(a.T, 65535));
   ev_before(a);
-  combine_kernel<<<grid, 128, 0, a.stream>>>(a);
+  if (launch_kernel(combine_kernel, grid, dim3(128), 0, a.stream, a.pdl != 0, a) != cudaSuccess) return -1;
   ev_after(a);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }

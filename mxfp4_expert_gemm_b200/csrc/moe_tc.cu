@@ -143,8 +143,7 @@ __global__ void __launch_bounds__(Cfg<BN, KS, S, SA, DG, CPS>::THREADS, CPS)
     tc_expert_kernel(const __grid_constant__ CUtensorMap tm_act, const TcParams p) {
   using C = Cfg<BN, KS, S, SA, DG, CPS>;
   extern __shared__ uint8_t smem_raw[];
-  const int n_items = *p.ntiles * p.n_rt;
-  if ((int)blockIdx.x >= n_items) return;  // uniform for the CTA
+  pdl_trigger();
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* epi = smem + S * C::STAGE_BYTES;
@@ -187,6 +186,9 @@ __global__ void __launch_bounds__(Cfg<BN, KS, S, SA, DG, CPS>::THREADS, CPS)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  // Everything above overlaps the previous kernel; the work list is its output.
+  pdl_wait();
+  const int n_items = *p.ntiles * p.n_rt;
 
   auto act_s = [&](int s) { return smem + s * C::STAGE_BYTES; };
   auto code_s = [&](int s) { return smem + s * C::STAGE_BYTES + C::CODE_OFF; };
@@ -589,9 +591,11 @@ int launch_one(const FwdArgs& a) {
   const int64_t max_items = (int64_t)((P + BN - 1) / BN + a.E) * prm.n_rt;
   const int grid = (int)std::min<int64_t>(max_items, (int64_t)sm_count() * CPS);
   ev_before(a);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, a.stream>>>(m_act, prm);
+  if (launch_kernel(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, a.stream, a.pdl != 0, m_act, prm) !=
+      cudaSuccess)
+    return -1;
   ev_after(a);
-  return cudaGetLastError() == cudaSuccess ? 1 : -1;
+  return 1;
 }
 
 // Pipeline shapes (compile-time; overridable with -D for tuning builds).

@@ -214,6 +214,49 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
 
+// ------------------------------------------------------------- block-scaled MMA (MX formats)
+// Instruction descriptor of kind::mxf8f6f4.block_scale with an E2M1 A operand, an E4M3 B
+// operand (both K-major), fp32 D and E8M0 scale factors.  sfa_id / sfb_id pick the byte of
+// each 32-bit scale-factor word in TMEM that this MMA (one 32-wide K block) uses.
+__host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(int M, int N, uint32_t sfa_id, uint32_t sfb_id) {
+  return ((sfb_id & 3u) << 4)            // B scale-factor byte
+         | (5u << 7)                     // A format: E2M1
+         | (0u << 10)                    // B format: E4M3
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | (1u << 23)                    // scale format: E8M0
+         | ((uint32_t)(M >> 4) << 24)    // M / 16
+         | ((sfa_id & 3u) << 29);        // A scale-factor byte
+}
+
+// D[tmem] (+)= (A * SFA)[smem desc] * (B * SFB)[smem desc]^T over one 32-wide K block,
+// kind::mxf8f6f4, one CTA.  sfa_tmem / sfb_tmem address the scale-factor columns.
+__device__ __forceinline__ void mma_mx_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// SMEM descriptor of an unswizzled K-major source of 16-byte rows: 8-row core matrices
+// stored back to back (128 bytes apart).
+__device__ __forceinline__ uint64_t smem_desc_k_rows16(const void* p) {
+  const uint64_t addr = smem_u32(p);
+  uint64_t d = (addr & 0x3FFFFull) >> 4;   // start address (16-byte units)
+  d |= 1ull << 16;                          // leading byte offset (one 16-byte column: unused)
+  d |= (uint64_t)(128 >> 4) << 32;          // stride byte offset: next 8-row core matrix
+  d |= 1ull << 46;                          // descriptor version (sm_100)
+  return d;                                 // layout type 0: no swizzle
+}
+
+// Copy 32 rows x 16 bytes from SMEM into TMEM lanes 0-31, columns taddr..taddr+3, and
+// the same data into the other three lane quarters (the scale-factor layout).
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
 // ----------------------------------------------------------------------------- E2M1
 // Four bytes (eight E2M1 codes, the even element in each low nibble) to four f16x2
 // words; each byte's high nibble becomes the upper half.
