@@ -33,12 +33,11 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous on that stream.  The returned status covers the synchronous
  *     argument checks and launch errors only; errors the kernels detect (a
- *     timed-out wait, non-finite input, a value outside the f16 tensor-core
- *     range) are recorded in the workspace status word: read them with
- *     moe_device_status().
+ *     timed-out wait, non-finite input) are recorded in the workspace status
+ *     word: read them with moe_device_status().
  *   - No call throws across the ABI or prints.
  *   - bf16 tensors are passed as uint16_t bit patterns.
- *   - Device pointers must be 16-byte aligned.
+ *   - Device pointers must be 16-byte aligned; MXFP4 code arrays 32-byte aligned.
  */
 #ifndef MOE_MXFP4_H
 #define MOE_MXFP4_H
@@ -60,17 +59,21 @@ typedef enum {
   MOE_ERR_CUDA = 4,              /* a CUDA runtime error at launch */
   MOE_ERR_TIMEOUT = 5,           /* (device) a pipeline wait gave up; the kernel exited cleanly */
   MOE_ERR_NONFINITE = 6,         /* (device) Inf/NaN in the input or the weights */
-  MOE_ERR_RANGE = 7,             /* (device) an MXFP4 scale or activation outside the range the
-                                    f16 tensor-core path represents exactly (see moe_forward) */
+                                 /* 7 is not used */
   MOE_ERR_DEVICE = 8             /* the current device is not sm_100 */
 } moe_status;
 
 typedef enum {
   MOE_PATH_AUTO = 0, /* GEMV when tokens per expert are few, else GEMM */
-  MOE_PATH_GEMV = 1, /* weight-streaming tcgen05 path with 16-token tiles (small batches) */
-  MOE_PATH_GEMM = 2, /* tcgen05 grouped GEMM with 128-token tiles (large batches) */
-  MOE_PATH_SIMT = 3  /* fp32 CUDA-core path (no tensor cores): a cross-check, not for speed */
+  MOE_PATH_GEMV = 1, /* weight-streaming path: 8-token tiles (small batches) */
+  MOE_PATH_GEMM = 2  /* grouped GEMM: 96-token tiles (large batches) */
 } moe_path;
+
+/* Which projection a weight tensor is (sets its row order in storage). */
+typedef enum {
+  MOE_WEIGHT_PLAIN = 0,   /* any [E][N][K], rows stored in order (W2, the down projection) */
+  MOE_WEIGHT_GATE_UP = 1  /* W1 [E][2I][d]: gate rows 0..I-1, up rows I..2I-1 */
+} moe_weight_role;
 
 typedef struct {
   int32_t d;            /* hidden size (gpt-oss: 2880)                                  */
@@ -84,33 +87,38 @@ typedef struct {
 } moe_dims;
 
 /* ---------------------------------------------------------------- MXFP4 storage
- * A weight tensor [E][N][K] (K = reduction axis; N and K multiples of 64) is stored in
- * blocks of 64 rows x 64 k, each block one contiguous run (exactly 4.25 bits/param):
- *   codes  [E][N/64][K/64][64 rows][32 bytes]: row r of a block keeps its 64 E2M1
- *          codes as two 16-byte chunks (k 0..31, k 32..63); chunk c is stored at
- *          chunk position c ^ ((r >> 2) & 1); byte j of a chunk holds k = 2j in the low
- *          nibble and k = 2j+1 in the high nibble.  Code bits: sign (bit 3), exponent
- *          (bits 2..1, bias 1), mantissa (bit 0).
- *   scales [E][N/64][K/64][2][64] bytes: E8M0 scale 2^(byte - 127) of row r for
- *          k = 32c .. 32c+31 of the block at index [c][r].
- * One block is what the tensor-core kernels stream per pipeline stage: 2048 contiguous
- * code bytes and 128 contiguous scale bytes, copied with single bulk copies.
- * W1 (gate_up) is [E][2I][d]: rows 0..I-1 are the gate projection, I..2I-1 the up
- * projection.  W2 (down) is [E][d][I].
+ * A weight tensor [E][N][K] (K = reduction axis, a multiple of 64; N a multiple of 64)
+ * is stored in the form the tensor cores' block-scaled MMA reads, in tiles of 128 rows
+ * x 128 k.  With NT = ceil(N/128) and KC = ceil(K/128):
+ *   codes  [E][NT][KC][128][64] bytes: one contiguous 8 KB block per tile; byte j of
+ *          row r of block [e][t][c] holds the E2M1 codes of row 128t + r at
+ *          k = 128c + 2j (low nibble) and k = 128c + 2j + 1 (high nibble); codes of
+ *          rows >= N or k >= K are 0.  Code bits: sign (bit 3), exponent (bits 2..1,
+ *          bias 1), mantissa (bit 0).
+ *   scales [E][NT][KC][512] bytes: the E8M0 scale 2^(byte - 127) of (row n, 32-value
+ *          block b) is byte (n%32)*16 + ((n%128)/32)*4 + b%4 of the 512-byte group
+ *          [e][n/128][b/4] (the tensor cores' scale-factor layout: 128 rows x 4
+ *          blocks); bytes of rows >= N or blocks >= K/32 are 127.
+ * For MOE_WEIGHT_GATE_UP the rows are stored in the order of 128-row tiles that each
+ * pair 64 gate rows with the 64 matching up rows: stored row 128*t + r holds gate row
+ * 64*t + r (r < 64) or up row I + 64*t + r - 64 (r >= 64); I must be a multiple of 64.
+ * Payload: 4.25 bits per parameter (plus the zero padding up to 128 rows and 128 k).
  */
-size_t moe_mxfp4_codes_bytes(int32_t E, int32_t N, int32_t K);  /* E*N*K/2 */
-size_t moe_mxfp4_scales_bytes(int32_t E, int32_t N, int32_t K); /* E*(K/32)*N */
+size_t moe_mxfp4_codes_bytes(int32_t E, int32_t N, int32_t K);  /* E*NT*KC*8192 */
+size_t moe_mxfp4_scales_bytes(int32_t E, int32_t N, int32_t K); /* E*NT*KC*512 */
 
-/* Quantize fp32 weights w [E][N][K] (device) to MXFP4 (codes, scales as above).
+/* Quantize fp32 weights w [E][N][K] (device, row-major) to MXFP4 (codes, scales as above).
  * Per 32-value block: s = clamp(floor(log2(amax)) - 2, -127, 127); each value
  * x * 2^-s is rounded to the nearest E2M1 value (ties to the even code), saturating
  * at +-6; the sign bit is set only on non-zero codes; an all-zero block gets s = 0.
  * (ewbang.com article, section 量化: 4-bit values, one 8-bit scale per 32.)
+ * role: a moe_weight_role (MOE_WEIGHT_GATE_UP needs N = 2I with I a multiple of 64).
  * status_word: optional device int32; MOE_ERR_NONFINITE is OR-ed into it when a
  * block holds Inf/NaN (that block's scale byte is then 0xFF, the E8M0 NaN).
- * Errors: MOE_ERR_INVALID_ARG (null/misaligned pointer, E/N/K <= 0),
- * MOE_ERR_UNSUPPORTED_SHAPE (N or K not a multiple of 64), MOE_ERR_CUDA. */
-moe_status moe_mxfp4_quantize(const float* w, int32_t E, int32_t N, int32_t K, uint8_t* codes,
+ * Errors: MOE_ERR_INVALID_ARG (null/misaligned pointer, E/N/K <= 0, bad role),
+ * MOE_ERR_UNSUPPORTED_SHAPE (N or K not a multiple of 64; GATE_UP with N/2 not a
+ * multiple of 64), MOE_ERR_CUDA. */
+moe_status moe_mxfp4_quantize(const float* w, int32_t E, int32_t N, int32_t K, int32_t role, uint8_t* codes,
                               uint8_t* scales, int32_t* status_word, void* stream);
 
 /* Bytes of device scratch moe_route / moe_forward need for T tokens.  The first 256
@@ -137,16 +145,17 @@ moe_status moe_route(const moe_dims* dims, int32_t T, const uint16_t* x, const f
                      void* stream);
 
 /* The whole layer: y [T][d] bf16 = x + MoE(RMSNorm(x)).
- *   w1_codes / w1_scales: W1 [E][2I][d] in the MXFP4 storage above
- *   w2_codes / w2_scales: W2 [E][d][I]
+ *   w1_codes / w1_scales: W1 [E][2I][d] in the MXFP4 storage above, role GATE_UP
+ *   w2_codes / w2_scales: W2 [E][d][I], role PLAIN
  * Optional outputs (device, NULL to skip): topk_idx_out [T][k], topk_w_out [T][k],
  * counts_out [E].
  * y may not alias x.  T >= 1 (T = 0 returns MOE_OK and launches nothing).
- * Tensor-core paths (GEMV, GEMM) multiply f16 operands with fp32 accumulation:
- * xe and h are bf16 values, exact in f16 when |v| <= 65504 (|h| <= L^2 always is);
- * a decoded weight E2M1 * 2^s is exact in f16 for s in [-23, 13] (scale bytes
- * 104..140).  Outside those ranges the call records MOE_ERR_RANGE instead of
- * returning a rounded result; MOE_PATH_SIMT has no such limit.
+ * Arithmetic: the expert projections run on the tensor cores' block-scaled MMA
+ * (E2M1 weights with their E8M0 scales, as stored) with fp32 accumulation.  Each
+ * activation (xe, then h) enters as two E4M3 terms with one E8M0 scale per 32 values
+ * each: hi = RN(v / 2^s1), lo = RN((v - hi * 2^s1) / 2^s2), s1 and s2 set by the
+ * largest |v| and the largest residual of the block.  hi + lo equals v whenever
+ * |v| >= 2^-13 * max|block|; smaller values are off by at most 2^-20 * max|block|.
  * Errors: as moe_route. */
 moe_status moe_forward(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
                        const float* router_w, const float* router_b, const uint8_t* w1_codes,
@@ -159,8 +168,10 @@ moe_status moe_forward(const moe_dims* dims, int32_t T, const uint16_t* x, const
  * just before the i-th kernel this call launches and event 2i+1 just after it, until
  * the array runs out.  Recording adds no synchronization; when `stream` is being captured
  * into a CUDA graph the events are recorded as external event nodes of the graph, so
- * that every replay records them.  The kernels of a call are,
- * in order: route (RMSNorm + router + top-k), group, gather, gate_up, down, combine.
+ * that every replay records them.  The kernels of a call are, in order: route
+ * (RMSNorm + router + top-k + E4M3 split of xe), group, tile scales, gate_up, down,
+ * combine; on the GEMV path with T <= 64, route (which then also groups and writes the
+ * tile scales), gate_up and down (which then also combines).
  * Errors: as moe_forward; MOE_ERR_INVALID_ARG if n_events < 0 or events is NULL with
  * n_events > 0. */
 moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
@@ -175,17 +186,23 @@ moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x,
 int32_t moe_resolve_path(const moe_dims* dims, int32_t T);
 
 /* Byte offsets of the workspace's sub-buffers for T tokens, for inspection by tests and
- * debuggers (layout may change between versions).  offsets[0..13] receive, in order:
- * status, counts (int32 [E], then internal counters), offsets, ntiles, tiles, topk_idx,
- * topk_w, perm, inv, w_sorted,
- * xe [T][d] f16, xs [T*k][d] f16 (xe in sorted pair order), h [T*k][I] f16 (SwiGLU
- * output, sorted order), ys [T*k][d] fp32 (weighted expert outputs, sorted order);
- * offsets[14] = total bytes.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE. */
+ * debuggers (layout may change between versions).  offsets[0..MOE_WS_FIELDS-2] receive,
+ * in order: status, counts (int32 [E], then internal counters), offsets, ntiles,
+ * tile_base (int32 [E]: first token tile of each expert), tiles, topk_idx, topk_w, perm,
+ * inv, w_sorted,
+ * xq  [T][2][dp] E4M3 (hi and lo terms of xe = bf16(xn) per token; dp = d rounded up to
+ *     a multiple of 128), xsf [T][2][dp/32] E8M0 (their scales),
+ * sfx (the scales of each token tile's columns, in the tensor cores' scale-factor layout),
+ * hq  [2*T*k][Ip] E4M3 (hi / lo terms of the SwiGLU output h, sorted order), sfh,
+ * ys  [T*k][d] fp32 (weighted expert outputs, sorted order);
+ * offsets[MOE_WS_FIELDS-1] = total bytes.  Errors: MOE_ERR_INVALID_ARG,
+ * MOE_ERR_UNSUPPORTED_SHAPE. */
+#define MOE_WS_FIELDS 18
 moe_status moe_workspace_layout(const moe_dims* dims, int32_t T, size_t* offsets);
 
 /* Synchronize `stream`, then read and clear the device status word of workspace `ws`
  * (device pointer).  Returns MOE_OK or the first device-side error recorded since the
- * last read (MOE_ERR_TIMEOUT, MOE_ERR_NONFINITE, MOE_ERR_RANGE), or MOE_ERR_CUDA. */
+ * last read (MOE_ERR_TIMEOUT, MOE_ERR_NONFINITE), or MOE_ERR_CUDA. */
 moe_status moe_device_status(void* ws, void* stream);
 
 /* Static description of a status code. */
@@ -203,7 +220,8 @@ int32_t moe_last_launch_count(void);
  * implicit synchronization once it is running -- use it instead of moe_forward.
  * Scratch: a fixed 16 MiB array in the library's own device memory, present on every GPU
  * that loads the library until the process exits.  T whose moe_workspace_bytes() exceed
- * 16 MiB is rejected with MOE_ERR_WORKSPACE (at d = I = 2880, top-4: up to 171 tokens).
+ * 16 MiB is rejected with MOE_ERR_WORKSPACE (at d = I = 2880, E = 32, top-4: up to 150
+ * tokens).
  * The first call on a device looks up the array's device address for that device
  * (cudaGetSymbolAddress); make that first call before any stream capture.
  * All calls share the one array and it keeps the previous call's contents; the device
@@ -217,8 +235,7 @@ moe_status moe_forward_no_alloc(const moe_dims* dims, int32_t T, const uint16_t*
                                 uint16_t* y, int32_t* status_out, void* stream);
 
 /* Test hook for the device-side failure path.  With enable != 0, the next moe_forward
- * (or moe_forward_timed) call on this host thread, if it takes a tensor-core path, launches
- * its gate_up kernel with one pipeline arrival withheld in its first CTA: that CTA's bounded
+ * (or moe_forward_timed) call on this host thread launches its gate_up kernel with one pipeline arrival withheld in its first CTA: that CTA's bounded
  * wait expires after about 2 s, the CTA drains its copies, frees its tensor memory and
  * exits, and the workspace status word records MOE_ERR_TIMEOUT (y of that call is then
  * unspecified).  The hook clears itself after that call; nothing faults or hangs. */

@@ -26,14 +26,16 @@ MOE_ERR_WORKSPACE = 3
 MOE_ERR_CUDA = 4
 MOE_ERR_TIMEOUT = 5
 MOE_ERR_NONFINITE = 6
-MOE_ERR_RANGE = 7
 MOE_ERR_DEVICE = 8
 
 MOE_PATH_AUTO = 0
 MOE_PATH_GEMV = 1
 MOE_PATH_GEMM = 2
-MOE_PATH_SIMT = 3
-PATHS = {"auto": MOE_PATH_AUTO, "gemv": MOE_PATH_GEMV, "gemm": MOE_PATH_GEMM, "simt": MOE_PATH_SIMT}
+PATHS = {"auto": MOE_PATH_AUTO, "gemv": MOE_PATH_GEMV, "gemm": MOE_PATH_GEMM}
+
+MOE_WEIGHT_PLAIN = 0
+MOE_WEIGHT_GATE_UP = 1
+ROLES = {"plain": MOE_WEIGHT_PLAIN, "down": MOE_WEIGHT_PLAIN, "gate_up": MOE_WEIGHT_GATE_UP}
 
 
 class MoeError(RuntimeError):
@@ -73,7 +75,7 @@ def lib():
             L.moe_mxfp4_codes_bytes.restype = sz
             L.moe_mxfp4_scales_bytes.argtypes = [i32, i32, i32]
             L.moe_mxfp4_scales_bytes.restype = sz
-            L.moe_mxfp4_quantize.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
+            L.moe_mxfp4_quantize.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
             L.moe_mxfp4_quantize.restype = ctypes.c_int
             L.moe_workspace_bytes.argtypes = [dp, i32]
             L.moe_workspace_bytes.restype = sz
@@ -148,15 +150,23 @@ def moe_mxfp4_scales_bytes(E: int, N: int, K: int) -> int:
     return lib().moe_mxfp4_scales_bytes(E, N, K)
 
 
+def kpad128(K: int) -> int:
+    return (K + 127) // 128 * 128
+
+
 def mxfp4_shapes(E: int, N: int, K: int):
-    """Tensor shapes of the library's MXFP4 block layout (see include/moe_mxfp4.h):
-    codes [E, N/64, K/64, 64, 32], scales [E, N/64, K/64, 2, 64] (uint8)."""
-    return (E, N // 64, K // 64, 64, 32), (E, N // 64, K // 64, 2, 64)
+    """Tensor shapes of the library's MXFP4 storage (see include/moe_mxfp4.h):
+    codes [E, NT, KC, 128, 64], scales [E, NT, KC, 512] (uint8), NT = ceil(N/128), KC = ceil(K/128)."""
+    NT, KC = (N + 127) // 128, kpad128(K) // 128
+    return (E, NT, KC, 128, 64), (E, NT, KC, 512)
 
 
 def moe_mxfp4_quantize(w: torch.Tensor, codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
-                       status_word: torch.Tensor | None = None, stream=None):
-    """fp32 weights [E, N, K] -> (codes, scales) in the library's MXFP4 block layout."""
+                       role: int | str = MOE_WEIGHT_PLAIN, status_word: torch.Tensor | None = None, stream=None):
+    """fp32 weights [E, N, K] -> (codes, scales) in the library's MXFP4 storage.
+    role: "gate_up" for W1 [E, 2I, d] (gate rows then up rows), "down"/"plain" otherwise."""
+    if isinstance(role, str):
+        role = ROLES[role]
     if w.dim() == 2:
         w = w.unsqueeze(0)
     _need(w, torch.float32, "w")
@@ -166,10 +176,10 @@ def moe_mxfp4_quantize(w: torch.Tensor, codes: torch.Tensor | None = None, scale
         codes = torch.empty(cs, dtype=torch.uint8, device=w.device)
     if scales is None:
         scales = torch.empty(ss, dtype=torch.uint8, device=w.device)
-    if codes.numel() != E * N * K // 2 or scales.numel() != E * N * K // 32:
+    if codes.numel() != moe_mxfp4_codes_bytes(E, N, K) or scales.numel() != moe_mxfp4_scales_bytes(E, N, K):
         raise ValueError("codes / scales have the wrong size")
-    _check(lib().moe_mxfp4_quantize(_ptr(w), E, N, K, _ptr(codes), _ptr(scales), _ptr(status_word), _stream(stream)),
-           "moe_mxfp4_quantize")
+    _check(lib().moe_mxfp4_quantize(_ptr(w), E, N, K, role, _ptr(codes), _ptr(scales), _ptr(status_word),
+                                    _stream(stream)), "moe_mxfp4_quantize")
     return codes, scales
 
 
@@ -223,13 +233,13 @@ def moe_forward(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scal
     return (y, r) if want_routing else y
 
 
-WS_FIELDS = ("status", "counts", "offsets", "ntiles", "tiles", "topk_idx", "topk_w", "perm", "inv", "w_sorted",
-             "xe", "xs", "h", "ys", "total")
+WS_FIELDS = ("status", "counts", "offsets", "ntiles", "tile_base", "tiles", "topk_idx", "topk_w", "perm", "inv",
+             "w_sorted", "xq", "xsf", "sfx", "hq", "sfh", "ys", "total")
 
 
 def moe_workspace_layout(dims: moe_dims, T: int) -> dict:
     """Byte offsets of the workspace sub-buffers (for tests and debugging)."""
-    arr = (ctypes.c_size_t * 15)()
+    arr = (ctypes.c_size_t * len(WS_FIELDS))()
     _check(lib().moe_workspace_layout(ctypes.byref(dims), T, arr), "moe_workspace_layout")
     return dict(zip(WS_FIELDS, list(arr)))
 

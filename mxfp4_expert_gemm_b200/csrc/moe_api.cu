@@ -13,6 +13,7 @@ thread_local int32_t g_last_launches = 0;
 thread_local int32_t g_inject_timeout = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // Compute capability check, remembered per device (bit set = checked and sm_100).
 std::atomic<uint64_t> g_device_ok{0};
@@ -32,7 +33,7 @@ moe_status check_device() {
 
 moe_status check_dims(const moe_dims* dm, int32_t T) {
   if (!dm || T < 0) return MOE_ERR_INVALID_ARG;
-  if (dm->path < MOE_PATH_AUTO || dm->path > MOE_PATH_SIMT) return MOE_ERR_INVALID_ARG;
+  if (dm->path < MOE_PATH_AUTO || dm->path > MOE_PATH_GEMM) return MOE_ERR_INVALID_ARG;
   if (!(dm->rms_eps >= 0.f) || !std::isfinite(dm->rms_eps)) return MOE_ERR_INVALID_ARG;
   if (!(dm->swiglu_limit > 0.f) || !std::isfinite(dm->swiglu_limit)) return MOE_ERR_INVALID_ARG;
   if (dm->block != 32) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -51,8 +52,10 @@ int resolve_path(const moe_dims& dm, int32_t T) {
   return per_expert <= 24.0 ? MOE_PATH_GEMV : MOE_PATH_GEMM;
 }
 
-int tile_tokens_of(int path) {
-  return path == MOE_PATH_SIMT ? moe::simt_tile_tokens() : moe::tc_tile_tokens(path);
+int tile_tokens_of(int path) { return moe::expert_tile_tokens(path); }
+
+moe::WsLayout layout_for(const moe_dims& dm, int32_t T) {
+  return moe::ws_layout(dm, T, tile_tokens_of(resolve_path(dm, T)));
 }
 
 moe_status prepare(const moe_dims* dm, int32_t T, const uint16_t* x, const float* norm_w, const float* router_w,
@@ -63,7 +66,7 @@ moe_status prepare(const moe_dims* dm, int32_t T, const uint16_t* x, const float
   if (!x || !norm_w || !router_w || !ws) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(norm_w) || !aligned16(router_w) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
   if (router_b && !aligned16(router_b)) return MOE_ERR_INVALID_ARG;
-  L = moe::ws_layout(*dm, T);
+  L = layout_for(*dm, T);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   st = check_device();
   if (st != MOE_OK) return st;
@@ -94,24 +97,25 @@ extern "C" {
 
 size_t moe_mxfp4_codes_bytes(int32_t E, int32_t N, int32_t K) {
   if (E <= 0 || N <= 0 || K <= 0) return 0;
-  return (size_t)E * N * (K / 2);
+  return (size_t)E * (size_t)((N + 127) / 128) * (size_t)(moe::kpad128(K) / moe::kKChunk) * moe::kCodeBlockBytes;
 }
 
 size_t moe_mxfp4_scales_bytes(int32_t E, int32_t N, int32_t K) {
   if (E <= 0 || N <= 0 || K <= 0) return 0;
-  return (size_t)E * (K / 32) * N;
+  return (size_t)E * (size_t)((N + 127) / 128) * (size_t)(moe::kpad128(K) / moe::kKChunk) * moe::kSfGroupBytes;
 }
 
-moe_status moe_mxfp4_quantize(const float* w, int32_t E, int32_t N, int32_t K, uint8_t* codes, uint8_t* scales,
-                              int32_t* status_word, void* stream) {
+moe_status moe_mxfp4_quantize(const float* w, int32_t E, int32_t N, int32_t K, int32_t role, uint8_t* codes,
+                              uint8_t* scales, int32_t* status_word, void* stream) {
   g_last_launches = 0;
   if (!w || !codes || !scales || E <= 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(w) || !aligned16(codes) || !aligned16(scales)) return MOE_ERR_INVALID_ARG;
+  if (role != MOE_WEIGHT_PLAIN && role != MOE_WEIGHT_GATE_UP) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned32(codes) || !aligned16(scales)) return MOE_ERR_INVALID_ARG;
   if (K % 64 || N % 64) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (role == MOE_WEIGHT_GATE_UP && (N / 2) % 64) return MOE_ERR_UNSUPPORTED_SHAPE;
   moe_status st = check_device();
   if (st != MOE_OK) return st;
-  const int n = moe::launch_quantize(w, (int64_t)E * N, N, K, E, codes, scales, status_word,
-                                     static_cast<cudaStream_t>(stream));
+  const int n = moe::launch_quantize(w, E, N, K, role, codes, scales, status_word, static_cast<cudaStream_t>(stream));
   if (n < 0) return MOE_ERR_CUDA;
   g_last_launches = n;
   return MOE_OK;
@@ -119,7 +123,7 @@ moe_status moe_mxfp4_quantize(const float* w, int32_t E, int32_t N, int32_t K, u
 
 size_t moe_workspace_bytes(const moe_dims* dims, int32_t T) {
   if (check_dims(dims, T) != MOE_OK) return 0;
-  return moe::ws_layout(*dims, T).total;
+  return layout_for(*dims, T).total;
 }
 
 moe_status moe_route(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
@@ -132,8 +136,7 @@ moe_status moe_route(const moe_dims* dims, int32_t T, const uint16_t* x, const f
   if (st != MOE_OK) return st;
   if (T == 0) return MOE_OK;
   a.stream = static_cast<cudaStream_t>(stream);
-  const int path = resolve_path(*dims, T);
-  const int n = moe::launch_route(a, tile_tokens_of(path));
+  const int n = moe::launch_route(a);
   if (n < 0) return MOE_ERR_CUDA;
   const size_t P = (size_t)T * dims->top_k;
   if ((st = copy_out(topk_idx, a.ws.topk_idx, 4 * P, a.stream)) != MOE_OK) return st;
@@ -161,16 +164,19 @@ moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x,
                              size_t ws_bytes, void* stream, void* const* events, int32_t n_events) {
   g_last_launches = 0;
   if (n_events < 0 || (n_events > 0 && !events)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_dims(dims, T);
+  if (st != MOE_OK) return st;
+  if (T > 0) {  // (argument errors come before any device query)
+    if (!w1_codes || !w1_scales || !w2_codes || !w2_scales || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned32(w1_codes) || !aligned16(w1_scales) || !aligned32(w2_codes) || !aligned16(w2_scales) ||
+        !aligned16(y))
+      return MOE_ERR_INVALID_ARG;
+    if ((const void*)y == (const void*)x) return MOE_ERR_INVALID_ARG;
+  }
   moe::FwdArgs a;
   moe::WsLayout L;
-  moe_status st = prepare(dims, T, x, norm_w, router_w, router_b, ws, ws_bytes, a, L);
+  st = prepare(dims, T, x, norm_w, router_w, router_b, ws, ws_bytes, a, L);
   if (st != MOE_OK) return st;
-  if (T == 0) return MOE_OK;
-  if (!w1_codes || !w1_scales || !w2_codes || !w2_scales || !y) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(w1_codes) || !aligned16(w1_scales) || !aligned16(w2_codes) || !aligned16(w2_scales) ||
-      !aligned16(y))
-    return MOE_ERR_INVALID_ARG;
-  if ((const void*)y == (const void*)x) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   a.w1c = w1_codes;
   a.w1s = w1_scales;
@@ -190,16 +196,15 @@ moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x,
   a.inject_timeout = g_inject_timeout;
   g_inject_timeout = 0;
   const int path = resolve_path(*dims, T);
-  // Small-batch path: fewer, fused kernels (routing + grouping + gather; down + combine).
+  // Small-batch path: fewer, fused kernels (routing + grouping + tile scales; down + combine).
   a.fuse_group = (path == MOE_PATH_GEMV && T <= moe::kFusedGroupMaxT) ? 1 : 0;
   a.fuse_combine = (path == MOE_PATH_GEMV) ? 1 : 0;
   // Overlap each kernel's launch and prologue with its predecessor, except when per-kernel
   // events are recorded between the kernels.
   a.pdl = (n_events == 0) ? 1 : 0;
-  int n = moe::launch_route(a, tile_tokens_of(path));
+  int n = moe::launch_route(a);
   if (n < 0) return MOE_ERR_CUDA;
-  const int ne = (path == MOE_PATH_SIMT) ? moe::launch_experts_simt(a)
-                                         : moe::launch_experts_tc(a, tile_tokens_of(path));
+  const int ne = moe::launch_experts(a);
   if (ne < 0) return MOE_ERR_CUDA;
   n += ne;
   if (!a.fuse_combine) {
@@ -224,10 +229,11 @@ moe_status moe_workspace_layout(const moe_dims* dims, int32_t T, size_t* offsets
   if (!offsets) return MOE_ERR_INVALID_ARG;
   const moe_status st = check_dims(dims, T);
   if (st != MOE_OK) return st;
-  const moe::WsLayout L = moe::ws_layout(*dims, T);
-  const size_t v[15] = {L.status, L.counts, L.offsets, L.ntiles, L.tiles, L.topk_idx, L.topk_w, L.perm,
-                        L.inv, L.w_sorted, L.xe, L.xs, L.h, L.ys, L.total};
-  for (int i = 0; i < 15; ++i) offsets[i] = v[i];
+  const moe::WsLayout L = layout_for(*dims, T);
+  const size_t v[MOE_WS_FIELDS] = {L.status, L.counts, L.offsets,  L.ntiles, L.tile_base, L.tiles,
+                                   L.topk_idx, L.topk_w, L.perm,   L.inv,      L.w_sorted, L.xq,
+                                   L.xsf,    L.sfx,    L.hq,       L.sfh,    L.ys,       L.total};
+  for (int i = 0; i < MOE_WS_FIELDS; ++i) offsets[i] = v[i];
   return MOE_OK;
 }
 
@@ -253,7 +259,6 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_TIMEOUT: return "device wait timed out";
     case MOE_ERR_NONFINITE: return "non-finite value";
-    case MOE_ERR_RANGE: return "value outside the f16 tensor-core range";
     case MOE_ERR_DEVICE: return "device is not sm_100";
   }
   return "unknown status";

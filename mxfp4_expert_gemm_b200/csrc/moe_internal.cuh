@@ -1,7 +1,9 @@
 // Internal declarations shared by the kernels and the C-ABI front end.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 
@@ -10,7 +12,9 @@
 namespace moe {
 
 constexpr int kStatusBytes = 256;
-constexpr int kMinTileTokens = 16;  // smallest token tile of any path (sizes the tile list)
+constexpr int kMinTileTokens = 8;   // smallest token tile of any path (sizes the tile list)
+constexpr int kKChunk = 128;        // reduction-axis chunk: one TMA box row, one scale-factor group
+constexpr int kSfGroupBytes = 512;  // scale factors of 128 rows x 4 blocks of 32
 
 // Token tile of the grouped expert kernels: rows [row0, row0 + rows) of the
 // expert-sorted pair list, all belonging to expert `e`.
@@ -21,6 +25,41 @@ struct Tile {
   int32_t pad;
 };
 
+__host__ __device__ __forceinline__ int64_t kpad128(int64_t K) { return (K + kKChunk - 1) / kKChunk * kKChunk; }
+
+// Byte offset, within one 512-byte scale-factor group, of row r (of 128) and 32-block b
+// (of 4): the layout the tensor cores' scale-factor copy (32 lanes x 16 bytes, repeated
+// for the four lane quarters) expects.
+__host__ __device__ __forceinline__ int sf_byte_in_group(int r, int b) {
+  return (r & 31) * 16 + ((r & 127) >> 5) * 4 + (b & 3);
+}
+
+// Scale-factor groups of one token tile: tile_tokens tokens give 2 * tile_tokens MMA
+// columns (hi and lo term of each token), 128 columns per group.
+__host__ __device__ __forceinline__ int sf_groups_of(int tile_tokens) { return (2 * tile_tokens + 127) / 128; }
+
+// ------------------------------------------------------------------ MXFP4 storage layout
+// Weights [E][N][K] (moe_mxfp4.h) in tiles of 128 rows x 128 k: codes [E][NT][KC][128][64]
+// (one contiguous 8 KB block per tile, row-major inside), scales [E][NT][KC][512] in the
+// scale-factor layout above; NT = ceil(N/128), KC = ceil(K/128).  Gate_up tensors store
+// rows in 128-row tiles of 64 gate rows + the 64 matching up rows.
+constexpr int kCodeBlockBytes = 128 * kKChunk / 2;   // 8 KB
+
+__host__ __device__ __forceinline__ int64_t mx_code_offset(int64_t e, int64_t row, int64_t k, int64_t N, int64_t K) {
+  const int64_t nt = (N + 127) / 128, kc = kpad128(K) / kKChunk;
+  return ((e * nt + row / 128) * kc + k / kKChunk) * kCodeBlockBytes + (row & 127) * (kKChunk / 2) +
+         (k % kKChunk) / 2;
+}
+__host__ __device__ __forceinline__ int64_t gate_up_stored_row(int64_t n, int64_t I) {
+  const int64_t part = n >= I ? 1 : 0, f = n - part * I;
+  return (f / 64) * 128 + part * 64 + f % 64;
+}
+
+__host__ __device__ __forceinline__ int64_t mx_scale_offset(int64_t e, int64_t row, int64_t b, int64_t N, int64_t K) {
+  const int64_t nt = (N + 127) / 128, kc = kpad128(K) / kKChunk;
+  return ((e * nt + row / 128) * kc + b / 4) * kSfGroupBytes + sf_byte_in_group((int)(row & 127), (int)(b & 3));
+}
+
 // Carve-up of the caller's workspace (byte offsets, 256-byte aligned).
 struct WsLayout {
   size_t status;    // int32 device status word (first device error wins)
@@ -28,26 +67,35 @@ struct WsLayout {
                     // [T * ceil(d/128)] combine arrivals; cleared at the start of every call
   size_t offsets;   // int32 [E+1]
   size_t ntiles;    // int32 [4]: number of token tiles
+  size_t tile_base; // int32 [E]: first token tile of each expert
   size_t tiles;     // Tile [max_tiles]
   size_t topk_idx;  // int32 [T*k]
   size_t topk_w;    // f32 [T*k]
   size_t perm;      // int32 [P]   sorted position -> t*k + slot
   size_t inv;       // int32 [P]   t*k + slot -> sorted position
   size_t w_sorted;  // f32 [P]     routing weight of each sorted pair
-  size_t xe;        // f16 [T][d]  bf16(RMSNorm(x)) held as f16
-  size_t xs;        // f16 [P][d]  xe gathered in sorted pair order
-  size_t h;         // f16 [P][I]  SwiGLU output (bf16 values) in sorted order
+  size_t xq;        // E4M3 [T][2][dp]   hi / lo terms of xe = bf16(RMSNorm(x))
+  size_t xsf;       // E8M0 [T][2][dp/32] their scales
+  size_t sfx;       // E8M0 [max_tiles][dp/128][G][512] scales of xq per token tile and column
+  size_t hq;        // E4M3 [2P][Ip]     hi / lo terms of h (sorted order)
+  size_t sfh;       // E8M0 [max_tiles][Ip/128][G][512]
   size_t ys;        // f32 [P][d]  routing-weighted expert outputs, sorted order
   size_t total;
   int64_t max_tiles;
+  int32_t tile_tokens;
+  int32_t dp, ip;   // d and I rounded up to 128
 };
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-inline WsLayout ws_layout(const moe_dims& dm, int64_t T) {
+inline WsLayout ws_layout(const moe_dims& dm, int64_t T, int tile_tokens) {
   WsLayout L{};
   const int64_t P = T * dm.top_k;
-  L.max_tiles = (P + kMinTileTokens - 1) / kMinTileTokens + dm.E;
+  L.tile_tokens = tile_tokens;
+  L.max_tiles = (P + tile_tokens - 1) / tile_tokens + dm.E;
+  L.dp = (int32_t)kpad128(dm.d);
+  L.ip = (int32_t)kpad128(dm.I);
+  const size_t G = (size_t)sf_groups_of(tile_tokens);
   size_t o = 0;
   auto take = [&](size_t bytes) {
     const size_t at = o;
@@ -58,15 +106,18 @@ inline WsLayout ws_layout(const moe_dims& dm, int64_t T) {
   L.counts = take(4 * ((size_t)dm.E + 4 + (size_t)T * ((dm.d + 127) / 128)));
   L.offsets = take(4 * (size_t)(dm.E + 1));
   L.ntiles = take(16);
+  L.tile_base = take(4 * (size_t)dm.E);
   L.tiles = take(sizeof(Tile) * (size_t)L.max_tiles);
   L.topk_idx = take(4 * (size_t)P);
   L.topk_w = take(4 * (size_t)P);
   L.perm = take(4 * (size_t)P);
   L.inv = take(4 * (size_t)P);
   L.w_sorted = take(4 * (size_t)P);
-  L.xe = take(2 * (size_t)T * dm.d);
-  L.xs = take(2 * (size_t)P * dm.d);
-  L.h = take(2 * (size_t)P * dm.I);
+  L.xq = take(2 * (size_t)T * L.dp);
+  L.xsf = take(2 * (size_t)T * (L.dp / 32));
+  L.sfx = take((size_t)L.max_tiles * (L.dp / kKChunk) * G * kSfGroupBytes);
+  L.hq = take(2 * (size_t)P * L.ip);
+  L.sfh = take((size_t)L.max_tiles * (L.ip / kKChunk) * G * kSfGroupBytes);
   L.ys = take(4 * (size_t)P * dm.d);
   L.total = o;
   return L;
@@ -80,17 +131,22 @@ struct Ws {
   int32_t* arrivals;   // [T][ceil(d/128)] expert outputs written per (token, 128 columns)
   int32_t* offsets;
   int32_t* ntiles;
+  int32_t* tile_base;
   Tile* tiles;
   int32_t* topk_idx;
   float* topk_w;
   int32_t* perm;
   int32_t* inv;
   float* w_sorted;
-  uint16_t* xe;
-  uint16_t* xs;
-  uint16_t* h;
+  uint8_t* xq;
+  uint8_t* xsf;
+  uint8_t* sfx;
+  uint8_t* hq;
+  uint8_t* sfh;
   float* ys;
   int64_t max_tiles;
+  int32_t tile_tokens;
+  int32_t dp, ip;
 };
 
 inline Ws ws_pointers(void* base, const WsLayout& L, int E) {
@@ -100,20 +156,95 @@ inline Ws ws_pointers(void* base, const WsLayout& L, int E) {
   w.counts = reinterpret_cast<int32_t*>(b + L.counts);
   w.offsets = reinterpret_cast<int32_t*>(b + L.offsets);
   w.ntiles = reinterpret_cast<int32_t*>(b + L.ntiles);
+  w.tile_base = reinterpret_cast<int32_t*>(b + L.tile_base);
   w.tiles = reinterpret_cast<Tile*>(b + L.tiles);
   w.topk_idx = reinterpret_cast<int32_t*>(b + L.topk_idx);
   w.topk_w = reinterpret_cast<float*>(b + L.topk_w);
   w.perm = reinterpret_cast<int32_t*>(b + L.perm);
   w.inv = reinterpret_cast<int32_t*>(b + L.inv);
   w.w_sorted = reinterpret_cast<float*>(b + L.w_sorted);
-  w.xe = reinterpret_cast<uint16_t*>(b + L.xe);
-  w.xs = reinterpret_cast<uint16_t*>(b + L.xs);
-  w.h = reinterpret_cast<uint16_t*>(b + L.h);
+  w.xq = reinterpret_cast<uint8_t*>(b + L.xq);
+  w.xsf = reinterpret_cast<uint8_t*>(b + L.xsf);
+  w.sfx = reinterpret_cast<uint8_t*>(b + L.sfx);
+  w.hq = reinterpret_cast<uint8_t*>(b + L.hq);
+  w.sfh = reinterpret_cast<uint8_t*>(b + L.sfh);
   w.ys = reinterpret_cast<float*>(b + L.ys);
   w.ticket = w.counts + E;
   w.arrivals = w.counts + E + 4;
   w.max_tiles = L.max_tiles;
+  w.tile_tokens = L.tile_tokens;
+  w.dp = L.dp;
+  w.ip = L.ip;
   return w;
+}
+
+// ------------------------------------------------------------ activations as E4M3 pairs
+// The block-scaled MMA takes E4M3 activations with one E8M0 scale per 32 values.  A
+// bf16 value v (8 significant bits) is carried as two terms: hi = RN_e4m3(v / 2^s1) and
+// lo = RN_e4m3((v - hi * 2^s1) / 2^s2), where 2^s1 puts the block's largest |v| in
+// [128, 256) and s2 = s1 - 4.  The residual is at most half a step of hi, i.e. at most
+// 8 * 2^s1, so (v - hi * 2^s1) / 2^s2 <= 128 fits E4M3; it has at most 4 significant
+// bits (bf16's 8 minus hi's 4), so lo is exact while it stays in E4M3's normal range.
+// Hence hi * 2^s1 + lo * 2^s2 == v for every v of the block within a factor 2^13 of the
+// largest, and within 2^-20 of the largest otherwise.
+
+// floor(log2(a)) for a finite a > 0 (normal or subnormal), exactly.
+__device__ __forceinline__ int floor_log2f(float a) {
+  const uint32_t bits = __float_as_uint(a);
+  const int e = (int)((bits >> 23) & 0xFF);
+  if (e != 0) return e - 127;
+  return (31 - __clz((int)(bits & 0x7FFFFF))) - 149;
+}
+
+// Scale exponent for a block whose largest magnitude is amax (0 for an all-zero block):
+// amax / 2^s lands in [128, 256); s is clamped to [-122, 126] so that s - 4 stays a
+// normal power of two (E8M0 bytes 1..253).
+__device__ __forceinline__ int e4m3_block_exp(float amax) {
+  if (!(amax > 0.f) || !(amax < INFINITY)) return 0;
+  return max(-122, min(126, floor_log2f(amax) - 7));
+}
+
+__device__ __forceinline__ float pow2f(int s) { return __uint_as_float((uint32_t)(s + 127) << 23); }  // s in [-126, 127]
+
+// Two fp32 values to E4M3 (round to nearest even, saturating); a in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// E4M3 byte (low byte of q) back to fp32 (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t q) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(q & 0xFFu)));
+  return __half2float(__ushort_as_half((uint16_t)(h2 & 0xFFFFu)));
+}
+
+// Warp-cooperative split of 32-value blocks: each lane holds V consecutive values of a
+// block spread over 32/V consecutive lanes (V = 1: one block per warp; V = 2: two).
+// Returns this lane's hi / lo bytes (value i in byte i) and the block's two scale bytes.
+template <int V>
+__device__ __forceinline__ void e4m3_split(const float (&v)[V], uint32_t& hi, uint32_t& lo, uint32_t& sf_hi,
+                                           uint32_t& sf_lo) {
+  constexpr int kLanes = 32 / V;
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < V; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+  for (int o = kLanes / 2; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const int s1 = e4m3_block_exp(amax), s2 = s1 - 4;
+  const float inv1 = pow2f(-s1), sc1 = pow2f(s1), inv2 = pow2f(-s2);
+  hi = 0u;
+  lo = 0u;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const uint32_t q = e4m3x2(v[i] * inv1, 0.f) & 0xFFu;
+    hi |= q << (8 * i);
+    const float r = v[i] - e4m3_to_f32(q) * sc1;   // exact
+    lo |= (e4m3x2(r * inv2, 0.f) & 0xFFu) << (8 * i);
+  }
+  sf_hi = (uint32_t)(s1 + 127);
+  sf_lo = (uint32_t)(s2 + 127);
 }
 
 // Optional per-kernel CUDA events supplied by the caller: event 2i is recorded just
@@ -148,7 +279,7 @@ struct FwdArgs {
   cudaStream_t stream;
   EventRec* ev;
   int32_t inject_timeout;  // test hook: withhold one pipeline arrival in the gate_up kernel
-  int32_t fuse_group;      // small batches: the routing kernel also groups and gathers
+  int32_t fuse_group;      // small batches: the routing kernel also groups (and scatters tile scales)
   int32_t fuse_combine;    // the down kernel also adds the k expert outputs and the residual
   int32_t pdl;             // launch dependent kernels with programmatic stream serialization
 };
@@ -189,35 +320,6 @@ inline void ev_after(const FwdArgs& a) {
   }
 }
 
-// ------------------------------------------------------------------ MXFP4 storage layout
-// Weights [E][N][K] are stored in blocks of 64 rows x 64 k (N % 64 == 0, K % 64 == 0):
-//   codes  [E][N/64][K/64][64 rows][32 bytes]   (one 2048-byte run per block)
-//   scales [E][N/64][K/64][2][64]               (one 128-byte run per block)
-// Row r of a block keeps its 64 codes as two 16-byte chunks (k 0..31 and k 32..63);
-// chunk c sits at chunk position c ^ ((r >> 2) & 1), so that consecutive rows read by
-// consecutive threads fall in different shared-memory banks.  Byte j of a chunk holds
-// k = 2j (low nibble) and k = 2j + 1 (high nibble).  Scale byte (c, r) is the E8M0
-// scale of row r, k = 32c .. 32c + 31 of the block.
-constexpr int kBlkRows = 64;
-constexpr int kBlkK = 64;
-constexpr int kBlkCodeBytes = kBlkRows * kBlkK / 2;   // 2048
-constexpr int kBlkScaleBytes = kBlkRows * kBlkK / 32; // 128
-
-__host__ __device__ __forceinline__ int64_t mx_block_index(int64_t e, int64_t rb, int64_t ks, int64_t N, int64_t K) {
-  return (e * (N / kBlkRows) + rb) * (K / kBlkK) + ks;
-}
-
-// Byte offset of the 16-byte code chunk holding k = 32*kb .. 32*kb+31 of row n.
-__host__ __device__ __forceinline__ int64_t mx_code_chunk_offset(int64_t e, int64_t n, int64_t kb, int64_t N,
-                                                                  int64_t K) {
-  const int64_t r = n % kBlkRows, c = kb & 1;
-  return mx_block_index(e, n / kBlkRows, kb >> 1, N, K) * kBlkCodeBytes + r * 32 + ((c ^ ((r >> 2) & 1)) << 4);
-}
-
-__host__ __device__ __forceinline__ int64_t mx_scale_offset(int64_t e, int64_t n, int64_t kb, int64_t N, int64_t K) {
-  return mx_block_index(e, n / kBlkRows, kb >> 1, N, K) * kBlkScaleBytes + (kb & 1) * kBlkRows + n % kBlkRows;
-}
-
 // Record the first device-side error in the status word.
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
@@ -225,13 +327,11 @@ __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
 
 // --------------------------------------------------------------------------- launchers
 // Each returns the number of kernels it launched (>= 0) or -1 on a launch error.
-int launch_quantize(const float* w, int64_t rows, int32_t N, int32_t K, int32_t E, uint8_t* codes,
+int launch_quantize(const float* w, int32_t E, int32_t N, int32_t K, int32_t role, uint8_t* codes,
                     uint8_t* scales, int32_t* status, cudaStream_t st);
-int launch_route(const FwdArgs& a, int tile_tokens);   // norm + router + top-k + grouping + gather
-int launch_combine(const FwdArgs& a);                  // y = x + sum_j ys[inv]
-int launch_experts_simt(const FwdArgs& a);             // CUDA-core expert MLPs
-int launch_experts_tc(const FwdArgs& a, int tile_tokens);  // tcgen05 expert MLPs
-int tc_tile_tokens(int path);                          // token tile of a tensor-core path
-int simt_tile_tokens();                                // token tile of the CUDA-core path
+int launch_route(const FwdArgs& a);     // norm + router + top-k + E4M3 split, grouping, tile scales
+int launch_combine(const FwdArgs& a);   // y = x + sum_j ys[inv]
+int launch_experts(const FwdArgs& a);   // block-scaled tcgen05 expert MLPs (gate_up, down)
+int expert_tile_tokens(int path);       // token tile of a path
 
 }  // namespace moe

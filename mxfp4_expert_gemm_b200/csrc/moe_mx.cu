@@ -1,0 +1,637 @@
+// Block-scaled tcgen05 grouped expert GEMMs: gate_up with the clamped-SwiGLU epilogue,
+// and down with the routing-weight epilogue.
+//
+// Layer definition: the SwiGLU expert of "From GPT-2 to gpt-oss" (新智元
+// translation), sec. 3 (three linears, silu(z) = z * sigmoid(z)), with
+// swiglu_limit 7 from the llm-atlas GPT-OSS 20B config table; MXFP4 weights per the
+// ewbang.com GPT-OSS article, section 量化 (E2M1 values, one E8M0 scale per 32).
+//
+// The tensor cores read the MXFP4 weights as stored: tcgen05.mma kind::mxf8f6f4 with an
+// E2M1 A operand (the weights, 128 rows per tile) scaled by its E8M0 block scales, and an
+// E4M3 B operand (the activations) scaled by theirs; fp32 accumulation in TMEM.  Each
+// activation vector is two B columns, its hi and lo E4M3 terms (see e4m3_split), so a
+// tile of BN tokens is an MMA of N = 2*BN and the epilogue adds column pairs.
+//
+// Persistent kernel, CPS CTAs per SM.  A work item is 128 weight rows x one token tile
+// over the whole reduction axis; CTA b takes items b, b + grid, ...  A pipeline stage
+// covers NP chunks of 128 along the reduction axis:
+//   warp 0     producer: per stage one TMA load of the weight codes (NP consecutive
+//              8 KB tile blocks; E2M1, unpacked by the copy to one byte per code in
+//              shared memory, 128B swizzle), the activation rows [NP][2*BN][128] (gate_up:
+//              tile::gather4 loads of the tile's tokens from the per-token rows, issued
+//              by all lanes; down: one 3D TMA load of the sorted rows of h), and one bulk
+//              copy each of the weight and the activation scale factors, both stored in
+//              the tensor cores' scale-factor layout;
+//   warp 1     TMEM allocation and the MMA issuer (one thread): per stage it copies the
+//              scale factors into TMEM (tcgen05.cp) and issues one block-scaled MMA
+//              per 32-wide block of the reduction axis;
+//   warps 2.. epilogue, EG warpgroups taking alternate 32-column reads: read the fp32
+//              accumulator (double-buffered in TMEM so that it overlaps the next item's
+//              main loop), gate_up: SwiGLU and the E4M3 split of h for the down GEMM;
+//              down: routing weight, and for small batches the combine
+//              y = x + sum_j w_j o_j.
+// Gate_up weights are stored in 128-row tiles of 64 gate rows (TMEM lanes 0..63) and the
+// 64 matching up rows (lanes 64..127), so g and u of one feature meet in the epilogue.
+//
+// Every wait is bounded (kWaitLimitNs).  When one gives up, the CTA raises its abort
+// flag, every role leaves its loop, in-flight copies and MMAs are drained (bounded),
+// TMEM is freed and MOE_ERR_TIMEOUT is recorded.
+#include <cuda.h>
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+
+#include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;                          // weight rows per tile (TMEM lanes)
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: a stuck pipeline, not a slow one
+
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
+
+struct MxParams {
+  const Tile* tiles;
+  const int32_t* ntiles;
+  const uint8_t* w_sf;     // weight scale-factor groups [E][NT][KC][512]
+  const uint8_t* a_sf;     // activation scale-factor groups per token tile [tiles][KC][G][512]
+  int32_t NT;              // 128-row tiles per expert
+  int32_t K;               // reduction length (d for gate_up, I for down)
+  int32_t KC;              // 128-chunks of the reduction axis (K rounded up)
+  int32_t n_rt;            // row tiles per token tile: I/64 (gate_up) or ceil(d/128) (down)
+  int32_t* status;
+  float limit;
+  int32_t inject_timeout;  // test hook: CTA 0 withholds its first stage
+  // gate_up output: h as E4M3 hi / lo rows [2P][ip] and their scale factors per token tile
+  uint8_t* hq;
+  uint8_t* sfh;
+  int32_t ip;              // I rounded up to 128 (row pitch of hq)
+  int32_t KCh;             // ip / 128
+  // down output: ys [P][d] fp32 = w * o; optionally y = bf16(x + sum_j ys[inv[t*k + j]])
+  // by the last writer of each (token, 128-column) block
+  float* ys;
+  int32_t d;
+  const float* w_sorted;
+  int32_t fuse_combine;
+  int32_t k;
+  const int32_t* perm;
+  const int32_t* inv;
+  const uint16_t* x;
+  uint16_t* y;
+  int32_t* arrivals;
+};
+
+#ifndef MOE_SF_SLOTS
+#define MOE_SF_SLOTS 2
+#endif
+constexpr int kSfSlots = MOE_SF_SLOTS;  // scale-factor TMEM slots, used stage after stage in turn
+
+template <int BN, int NP, int S, int CPS, int EG>
+struct MxCfg {
+  static constexpr int N2 = 2 * BN;                     // MMA N: hi and lo column per token
+  static constexpr int G = (N2 + 127) / 128;            // scale-factor groups of the B operand
+  static constexpr int A_PANEL = kBM * kKChunk;         // 128 rows x 128 codes, one byte each
+  static constexpr int B_PANEL = N2 * kKChunk;          // N2 rows x 128 E4M3
+  static constexpr int B_OFF = NP * A_PANEL;
+  static constexpr int SFA_OFF = B_OFF + NP * B_PANEL;
+  static constexpr int SFB_OFF = SFA_OFF + NP * kSfGroupBytes;
+  static constexpr int STAGE_BYTES = ((SFB_OFF + NP * G * kSfGroupBytes + 1023) / 1024) * 1024;
+  static constexpr int A_TX = NP * kBM * kKChunk / 2;   // the weight box counts packed bytes
+  static constexpr int B_TX = NP * B_PANEL;
+  static constexpr int CW = N2 < 32 ? N2 : 32;          // accumulator columns per epilogue read
+  static constexpr int TC = CW / 2;                     // tokens per epilogue read
+  static constexpr int HT = TC / 2;                     // tokens each side (gate / up) finishes
+  static constexpr int ACC_COLS = N2 < 32 ? 32 : N2;    // one accumulator buffer
+  static constexpr int SF_SLOT_COLS = 4 * NP * (1 + G);         // A then B scale factors of a stage
+  static constexpr int SFA_COL = 2 * ACC_COLS;                   // + slot * SF_SLOT_COLS
+  static constexpr int SFB_COL = SFA_COL + 4 * NP;
+  static constexpr int COLS_NEEDED = 2 * ACC_COLS + kSfSlots * SF_SLOT_COLS;
+  static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 : COLS_NEEDED <= 128 ? 128
+                                   : COLS_NEEDED <= 256 ? 256 : 512;
+  static constexpr int EPI_GROUP_BYTES = TC * 64 * 4 + TC * 4;  // g / u exchange; token list (down)
+  static constexpr int EPI_BYTES = EG * EPI_GROUP_BYTES;
+  static constexpr int BAR_BYTES = 8 * (2 * S + 5) + 16;
+  static constexpr int SMEM_BYTES = S * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024 /*align slack*/;
+  static constexpr int EPI_THREADS = 128 * EG;
+  static constexpr int THREADS = 64 + EPI_THREADS;
+  static_assert(N2 == 16 || (N2 % 32 == 0 && N2 <= 256), "MMA N: 16 or a multiple of 32 up to 256");
+  static_assert(COLS_NEEDED <= 512 && TMEM_COLS * CPS <= 512, "TMEM budget of CPS co-resident CTAs");
+  static_assert(SMEM_BYTES * CPS <= 227 * 1024, "shared memory budget of CPS co-resident CTAs");
+  static_assert(kBM * NP <= 256, "TMA box height");
+  static_assert(EG == 1 || EG == 2, "one or two epilogue warpgroups");
+  static_assert(N2 % 4 == 0 && N2 / 4 <= 64, "gather4 columns: two instructions per producer lane");
+};
+
+template <int BN, int NP, int S, int CPS, int EG, int MODE>
+__global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
+    mx_expert_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_act,
+                     const MxParams p) {
+  using C = MxCfg<BN, NP, S, CPS, EG>;
+  extern __shared__ uint8_t smem_raw[];
+  pdl_trigger();
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* epi = smem + S * C::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi + C::EPI_BYTES);
+  uint64_t* sfree = full + S;       // stage consumed (its MMAs done)
+  uint64_t* accf = sfree + S;       // [2] accumulator ready
+  uint64_t* acce = accf + 2;        // [2] accumulator drained by the epilogue
+  uint64_t* drain = acce + 2;       // final MMA drain
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nst = (p.KC + NP - 1) / NP;   // stages per item
+  const int kblocks = p.K / 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&sfree[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&accf[b], 1);
+      ptx::mbar_init(&acce[b], C::EPI_THREADS);
+    }
+    ptx::mbar_init(drain, 1);
+    *s_abort = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tensormap(&tm_w);
+    ptx::prefetch_tensormap(&tm_act);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(s_tmem, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+    ptx::tc_fence_before();
+  }
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  // Everything above overlaps the previous kernel; the work list is its output.
+  pdl_wait();
+  const int n_items = *p.ntiles * p.n_rt;
+
+  auto a_s = [&](int s) { return smem + s * C::STAGE_BYTES; };
+  auto b_s = [&](int s) { return smem + s * C::STAGE_BYTES + C::B_OFF; };
+  auto sfa_s = [&](int s) { return smem + s * C::STAGE_BYTES + C::SFA_OFF; };
+  auto sfb_s = [&](int s) { return smem + s * C::STAGE_BYTES + C::SFB_OFF; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    // Lane 0 owns the ring and issues the weight load and the scale-factor copies; for
+    // gate_up every lane also gathers activation rows (tile::gather4, four MMA columns
+    // per instruction) straight from the per-token rows of xq, in the tile's token order.
+    int64_t g = 0;  // global stage counter of this CTA
+    bool stop = false, withheld = false;
+    for (int i = blockIdx.x; i < n_items && !stop; i += gridDim.x) {
+      const int tt = i / p.n_rt, rt = i - tt * p.n_rt;
+      const Tile tl = p.tiles[tt];
+      // gate_up: xq rows (2 t + term) of MMA columns 4 i4 .. 4 i4 + 3, i4 = lane, lane + 32
+      // (columns past the tile's tokens repeat its last token; their outputs are dropped)
+      int xr[2][4];
+      if (MODE == MODE_GATE_UP) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int n = 4 * (lane + 32 * u) + r;
+            const int j = min(n >> 1, tl.rows - 1);
+            xr[u][r] = (n < C::N2) ? 2 * (p.perm[tl.row0 + j] / p.k) + (n & 1) : 0;
+          }
+      }
+      for (int st = 0; st < nst; ++st, ++g) {
+        const int s = (int)(g % S);
+        bool ok = true;
+        if (lane == 0 && g >= S)
+          ok = ptx::mbar_wait_bounded(&sfree[s], (uint32_t)((g / S) - 1) & 1, s_abort, kWaitLimitNs);
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+          stop = true;
+          break;
+        }
+        if (p.inject_timeout && blockIdx.x == 0 && g == 0) {
+          withheld = true;  // this stage never fills: the MMA issuer's wait gives up
+          continue;
+        }
+        const int c0 = st * NP, nck = min(NP, p.KC - c0);
+        if (lane == 0) {
+          const int b_tx = (MODE == MODE_GATE_UP) ? nck * C::B_PANEL : C::B_TX;
+          ptx::mbar_arrive_expect_tx(&full[s], C::A_TX + b_tx + nck * (1 + C::G) * kSfGroupBytes);
+          ptx::tma_load_2d(a_s(s), &tm_w, 0, (int)(((int64_t)tl.e * p.NT + rt) * p.KC + c0) * kBM, &full[s]);
+          if (MODE == MODE_DOWN) ptx::tma_load_3d(b_s(s), &tm_act, 0, 2 * tl.row0, c0, &full[s]);
+          ptx::bulk_load(sfa_s(s), p.w_sf + ((int64_t)(tl.e * p.NT + rt) * p.KC + c0) * kSfGroupBytes,
+                         nck * kSfGroupBytes, &full[s]);
+          ptx::bulk_load(sfb_s(s), p.a_sf + ((int64_t)tt * p.KC + c0) * C::G * kSfGroupBytes,
+                         nck * C::G * kSfGroupBytes, &full[s]);
+        }
+        __syncwarp();
+        if (MODE == MODE_GATE_UP) {
+          for (int c = 0; c < nck; ++c)
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int i4 = lane + 32 * u;
+              if (4 * i4 < C::N2)
+                ptx::tma_gather4(b_s(s) + c * C::B_PANEL + i4 * 4 * kKChunk, &tm_act, (c0 + c) * kKChunk,
+                                 xr[u][0], xr[u][1], xr[u][2], xr[u][3], &full[s]);
+            }
+        }
+      }
+    }
+    // Never leave copies in flight when the CTA exits (consumers may have aborted before
+    // waiting for them): wait, bounded, for the last fill of every slot.  On the normal
+    // path these have all landed already.
+    if (lane == 0) {
+      volatile int local_abort = 0;
+      for (int64_t q = (g > S ? g - S : 0); q < g; ++q) {
+        if (withheld && q == 0) continue;
+        ptx::mbar_wait_bounded(&full[q % S], (uint32_t)(q / S) & 1, &local_abort, kWaitLimitNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int64_t g = 0;
+      int li = 0;
+      bool stop = false;
+      for (int i = blockIdx.x; i < n_items && !stop; i += gridDim.x, ++li) {
+        const int b = li & 1;
+        if (li >= 2 && !ptx::mbar_wait_bounded(&acce[b], (uint32_t)((li >> 1) - 1) & 1, s_abort, kWaitLimitNs))
+          break;
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem + b * C::ACC_COLS;
+        for (int st = 0; st < nst; ++st, ++g) {
+          const int s = (int)(g % S);
+          if (!ptx::mbar_wait_bounded(&full[s], (uint32_t)(g / S) & 1, s_abort, kWaitLimitNs)) {
+            stop = true;
+            break;
+          }
+          ptx::tc_fence_after();
+          const int c0 = st * NP, nck = min(NP, p.KC - c0);
+          // scale factors of this stage into their TMEM slot (the tensor pipe runs one
+          // thread's copies and MMAs in issue order; with two slots a copy does not
+          // overwrite columns the previous stage's MMAs still read)
+          const uint32_t sf_slot = tmem + (uint32_t)((g % kSfSlots) * C::SF_SLOT_COLS);
+          for (int c = 0; c < nck; ++c) {
+            ptx::tc_cp_32x128b_x4(sf_slot + C::SFA_COL + 4 * c, ptx::smem_desc_k_rows16(sfa_s(s) + c * kSfGroupBytes));
+#pragma unroll
+            for (int gg = 0; gg < C::G; ++gg)
+              ptx::tc_cp_32x128b_x4(sf_slot + C::SFB_COL + 4 * (c * C::G + gg),
+                                    ptx::smem_desc_k_rows16(sfb_s(s) + (c * C::G + gg) * kSfGroupBytes));
+          }
+          for (int c = 0; c < nck; ++c) {
+            const int nkb = min(4, kblocks - 4 * (c0 + c));
+            const uint64_t adesc = ptx::smem_desc_k_sw128(a_s(s) + c * C::A_PANEL);
+            const uint64_t bdesc = ptx::smem_desc_k_sw128(b_s(s) + c * C::B_PANEL);
+            const uint32_t sfa = sf_slot + C::SFA_COL + 4 * c, sfb = sf_slot + C::SFB_COL + 4 * c * C::G;
+            for (int kk = 0; kk < nkb; ++kk)
+              ptx::mma_mx_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
+                             ptx::idesc_mx_e2m1_e4m3(kBM, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
+                             (st | c | kk) != 0);
+          }
+          ptx::tc_commit(&sfree[s]);
+        }
+        if (!stop) ptx::tc_commit(&accf[b]);
+      }
+      // Every MMA issued above completes before the drain barrier fires.
+      ptx::tc_commit(drain);
+      volatile int local_abort = 0;
+      ptx::mbar_wait_bounded(drain, 0, &local_abort, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue warps
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int row = 32 * q + lane;       // weight row of the tile == TMEM lane
+    const int eg = (warp - 2) >> 2;      // epilogue warpgroup: reads c0 = (eg + EG*m) * CW
+    const int et = threadIdx.x - 64 - 128 * eg;  // 0..127 within the group
+    const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+    uint8_t* gepi = epi + eg * C::EPI_GROUP_BYTES;
+    auto group_sync = [&]() {            // the group's named barrier (128 threads)
+      if (eg == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
+      else asm volatile("bar.sync 2, 128;" ::: "memory");
+    };
+    int li = 0;
+    for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++li) {
+      const int b = li & 1;
+      const bool ready = !*s_abort && ptx::mbar_wait_bounded(&accf[b], (uint32_t)(li >> 1) & 1, s_abort,
+                                                             kWaitLimitNs);
+      // All epilogue warps take the same branch (the abort flag may be raised by another
+      // role at any time; the barrier reduction freezes one answer for all).
+      if (ptx::bar_or<3, C::EPI_THREADS>(!ready)) break;
+      ptx::tc_fence_after();
+      const int tt = i / p.n_rt, rt = i - tt * p.n_rt;
+      const Tile tl = p.tiles[tt];
+      const uint32_t acc = tmem + lane_addr + b * C::ACC_COLS;
+      if (MODE == MODE_GATE_UP) {
+        // Per read of TC tokens the gate thread of feature f (lane row f < 64) and the up
+        // thread of f (row f + 64) trade: the gate side finishes the first HT tokens, the
+        // up side the rest.  Each warp then holds one 32-feature block of h per token and
+        // splits it into E4M3 hi / lo terms for the down GEMM.
+        float* s_x = reinterpret_cast<float*>(gepi);  // [TC tokens][64 features]
+        const float L = p.limit;
+        const bool gate_side = q < 2;
+        const int f = 32 * (q & 1) + lane;           // feature within the item's 64
+        const int kb = 2 * rt + (q & 1);             // its 32-block along the down GEMM's K
+        if (eg * C::CW >= C::N2) {  // nothing for this group to read
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&acce[b]);
+        }
+        for (int c0 = eg * C::CW; c0 < C::N2; c0 += EG * C::CW) {
+          uint32_t v[32];
+          ptx::tmem_ld32(acc + c0, v);
+          ptx::tmem_wait_ld();
+          if (c0 + EG * C::CW >= C::N2) {  // last read: the accumulator goes back to the MMA issuer
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&acce[b]);
+          }
+          // (register indices stay compile-time constants: select values, not indices)
+#pragma unroll
+          for (int c = 0; c < C::HT; ++c) {
+            const int jj = gate_side ? C::HT + c : c;  // token the other side finishes
+            const float val = gate_side ? __uint_as_float(v[2 * (C::HT + c)]) + __uint_as_float(v[2 * (C::HT + c) + 1])
+                                        : __uint_as_float(v[2 * c]) + __uint_as_float(v[2 * c + 1]);
+            s_x[jj * 64 + f] = val;
+          }
+          group_sync();
+#pragma unroll
+          for (int c = 0; c < C::HT; ++c) {
+            const int jj = gate_side ? c : C::HT + c;  // token this side finishes
+            const float mine = gate_side ? __uint_as_float(v[2 * c]) + __uint_as_float(v[2 * c + 1])
+                                         : __uint_as_float(v[2 * (C::HT + c)]) +
+                                               __uint_as_float(v[2 * (C::HT + c) + 1]);
+            const float other = s_x[jj * 64 + f];
+            const float gv = fminf(gate_side ? mine : other, L);
+            const float uv = fminf(fmaxf(gate_side ? other : mine, -L), L);
+            float hv = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;   // silu(g) * u
+            uint32_t bits = __float_as_uint(hv);
+            bits = (bits + 0x7FFFu + ((bits >> 16) & 1u)) & 0xFFFF0000u;    // round to bf16
+            hv = __uint_as_float(bits);
+            const float vv[1] = {hv};
+            uint32_t hi, lo, s1, s2;
+            e4m3_split<1>(vv, hi, lo, s1, s2);
+            const int j = c0 / 2 + jj;                 // token within the tile
+            if (j < tl.rows) {
+              const int64_t prow = tl.row0 + j;
+              p.hq[(2 * prow) * p.ip + 64 * rt + f] = (uint8_t)hi;
+              p.hq[(2 * prow + 1) * p.ip + 64 * rt + f] = (uint8_t)lo;
+              if (lane == 0) {
+                uint8_t* grp = p.sfh + ((int64_t)tt * p.KCh + kb / 4) * C::G * kSfGroupBytes;
+                const int nh = 2 * j, nl = 2 * j + 1;
+                grp[(nh >> 7) * kSfGroupBytes + sf_byte_in_group(nh, kb)] = (uint8_t)s1;
+                grp[(nl >> 7) * kSfGroupBytes + sf_byte_in_group(nl, kb)] = (uint8_t)s2;
+              }
+            }
+          }
+          group_sync();  // s_x is reused by the next read
+        }
+      } else {
+        int* s_tok = reinterpret_cast<int*>(gepi + C::TC * 64 * 4);  // [TC]
+        const int m = kBM * rt + row;                                // output feature
+        const int ncol = min(kBM, p.d - kBM * rt);
+        if (eg * C::CW >= C::N2) {
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&acce[b]);
+        }
+        for (int c0 = eg * C::CW; c0 < C::N2; c0 += EG * C::CW) {
+          uint32_t v[32];
+          ptx::tmem_ld32(acc + c0, v);
+          ptx::tmem_wait_ld();
+          if (c0 + EG * C::CW >= C::N2) {
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&acce[b]);
+          }
+          const int jbase = c0 / 2;
+          const int nt = min(C::TC, tl.rows - jbase);   // tokens of this read (may be <= 0)
+#pragma unroll
+          for (int c = 0; c < C::TC; ++c) {
+            if (c < nt && m < p.d) {
+              const int64_t prow = tl.row0 + jbase + c;
+              const float o = __uint_as_float(v[2 * c]) + __uint_as_float(v[2 * c + 1]);
+              p.ys[prow * p.d + m] = o * p.w_sorted[prow];
+            }
+          }
+          if (p.fuse_combine) {
+            // Publish this read's outputs, count them per (token, column block); the writer of
+            // a token's k-th contribution adds the k outputs in slot order plus the residual.
+            __threadfence();
+            group_sync();
+            if (et < nt) {
+              const int tok = p.perm[tl.row0 + jbase + et] / p.k;
+              const int prev = atomicAdd(p.arrivals + (int64_t)tok * p.n_rt + rt, 1);
+              s_tok[et] = (prev == p.k - 1) ? tok : -1;
+            }
+            group_sync();
+            __threadfence();
+            for (int t = 0; t < nt; ++t) {
+              const int tok = s_tok[t];
+              if (tok < 0) continue;
+              for (int col = et; col < ncol; col += 128) {
+                const int64_t gc = kBM * rt + col;
+                float accv = __uint_as_float((uint32_t)p.x[(int64_t)tok * p.d + gc] << 16);
+                for (int j = 0; j < p.k; ++j) {
+                  const int srow = p.inv[(int64_t)tok * p.k + j];
+                  accv += __ldcg(p.ys + (int64_t)srow * p.d + gc);
+                }
+                uint32_t bb = __float_as_uint(accv);
+                bb = (bb + 0x7FFFu + ((bb >> 16) & 1u)) >> 16;   // round to bf16
+                p.y[(int64_t)tok * p.d + gc] = (uint16_t)bb;
+              }
+            }
+            group_sync();
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (*s_abort && threadIdx.x == 0) set_status(p.status, MOE_ERR_TIMEOUT);
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[4], gs[3];
+  cuuint32_t bx[4], es[4] = {1, 1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  return fn(m, dt, rank, const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+template <int MODE, int BN, int NP, int S, int CPS, int EG>
+int launch_one(const FwdArgs& a) {
+  using C = MxCfg<BN, NP, S, CPS, EG>;
+  const int P = a.T * a.k;
+  const int K = (MODE == MODE_GATE_UP) ? a.d : a.I;
+  const int N = (MODE == MODE_GATE_UP) ? 2 * a.I : a.d;  // weight rows per expert
+  const int64_t Kp = kpad128(K);
+  const int KC = (int)(Kp / kKChunk);
+  const uint8_t* codes = (MODE == MODE_GATE_UP) ? a.w1c : a.w2c;
+  const uint8_t* scales = (MODE == MODE_GATE_UP) ? a.w1s : a.w2s;
+  const uint8_t* act = (MODE == MODE_GATE_UP) ? a.ws.xq : a.ws.hq;
+  const int act_pitch = (MODE == MODE_GATE_UP) ? a.ws.dp : a.ws.ip;
+
+  // Weight codes [E][NT][KC][128][64] viewed as rows of 128 codes (E2M1, unpacked by the
+  // copy): one box brings NP consecutive tile blocks (NP x 128 rows), each a
+  // 128B-swizzled [128][128] panel in shared memory.
+  CUtensorMap m_w, m_act;
+  {
+    const int NT = (N + kBM - 1) / kBM;
+    const uint64_t dims[2] = {(uint64_t)kKChunk, (uint64_t)a.E * NT * KC * kBM};
+    const uint64_t str[1] = {(uint64_t)kKChunk / 2};
+    const uint32_t box[2] = {kKChunk, (uint32_t)(kBM * NP)};
+    if (!make_map(&m_w, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, codes, dims, str, box)) return -1;
+  }
+  if (MODE == MODE_GATE_UP) {
+    // Per-token rows xq [2T][dp] E4M3 (hi, lo): gathered four rows at a time, one row high.
+    const uint64_t dims[2] = {(uint64_t)act_pitch, (uint64_t)2 * a.T};
+    const uint64_t str[1] = {(uint64_t)act_pitch};
+    const uint32_t box[2] = {kKChunk, 1};
+    if (!make_map(&m_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, act, dims, str, box)) return -1;
+  } else {
+    // Sorted rows of h [2P][ip] E4M3 viewed as [chunks][2P rows][128]: one box brings NP
+    // chunks of the tile's 2*BN rows.
+    const uint64_t dims[3] = {(uint64_t)kKChunk, (uint64_t)2 * P, (uint64_t)act_pitch / kKChunk};
+    const uint64_t str[2] = {(uint64_t)act_pitch, (uint64_t)kKChunk};
+    const uint32_t box[3] = {kKChunk, (uint32_t)C::N2, (uint32_t)NP};
+    if (!make_map(&m_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, act, dims, str, box)) return -1;
+  }
+  MxParams prm;
+  prm.tiles = a.ws.tiles;
+  prm.ntiles = a.ws.ntiles;
+  prm.w_sf = scales;
+  prm.a_sf = (MODE == MODE_GATE_UP) ? a.ws.sfx : a.ws.sfh;
+  prm.NT = (N + kBM - 1) / kBM;
+  prm.K = K;
+  prm.KC = KC;
+  prm.n_rt = (MODE == MODE_GATE_UP) ? a.I / 64 : (a.d + kBM - 1) / kBM;
+  prm.status = a.ws.status;
+  prm.limit = a.limit;
+  prm.inject_timeout = (MODE == MODE_GATE_UP) ? a.inject_timeout : 0;
+  prm.hq = a.ws.hq;
+  prm.sfh = a.ws.sfh;
+  prm.ip = a.ws.ip;
+  prm.KCh = a.ws.ip / kKChunk;
+  prm.ys = a.ws.ys;
+  prm.d = a.d;
+  prm.w_sorted = a.ws.w_sorted;
+  prm.fuse_combine = (MODE == MODE_DOWN) ? a.fuse_combine : 0;
+  prm.k = a.k;
+  prm.perm = a.ws.perm;
+  prm.inv = a.ws.inv;
+  prm.x = a.x;
+  prm.y = a.y;
+  prm.arrivals = a.ws.arrivals;
+
+  auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, MODE>;
+  static std::atomic<uint64_t> attr_done{0};   // per-device "attribute set" bits
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return -1;
+    attr_done.fetch_or(bit, std::memory_order_release);
+  }
+  const int64_t max_items = (int64_t)((P + BN - 1) / BN + a.E) * prm.n_rt;
+  const int grid = (int)std::min<int64_t>(max_items, (int64_t)sm_count() * CPS);
+  ev_before(a);
+  if (launch_kernel(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, a.stream, a.pdl != 0, m_w, m_act, prm) !=
+      cudaSuccess)
+    return -1;
+  ev_after(a);
+  return 1;
+}
+
+// Pipeline shapes (compile-time; overridable with -D for tuning builds).
+// Small batches (few tokens per expert): 8-token tiles (MMA N = 16), two independent
+// pipelines (CTAs) per SM.
+#ifndef MOE_GEMV_NP
+#define MOE_GEMV_NP 1
+#endif
+#ifndef MOE_GEMV_S
+#define MOE_GEMV_S 5
+#endif
+#ifndef MOE_GEMV_CPS
+#define MOE_GEMV_CPS 2
+#endif
+#ifndef MOE_GEMV_EG
+#define MOE_GEMV_EG 1
+#endif
+// Large batches: 96-token tiles (MMA N = 192).
+#ifndef MOE_GEMM_NP
+#define MOE_GEMM_NP 1
+#endif
+#ifndef MOE_GEMM_S
+#define MOE_GEMM_S 4
+#endif
+#ifndef MOE_GEMM_CPS
+#define MOE_GEMM_CPS 1
+#endif
+#ifndef MOE_GEMM_EG
+#define MOE_GEMM_EG 2
+#endif
+constexpr int kGemvBN = 8, kGemvNP = MOE_GEMV_NP, kGemvS = MOE_GEMV_S, kGemvCPS = MOE_GEMV_CPS,
+              kGemvEG = MOE_GEMV_EG;
+constexpr int kGemmBN = 96, kGemmNP = MOE_GEMM_NP, kGemmS = MOE_GEMM_S, kGemmCPS = MOE_GEMM_CPS,
+              kGemmEG = MOE_GEMM_EG;
+static_assert(kGemvBN >= kMinTileTokens, "tile list sized for the smallest tile");
+
+}  // namespace
+
+int expert_tile_tokens(int path) { return path == MOE_PATH_GEMV ? kGemvBN : kGemmBN; }
+
+int launch_experts(const FwdArgs& a) {
+  int n1, n2;
+  if (a.ws.tile_tokens == kGemvBN) {
+    n1 = launch_one<MODE_GATE_UP, kGemvBN, kGemvNP, kGemvS, kGemvCPS, kGemvEG>(a);
+    if (n1 < 0) return -1;
+    n2 = launch_one<MODE_DOWN, kGemvBN, kGemvNP, kGemvS, kGemvCPS, kGemvEG>(a);
+  } else {
+    n1 = launch_one<MODE_GATE_UP, kGemmBN, kGemmNP, kGemmS, kGemmCPS, kGemmEG>(a);
+    if (n1 < 0) return -1;
+    n2 = launch_one<MODE_DOWN, kGemmBN, kGemmNP, kGemmS, kGemmCPS, kGemmEG>(a);
+  }
+  if (n2 < 0) return -1;
+  return n1 + n2;
+}
+
+}  // namespace moe

@@ -1,4 +1,4 @@
-// MXFP4 quantization, RMSNorm + router + top-k, grouping, gather and combine.
+// MXFP4 quantization, RMSNorm + router + top-k, grouping, tile scales and combine.
 //
 // Layer definition (web pages on gpt-oss):
 //  - RMSNorm: "From GPT-2 to gpt-oss" (新智元 translation), sec. 7: divide by the
@@ -49,9 +49,8 @@ __device__ __forceinline__ int e2m1_code_of(float a) {
   return c;
 }
 
-__global__ void quantize_kernel(const float* __restrict__ w, int64_t nblocks, int32_t N, int32_t K,
-                                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                                int32_t* status) {
+__global__ void quantize_kernel(const float* __restrict__ w, int64_t nblocks, int32_t N, int32_t K, int32_t role,
+                                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int32_t* status) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -83,10 +82,10 @@ __global__ void quantize_kernel(const float* __restrict__ w, int64_t nblocks, in
     const int hi = __shfl_down_sync(0xffffffffu, c, 1);
     const int64_t e_idx = row / N;
     const int64_t n = row - e_idx * N;
-    if ((lane & 1) == 0)
-      codes[mx_code_chunk_offset(e_idx, n, kb, N, K) + (lane >> 1)] = (uint8_t)(c | (hi << 4));
+    const int64_t srow = role == MOE_WEIGHT_GATE_UP ? gate_up_stored_row(n, N / 2) : n;
+    if ((lane & 1) == 0) codes[mx_code_offset(e_idx, srow, 32 * kb + lane, N, K)] = (uint8_t)(c | (hi << 4));
     if (lane == 0) {
-      scales[mx_scale_offset(e_idx, n, kb, N, K)] = all_finite ? (uint8_t)(s + 127) : (uint8_t)0xFF;
+      scales[mx_scale_offset(e_idx, srow, kb, N, K)] = all_finite ? (uint8_t)(s + 127) : (uint8_t)0xFF;
       if (!all_finite) set_status(status, MOE_ERR_NONFINITE);
     }
   }
@@ -151,17 +150,33 @@ __device__ __forceinline__ void warp_topk_softmax(float (&l)[NJ], int E, int k, 
 }
 
 // ----------------------------------------------------------------------------------
-// Grouping and gather for a small batch, run by the routing CTA that finished last
-// (all others have published their top-k, counts and xe rows before taking a ticket).
+// Grouping (and the tile scales) for a small batch, run by the routing CTA that finished last
+// (all others have published their top-k, counts and xq rows before taking a ticket).
 // Pairs are listed per expert in token order: one warp walks the tokens in order and
 // hands each of a token's k (distinct) experts the next free position of that expert.
 // Deterministic: positions depend on counts and token order only.
 // ----------------------------------------------------------------------------------
-__device__ void group_and_gather_block(const FwdArgs& a, int tile_tokens) {
+// Token t's activation scales (hi and lo term) into the scale-factor groups of token
+// tile `tile`, MMA columns 2*col (hi) and 2*col + 1 (lo).  One warp.  (The expert kernel
+// gathers the activation rows themselves from xq.)
+__device__ __forceinline__ void scatter_pair_scales(const FwdArgs& a, int t, int tile, int col) {
+  const int lane = threadIdx.x & 31;
+  const int dp = a.ws.dp, nb = a.d / 32, G = sf_groups_of(a.ws.tile_tokens), kc = dp / kKChunk;
+  const uint8_t* sf = a.ws.xsf + (int64_t)t * 2 * (dp / 32);
+  const int n_hi = 2 * col, n_lo = 2 * col + 1;
+  for (int b = lane; b < nb; b += 32) {
+    uint8_t* grp = a.ws.sfx + ((int64_t)tile * kc + b / 4) * G * kSfGroupBytes;
+    grp[(n_hi >> 7) * kSfGroupBytes + sf_byte_in_group(n_hi, b)] = __ldcg(sf + b);
+    grp[(n_lo >> 7) * kSfGroupBytes + sf_byte_in_group(n_lo, b)] = __ldcg(sf + dp / 32 + b);
+  }
+}
+
+__device__ void group_block(const FwdArgs& a, int tile_tokens) {
   __shared__ int s_off[257];
   __shared__ int s_cur[256];
   __shared__ int s_tb[257];
   __shared__ int s_perm_tok[kFusedGroupMaxT * 32];
+  __shared__ int s_perm_e[kFusedGroupMaxT * 32];
   const int E = a.E, k = a.k, T = a.T, P = T * k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (warp == 0) {
@@ -193,6 +208,7 @@ __device__ void group_and_gather_block(const FwdArgs& a, int tile_tokens) {
         s_tb[e] = ot;
         s_cur[e] = 0;
         a.ws.offsets[e] = oc;
+        a.ws.tile_base[e] = ot;
       }
       oc += c[j];
       ot += nt[j];
@@ -216,27 +232,38 @@ __device__ void group_and_gather_block(const FwdArgs& a, int tile_tokens) {
       a.ws.tiles[base + i] = tl;
     }
   }
+  // every pair's expert id, loaded once (staged in s_perm_tok until the walk is done)
+  for (int q = tid; q < P; q += blockDim.x) s_perm_tok[q] = __ldcg(a.ws.topk_idx + q);
+  __syncthreads();
   if (warp == 0) {
     for (int t = 0; t < T; ++t) {
       if (lane < k) {
         const int q = t * k + lane;
-        const int e = __ldcg(a.ws.topk_idx + q);
-        const int pos = s_off[e] + s_cur[e]++;
-        a.ws.perm[pos] = q;
-        a.ws.inv[q] = pos;
-        a.ws.w_sorted[pos] = __ldcg(a.ws.topk_w + q);
-        s_perm_tok[pos] = t;
+        const int e = s_perm_tok[q];
+        const int pos = s_off[e] + s_cur[e]++;   // a token's k experts are distinct
+        s_perm_e[pos] = e | (q << 9);            // (E <= 256, q < 64 * 32)
       }
       __syncwarp();
     }
   }
   __syncthreads();
-  // xs[p] = xe[token of p]: 16-byte copies over all pairs
-  const int n16 = a.d / 8;
-  for (int idx = tid; idx < P * n16; idx += blockDim.x) {
-    const int p = idx / n16, c = idx - p * n16;
-    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.ws.xe + (int64_t)s_perm_tok[p] * a.d) + c);
-    reinterpret_cast<uint4*>(a.ws.xs + (int64_t)p * a.d)[c] = v;
+  for (int pos = tid; pos < P; pos += blockDim.x) {
+    const int v = s_perm_e[pos], q = v >> 9;
+    a.ws.perm[pos] = q;
+    a.ws.inv[q] = pos;
+    a.ws.w_sorted[pos] = __ldcg(a.ws.topk_w + q);
+  }
+  __syncthreads();
+  for (int pos = tid; pos < P; pos += blockDim.x) {
+    const int v = s_perm_e[pos];
+    s_perm_tok[pos] = (v >> 9) / k;
+    s_perm_e[pos] = v & 511;
+  }
+  __syncthreads();
+  // activation scales per token tile, one warp per pair
+  for (int p = warp; p < P; p += blockDim.x >> 5) {
+    const int e = s_perm_e[p], j = p - s_off[e];
+    scatter_pair_scales(a, s_perm_tok[p], s_tb[e] + j / tile_tokens, j % tile_tokens);
   }
 }
 
@@ -282,17 +309,28 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
 #pragma unroll
   for (int w = 0; w < kTokWarps; ++w) tot += s_red[w];
   const float r = 1.0f / sqrtf(tot / (float)d + a.eps);
-  bool range_bad = false;
   for (int i = tid * 2; i < d; i += 2 * kTokThreads) {
-    const float v0 = s_xn[i] * r * a.norm_w[i], v1 = s_xn[i + 1] * r * a.norm_w[i + 1];
-    s_xn[i] = v0;
-    s_xn[i + 1] = v1;
-    const float b0 = bf16_to_f32(f32_to_bf16_rne(v0)), b1 = bf16_to_f32(f32_to_bf16_rne(v1));
-    range_bad |= fabsf(b0) > 65504.f || fabsf(b1) > 65504.f;
-    *reinterpret_cast<__half2*>(a.ws.xe + t * d + i) = __floats2half2_rn(b0, b1);
+    s_xn[i] = s_xn[i] * r * a.norm_w[i];
+    s_xn[i + 1] = s_xn[i + 1] * r * a.norm_w[i + 1];
   }
-  if (range_bad) set_status(a.ws.status, MOE_ERR_RANGE);
   __syncthreads();
+  {
+    // xe = bf16(xn) as E4M3 hi / lo terms: warp w splits 32-blocks w, w + 32, ...
+    const int dp = a.ws.dp;
+    uint8_t* xq = a.ws.xq + t * 2 * dp;
+    uint8_t* sf = a.ws.xsf + t * 2 * (dp / 32);
+    for (int b = warp; b < d / 32; b += kTokWarps) {
+      const float v[1] = {bf16_to_f32(f32_to_bf16_rne(s_xn[32 * b + lane]))};
+      uint32_t hi, lo, s1, s2;
+      e4m3_split<1>(v, hi, lo, s1, s2);
+      xq[32 * b + lane] = (uint8_t)hi;
+      xq[dp + 32 * b + lane] = (uint8_t)lo;
+      if (lane == 0) {
+        sf[b] = (uint8_t)s1;
+        sf[dp / 32 + b] = (uint8_t)s2;
+      }
+    }
+  }
   const int n4 = d / 4;
   for (int e = warp; e < E; e += kTokWarps) {
     const float4* wr = reinterpret_cast<const float4*>(a.router_w + (int64_t)e * d);
@@ -329,7 +367,7 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
     warp_topk_softmax<NJ>(l, E, a.k, t, a);
   }
   if (a.fuse_group) {
-    // Publish this token (top-k, counts, xe row), then take a ticket; the last CTA groups.
+    // Publish this token (top-k, counts, xq rows), then take a ticket; the last CTA groups.
     __shared__ int s_last;
     __threadfence();
     __syncthreads();
@@ -337,14 +375,14 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
     __syncthreads();
     if (s_last) {
       __threadfence();
-      group_and_gather_block(a, a.fuse_group);
+      group_block(a, a.fuse_group);
     }
   }
 }
 
 // ----------------------------------------------------------------------------------
 // Fused RMSNorm + router GEMV + top-k + softmax, 32 tokens per CTA, 256 threads.
-// Outputs: xe (f16 copy of bf16(xn)), topk_idx, topk_w, expert histogram.
+// Outputs: xq / xsf (E4M3 terms of bf16(xn)), topk_idx, topk_w, expert histogram.
 // ----------------------------------------------------------------------------------
 constexpr int RT = 32;   // tokens per CTA (tiled kernel)
 constexpr int kTokenKernelMaxT = 1024;  // up to this many tokens: one CTA per token
@@ -393,7 +431,6 @@ __global__ void __launch_bounds__(256) route_kernel(FwdArgs a) {
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
-  bool range_bad = false;
 
   // Register prefetch of the next d-chunk overlaps its global loads with the FMAs.
   constexpr int XQ = RT * (RK / 2) / 256;   // bf16 pairs of x per thread per chunk
@@ -421,13 +458,23 @@ __global__ void __launch_bounds__(256) route_kernel(FwdArgs a) {
       const int q = tid + 256 * u;
       const int tt = q / (RK / 2), c2 = (q % (RK / 2)) * 2;
       float v0 = 0.f, v1 = 0.f;
-      if (tt < nt) {
+      if (tt < nt) {  // uniform per warp: a warp covers one token's 64 values
         const float r = s_r[tt];
         v0 = __uint_as_float(px[u] << 16) * r * a.norm_w[k0 + c2];
         v1 = __uint_as_float(px[u] & 0xFFFF0000u) * r * a.norm_w[k0 + c2 + 1];
-        const float b0 = bf16_to_f32(f32_to_bf16_rne(v0)), b1 = bf16_to_f32(f32_to_bf16_rne(v1));
-        range_bad |= fabsf(b0) > 65504.f || fabsf(b1) > 65504.f;
-        *reinterpret_cast<__half2*>(a.ws.xe + (int64_t)(t0 + tt) * d + k0 + c2) = __floats2half2_rn(b0, b1);
+        const float v[2] = {bf16_to_f32(f32_to_bf16_rne(v0)), bf16_to_f32(f32_to_bf16_rne(v1))};
+        uint32_t hi, lo, s1, s2;
+        e4m3_split<2>(v, hi, lo, s1, s2);   // lanes 0-15: block k0/32, lanes 16-31: the next
+        const int dp = a.ws.dp;
+        uint8_t* xq = a.ws.xq + (int64_t)(t0 + tt) * 2 * dp;
+        *reinterpret_cast<uint16_t*>(xq + k0 + c2) = (uint16_t)hi;
+        *reinterpret_cast<uint16_t*>(xq + dp + k0 + c2) = (uint16_t)lo;
+        if ((lane & 15) == 0) {
+          uint8_t* sf = a.ws.xsf + (int64_t)(t0 + tt) * 2 * (dp / 32);
+          const int b = (k0 + c2) / 32;
+          sf[b] = (uint8_t)s1;
+          sf[dp / 32 + b] = (uint8_t)s2;
+        }
       }
       s_x[tt * (RK + 1) + c2] = v0;
       s_x[tt * (RK + 1) + c2 + 1] = v1;
@@ -454,7 +501,6 @@ __global__ void __launch_bounds__(256) route_kernel(FwdArgs a) {
     }
     __syncthreads();
   }
-  if (range_bad) set_status(a.ws.status, MOE_ERR_RANGE);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -507,6 +553,7 @@ __global__ void __launch_bounds__(1024) group_kernel(FwdArgs a, int tile_tokens)
   a.ws.offsets[e] = off;
   if (e == E - 1) a.ws.offsets[E] = off + cnt;
   if (e == 0) a.ws.ntiles[0] = s_total_tiles;
+  if (tid == 0) a.ws.tile_base[e] = s_tile_base;
   for (int i = tid; i * tile_tokens < cnt; i += blockDim.x) {
     Tile tl;
     tl.e = e;
@@ -548,18 +595,17 @@ __global__ void __launch_bounds__(1024) group_kernel(FwdArgs a, int tile_tokens)
   }
 }
 
-// xs[p] = xe[perm[p] / k]: 16-byte copies, one warp per row.
-__global__ void gather_kernel(FwdArgs a) {
+// Activation scales of every pair into its token tile's scale-factor groups.  One warp
+// per pair.
+__global__ void tile_scales_kernel(FwdArgs a) {
   pdl_trigger();
   pdl_wait();
-  const int P = a.T * a.k;
-  const int lane = threadIdx.x & 31;
-  const int n16 = a.d / 8;
+  const int P = a.T * a.k, bt = a.ws.tile_tokens;
   for (int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x >> 5)) {
-    const int t = a.ws.perm[p] / a.k;
-    const uint4* src = reinterpret_cast<const uint4*>(a.ws.xe + (int64_t)t * a.d);
-    uint4* dst = reinterpret_cast<uint4*>(a.ws.xs + (int64_t)p * a.d);
-    for (int i = lane; i < n16; i += 32) dst[i] = src[i];
+    const int q = a.ws.perm[p];
+    const int e = a.ws.topk_idx[q];
+    const int j = p - a.ws.offsets[e];
+    scatter_pair_scales(a, q / a.k, a.ws.tile_base[e] + j / bt, j % bt);
   }
 }
 
@@ -625,17 +671,24 @@ int launch_route_nj(const FwdArgs& a) {
 
 }  // namespace
 
-int launch_quantize(const float* w, int64_t rows, int32_t N, int32_t K, int32_t E, uint8_t* codes,
+int launch_quantize(const float* w, int32_t E, int32_t N, int32_t K, int32_t role, uint8_t* codes,
                     uint8_t* scales, int32_t* status, cudaStream_t st) {
-  (void)E;
-  const int64_t nblocks = rows * (K / 32);
+  const int64_t Kp = kpad128(K);
+  // padding (rows past N, k past K): codes 0, scale bytes 127 (2^0)
+  const size_t blocks = (size_t)E * ((N + 127) / 128) * (Kp / kKChunk);
+  if (Kp != K || N % 128) {
+    if (cudaMemsetAsync(codes, 0, blocks * kCodeBlockBytes, st) != cudaSuccess) return -1;
+    if (cudaMemsetAsync(scales, 127, blocks * kSfGroupBytes, st) != cudaSuccess) return -1;
+  }
+  const int64_t nblocks = (int64_t)E * N * (K / 32);
   const int64_t want = (nblocks + 7) / 8;
   const int grid = (int)std::min<int64_t>(want, 148 * 64);
-  quantize_kernel<<<grid, 256, 0, st>>>(w, nblocks, N, K, codes, scales, status);
+  quantize_kernel<<<grid, 256, 0, st>>>(w, nblocks, N, K, role, codes, scales, status);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 
-int launch_route(const FwdArgs& a_in, int tile_tokens) {
+int launch_route(const FwdArgs& a_in) {
+  const int tile_tokens = a_in.ws.tile_tokens;
   int n = 0;
   FwdArgs a = a_in;
   // fuse_group carries the token-tile size into the routing kernel (0 = separate kernels)
@@ -657,8 +710,8 @@ int launch_route(const FwdArgs& a_in, int tile_tokens) {
   ++n;
   const int P = a.T * a.k;
   ev_before(a);
-  if (launch_kernel(gather_kernel, dim3(std::min((P + 7) / 8, 148 * 16)), dim3(256), 0, a.stream, a.pdl != 0, a) !=
-      cudaSuccess)
+  if (launch_kernel(tile_scales_kernel, dim3(std::min((P + 7) / 8, 148 * 16)), dim3(256), 0, a.stream, a.pdl != 0,
+                    a) != cudaSuccess)
     return -1;
   ev_after(a);
   ++n;

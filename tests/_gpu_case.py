@@ -18,19 +18,48 @@ import synth
 from _inputs import routed_inputs
 
 
-def blocks_to_rowmajor(codes: np.ndarray, scales: np.ndarray, N: int, K: int):
-    """Library MXFP4 block layout -> the oracle's row-major layout.
+# Token tile of each path (moe_mxfp4.h: "8-token tiles", "96-token tiles").
+TILE_TOKENS = {"gemv": 8, "gemm": 96}
 
-    codes [E, N/64, K/64, 64, 32] -> [E, N, K/2]; scales [E, N/64, K/64, 2, 64] -> [E, N, K/32].
-    In a block, row r's logical 16-byte chunk c is stored at chunk c ^ ((r >> 2) & 1).
+
+def decode_e4m3(b: np.ndarray) -> np.ndarray:
+    """E4M3 bytes -> float64 from the format's fields: sign bit 7, exponent bits 6..3
+    (bias 7), mantissa bits 2..0; exponent 0 is subnormal (m/8 * 2^-6); 0x7F / 0xFF NaN."""
+    b = b.astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 15
+    m = (b & 7).astype(np.float64)
+    v = np.where(e == 0, m / 8 * 2.0 ** -6, (1 + m / 8) * np.exp2(e.astype(np.float64) - 7))
+    v = np.where((e == 15) & (m == 7), np.nan, v)
+    return sign * v
+
+
+def stored_row_of(N: int, role: str) -> np.ndarray:
+    """Stored row of each logical row n: gate_up tensors pair 64 gate rows with the 64
+    matching up rows in every 128-row tile; other tensors keep their order."""
+    n = np.arange(N)
+    if role != "gate_up":
+        return n
+    I = N // 2
+    part = (n >= I).astype(np.int64)
+    f = n - part * I
+    return (f // 64) * 128 + part * 64 + f % 64
+
+
+def stored_to_rowmajor(codes: np.ndarray, scales: np.ndarray, N: int, K: int, role: str):
+    """Library MXFP4 storage -> the oracle's row-major layout.
+
+    codes [E, NT, KC, 128, 64] -> [E, N, K/2] (row r's bytes for k = 128c .. 128c+127 are
+    block [r//128, c], row r%128); scales [E, NT, KC, 512] -> [E, N, K/32], where the scale of
+    (stored row r, block b) is byte (r%32)*16 + ((r%128)//32)*4 + b%4 of group [r//128, b//4].
     """
-    E = codes.shape[0]
-    c = codes.reshape(E, N // 64, K // 64, 64, 2, 16)
-    r = np.arange(64)
-    phys = np.stack([(0 ^ ((r >> 2) & 1)), (1 ^ ((r >> 2) & 1))], axis=1)  # [64, 2] physical chunk of logical c
-    logical = np.take_along_axis(c, phys[None, None, None, :, :, None], axis=4)
-    rows = logical.reshape(E, N // 64, K // 64, 64, 32).transpose(0, 1, 3, 2, 4).reshape(E, N, K // 2)
-    sc = scales.reshape(E, N // 64, K // 64, 2, 64).transpose(0, 1, 4, 2, 3).reshape(E, N, K // 32)
+    E, KC = codes.shape[0], codes.shape[2]
+    sr = stored_row_of(N, role)
+    # (advanced indices split by a slice put the row axis first: [N, E, KC, 64])
+    rows = codes[:, sr // 128, :, sr % 128, :].transpose(1, 0, 2, 3).reshape(E, N, KC * 64)[:, :, : K // 2]
+    b = np.arange(K // 32)
+    byte = ((sr % 32) * 16 + ((sr % 128) // 32) * 4)[:, None] + (b % 4)[None, :]
+    sc = scales[:, (sr // 128)[:, None], (b // 4)[None, :], byte]
     return np.ascontiguousarray(rows), np.ascontiguousarray(sc)
 
 
@@ -60,12 +89,12 @@ def weights(seed: int, E: int, d: int, I: int, w1_mul: float):
     mismatches = 0
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     for e in range(E):
-        for w, gc, gs, oc, os_ in ((synth.w1_expert(cfg, e), g1c, g1s, o1c, o1s),
-                                   (synth.w2_expert(cfg, e), g2c, g2s, o2c, o2s)):
+        for w, gc, gs, oc, os_, role in ((synth.w1_expert(cfg, e), g1c, g1s, o1c, o1s, "gate_up"),
+                                         (synth.w2_expert(cfg, e), g2c, g2s, o2c, o2s, "down")):
             wt = torch.from_numpy(w).cuda()
-            moe.moe_mxfp4_quantize(wt, gc[e:e + 1], gs[e:e + 1], status_word=status)
+            moe.moe_mxfp4_quantize(wt, gc[e:e + 1], gs[e:e + 1], role=role, status_word=status)
             oc[e], os_[e] = oracle.quantize(w)
-            rc, rs = blocks_to_rowmajor(gc[e:e + 1].cpu().numpy(), gs[e:e + 1].cpu().numpy(), *w.shape)
+            rc, rs = stored_to_rowmajor(gc[e:e + 1].cpu().numpy(), gs[e:e + 1].cpu().numpy(), *w.shape, role)
             mismatches += int(np.count_nonzero(rc[0] != oc[e]))
             mismatches += int(np.count_nonzero(rs[0] != os_[e]))
     torch.cuda.synchronize()

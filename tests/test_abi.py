@@ -23,14 +23,22 @@ def test_every_header_symbol_is_exported(L):
 
 
 def test_storage_sizes(L):
-    assert moe.moe_mxfp4_codes_bytes(1, 5760, 2880) == 8_294_400
-    assert moe.moe_mxfp4_scales_bytes(1, 5760, 2880) == 518_400
-    assert moe.moe_mxfp4_codes_bytes(32, 5760, 2880) == 32 * 8_294_400
+    # K a multiple of 128 and N of 128: exactly 4.25 bits per parameter
+    assert moe.moe_mxfp4_codes_bytes(1, 256, 4096) == 256 * 4096 // 2
+    assert moe.moe_mxfp4_scales_bytes(1, 256, 4096) == 256 * 4096 // 32
+    # gpt-oss W1 [2I=5760][d=2880]: rows padded to 2944 codes, scale groups of 128 rows x 128
+    assert moe.moe_mxfp4_codes_bytes(1, 5760, 2880) == 45 * 23 * 8192
+    assert moe.moe_mxfp4_scales_bytes(1, 5760, 2880) == 45 * 23 * 512
+    # W2 [d=2880][I=2880]: 22.5 row tiles -> 23
+    assert moe.moe_mxfp4_codes_bytes(1, 2880, 2880) == 23 * 23 * 8192
+    assert moe.moe_mxfp4_scales_bytes(1, 2880, 2880) == 23 * 23 * 512
+    assert moe.moe_mxfp4_codes_bytes(32, 5760, 2880) == 32 * 45 * 23 * 8192
     assert moe.moe_mxfp4_codes_bytes(0, 5760, 2880) == 0
+    assert moe.mxfp4_shapes(2, 2880, 2880) == ((2, 23, 23, 128, 64), (2, 23, 23, 512))
 
 
 def test_status_strings(L):
-    for s in range(9):
+    for s in (0, 1, 2, 3, 4, 5, 6, 8):
         assert moe.status_string(s) and moe.status_string(s) != "unknown status"
     assert moe.status_string(99) == "unknown status"
 
@@ -47,7 +55,7 @@ def test_workspace_size_and_layout(L):
     assert moe.moe_workspace_bytes(moe.make_dims(2880, 2880, 32, 4, block=16), 16) == 0
 
 
-def _call_forward(L, dims, T, ptr=16, ws_bytes=1 << 40):
+def _call_forward(L, dims, T, ptr=256, ws_bytes=1 << 40):
     p = ctypes.c_void_p(ptr)
     return L.moe_forward(ctypes.byref(dims), T, p, p, p, p, p, p, p, p, ctypes.c_void_p(ptr + 4096), None, None,
                          None, p, ws_bytes, None)
@@ -67,9 +75,13 @@ def test_argument_checks_before_device(L):
     assert _call_forward(L, ok, 4, ptr=0) == moe.MOE_ERR_INVALID_ARG          # null
     assert _call_forward(L, ok, 4096, ws_bytes=1024) == moe.MOE_ERR_WORKSPACE
     assert L.moe_forward(None, 4, *([None] * 13), 0, None) == moe.MOE_ERR_INVALID_ARG
-    p = ctypes.c_void_p(16)
-    assert L.moe_mxfp4_quantize(p, 1, 64, 48, p, p, None, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
-    assert L.moe_mxfp4_quantize(None, 1, 64, 64, p, p, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert _call_forward(L, ok, 4, ptr=16) == moe.MOE_ERR_INVALID_ARG         # codes need 32-byte alignment
+    p = ctypes.c_void_p(256)
+    assert L.moe_mxfp4_quantize(p, 1, 64, 48, 0, p, p, None, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_mxfp4_quantize(None, 1, 64, 64, 0, p, p, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_mxfp4_quantize(p, 1, 64, 64, 7, p, p, None, None) == moe.MOE_ERR_INVALID_ARG     # bad role
+    assert L.moe_mxfp4_quantize(p, 1, 64, 64, 1, p, p, None, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE  # I = 32
+    assert L.moe_mxfp4_quantize(p, 1, 128, 64, 1, ctypes.c_void_p(272), p, None, None) == moe.MOE_ERR_INVALID_ARG
 
 
 def test_no_device_is_an_error_not_a_fallback(L):

@@ -11,8 +11,8 @@ import torch
 import mxfp4_expert_gemm_b200 as moe
 import oracle
 import synth
-from _gpu_case import (assert_parity, bf16_dev, bf16_host, blocks_to_rowmajor, case, oracle_rows, parity_stats,
-                       run_gpu, weights)
+from _gpu_case import (TILE_TOKENS, assert_parity, bf16_dev, bf16_host, case, decode_e4m3, oracle_rows, parity_stats, run_gpu,
+                       stored_row_of, stored_to_rowmajor, weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +27,7 @@ SMALL = {
     "mid_ragged": synth.MoEConfig("mid_ragged", T=200, d=2880, I=2880, E=8, k=4),
     "clamp": synth.MoEConfig("clamp", T=32, d=2880, I=2880, E=4, k=2, w1_mul=8.0),
 }
-PATHS = ["simt", "gemv", "gemm"]
+PATHS = ["gemv", "gemm"]
 
 
 def _pairs(idx: np.ndarray, perm: np.ndarray, k: int):
@@ -60,11 +60,34 @@ def test_quantize_special_values_bit_exact():
     w = np.stack(rows).astype(np.float32)
     w = np.concatenate([w, (rng.standard_normal((58, 32)) * 0.02).astype(np.float32)])  # 64 rows
     w = np.tile(w, (1, 2))  # K = 64
-    codes, scales = moe.moe_mxfp4_quantize(torch.from_numpy(w).cuda())
     oc, os_ = oracle.quantize(w)
-    rc, rs = blocks_to_rowmajor(codes.cpu().numpy(), scales.cpu().numpy(), *w.shape)
+    codes, scales = moe.moe_mxfp4_quantize(torch.from_numpy(w).cuda())
+    rc, rs = stored_to_rowmajor(codes.cpu().numpy(), scales.cpu().numpy(), *w.shape, "plain")
     np.testing.assert_array_equal(rc[0], oc)
     np.testing.assert_array_equal(rs[0], os_)
+    # the same rows as a gate_up tensor [2I = 128][64]: only the stored row order changes
+    w2 = np.concatenate([w, w[::-1]])
+    oc2, os2 = oracle.quantize(w2)
+    codes, scales = moe.moe_mxfp4_quantize(torch.from_numpy(w2).cuda(), role="gate_up")
+    rc, rs = stored_to_rowmajor(codes.cpu().numpy(), scales.cpu().numpy(), *w2.shape, "gate_up")
+    np.testing.assert_array_equal(rc[0], oc2)
+    np.testing.assert_array_equal(rs[0], os2)
+
+
+def test_quantize_padding():
+    """N = K = 192 pads to 2 x 2 tiles of 128 x 128: padding codes 0, padding scale bytes 127."""
+    w = (np.random.default_rng(3).standard_normal((2, 192, 192)) * 0.02).astype(np.float32)
+    codes, scales = moe.moe_mxfp4_quantize(torch.from_numpy(w).cuda())
+    c, sc = codes.cpu().numpy(), scales.cpu().numpy()
+    assert c.shape == (2, 2, 2, 128, 64) and sc.shape == (2, 2, 2, 512)
+    assert np.all(c[:, 1, :, 64:, :] == 0)          # rows 192..255
+    assert np.all(c[:, :, 1, :, 32:] == 0)          # k 192..255
+    sr = stored_row_of(192, "plain")
+    mask = np.zeros(sc.shape, bool)
+    for b in range(6):
+        byte = (sr % 32) * 16 + ((sr % 128) // 32) * 4 + b % 4
+        mask[:, sr // 128, b // 4, byte] = True
+    assert np.all(sc[~mask] == 127)
 
 
 def test_quantize_non_finite_is_flagged():
@@ -74,7 +97,7 @@ def test_quantize_non_finite_is_flagged():
     codes, scales = moe.moe_mxfp4_quantize(torch.from_numpy(w).cuda(), status_word=status)
     torch.cuda.synchronize()
     assert int(status.item()) == moe.MOE_ERR_NONFINITE
-    _, rs = blocks_to_rowmajor(codes.cpu().numpy(), scales.cpu().numpy(), *w.shape)
+    _, rs = stored_to_rowmajor(codes.cpu().numpy(), scales.cpu().numpy(), *w.shape, "plain")
     assert rs[0, 3, 1] == 0xFF and rs[0, 3, 0] != 0xFF and rs[0, 2, 1] != 0xFF
 
 
@@ -126,15 +149,46 @@ def test_forward_parity(name, path):
     np.testing.assert_array_equal(np.sort(g["routing"]["topk_idx"].cpu().numpy(), 1), np.sort(ref["idx"], 1))
 
 
-@pytest.mark.parametrize("path", ["gemv", "gemm", "simt"])
+def _h_from_workspace(g, cfg):
+    """h [P, I] (sorted pairs) rebuilt from the workspace's E4M3 hi / lo rows and the
+    token tiles' scale-factor groups."""
+    dims, ws, T = g["dims"], g["ws"], cfg.T
+    P = T * cfg.k
+    Ip = moe.kpad128(cfg.I)
+    bt = TILE_TOKENS[moe.resolved_path(dims, T)]
+    G = (2 * bt + 127) // 128
+    view = lambda f, dt, sh: moe.workspace_view(ws, dims, T, f, dt, sh).cpu().numpy()
+    hq = view("hq", torch.uint8, (2 * P, Ip))[:, :cfg.I]
+    offsets = view("offsets", torch.int32, (cfg.E + 1,))
+    tbase = view("tile_base", torch.int32, (cfg.E,))
+    n_tiles = (P + bt - 1) // bt + cfg.E
+    sfh = view("sfh", torch.uint8, (n_tiles, Ip // 128, G, 512))
+    h = np.empty((P, cfg.I))
+    b = np.arange(cfg.I // 32)
+    for p in range(P):
+        e = int(np.searchsorted(offsets, p, side="right") - 1)
+        j = p - offsets[e]
+        tile, col = tbase[e] + j // bt, j % bt
+        sc = []
+        for n in (2 * col, 2 * col + 1):
+            byte = (n % 32) * 16 + ((n % 128) // 32) * 4 + b % 4
+            sc.append(sfh[tile, b // 4, n // 128, byte].astype(np.float64) - 127)
+        s_hi = np.repeat(np.exp2(sc[0]), 32)
+        s_lo = np.repeat(np.exp2(sc[1]), 32)
+        h[p] = decode_e4m3(hq[2 * p]) * s_hi + decode_e4m3(hq[2 * p + 1]) * s_lo
+    return h
+
+
+@pytest.mark.parametrize("path", PATHS)
 def test_swiglu_output_h_matches_oracle(path):
-    """The gate_up stage alone: h (bf16 values) in the workspace vs the oracle's h."""
+    """The gate_up stage alone: h rebuilt from its E4M3 hi / lo terms vs the oracle's h;
+    the two terms carry bf16 values exactly (up to the block's dynamic range)."""
     c = case(SMALL["mid_ragged"])
     cfg = c["cfg"]
     g = run_gpu(c, path)
     assert g["status"] == moe.MOE_OK
     P = cfg.T * cfg.k
-    h = moe.workspace_view(g["ws"], g["dims"], cfg.T, "h", torch.float16, (P, cfg.I)).float().cpu().numpy()
+    h = _h_from_workspace(g, cfg)
     inv = moe.workspace_view(g["ws"], g["dims"], cfg.T, "inv", torch.int32, (P,)).cpu().numpy()
     idx = g["routing"]["topk_idx"].cpu().numpy()
     ref = oracle_rows(c, want_h=True)
@@ -147,6 +201,11 @@ def test_swiglu_output_h_matches_oracle(path):
             num += float(diff @ diff)
             den += float(href[t, so] @ href[t, so])
     assert np.sqrt(num / den) <= 1e-2
+    # hi + lo reproduce bf16 values: round-tripping through bf16 changes (almost) nothing
+    h32 = h.astype(np.float32)
+    u = h32.view(np.uint32).astype(np.uint64)
+    hb = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32).view(np.float32)
+    assert np.mean(hb == h32) >= 0.999, np.mean(hb == h32)
 
 
 @pytest.mark.parametrize("name,path,n_sample", [
@@ -179,7 +238,7 @@ def test_full_size_sampled(name, path, n_sample):
 def test_T_zero_and_one():
     c = case(SMALL["tiny"])
     cfg = c["cfg"]
-    for path in ("gemv", "gemm", "simt"):
+    for path in PATHS:
         dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path=path)
         ws = moe.new_workspace(dims, 1)
         y = moe.moe_forward(dims, c["x_dev"][:1], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws)
@@ -199,16 +258,35 @@ def test_deterministic():
         np.testing.assert_array_equal(a, b)
 
 
-def test_scale_out_of_f16_range_is_reported():
+def _set_scale(scales_gpu, scales_or, e, n, b, value, N, K, role):
+    """Set the E8M0 scale of (expert e, logical row n, block b) on both sides."""
+    sr = int(stored_row_of(N, role)[n])
+    byte = (sr % 32) * 16 + ((sr % 128) // 32) * 4 + b % 4
+    scales_gpu[e, sr // 128, b // 4, byte] = value
+    scales_or[e, n, b] = value
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_extreme_scales_stay_exact(path):
+    """The tensor cores apply E8M0 scales exactly over their whole range: blocks scaled by
+    2^+-40 (far outside f16) still match the oracle."""
     c = case(SMALL["tiny"])
     cfg = c["cfg"]
     g1c, g1s, g2c, g2s = (t.clone() for t in c["W"]["gpu"])
-    g1s.view(-1)[0] = 127 + 20   # a scale of 2^20: E2M1 * 2^20 is not exact in f16
-    for path, expect in (("gemm", moe.MOE_ERR_RANGE), ("gemv", moe.MOE_ERR_RANGE), ("simt", moe.MOE_OK)):
-        dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path=path)
-        ws = moe.new_workspace(dims, cfg.T)
-        moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], g1c, g1s, g2c, g2s, ws)
-        assert moe.moe_device_status(ws) == expect, path
+    o1c, o1s, o2c, o2s = (a.copy() for a in c["W"]["oracle"])
+    rng = np.random.default_rng(11)
+    for _ in range(6):
+        e, n, b = int(rng.integers(cfg.E)), int(rng.integers(2 * cfg.I)), int(rng.integers(cfg.d // 32))
+        _set_scale(g1s, o1s, e, n, b, int(o1s[e, n, b]) + 40, 2 * cfg.I, cfg.d, "gate_up")  # g / u saturate
+        e, n, b = int(rng.integers(cfg.E)), int(rng.integers(cfg.d)), int(rng.integers(cfg.I // 32))
+        _set_scale(g2s, o2s, e, n, b, int(o2s[e, n, b]) - 40, cfg.d, cfg.I, "down")
+    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path=path)
+    ws = moe.new_workspace(dims, cfg.T)
+    y = moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], g1c, g1s, g2c, g2s, ws)
+    assert moe.moe_device_status(ws) == moe.MOE_OK
+    ref = oracle.moe_forward(c["x"], c["gamma"], c["rw"], c["rb"], o1c, o1s, o2c, o2s, I=cfg.I, k=cfg.k,
+                             eps=cfg.rms_eps, limit=cfg.swiglu_limit)
+    assert_parity(parity_stats(bf16_host(y), ref["y"], c["x"]), path)
 
 
 def test_non_finite_input_is_reported():
@@ -227,8 +305,7 @@ def test_launch_count_reported():
     c = case(SMALL["tiny"])
     cfg = c["cfg"]
     for path, n in (("gemm", 6),   # route, group, gather, gate_up, down, combine
-                    ("gemv", 3),   # route (+ grouping + gather), gate_up, down (+ combine)
-                    ("simt", 6)):
+                    ("gemv", 3)):  # route (+ grouping + gather), gate_up, down (+ combine)
         dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path=path)
         ws = moe.new_workspace(dims, cfg.T)
         moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws)
