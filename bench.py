@@ -42,7 +42,7 @@ WORKLOAD_TEXT = {
     "moe_120b": "gpt-oss-120b MoE layer: T=8192, d=2880, I=2880, E=128, top-4, MXFP4 experts",
     "skew_120b": "skewed routing: T=16384, d=I=2880, E=128, top-4, Zipf(1.2) router bias, MXFP4 experts",
 }
-KERNELS = ["route", "group", "tile_scales", "gate_up", "down", "combine"]
+KERNELS = ["route", "group", "pack", "gate_up", "down", "combine"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_DENSE_NOMINAL_TFLOPS = 9000.0
 

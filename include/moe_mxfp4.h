@@ -169,9 +169,9 @@ moe_status moe_forward(const moe_dims* dims, int32_t T, const uint16_t* x, const
  * the array runs out.  Recording adds no synchronization; when `stream` is being captured
  * into a CUDA graph the events are recorded as external event nodes of the graph, so
  * that every replay records them.  The kernels of a call are, in order: route
- * (RMSNorm + router + top-k + E4M3 split of xe), group, tile scales, gate_up, down,
- * combine; on the GEMV path with T <= 64, route (which then also groups and writes the
- * tile scales), gate_up and down (which then also combines).
+ * (RMSNorm + router + top-k + E4M3 split of xe), group, pack (the token tiles' packed
+ * activation blocks), gate_up, down, combine; on the GEMV path with T <= 64, route (which
+ * then also groups and packs), gate_up and down (which then also combines).
  * Errors: as moe_forward; MOE_ERR_INVALID_ARG if n_events < 0 or events is NULL with
  * n_events > 0. */
 moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
@@ -192,12 +192,15 @@ int32_t moe_resolve_path(const moe_dims* dims, int32_t T);
  * inv, w_sorted,
  * xq  [T][2][dp] E4M3 (hi and lo terms of xe = bf16(xn) per token; dp = d rounded up to
  *     a multiple of 128), xsf [T][2][dp/32] E8M0 (their scales),
- * sfx (the scales of each token tile's columns, in the tensor cores' scale-factor layout),
- * hq  [2*T*k][Ip] E4M3 (hi / lo terms of the SwiGLU output h, sorted order), sfh,
- * ys  [T*k][d] fp32 (weighted expert outputs, sorted order);
+ * bpx / bph: packed activation blocks of xe and of the SwiGLU output h, per token tile
+ *     and 128-chunk: the tile's 2 * BN E4M3 rows (hi / lo term of each token) in the
+ *     tensor cores' 128-byte-swizzled order, then their scales (BN = 8 on the GEMV path,
+ *     96 on the GEMM path),
+ * ys  [S][T*k][d] fp32 (weighted expert outputs, sorted order; S = 2 partial sums on the
+ *     GEMV path, whose down GEMM splits its reduction axis in two, else 1);
  * offsets[MOE_WS_FIELDS-1] = total bytes.  Errors: MOE_ERR_INVALID_ARG,
  * MOE_ERR_UNSUPPORTED_SHAPE. */
-#define MOE_WS_FIELDS 18
+#define MOE_WS_FIELDS 17
 moe_status moe_workspace_layout(const moe_dims* dims, int32_t T, size_t* offsets);
 
 /* Synchronize `stream`, then read and clear the device status word of workspace `ws`
@@ -220,7 +223,7 @@ int32_t moe_last_launch_count(void);
  * implicit synchronization once it is running -- use it instead of moe_forward.
  * Scratch: a fixed 16 MiB array in the library's own device memory, present on every GPU
  * that loads the library until the process exits.  T whose moe_workspace_bytes() exceed
- * 16 MiB is rejected with MOE_ERR_WORKSPACE (at d = I = 2880, E = 32, top-4: up to 150
+ * 16 MiB is rejected with MOE_ERR_WORKSPACE (at d = I = 2880, E = 32, top-4: up to 119
  * tokens).
  * The first call on a device looks up the array's device address for that device
  * (cudaGetSymbolAddress); make that first call before any stream capture.

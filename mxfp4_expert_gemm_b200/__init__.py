@@ -234,7 +234,7 @@ def moe_forward(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scal
 
 
 WS_FIELDS = ("status", "counts", "offsets", "ntiles", "tile_base", "tiles", "topk_idx", "topk_w", "perm", "inv",
-             "w_sorted", "xq", "xsf", "sfx", "hq", "sfh", "ys", "total")
+             "w_sorted", "xq", "xsf", "bpx", "bph", "ys", "total")
 
 
 def moe_workspace_layout(dims: moe_dims, T: int) -> dict:

@@ -55,7 +55,8 @@ int resolve_path(const moe_dims& dm, int32_t T) {
 int tile_tokens_of(int path) { return moe::expert_tile_tokens(path); }
 
 moe::WsLayout layout_for(const moe_dims& dm, int32_t T) {
-  return moe::ws_layout(dm, T, tile_tokens_of(resolve_path(dm, T)));
+  const int path = resolve_path(dm, T);
+  return moe::ws_layout(dm, T, tile_tokens_of(path), moe::expert_down_split(path));
 }
 
 moe_status prepare(const moe_dims* dm, int32_t T, const uint16_t* x, const float* norm_w, const float* router_w,
@@ -232,7 +233,7 @@ moe_status moe_workspace_layout(const moe_dims* dims, int32_t T, size_t* offsets
   const moe::WsLayout L = layout_for(*dims, T);
   const size_t v[MOE_WS_FIELDS] = {L.status, L.counts, L.offsets,  L.ntiles, L.tile_base, L.tiles,
                                    L.topk_idx, L.topk_w, L.perm,   L.inv,      L.w_sorted, L.xq,
-                                   L.xsf,    L.sfx,    L.hq,       L.sfh,    L.ys,       L.total};
+                                   L.xsf,    L.bpx,    L.bph,      L.ys,     L.total};
   for (int i = 0; i < MOE_WS_FIELDS; ++i) offsets[i] = v[i];
   return MOE_OK;
 }

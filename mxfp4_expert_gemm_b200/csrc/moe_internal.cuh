@@ -36,7 +36,20 @@ __host__ __device__ __forceinline__ int sf_byte_in_group(int r, int b) {
 
 // Scale-factor groups of one token tile: tile_tokens tokens give 2 * tile_tokens MMA
 // columns (hi and lo term of each token), 128 columns per group.
-__host__ __device__ __forceinline__ int sf_groups_of(int tile_tokens) { return (2 * tile_tokens + 127) / 128; }
+__host__ __device__ constexpr int sf_groups_of(int tile_tokens) { return (2 * tile_tokens + 127) / 128; }
+
+// Packed activation block of one token tile and one 128-chunk of the reduction axis: the
+// tile's 2 * tile_tokens E4M3 rows of 128 bytes (row n = MMA column n = hi / lo term of
+// token n / 2) in the 128-byte-swizzled order the MMA reads (16-byte unit u of row n at
+// unit u ^ (n % 8)), then the tile's scale-factor groups for the chunk's four 32-blocks,
+// padded to a multiple of 1 KB.  One contiguous copy brings a block into shared memory.
+__host__ __device__ constexpr int packed_block_bytes(int tile_tokens) {
+  return (2 * tile_tokens * kKChunk + sf_groups_of(tile_tokens) * kSfGroupBytes + 1023) / 1024 * 1024;
+}
+__host__ __device__ __forceinline__ int packed_unit_offset(int n, int u) { return n * kKChunk + ((u ^ (n & 7)) << 4); }
+__host__ __device__ __forceinline__ int packed_sf_offset(int tile_tokens, int n, int b) {
+  return 2 * tile_tokens * kKChunk + (n >> 7) * kSfGroupBytes + sf_byte_in_group(n & 127, b & 3);
+}
 
 // ------------------------------------------------------------------ MXFP4 storage layout
 // Weights [E][N][K] (moe_mxfp4.h) in tiles of 128 rows x 128 k: codes [E][NT][KC][128][64]
@@ -76,26 +89,27 @@ struct WsLayout {
   size_t w_sorted;  // f32 [P]     routing weight of each sorted pair
   size_t xq;        // E4M3 [T][2][dp]   hi / lo terms of xe = bf16(RMSNorm(x))
   size_t xsf;       // E8M0 [T][2][dp/32] their scales
-  size_t sfx;       // E8M0 [max_tiles][dp/128][G][512] scales of xq per token tile and column
-  size_t hq;        // E4M3 [2P][Ip]     hi / lo terms of h (sorted order)
-  size_t sfh;       // E8M0 [max_tiles][Ip/128][G][512]
-  size_t ys;        // f32 [P][d]  routing-weighted expert outputs, sorted order
+  size_t bpx;       // packed blocks [max_tiles][dp/128] of xe per token tile (gate_up's B)
+  size_t bph;       // packed blocks [max_tiles][ip/128] of h per token tile (down's B)
+  size_t ys;        // f32 [ksplit][P][d]  routing-weighted expert outputs (partial sums per
+                    // reduction-axis split of the down GEMM), sorted order
   size_t total;
   int64_t max_tiles;
   int32_t tile_tokens;
+  int32_t ksplit;   // down GEMM reduction-axis splits (ys planes)
   int32_t dp, ip;   // d and I rounded up to 128
 };
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-inline WsLayout ws_layout(const moe_dims& dm, int64_t T, int tile_tokens) {
+inline WsLayout ws_layout(const moe_dims& dm, int64_t T, int tile_tokens, int ksplit) {
   WsLayout L{};
   const int64_t P = T * dm.top_k;
   L.tile_tokens = tile_tokens;
+  L.ksplit = ksplit;
   L.max_tiles = (P + tile_tokens - 1) / tile_tokens + dm.E;
   L.dp = (int32_t)kpad128(dm.d);
   L.ip = (int32_t)kpad128(dm.I);
-  const size_t G = (size_t)sf_groups_of(tile_tokens);
   size_t o = 0;
   auto take = [&](size_t bytes) {
     const size_t at = o;
@@ -115,10 +129,9 @@ inline WsLayout ws_layout(const moe_dims& dm, int64_t T, int tile_tokens) {
   L.w_sorted = take(4 * (size_t)P);
   L.xq = take(2 * (size_t)T * L.dp);
   L.xsf = take(2 * (size_t)T * (L.dp / 32));
-  L.sfx = take((size_t)L.max_tiles * (L.dp / kKChunk) * G * kSfGroupBytes);
-  L.hq = take(2 * (size_t)P * L.ip);
-  L.sfh = take((size_t)L.max_tiles * (L.ip / kKChunk) * G * kSfGroupBytes);
-  L.ys = take(4 * (size_t)P * dm.d);
+  L.bpx = take((size_t)L.max_tiles * (L.dp / kKChunk) * packed_block_bytes(tile_tokens));
+  L.bph = take((size_t)L.max_tiles * (L.ip / kKChunk) * packed_block_bytes(tile_tokens));
+  L.ys = take(4 * (size_t)ksplit * P * dm.d);
   L.total = o;
   return L;
 }
@@ -140,12 +153,12 @@ struct Ws {
   float* w_sorted;
   uint8_t* xq;
   uint8_t* xsf;
-  uint8_t* sfx;
-  uint8_t* hq;
-  uint8_t* sfh;
+  uint8_t* bpx;
+  uint8_t* bph;
   float* ys;
   int64_t max_tiles;
   int32_t tile_tokens;
+  int32_t ksplit;
   int32_t dp, ip;
 };
 
@@ -165,14 +178,14 @@ inline Ws ws_pointers(void* base, const WsLayout& L, int E) {
   w.w_sorted = reinterpret_cast<float*>(b + L.w_sorted);
   w.xq = reinterpret_cast<uint8_t*>(b + L.xq);
   w.xsf = reinterpret_cast<uint8_t*>(b + L.xsf);
-  w.sfx = reinterpret_cast<uint8_t*>(b + L.sfx);
-  w.hq = reinterpret_cast<uint8_t*>(b + L.hq);
-  w.sfh = reinterpret_cast<uint8_t*>(b + L.sfh);
+  w.bpx = reinterpret_cast<uint8_t*>(b + L.bpx);
+  w.bph = reinterpret_cast<uint8_t*>(b + L.bph);
   w.ys = reinterpret_cast<float*>(b + L.ys);
   w.ticket = w.counts + E;
   w.arrivals = w.counts + E + 4;
   w.max_tiles = L.max_tiles;
   w.tile_tokens = L.tile_tokens;
+  w.ksplit = L.ksplit;
   w.dp = L.dp;
   w.ip = L.ip;
   return w;
@@ -279,7 +292,7 @@ struct FwdArgs {
   cudaStream_t stream;
   EventRec* ev;
   int32_t inject_timeout;  // test hook: withhold one pipeline arrival in the gate_up kernel
-  int32_t fuse_group;      // small batches: the routing kernel also groups (and scatters tile scales)
+  int32_t fuse_group;      // small batches: the routing kernel also groups (and packs the tiles)
   int32_t fuse_combine;    // the down kernel also adds the k expert outputs and the residual
   int32_t pdl;             // launch dependent kernels with programmatic stream serialization
 };
@@ -329,9 +342,10 @@ __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
 // Each returns the number of kernels it launched (>= 0) or -1 on a launch error.
 int launch_quantize(const float* w, int32_t E, int32_t N, int32_t K, int32_t role, uint8_t* codes,
                     uint8_t* scales, int32_t* status, cudaStream_t st);
-int launch_route(const FwdArgs& a);     // norm + router + top-k + E4M3 split, grouping, tile scales
+int launch_route(const FwdArgs& a);     // norm + router + top-k + E4M3 split, grouping, packing
 int launch_combine(const FwdArgs& a);   // y = x + sum_j ys[inv]
 int launch_experts(const FwdArgs& a);   // block-scaled tcgen05 expert MLPs (gate_up, down)
 int expert_tile_tokens(int path);       // token tile of a path
+int expert_down_split(int path);        // reduction-axis splits of a path's down GEMM
 
 }  // namespace moe

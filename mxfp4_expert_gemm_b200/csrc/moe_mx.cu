@@ -15,13 +15,12 @@
 // Persistent kernel, CPS CTAs per SM.  A work item is 128 weight rows x one token tile
 // over the whole reduction axis; CTA b takes items b, b + grid, ...  A pipeline stage
 // covers NP chunks of 128 along the reduction axis:
-//   warp 0     producer: per stage one TMA load of the weight codes (NP consecutive
+//   warps 0..  producers: per stage one TMA load of the weight codes (NP consecutive
 //              8 KB tile blocks; E2M1, unpacked by the copy to one byte per code in
-//              shared memory, 128B swizzle), the activation rows [NP][2*BN][128] (gate_up:
-//              tile::gather4 loads of the tile's tokens from the per-token rows, issued
-//              by all lanes; down: one 3D TMA load of the sorted rows of h), and one bulk
-//              copy each of the weight and the activation scale factors, both stored in
-//              the tensor cores' scale-factor layout;
+//              shared memory, 128B swizzle), one bulk copy of the token tile's packed
+//              activation blocks (2*BN E4M3 rows per chunk, already in the swizzled order,
+//              followed by their scale factors) and one bulk copy of the weight scale
+//              factors (stored in the tensor cores' scale-factor layout);
 //   warp 1     TMEM allocation and the MMA issuer (one thread): per stage it copies the
 //              scale factors into TMEM (tcgen05.cp) and issues one block-scaled MMA
 //              per 32-wide block of the reduction axis;
@@ -56,21 +55,22 @@ struct MxParams {
   const Tile* tiles;
   const int32_t* ntiles;
   const uint8_t* w_sf;     // weight scale-factor groups [E][NT][KC][512]
-  const uint8_t* a_sf;     // activation scale-factor groups per token tile [tiles][KC][G][512]
+  const uint8_t* bp_in;    // packed activation blocks of this GEMM [tiles][KC][block]
   int32_t NT;              // 128-row tiles per expert
   int32_t K;               // reduction length (d for gate_up, I for down)
   int32_t KC;              // 128-chunks of the reduction axis (K rounded up)
   int32_t n_rt;            // row tiles per token tile: I/64 (gate_up) or ceil(d/128) (down)
+  int32_t ksplit;          // reduction-axis splits per (token tile, row tile) (down only; >= 1)
+  int32_t P;               // pairs (rows of ys per split)
   int32_t* status;
   float limit;
   int32_t inject_timeout;  // test hook: CTA 0 withholds its first stage
-  // gate_up output: h as E4M3 hi / lo rows [2P][ip] and their scale factors per token tile
-  uint8_t* hq;
-  uint8_t* sfh;
-  int32_t ip;              // I rounded up to 128 (row pitch of hq)
-  int32_t KCh;             // ip / 128
-  // down output: ys [P][d] fp32 = w * o; optionally y = bf16(x + sum_j ys[inv[t*k + j]])
-  // by the last writer of each (token, 128-column) block
+  // gate_up output: h as packed activation blocks of the down GEMM [tiles][KCo][block]
+  uint8_t* bp_out;
+  int32_t KCo;             // 128-chunks of I
+  // down output: ys [ksplit][P][d] fp32 = w * (partial) o; optionally
+  // y = bf16(x + sum_j sum_s ys[s][inv[t*k + j]]) by the last writer of each (token,
+  // 128-column) block
   float* ys;
   int32_t d;
   const float* w_sorted;
@@ -88,18 +88,17 @@ struct MxParams {
 #endif
 constexpr int kSfSlots = MOE_SF_SLOTS;  // scale-factor TMEM slots, used stage after stage in turn
 
-template <int BN, int NP, int S, int CPS, int EG>
+template <int BN, int NP, int S, int CPS, int EG, int NPW>
 struct MxCfg {
   static constexpr int N2 = 2 * BN;                     // MMA N: hi and lo column per token
   static constexpr int G = (N2 + 127) / 128;            // scale-factor groups of the B operand
   static constexpr int A_PANEL = kBM * kKChunk;         // 128 rows x 128 codes, one byte each
   static constexpr int B_PANEL = N2 * kKChunk;          // N2 rows x 128 E4M3
+  static constexpr int B_BLOCK = packed_block_bytes(BN);  // B panel + its scale factors, padded
   static constexpr int B_OFF = NP * A_PANEL;
-  static constexpr int SFA_OFF = B_OFF + NP * B_PANEL;
-  static constexpr int SFB_OFF = SFA_OFF + NP * kSfGroupBytes;
-  static constexpr int STAGE_BYTES = ((SFB_OFF + NP * G * kSfGroupBytes + 1023) / 1024) * 1024;
+  static constexpr int SFA_OFF = B_OFF + NP * B_BLOCK;
+  static constexpr int STAGE_BYTES = ((SFA_OFF + NP * kSfGroupBytes + 1023) / 1024) * 1024;
   static constexpr int A_TX = NP * kBM * kKChunk / 2;   // the weight box counts packed bytes
-  static constexpr int B_TX = NP * B_PANEL;
   static constexpr int CW = N2 < 32 ? N2 : 32;          // accumulator columns per epilogue read
   static constexpr int TC = CW / 2;                     // tokens per epilogue read
   static constexpr int HT = TC / 2;                     // tokens each side (gate / up) finishes
@@ -115,20 +114,37 @@ struct MxCfg {
   static constexpr int BAR_BYTES = 8 * (2 * S + 5) + 16;
   static constexpr int SMEM_BYTES = S * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024 /*align slack*/;
   static constexpr int EPI_THREADS = 128 * EG;
-  static constexpr int THREADS = 64 + EPI_THREADS;
+  static constexpr int MMA_WARP = NPW;                // warps 0..NPW-1 produce
+  static constexpr int EPI_WARP0 = NPW + 1;
+  static constexpr int THREADS = 32 * EPI_WARP0 + EPI_THREADS;
   static_assert(N2 == 16 || (N2 % 32 == 0 && N2 <= 256), "MMA N: 16 or a multiple of 32 up to 256");
   static_assert(COLS_NEEDED <= 512 && TMEM_COLS * CPS <= 512, "TMEM budget of CPS co-resident CTAs");
   static_assert(SMEM_BYTES * CPS <= 227 * 1024, "shared memory budget of CPS co-resident CTAs");
   static_assert(kBM * NP <= 256, "TMA box height");
   static_assert(EG == 1 || EG == 2, "one or two epilogue warpgroups");
-  static_assert(N2 % 4 == 0 && N2 / 4 <= 64, "gather4 columns: two instructions per producer lane");
+  static_assert(NPW >= 1 && NPW <= 4, "producer warps");
 };
 
-template <int BN, int NP, int S, int CPS, int EG, int MODE>
-__global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
-    mx_expert_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_act,
-                     const MxParams p) {
-  using C = MxCfg<BN, NP, S, CPS, EG>;
+// Work item i: token tile tt, row tile rt, and the chunk range [kc0, kc1) of split ks.
+struct Item {
+  int tt, rt, ks, kc0, kc1;
+};
+
+__device__ __forceinline__ Item item_of(const MxParams& p, int i) {
+  Item it;
+  const int r = i / p.ksplit;
+  it.ks = i - r * p.ksplit;
+  it.tt = r / p.n_rt;
+  it.rt = r - it.tt * p.n_rt;
+  it.kc0 = it.ks * p.KC / p.ksplit;
+  it.kc1 = (it.ks + 1) * p.KC / p.ksplit;
+  return it;
+}
+
+template <int BN, int NP, int S, int CPS, int EG, int NPW, int MODE>
+__global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
+    mx_expert_kernel(const __grid_constant__ CUtensorMap tm_w, const MxParams p) {
+  using C = MxCfg<BN, NP, S, CPS, EG, NPW>;
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
 
@@ -143,7 +159,6 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nst = (p.KC + NP - 1) / NP;   // stages per item
   const int kblocks = p.K / 32;
 
   if (threadIdx.x == 0) {
@@ -159,9 +174,8 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
     *s_abort = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tm_w);
-    ptx::prefetch_tensormap(&tm_act);
   }
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     ptx::tmem_alloc(s_tmem, C::TMEM_COLS);
     ptx::tmem_relinquish();
     ptx::tc_fence_before();
@@ -171,42 +185,29 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
   const uint32_t tmem = *s_tmem;
   // Everything above overlaps the previous kernel; the work list is its output.
   pdl_wait();
-  const int n_items = *p.ntiles * p.n_rt;
+  const int n_items = *p.ntiles * p.n_rt * p.ksplit;
 
   auto a_s = [&](int s) { return smem + s * C::STAGE_BYTES; };
   auto b_s = [&](int s) { return smem + s * C::STAGE_BYTES + C::B_OFF; };
   auto sfa_s = [&](int s) { return smem + s * C::STAGE_BYTES + C::SFA_OFF; };
-  auto sfb_s = [&](int s) { return smem + s * C::STAGE_BYTES + C::SFB_OFF; };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ producer
-    // Lane 0 owns the ring and issues the weight load and the scale-factor copies; for
-    // gate_up every lane also gathers activation rows (tile::gather4, four MMA columns
-    // per instruction) straight from the per-token rows of xq, in the tile's token order.
+  if (warp < NPW) {
+    // ------------------------------------------------------------------ producers
+    // Producer warp w fills the stages g with g % NPW == w; the warp waits converged and
+    // lane 0 issues the three copies of a stage.
     int64_t g = 0;  // global stage counter of this CTA
     bool stop = false, withheld = false;
     for (int i = blockIdx.x; i < n_items && !stop; i += gridDim.x) {
-      const int tt = i / p.n_rt, rt = i - tt * p.n_rt;
+      const Item it = item_of(p, i);
+      const int tt = it.tt, rt = it.rt;
+      const int nst = (it.kc1 - it.kc0 + NP - 1) / NP;   // stages of this item
       const Tile tl = p.tiles[tt];
-      // gate_up: xq rows (2 t + term) of MMA columns 4 i4 .. 4 i4 + 3, i4 = lane, lane + 32
-      // (columns past the tile's tokens repeat its last token; their outputs are dropped)
-      int xr[2][4];
-      if (MODE == MODE_GATE_UP) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int n = 4 * (lane + 32 * u) + r;
-            const int j = min(n >> 1, tl.rows - 1);
-            xr[u][r] = (n < C::N2) ? 2 * (p.perm[tl.row0 + j] / p.k) + (n & 1) : 0;
-          }
-      }
       for (int st = 0; st < nst; ++st, ++g) {
+        if ((int)(g % NPW) != warp) continue;
         const int s = (int)(g % S);
         bool ok = true;
-        if (lane == 0 && g >= S)
-          ok = ptx::mbar_wait_bounded(&sfree[s], (uint32_t)((g / S) - 1) & 1, s_abort, kWaitLimitNs);
-        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+        if (g >= S) ok = ptx::mbar_wait_bounded(&sfree[s], (uint32_t)((g / S) - 1) & 1, s_abort, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) {
           stop = true;
           break;
         }
@@ -214,88 +215,88 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
           withheld = true;  // this stage never fills: the MMA issuer's wait gives up
           continue;
         }
-        const int c0 = st * NP, nck = min(NP, p.KC - c0);
+        const int c0 = it.kc0 + st * NP, nck = min(NP, it.kc1 - c0);
         if (lane == 0) {
-          const int b_tx = (MODE == MODE_GATE_UP) ? nck * C::B_PANEL : C::B_TX;
-          ptx::mbar_arrive_expect_tx(&full[s], C::A_TX + b_tx + nck * (1 + C::G) * kSfGroupBytes);
+          ptx::mbar_arrive_expect_tx(&full[s], C::A_TX + nck * (C::B_BLOCK + kSfGroupBytes));
           ptx::tma_load_2d(a_s(s), &tm_w, 0, (int)(((int64_t)tl.e * p.NT + rt) * p.KC + c0) * kBM, &full[s]);
-          if (MODE == MODE_DOWN) ptx::tma_load_3d(b_s(s), &tm_act, 0, 2 * tl.row0, c0, &full[s]);
+          ptx::bulk_load(b_s(s), p.bp_in + ((int64_t)tt * p.KC + c0) * C::B_BLOCK, nck * C::B_BLOCK, &full[s]);
           ptx::bulk_load(sfa_s(s), p.w_sf + ((int64_t)(tl.e * p.NT + rt) * p.KC + c0) * kSfGroupBytes,
                          nck * kSfGroupBytes, &full[s]);
-          ptx::bulk_load(sfb_s(s), p.a_sf + ((int64_t)tt * p.KC + c0) * C::G * kSfGroupBytes,
-                         nck * C::G * kSfGroupBytes, &full[s]);
         }
         __syncwarp();
-        if (MODE == MODE_GATE_UP) {
-          for (int c = 0; c < nck; ++c)
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int i4 = lane + 32 * u;
-              if (4 * i4 < C::N2)
-                ptx::tma_gather4(b_s(s) + c * C::B_PANEL + i4 * 4 * kKChunk, &tm_act, (c0 + c) * kKChunk,
-                                 xr[u][0], xr[u][1], xr[u][2], xr[u][3], &full[s]);
-            }
-        }
       }
     }
     // Never leave copies in flight when the CTA exits (consumers may have aborted before
     // waiting for them): wait, bounded, for the last fill of every slot.  On the normal
     // path these have all landed already.
-    if (lane == 0) {
+    {
       volatile int local_abort = 0;
       for (int64_t q = (g > S ? g - S : 0); q < g; ++q) {
-        if (withheld && q == 0) continue;
+        if ((int)(q % NPW) != warp || (withheld && q == 0)) continue;
         ptx::mbar_wait_bounded(&full[q % S], (uint32_t)(q / S) & 1, &local_abort, kWaitLimitNs);
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The warp waits converged; lane 0 issues the copies into TMEM, the MMAs and the
+    // commits.
+    {
       int64_t g = 0;
       int li = 0;
       bool stop = false;
       for (int i = blockIdx.x; i < n_items && !stop; i += gridDim.x, ++li) {
         const int b = li & 1;
-        if (li >= 2 && !ptx::mbar_wait_bounded(&acce[b], (uint32_t)((li >> 1) - 1) & 1, s_abort, kWaitLimitNs))
+        if (li >= 2 &&
+            !__all_sync(0xffffffffu,
+                        ptx::mbar_wait_bounded(&acce[b], (uint32_t)((li >> 1) - 1) & 1, s_abort, kWaitLimitNs)))
           break;
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + b * C::ACC_COLS;
+        const Item it = item_of(p, i);
+        const int nst = (it.kc1 - it.kc0 + NP - 1) / NP;
         for (int st = 0; st < nst; ++st, ++g) {
           const int s = (int)(g % S);
-          if (!ptx::mbar_wait_bounded(&full[s], (uint32_t)(g / S) & 1, s_abort, kWaitLimitNs)) {
+          if (!__all_sync(0xffffffffu,
+                          ptx::mbar_wait_bounded(&full[s], (uint32_t)(g / S) & 1, s_abort, kWaitLimitNs))) {
             stop = true;
             break;
           }
           ptx::tc_fence_after();
-          const int c0 = st * NP, nck = min(NP, p.KC - c0);
-          // scale factors of this stage into their TMEM slot (the tensor pipe runs one
-          // thread's copies and MMAs in issue order; with two slots a copy does not
-          // overwrite columns the previous stage's MMAs still read)
-          const uint32_t sf_slot = tmem + (uint32_t)((g % kSfSlots) * C::SF_SLOT_COLS);
-          for (int c = 0; c < nck; ++c) {
-            ptx::tc_cp_32x128b_x4(sf_slot + C::SFA_COL + 4 * c, ptx::smem_desc_k_rows16(sfa_s(s) + c * kSfGroupBytes));
+          const int c0 = it.kc0 + st * NP, nck = min(NP, it.kc1 - c0);
+          if (lane == 0) {
+            // scale factors of this stage into their TMEM slot (the tensor pipe runs one
+            // thread's copies and MMAs in issue order; with two slots a copy does not
+            // overwrite columns the previous stage's MMAs still read)
+            const uint32_t sf_slot = tmem + (uint32_t)((g % kSfSlots) * C::SF_SLOT_COLS);
+            for (int c = 0; c < nck; ++c) {
+              ptx::tc_cp_32x128b_x4(sf_slot + C::SFA_COL + 4 * c,
+                                    ptx::smem_desc_k_rows16(sfa_s(s) + c * kSfGroupBytes));
 #pragma unroll
-            for (int gg = 0; gg < C::G; ++gg)
-              ptx::tc_cp_32x128b_x4(sf_slot + C::SFB_COL + 4 * (c * C::G + gg),
-                                    ptx::smem_desc_k_rows16(sfb_s(s) + (c * C::G + gg) * kSfGroupBytes));
+              for (int gg = 0; gg < C::G; ++gg)
+                ptx::tc_cp_32x128b_x4(sf_slot + C::SFB_COL + 4 * (c * C::G + gg),
+                                      ptx::smem_desc_k_rows16(b_s(s) + c * C::B_BLOCK + C::B_PANEL + gg * kSfGroupBytes));
+            }
+            for (int c = 0; c < nck; ++c) {
+              const int nkb = min(4, kblocks - 4 * (c0 + c));
+              const uint64_t adesc = ptx::smem_desc_k_sw128(a_s(s) + c * C::A_PANEL);
+              const uint64_t bdesc = ptx::smem_desc_k_sw128(b_s(s) + c * C::B_BLOCK);
+              const uint32_t sfa = sf_slot + C::SFA_COL + 4 * c, sfb = sf_slot + C::SFB_COL + 4 * c * C::G;
+              for (int kk = 0; kk < nkb; ++kk)
+                ptx::mma_mx_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
+                               ptx::idesc_mx_e2m1_e4m3(kBM, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
+                               (st | c | kk) != 0);
+            }
+            ptx::tc_commit(&sfree[s]);
           }
-          for (int c = 0; c < nck; ++c) {
-            const int nkb = min(4, kblocks - 4 * (c0 + c));
-            const uint64_t adesc = ptx::smem_desc_k_sw128(a_s(s) + c * C::A_PANEL);
-            const uint64_t bdesc = ptx::smem_desc_k_sw128(b_s(s) + c * C::B_PANEL);
-            const uint32_t sfa = sf_slot + C::SFA_COL + 4 * c, sfb = sf_slot + C::SFB_COL + 4 * c * C::G;
-            for (int kk = 0; kk < nkb; ++kk)
-              ptx::mma_mx_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
-                             ptx::idesc_mx_e2m1_e4m3(kBM, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
-                             (st | c | kk) != 0);
-          }
-          ptx::tc_commit(&sfree[s]);
+          __syncwarp();
         }
-        if (!stop) ptx::tc_commit(&accf[b]);
+        if (!stop && lane == 0) ptx::tc_commit(&accf[b]);
+        __syncwarp();
       }
       // Every MMA issued above completes before the drain barrier fires.
-      ptx::tc_commit(drain);
+      if (lane == 0) ptx::tc_commit(drain);
+      __syncwarp();
       volatile int local_abort = 0;
       ptx::mbar_wait_bounded(drain, 0, &local_abort, kWaitLimitNs);
     }
@@ -304,8 +305,8 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
     // ------------------------------------------------------------------ epilogue warps
     const int q = warp & 3;              // TMEM lane quarter this warp may access
     const int row = 32 * q + lane;       // weight row of the tile == TMEM lane
-    const int eg = (warp - 2) >> 2;      // epilogue warpgroup: reads c0 = (eg + EG*m) * CW
-    const int et = threadIdx.x - 64 - 128 * eg;  // 0..127 within the group
+    const int eg = (warp - C::EPI_WARP0) >> 2;   // epilogue warpgroup: reads c0 = (eg + EG*m) * CW
+    const int et = threadIdx.x - 32 * C::EPI_WARP0 - 128 * eg;  // 0..127 within the group
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     uint8_t* gepi = epi + eg * C::EPI_GROUP_BYTES;
     auto group_sync = [&]() {            // the group's named barrier (128 threads)
@@ -321,7 +322,8 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
       // role at any time; the barrier reduction freezes one answer for all).
       if (ptx::bar_or<3, C::EPI_THREADS>(!ready)) break;
       ptx::tc_fence_after();
-      const int tt = i / p.n_rt, rt = i - tt * p.n_rt;
+      const Item it = item_of(p, i);
+      const int tt = it.tt, rt = it.rt;
       const Tile tl = p.tiles[tt];
       const uint32_t acc = tmem + lane_addr + b * C::ACC_COLS;
       if (MODE == MODE_GATE_UP) {
@@ -373,14 +375,15 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
             e4m3_split<1>(vv, hi, lo, s1, s2);
             const int j = c0 / 2 + jj;                 // token within the tile
             if (j < tl.rows) {
-              const int64_t prow = tl.row0 + j;
-              p.hq[(2 * prow) * p.ip + 64 * rt + f] = (uint8_t)hi;
-              p.hq[(2 * prow + 1) * p.ip + 64 * rt + f] = (uint8_t)lo;
+              // the down GEMM's packed block: chunk kb / 4, rows 2j (hi) and 2j + 1 (lo),
+              // byte f' = 32 (kb % 4) + lane of the 128-byte row
+              uint8_t* blk = p.bp_out + ((int64_t)tt * p.KCo + kb / 4) * C::B_BLOCK;
+              const int u = 2 * (kb & 3) + (lane >> 4);
+              blk[packed_unit_offset(2 * j, u) + (lane & 15)] = (uint8_t)hi;
+              blk[packed_unit_offset(2 * j + 1, u) + (lane & 15)] = (uint8_t)lo;
               if (lane == 0) {
-                uint8_t* grp = p.sfh + ((int64_t)tt * p.KCh + kb / 4) * C::G * kSfGroupBytes;
-                const int nh = 2 * j, nl = 2 * j + 1;
-                grp[(nh >> 7) * kSfGroupBytes + sf_byte_in_group(nh, kb)] = (uint8_t)s1;
-                grp[(nl >> 7) * kSfGroupBytes + sf_byte_in_group(nl, kb)] = (uint8_t)s2;
+                blk[packed_sf_offset(BN, 2 * j, kb)] = (uint8_t)s1;
+                blk[packed_sf_offset(BN, 2 * j + 1, kb)] = (uint8_t)s2;
               }
             }
           }
@@ -388,6 +391,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
         }
       } else {
         int* s_tok = reinterpret_cast<int*>(gepi + C::TC * 64 * 4);  // [TC]
+        float* ys = p.ys + (int64_t)it.ks * p.P * p.d;               // this split's partial sums
         const int m = kBM * rt + row;                                // output feature
         const int ncol = min(kBM, p.d - kBM * rt);
         if (eg * C::CW >= C::N2) {
@@ -409,7 +413,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
             if (c < nt && m < p.d) {
               const int64_t prow = tl.row0 + jbase + c;
               const float o = __uint_as_float(v[2 * c]) + __uint_as_float(v[2 * c + 1]);
-              p.ys[prow * p.d + m] = o * p.w_sorted[prow];
+              ys[prow * p.d + m] = o * p.w_sorted[prow];
             }
           }
           if (p.fuse_combine) {
@@ -420,7 +424,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
             if (et < nt) {
               const int tok = p.perm[tl.row0 + jbase + et] / p.k;
               const int prev = atomicAdd(p.arrivals + (int64_t)tok * p.n_rt + rt, 1);
-              s_tok[et] = (prev == p.k - 1) ? tok : -1;
+              s_tok[et] = (prev == p.k * p.ksplit - 1) ? tok : -1;
             }
             group_sync();
             __threadfence();
@@ -432,7 +436,8 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
                 float accv = __uint_as_float((uint32_t)p.x[(int64_t)tok * p.d + gc] << 16);
                 for (int j = 0; j < p.k; ++j) {
                   const int srow = p.inv[(int64_t)tok * p.k + j];
-                  accv += __ldcg(p.ys + (int64_t)srow * p.d + gc);
+                  for (int sp = 0; sp < p.ksplit; ++sp)
+                    accv += __ldcg(p.ys + ((int64_t)sp * p.P + srow) * p.d + gc);
                 }
                 uint32_t bb = __float_as_uint(accv);
                 bb = (bb + 0x7FFFu + ((bb >> 16) & 1u)) >> 16;   // round to bf16
@@ -448,7 +453,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG>::THREADS, CPS)
 
   __syncthreads();
   if (*s_abort && threadIdx.x == 0) set_status(p.status, MOE_ERR_TIMEOUT);
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -496,9 +501,9 @@ int sm_count() {
   return n;
 }
 
-template <int MODE, int BN, int NP, int S, int CPS, int EG>
+template <int MODE, int BN, int NP, int S, int CPS, int EG, int NPW, int KSPLIT>
 int launch_one(const FwdArgs& a) {
-  using C = MxCfg<BN, NP, S, CPS, EG>;
+  using C = MxCfg<BN, NP, S, CPS, EG, NPW>;
   const int P = a.T * a.k;
   const int K = (MODE == MODE_GATE_UP) ? a.d : a.I;
   const int N = (MODE == MODE_GATE_UP) ? 2 * a.I : a.d;  // weight rows per expert
@@ -506,13 +511,11 @@ int launch_one(const FwdArgs& a) {
   const int KC = (int)(Kp / kKChunk);
   const uint8_t* codes = (MODE == MODE_GATE_UP) ? a.w1c : a.w2c;
   const uint8_t* scales = (MODE == MODE_GATE_UP) ? a.w1s : a.w2s;
-  const uint8_t* act = (MODE == MODE_GATE_UP) ? a.ws.xq : a.ws.hq;
-  const int act_pitch = (MODE == MODE_GATE_UP) ? a.ws.dp : a.ws.ip;
 
   // Weight codes [E][NT][KC][128][64] viewed as rows of 128 codes (E2M1, unpacked by the
   // copy): one box brings NP consecutive tile blocks (NP x 128 rows), each a
   // 128B-swizzled [128][128] panel in shared memory.
-  CUtensorMap m_w, m_act;
+  CUtensorMap m_w;
   {
     const int NT = (N + kBM - 1) / kBM;
     const uint64_t dims[2] = {(uint64_t)kKChunk, (uint64_t)a.E * NT * KC * kBM};
@@ -520,36 +523,22 @@ int launch_one(const FwdArgs& a) {
     const uint32_t box[2] = {kKChunk, (uint32_t)(kBM * NP)};
     if (!make_map(&m_w, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, codes, dims, str, box)) return -1;
   }
-  if (MODE == MODE_GATE_UP) {
-    // Per-token rows xq [2T][dp] E4M3 (hi, lo): gathered four rows at a time, one row high.
-    const uint64_t dims[2] = {(uint64_t)act_pitch, (uint64_t)2 * a.T};
-    const uint64_t str[1] = {(uint64_t)act_pitch};
-    const uint32_t box[2] = {kKChunk, 1};
-    if (!make_map(&m_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, act, dims, str, box)) return -1;
-  } else {
-    // Sorted rows of h [2P][ip] E4M3 viewed as [chunks][2P rows][128]: one box brings NP
-    // chunks of the tile's 2*BN rows.
-    const uint64_t dims[3] = {(uint64_t)kKChunk, (uint64_t)2 * P, (uint64_t)act_pitch / kKChunk};
-    const uint64_t str[2] = {(uint64_t)act_pitch, (uint64_t)kKChunk};
-    const uint32_t box[3] = {kKChunk, (uint32_t)C::N2, (uint32_t)NP};
-    if (!make_map(&m_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, act, dims, str, box)) return -1;
-  }
   MxParams prm;
   prm.tiles = a.ws.tiles;
   prm.ntiles = a.ws.ntiles;
   prm.w_sf = scales;
-  prm.a_sf = (MODE == MODE_GATE_UP) ? a.ws.sfx : a.ws.sfh;
+  prm.bp_in = (MODE == MODE_GATE_UP) ? a.ws.bpx : a.ws.bph;
   prm.NT = (N + kBM - 1) / kBM;
   prm.K = K;
   prm.KC = KC;
   prm.n_rt = (MODE == MODE_GATE_UP) ? a.I / 64 : (a.d + kBM - 1) / kBM;
+  prm.ksplit = std::max(1, std::min(KSPLIT, KC));   // every split keeps at least one chunk
+  prm.P = P;
   prm.status = a.ws.status;
   prm.limit = a.limit;
   prm.inject_timeout = (MODE == MODE_GATE_UP) ? a.inject_timeout : 0;
-  prm.hq = a.ws.hq;
-  prm.sfh = a.ws.sfh;
-  prm.ip = a.ws.ip;
-  prm.KCh = a.ws.ip / kKChunk;
+  prm.bp_out = a.ws.bph;
+  prm.KCo = a.ws.ip / kKChunk;
   prm.ys = a.ws.ys;
   prm.d = a.d;
   prm.w_sorted = a.ws.w_sorted;
@@ -561,7 +550,7 @@ int launch_one(const FwdArgs& a) {
   prm.y = a.y;
   prm.arrivals = a.ws.arrivals;
 
-  auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, MODE>;
+  auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, NPW, MODE>;
   static std::atomic<uint64_t> attr_done{0};   // per-device "attribute set" bits
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -571,10 +560,10 @@ int launch_one(const FwdArgs& a) {
       return -1;
     attr_done.fetch_or(bit, std::memory_order_release);
   }
-  const int64_t max_items = (int64_t)((P + BN - 1) / BN + a.E) * prm.n_rt;
+  const int64_t max_items = (int64_t)((P + BN - 1) / BN + a.E) * prm.n_rt * prm.ksplit;
   const int grid = (int)std::min<int64_t>(max_items, (int64_t)sm_count() * CPS);
   ev_before(a);
-  if (launch_kernel(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, a.stream, a.pdl != 0, m_w, m_act, prm) !=
+  if (launch_kernel(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, a.stream, a.pdl != 0, m_w, prm) !=
       cudaSuccess)
     return -1;
   ev_after(a);
@@ -582,26 +571,33 @@ int launch_one(const FwdArgs& a) {
 }
 
 // Pipeline shapes (compile-time; overridable with -D for tuning builds).
-// Small batches (few tokens per expert): 8-token tiles (MMA N = 16), two independent
-// pipelines (CTAs) per SM.
+// Small batches (few tokens per expert): 8-token tiles (MMA N = 16), three independent
+// pipelines (CTAs) per SM: each CTA's copies are served in order, so more CTAs keep
+// more of HBM's requests in flight.
 #ifndef MOE_GEMV_NP
 #define MOE_GEMV_NP 1
 #endif
 #ifndef MOE_GEMV_S
-#define MOE_GEMV_S 5
+#define MOE_GEMV_S 3
 #endif
 #ifndef MOE_GEMV_CPS
-#define MOE_GEMV_CPS 2
+#define MOE_GEMV_CPS 3
 #endif
 #ifndef MOE_GEMV_EG
 #define MOE_GEMV_EG 1
 #endif
+#ifndef MOE_GEMV_NPW
+#define MOE_GEMV_NPW 1
+#endif
+#ifndef MOE_GEMV_DOWN_SPLIT
+#define MOE_GEMV_DOWN_SPLIT 2
+#endif
 // Large batches: 96-token tiles (MMA N = 192).
 #ifndef MOE_GEMM_NP
-#define MOE_GEMM_NP 1
+#define MOE_GEMM_NP 2
 #endif
 #ifndef MOE_GEMM_S
-#define MOE_GEMM_S 4
+#define MOE_GEMM_S 2
 #endif
 #ifndef MOE_GEMM_CPS
 #define MOE_GEMM_CPS 1
@@ -609,26 +605,31 @@ int launch_one(const FwdArgs& a) {
 #ifndef MOE_GEMM_EG
 #define MOE_GEMM_EG 2
 #endif
+#ifndef MOE_GEMM_NPW
+#define MOE_GEMM_NPW 1
+#endif
 constexpr int kGemvBN = 8, kGemvNP = MOE_GEMV_NP, kGemvS = MOE_GEMV_S, kGemvCPS = MOE_GEMV_CPS,
-              kGemvEG = MOE_GEMV_EG;
+              kGemvEG = MOE_GEMV_EG, kGemvNPW = MOE_GEMV_NPW, kGemvDownSplit = MOE_GEMV_DOWN_SPLIT;
 constexpr int kGemmBN = 96, kGemmNP = MOE_GEMM_NP, kGemmS = MOE_GEMM_S, kGemmCPS = MOE_GEMM_CPS,
-              kGemmEG = MOE_GEMM_EG;
+              kGemmEG = MOE_GEMM_EG, kGemmNPW = MOE_GEMM_NPW;
 static_assert(kGemvBN >= kMinTileTokens, "tile list sized for the smallest tile");
 
 }  // namespace
 
 int expert_tile_tokens(int path) { return path == MOE_PATH_GEMV ? kGemvBN : kGemmBN; }
 
+int expert_down_split(int path) { return path == MOE_PATH_GEMV ? kGemvDownSplit : 1; }
+
 int launch_experts(const FwdArgs& a) {
   int n1, n2;
   if (a.ws.tile_tokens == kGemvBN) {
-    n1 = launch_one<MODE_GATE_UP, kGemvBN, kGemvNP, kGemvS, kGemvCPS, kGemvEG>(a);
+    n1 = launch_one<MODE_GATE_UP, kGemvBN, kGemvNP, kGemvS, kGemvCPS, kGemvEG, kGemvNPW, 1>(a);
     if (n1 < 0) return -1;
-    n2 = launch_one<MODE_DOWN, kGemvBN, kGemvNP, kGemvS, kGemvCPS, kGemvEG>(a);
+    n2 = launch_one<MODE_DOWN, kGemvBN, kGemvNP, kGemvS, kGemvCPS, kGemvEG, kGemvNPW, kGemvDownSplit>(a);
   } else {
-    n1 = launch_one<MODE_GATE_UP, kGemmBN, kGemmNP, kGemmS, kGemmCPS, kGemmEG>(a);
+    n1 = launch_one<MODE_GATE_UP, kGemmBN, kGemmNP, kGemmS, kGemmCPS, kGemmEG, kGemmNPW, 1>(a);
     if (n1 < 0) return -1;
-    n2 = launch_one<MODE_DOWN, kGemmBN, kGemmNP, kGemmS, kGemmCPS, kGemmEG>(a);
+    n2 = launch_one<MODE_DOWN, kGemmBN, kGemmNP, kGemmS, kGemmCPS, kGemmEG, kGemmNPW, 1>(a);
   }
   if (n2 < 0) return -1;
   return n1 + n2;

@@ -1,4 +1,4 @@
-// MXFP4 quantization, RMSNorm + router + top-k, grouping, tile scales and combine.
+// MXFP4 quantization, RMSNorm + router + top-k, grouping, tile packing and combine.
 //
 // Layer definition (web pages on gpt-oss):
 //  - RMSNorm: "From GPT-2 to gpt-oss" (新智元 translation), sec. 7: divide by the
@@ -150,24 +150,31 @@ __device__ __forceinline__ void warp_topk_softmax(float (&l)[NJ], int E, int k, 
 }
 
 // ----------------------------------------------------------------------------------
-// Grouping (and the tile scales) for a small batch, run by the routing CTA that finished last
+// Grouping (and the tile packing) for a small batch, run by the routing CTA that finished last
 // (all others have published their top-k, counts and xq rows before taking a ticket).
 // Pairs are listed per expert in token order: one warp walks the tokens in order and
 // hands each of a token's k (distinct) experts the next free position of that expert.
 // Deterministic: positions depend on counts and token order only.
 // ----------------------------------------------------------------------------------
-// Token t's activation scales (hi and lo term) into the scale-factor groups of token
-// tile `tile`, MMA columns 2*col (hi) and 2*col + 1 (lo).  One warp.  (The expert kernel
-// gathers the activation rows themselves from xq.)
-__device__ __forceinline__ void scatter_pair_scales(const FwdArgs& a, int t, int tile, int col) {
+// Token t's E4M3 rows (hi, lo) and their scales into the packed blocks of token tile
+// `tile`, MMA columns 2*col (hi) and 2*col + 1 (lo).  One warp.
+__device__ __forceinline__ void pack_pair(const FwdArgs& a, int t, int tile, int col) {
   const int lane = threadIdx.x & 31;
-  const int dp = a.ws.dp, nb = a.d / 32, G = sf_groups_of(a.ws.tile_tokens), kc = dp / kKChunk;
+  const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk;
+  const int bb = packed_block_bytes(bt);
+  uint8_t* blocks = a.ws.bpx + (int64_t)tile * kc * bb;
+  const uint8_t* rows = a.ws.xq + (int64_t)t * 2 * dp;
+  // 16-byte units: chunk c, term, unit u (the units past d are never read by the MMAs)
+  for (int i = lane; i < kc * 16; i += 32) {
+    const int c = i >> 4, term = (i >> 3) & 1, u = i & 7;
+    const int n = 2 * col + term;
+    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(rows + term * dp + c * kKChunk) + u);
+    *reinterpret_cast<uint4*>(blocks + (int64_t)c * bb + packed_unit_offset(n, u)) = v;
+  }
   const uint8_t* sf = a.ws.xsf + (int64_t)t * 2 * (dp / 32);
-  const int n_hi = 2 * col, n_lo = 2 * col + 1;
-  for (int b = lane; b < nb; b += 32) {
-    uint8_t* grp = a.ws.sfx + ((int64_t)tile * kc + b / 4) * G * kSfGroupBytes;
-    grp[(n_hi >> 7) * kSfGroupBytes + sf_byte_in_group(n_hi, b)] = __ldcg(sf + b);
-    grp[(n_lo >> 7) * kSfGroupBytes + sf_byte_in_group(n_lo, b)] = __ldcg(sf + dp / 32 + b);
+  for (int i = lane; i < 2 * nb; i += 32) {
+    const int term = i / nb, b = i - term * nb;
+    blocks[(int64_t)(b / 4) * bb + packed_sf_offset(bt, 2 * col + term, b)] = __ldcg(sf + term * (dp / 32) + b);
   }
 }
 
@@ -260,10 +267,10 @@ __device__ void group_block(const FwdArgs& a, int tile_tokens) {
     s_perm_e[pos] = v & 511;
   }
   __syncthreads();
-  // activation scales per token tile, one warp per pair
+  // packed activation blocks per token tile, one warp per pair
   for (int p = warp; p < P; p += blockDim.x >> 5) {
     const int e = s_perm_e[p], j = p - s_off[e];
-    scatter_pair_scales(a, s_perm_tok[p], s_tb[e] + j / tile_tokens, j % tile_tokens);
+    pack_pair(a, s_perm_tok[p], s_tb[e] + j / tile_tokens, j % tile_tokens);
   }
 }
 
@@ -595,9 +602,9 @@ __global__ void __launch_bounds__(1024) group_kernel(FwdArgs a, int tile_tokens)
   }
 }
 
-// Activation scales of every pair into its token tile's scale-factor groups.  One warp
+// Every pair's activation rows and scales into its token tile's packed blocks.  One warp
 // per pair.
-__global__ void tile_scales_kernel(FwdArgs a) {
+__global__ void pack_kernel(FwdArgs a) {
   pdl_trigger();
   pdl_wait();
   const int P = a.T * a.k, bt = a.ws.tile_tokens;
@@ -605,11 +612,11 @@ __global__ void tile_scales_kernel(FwdArgs a) {
     const int q = a.ws.perm[p];
     const int e = a.ws.topk_idx[q];
     const int j = p - a.ws.offsets[e];
-    scatter_pair_scales(a, q / a.k, a.ws.tile_base[e] + j / bt, j % bt);
+    pack_pair(a, q / a.k, a.ws.tile_base[e] + j / bt, j % bt);
   }
 }
 
-// y[t] = bf16(x[t] + sum_j ys[inv[t*k + j]]), j in slot order.
+// y[t] = bf16(x[t] + sum_j sum_s ys[s][inv[t*k + j]]), j in slot order, then split order.
 __global__ void combine_kernel(FwdArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -619,13 +626,16 @@ __global__ void combine_kernel(FwdArgs a) {
   const uint2 xr = *reinterpret_cast<const uint2*>(a.x + (int64_t)t * a.d + i4);
   float v[4] = {__uint_as_float(xr.x << 16), __uint_as_float(xr.x & 0xFFFF0000u), __uint_as_float(xr.y << 16),
                 __uint_as_float(xr.y & 0xFFFF0000u)};
+  const int64_t P = (int64_t)a.T * a.k;
   for (int j = 0; j < a.k; ++j) {
     const int p = a.ws.inv[(int64_t)t * a.k + j];
-    const float4 o = *reinterpret_cast<const float4*>(a.ws.ys + (int64_t)p * a.d + i4);
-    v[0] += o.x;
-    v[1] += o.y;
-    v[2] += o.z;
-    v[3] += o.w;
+    for (int sp = 0; sp < a.ws.ksplit; ++sp) {   // partial sums of a split down GEMM
+      const float4 o = *reinterpret_cast<const float4*>(a.ws.ys + (sp * P + p) * a.d + i4);
+      v[0] += o.x;
+      v[1] += o.y;
+      v[2] += o.z;
+      v[3] += o.w;
+    }
   }
   uint2 out;
   out.x = (uint32_t)f32_to_bf16_rne(v[0]) | ((uint32_t)f32_to_bf16_rne(v[1]) << 16);
@@ -710,8 +720,8 @@ int launch_route(const FwdArgs& a_in) {
   ++n;
   const int P = a.T * a.k;
   ev_before(a);
-  if (launch_kernel(tile_scales_kernel, dim3(std::min((P + 7) / 8, 148 * 16)), dim3(256), 0, a.stream, a.pdl != 0,
-                    a) != cudaSuccess)
+  if (launch_kernel(pack_kernel, dim3(std::min((P + 7) / 8, 148 * 16)), dim3(256), 0, a.stream, a.pdl != 0, a) !=
+      cudaSuccess)
     return -1;
   ev_after(a);
   ++n;

@@ -150,32 +150,38 @@ def test_forward_parity(name, path):
 
 
 def _h_from_workspace(g, cfg):
-    """h [P, I] (sorted pairs) rebuilt from the workspace's E4M3 hi / lo rows and the
-    token tiles' scale-factor groups."""
+    """h [P, I] (sorted pairs) rebuilt from the down GEMM's packed activation blocks: per
+    token tile and 128-chunk, 2*BN E4M3 rows (row n = hi / lo term of token n // 2, 16-byte
+    unit u stored at unit u ^ (n % 8)), then the scale-factor groups (byte
+    (n%32)*16 + ((n%128)//32)*4 + b%4 of group n // 128 for 32-block b)."""
     dims, ws, T = g["dims"], g["ws"], cfg.T
     P = T * cfg.k
     Ip = moe.kpad128(cfg.I)
+    KC = Ip // 128
     bt = TILE_TOKENS[moe.resolved_path(dims, T)]
     G = (2 * bt + 127) // 128
+    BB = (2 * bt * 128 + G * 512 + 1023) // 1024 * 1024
     view = lambda f, dt, sh: moe.workspace_view(ws, dims, T, f, dt, sh).cpu().numpy()
-    hq = view("hq", torch.uint8, (2 * P, Ip))[:, :cfg.I]
     offsets = view("offsets", torch.int32, (cfg.E + 1,))
     tbase = view("tile_base", torch.int32, (cfg.E,))
     n_tiles = (P + bt - 1) // bt + cfg.E
-    sfh = view("sfh", torch.uint8, (n_tiles, Ip // 128, G, 512))
+    bph = view("bph", torch.uint8, (n_tiles, KC, BB))
     h = np.empty((P, cfg.I))
     b = np.arange(cfg.I // 32)
+    u = np.arange(8)
     for p in range(P):
         e = int(np.searchsorted(offsets, p, side="right") - 1)
         j = p - offsets[e]
         tile, col = tbase[e] + j // bt, j % bt
-        sc = []
+        terms = []
         for n in (2 * col, 2 * col + 1):
-            byte = (n % 32) * 16 + ((n % 128) // 32) * 4 + b % 4
-            sc.append(sfh[tile, b // 4, n // 128, byte].astype(np.float64) - 127)
-        s_hi = np.repeat(np.exp2(sc[0]), 32)
-        s_lo = np.repeat(np.exp2(sc[1]), 32)
-        h[p] = decode_e4m3(hq[2 * p]) * s_hi + decode_e4m3(hq[2 * p + 1]) * s_lo
+            phys = n * 128 + ((u ^ (n % 8)) << 4)                                    # [8]
+            rows = bph[tile][:, (phys[:, None] + np.arange(16)[None, :]).ravel()]     # [KC, 128]
+            codes = rows.reshape(-1)[: cfg.I]
+            sfo = 2 * bt * 128 + (n // 128) * 512 + (n % 32) * 16 + ((n % 128) // 32) * 4 + b % 4
+            sc = bph[tile, b // 4, sfo].astype(np.float64) - 127
+            terms.append(decode_e4m3(codes) * np.repeat(np.exp2(sc), 32))
+        h[p] = terms[0] + terms[1]
     return h
 
 
