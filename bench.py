@@ -330,7 +330,7 @@ def run_ours(args, rank, world, local_rank):
         with torch.cuda.graph(kgraph):
             step(kev[0])
     n_timed = moe.last_launch_count()
-    names = KERNELS if n_timed == len(KERNELS) else ["route", "gate_up", "down"]
+    names = KERNELS if n_timed == len(KERNELS) else ["route", "pack", "gate_up", "down"]
     per_kernel = {name: [] for name in names[:n_timed]}
     for i in range(K):
         flush.zero_()

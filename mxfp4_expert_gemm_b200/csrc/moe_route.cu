@@ -150,31 +150,29 @@ __device__ __forceinline__ void warp_topk_softmax(float (&l)[NJ], int E, int k, 
 }
 
 // ----------------------------------------------------------------------------------
-// Grouping (and the tile packing) for a small batch, run by the routing CTA that finished last
+// Grouping for a small batch, run by the routing CTA that finished last
 // (all others have published their top-k, counts and xq rows before taking a ticket).
 // Pairs are listed per expert in token order: one warp walks the tokens in order and
 // hands each of a token's k (distinct) experts the next free position of that expert.
 // Deterministic: positions depend on counts and token order only.
 // ----------------------------------------------------------------------------------
-// Token t's E4M3 rows (hi, lo) and their scales into the packed blocks of token tile
-// `tile`, MMA columns 2*col (hi) and 2*col + 1 (lo).  One warp.
-__device__ __forceinline__ void pack_pair(const FwdArgs& a, int t, int tile, int col) {
+// Chunk c of token t's E4M3 rows (hi, lo) and their scales into the packed block of
+// token tile `tile`, MMA columns 2*col (hi) and 2*col + 1 (lo).  One warp: lanes 0-15
+// move the 16 16-byte units, lanes 16-23 the eight scale bytes.
+__device__ __forceinline__ void pack_pair_chunk(const FwdArgs& a, int t, int tile, int col, int c) {
   const int lane = threadIdx.x & 31;
   const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk;
-  const int bb = packed_block_bytes(bt);
-  uint8_t* blocks = a.ws.bpx + (int64_t)tile * kc * bb;
-  const uint8_t* rows = a.ws.xq + (int64_t)t * 2 * dp;
-  // 16-byte units: chunk c, term, unit u (the units past d are never read by the MMAs)
-  for (int i = lane; i < kc * 16; i += 32) {
-    const int c = i >> 4, term = (i >> 3) & 1, u = i & 7;
-    const int n = 2 * col + term;
-    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(rows + term * dp + c * kKChunk) + u);
-    *reinterpret_cast<uint4*>(blocks + (int64_t)c * bb + packed_unit_offset(n, u)) = v;
-  }
-  const uint8_t* sf = a.ws.xsf + (int64_t)t * 2 * (dp / 32);
-  for (int i = lane; i < 2 * nb; i += 32) {
-    const int term = i / nb, b = i - term * nb;
-    blocks[(int64_t)(b / 4) * bb + packed_sf_offset(bt, 2 * col + term, b)] = __ldcg(sf + term * (dp / 32) + b);
+  uint8_t* block = a.ws.bpx + ((int64_t)tile * kc + c) * packed_block_bytes(bt);
+  if (lane < 16) {   // (units past d are never read by the MMAs)
+    const int term = lane >> 3, u = lane & 7;
+    const uint4 v =
+        __ldcg(reinterpret_cast<const uint4*>(a.ws.xq + (int64_t)t * 2 * dp + term * dp + c * kKChunk) + u);
+    *reinterpret_cast<uint4*>(block + packed_unit_offset(2 * col + term, u)) = v;
+  } else if (lane < 24) {
+    const int term = (lane - 16) >> 2, b = 4 * c + ((lane - 16) & 3);
+    if (b < nb)
+      block[packed_sf_offset(bt, 2 * col + term, b)] =
+          __ldcg(a.ws.xsf + (int64_t)t * 2 * (dp / 32) + term * (dp / 32) + b);
   }
 }
 
@@ -259,18 +257,6 @@ __device__ void group_block(const FwdArgs& a, int tile_tokens) {
     a.ws.perm[pos] = q;
     a.ws.inv[q] = pos;
     a.ws.w_sorted[pos] = __ldcg(a.ws.topk_w + q);
-  }
-  __syncthreads();
-  for (int pos = tid; pos < P; pos += blockDim.x) {
-    const int v = s_perm_e[pos];
-    s_perm_tok[pos] = (v >> 9) / k;
-    s_perm_e[pos] = v & 511;
-  }
-  __syncthreads();
-  // packed activation blocks per token tile, one warp per pair
-  for (int p = warp; p < P; p += blockDim.x >> 5) {
-    const int e = s_perm_e[p], j = p - s_off[e];
-    pack_pair(a, s_perm_tok[p], s_tb[e] + j / tile_tokens, j % tile_tokens);
   }
 }
 
@@ -388,29 +374,82 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
 }
 
 // ----------------------------------------------------------------------------------
-// Fused RMSNorm + router GEMV + top-k + softmax, 32 tokens per CTA, 256 threads.
-// Outputs: xq / xsf (E4M3 terms of bf16(xn)), topk_idx, topk_w, expert histogram.
+// Large batches: fused RMSNorm + router + top-k + softmax, kRT tokens per CTA, 256
+// threads.  The reduction axis is walked in chunks of RK through a ring of kNS cp.async
+// stages, each holding the chunk's bf16 x rows of the CTA's tokens and the router rows
+// [E][RK] (fp32, rows padded by 4 floats so that the float4 reads of 32 consecutive
+// experts hit distinct banks).  Per chunk, warp w first normalizes tokens 2w and 2w + 1
+// (xn = x / rms * gamma, fp32) and stores their E4M3 hi / lo terms and scales; then warp
+// w takes the chunk's columns [RK/8 w, RK/8 (w + 1)): each lane keeps those router
+// values of its experts (lane + 32 j) in registers and accumulates them against every
+// token's xn (broadcast reads).  The eight warps' partial logits are added at the end
+// in warp order.  Outputs: xq / xsf, topk_idx, topk_w, expert histogram.
 // ----------------------------------------------------------------------------------
-constexpr int RT = 32;   // tokens per CTA (tiled kernel)
-constexpr int kTokenKernelMaxT = 1024;  // up to this many tokens: one CTA per token
-constexpr int RK = 64;   // d-chunk
+constexpr int kRT = 16;                  // tokens per CTA
+constexpr int kNS = 4;                   // cp.async stages
+constexpr int kTokenKernelMaxT = 256;    // up to this many tokens: one CTA per token
 
-template <int NJ>  // experts per lane group: E <= 32*NJ
-__global__ void __launch_bounds__(256) route_kernel(FwdArgs a) {
-  extern __shared__ float smem[];
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int NJ, int RK>
+struct RouteTilesCfg {
+  static constexpr int EP = 32 * NJ;
+  static constexpr int WST = RK + 4;                       // router row stride (floats)
+  static constexpr int W_FLOATS = EP * WST;                // one stage of router rows
+  static constexpr int X_HALVES = kRT * RK;                // one stage of x (bf16)
+  static constexpr int KW = RK / 8;                        // columns of a chunk per warp
+  static constexpr size_t STAGES = sizeof(float) * (kNS * W_FLOATS + kRT * RK) + 2 * kNS * X_HALVES;
+  // RMSNorm weights (d floats) follow the stages / partials
+  static constexpr size_t PARTIALS = sizeof(float) * 8 * kRT * EP;   // final reduction (reuses the stages)
+  static constexpr size_t MAIN = STAGES > PARTIALS ? STAGES : PARTIALS;
+  static size_t smem(int d) { return MAIN + sizeof(float) * (size_t)d; }
+  static_assert(KW % 4 == 0, "float4 columns per warp");
+};
+
+template <int NJ, int RK>
+__global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
+  using C = RouteTilesCfg<NJ, RK>;
+  extern __shared__ __align__(16) float smem[];
+  float* s_w = smem;                                        // [kNS][EP][WST]
+  float* s_xn = smem + kNS * C::W_FLOATS;                   // [kRT][RK]
+  uint16_t* s_x = reinterpret_cast<uint16_t*>(s_xn + kRT * RK);  // [kNS][kRT][RK]
+  float* s_g = smem + C::MAIN / sizeof(float);             // [d] RMSNorm weights
+  __shared__ float s_r[kRT];
   pdl_trigger();
   const int E = a.E, d = a.d, k = a.k;
-  const int EP = 32 * NJ;
-  float* s_r = smem;                         // [RT]
-  float* s_x = s_r + RT;                     // [RT][RK+1]
-  float* s_w = s_x + RT * (RK + 1);          // [RK][EP+1]
-  float* s_l = s_w + RK * (EP + 1);          // [RT][EP+1]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = blockIdx.x * RT;
-  const int nt = min(RT, a.T - t0);
+  const int t0 = blockIdx.x * kRT;
+  const int nt = min(kRT, a.T - t0);
+  const int nchunks = d / RK;
+  const int dp = a.ws.dp;
 
-  // Phase A: 1/rms per token (warp w: tokens w, w+8, ...).
-  for (int tt = warp; tt < RT; tt += 8) {
+  auto issue = [&](int c) {   // chunk c into stage c % kNS
+    const int st = c % kNS, k0 = c * RK;
+    for (int i = tid; i < kRT * (RK / 8); i += 256) {   // x: 16-byte pieces
+      const int tt = i / (RK / 8), q = i - tt * (RK / 8);
+      if (tt < nt) cp_async16(s_x + (st * kRT + tt) * RK + q * 8, a.x + (int64_t)(t0 + tt) * d + k0 + q * 8);
+    }
+    for (int i = tid; i < E * (RK / 4); i += 256) {     // router rows: 16-byte pieces
+      const int e = i / (RK / 4), q = i - e * (RK / 4);
+      cp_async16(s_w + (st * C::EP + e) * C::WST + q * 4, a.router_w + (int64_t)e * d + k0 + q * 4);
+    }
+  };
+  for (int c = 0; c < kNS - 1; ++c) {
+    if (c < nchunks) issue(c);
+    cp_async_commit();
+  }
+
+  for (int i = tid * 4; i < d; i += 256 * 4) *reinterpret_cast<float4*>(s_g + i) = *reinterpret_cast<const float4*>(a.norm_w + i);
+  // 1 / rms of the warp's two tokens (overlaps the first chunks' copies)
+  for (int h = 0; h < 2; ++h) {
+    const int tt = 2 * warp + h;
     float ss = 0.f;
     if (tt < nt) {
       const uint16_t* xr = a.x + (int64_t)(t0 + tt) * d;
@@ -429,100 +468,103 @@ __global__ void __launch_bounds__(256) route_kernel(FwdArgs a) {
     for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) s_r[tt] = 1.0f / sqrtf(ss / (float)d + a.eps);
   }
-  __syncthreads();
+  __syncwarp();
 
-  // Phase B: router logits, d in chunks of RK.  Thread = (token group tg of 4, lane).
-  const int tg = warp;  // tokens 4*tg .. 4*tg+3
-  float acc[4][NJ];
+  float acc[kRT][NJ];   // partial logits of this warp's columns, all tokens
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int t = 0; t < kRT; ++t)
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < NJ; ++j) acc[t][j] = 0.f;
 
-  // Register prefetch of the next d-chunk overlaps its global loads with the FMAs.
-  constexpr int XQ = RT * (RK / 2) / 256;   // bf16 pairs of x per thread per chunk
-  constexpr int WQ = RK * 32 * NJ / 256;    // router weights per thread per chunk
-  uint32_t px[XQ];
-  float pw[WQ];
-  auto load_chunk = [&](int k0) {
+  for (int c = 0; c < nchunks; ++c) {
+    if (c + kNS - 1 < nchunks) issue(c + kNS - 1);
+    cp_async_commit();
+    cp_async_wait<kNS - 1>();
+    __syncthreads();
+    const int st = c % kNS, k0 = c * RK;
+    // normalize this warp's tokens, split into E4M3 terms (warp-private rows of s_xn)
 #pragma unroll
-    for (int u = 0; u < XQ; ++u) {
-      const int q = tid + 256 * u;
-      const int tt = q / (RK / 2), c2 = (q % (RK / 2)) * 2;
-      px[u] = (tt < nt) ? *reinterpret_cast<const uint32_t*>(a.x + (int64_t)(t0 + tt) * d + k0 + c2) : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < WQ; ++u) {
-      const int q = tid + 256 * u;
-      const int e = q / RK, kk = q % RK;
-      pw[u] = (e < E) ? a.router_w[(int64_t)e * d + k0 + kk] : 0.f;
-    }
-  };
-  load_chunk(0);
-  for (int k0 = 0; k0 < d; k0 += RK) {
-#pragma unroll
-    for (int u = 0; u < XQ; ++u) {
-      const int q = tid + 256 * u;
-      const int tt = q / (RK / 2), c2 = (q % (RK / 2)) * 2;
-      float v0 = 0.f, v1 = 0.f;
-      if (tt < nt) {  // uniform per warp: a warp covers one token's 64 values
+    for (int h = 0; h < 2; ++h) {
+      const int tt = 2 * warp + h;
+      if (tt < nt) {   // uniform per warp
         const float r = s_r[tt];
-        v0 = __uint_as_float(px[u] << 16) * r * a.norm_w[k0 + c2];
-        v1 = __uint_as_float(px[u] & 0xFFFF0000u) * r * a.norm_w[k0 + c2 + 1];
-        const float v[2] = {bf16_to_f32(f32_to_bf16_rne(v0)), bf16_to_f32(f32_to_bf16_rne(v1))};
-        uint32_t hi, lo, s1, s2;
-        e4m3_split<2>(v, hi, lo, s1, s2);   // lanes 0-15: block k0/32, lanes 16-31: the next
-        const int dp = a.ws.dp;
         uint8_t* xq = a.ws.xq + (int64_t)(t0 + tt) * 2 * dp;
-        *reinterpret_cast<uint16_t*>(xq + k0 + c2) = (uint16_t)hi;
-        *reinterpret_cast<uint16_t*>(xq + dp + k0 + c2) = (uint16_t)lo;
-        if ((lane & 15) == 0) {
-          uint8_t* sf = a.ws.xsf + (int64_t)(t0 + tt) * 2 * (dp / 32);
-          const int b = (k0 + c2) / 32;
-          sf[b] = (uint8_t)s1;
-          sf[dp / 32 + b] = (uint8_t)s2;
+        uint8_t* sf = a.ws.xsf + (int64_t)(t0 + tt) * 2 * (dp / 32);
+        if (RK == 64) {
+          const int kk = 2 * lane;
+          const uint32_t pr = *reinterpret_cast<const uint32_t*>(s_x + (st * kRT + tt) * RK + kk);
+          const float v0 = __uint_as_float(pr << 16) * r * s_g[k0 + kk];
+          const float v1 = __uint_as_float(pr & 0xFFFF0000u) * r * s_g[k0 + kk + 1];
+          s_xn[tt * RK + kk] = v0;
+          s_xn[tt * RK + kk + 1] = v1;
+          const float v[2] = {bf16_to_f32(f32_to_bf16_rne(v0)), bf16_to_f32(f32_to_bf16_rne(v1))};
+          uint32_t hi, lo, s1, s2;
+          e4m3_split<2>(v, hi, lo, s1, s2);   // lanes 0-15: block k0/32, 16-31: the next
+          *reinterpret_cast<uint16_t*>(xq + k0 + kk) = (uint16_t)hi;
+          *reinterpret_cast<uint16_t*>(xq + dp + k0 + kk) = (uint16_t)lo;
+          if ((lane & 15) == 0) {
+            sf[(k0 + kk) / 32] = (uint8_t)s1;
+            sf[dp / 32 + (k0 + kk) / 32] = (uint8_t)s2;
+          }
+        } else {   // RK == 32: one 32-block per chunk, one value per lane
+          const float v0 = bf16_to_f32(s_x[(st * kRT + tt) * RK + lane]) * r * s_g[k0 + lane];
+          s_xn[tt * RK + lane] = v0;
+          const float v[1] = {bf16_to_f32(f32_to_bf16_rne(v0))};
+          uint32_t hi, lo, s1, s2;
+          e4m3_split<1>(v, hi, lo, s1, s2);
+          xq[k0 + lane] = (uint8_t)hi;
+          xq[dp + k0 + lane] = (uint8_t)lo;
+          if (lane == 0) {
+            sf[k0 / 32] = (uint8_t)s1;
+            sf[dp / 32 + k0 / 32] = (uint8_t)s2;
+          }
         }
       }
-      s_x[tt * (RK + 1) + c2] = v0;
-      s_x[tt * (RK + 1) + c2 + 1] = v1;
     }
+    __syncthreads();   // every warp's xn rows of this chunk are in place
+    // acc[t][j] += router_w[lane + 32 j][columns of warp w] . xn[t][same columns]
+    const float* wst = s_w + st * C::W_FLOATS;
+    const int kw = warp * C::KW;
 #pragma unroll
-    for (int u = 0; u < WQ; ++u) {
-      const int q = tid + 256 * u;
-      const int e = q / RK, kk = q % RK;
-      s_w[kk * (EP + 1) + e] = pw[u];
-    }
-    __syncthreads();
-    if (k0 + RK < d) load_chunk(k0 + RK);
-#pragma unroll 4
-    for (int kk = 0; kk < RK; ++kk) {
-      float xv[4];
+    for (int q = 0; q < C::KW; q += 4) {
+      float4 w4[NJ];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) xv[i] = s_x[(4 * tg + i) * (RK + 1) + kk];
+      for (int j = 0; j < NJ; ++j) w4[j] = *reinterpret_cast<const float4*>(wst + (lane + 32 * j) * C::WST + kw + q);
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const float wv = s_w[kk * (EP + 1) + lane + 32 * j];
+      for (int t = 0; t < kRT; ++t) {
+        const float4 xv = *reinterpret_cast<const float4*>(s_xn + t * RK + kw + q);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(xv[i], wv, acc[i][j]);
+        for (int j = 0; j < NJ; ++j)
+          acc[t][j] = fmaf(w4[j].x, xv.x, fmaf(w4[j].y, xv.y, fmaf(w4[j].z, xv.z, fmaf(w4[j].w, xv.w, acc[t][j]))));
       }
     }
-    __syncthreads();
+    __syncthreads();   // stage st and the xn rows are refilled by the next iteration
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      const int e = lane + 32 * j;
-      s_l[(4 * tg + i) * (EP + 1) + e] = (e < E) ? acc[i][j] + (a.router_b ? a.router_b[e] : 0.f) : -INFINITY;
-    }
-  __syncthreads();
+  cp_async_wait<0>();
 
-  // Phase C: top-k + softmax per token (warp w: tokens w, w+8, ...).
-  for (int tt = warp; tt < nt; tt += 8) {
-    float l[NJ];
+  // add the warps' partial logits in warp order (router stages reused: [8][kRT][EP])
+  float* s_part = s_w;
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) l[j] = s_l[tt * (EP + 1) + lane + 32 * j];
-    warp_topk_softmax<NJ>(l, E, k, t0 + tt, a);
+  for (int t = 0; t < kRT; ++t)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) s_part[(warp * kRT + t) * C::EP + lane + 32 * j] = acc[t][j];
+  __syncthreads();
+  // top-k + softmax: warp w takes tokens 2w and 2w + 1 (lane holds experts lane + 32 j)
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int tt = 2 * warp + h;
+    if (tt < nt) {
+      float l[NJ];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int e = lane + 32 * j;
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) v += s_part[(w * kRT + tt) * C::EP + e];
+        l[j] = (e < E) ? v + (a.router_b ? a.router_b[e] : 0.f) : -INFINITY;
+      }
+      warp_topk_softmax<NJ>(l, E, k, t0 + tt, a);
+    }
   }
 }
 
@@ -602,17 +644,66 @@ __global__ void __launch_bounds__(1024) group_kernel(FwdArgs a, int tile_tokens)
   }
 }
 
-// Every pair's activation rows and scales into its token tile's packed blocks.  One warp
-// per pair.
+// All chunks of token t's rows and scales into token tile `tile`'s packed blocks.  One
+// warp; each lane keeps four 16-byte copies in flight.
+__device__ __forceinline__ void pack_pair(const FwdArgs& a, int t, int tile, int col) {
+  const int lane = threadIdx.x & 31;
+  const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk;
+  const int bb = packed_block_bytes(bt);
+  uint8_t* blocks = a.ws.bpx + (int64_t)tile * kc * bb;
+  const uint8_t* rows = a.ws.xq + (int64_t)t * 2 * dp;
+  const int units = kc * 16;   // (chunk, term, unit); units past d are never read by the MMAs
+  for (int i0 = lane; i0 < units; i0 += 128) {
+    uint4 v[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int i = i0 + 32 * r;
+      if (i < units) {
+        const int c = i >> 4, term = (i >> 3) & 1, u = i & 7;
+        v[r] = __ldcg(reinterpret_cast<const uint4*>(rows + term * dp + c * kKChunk) + u);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int i = i0 + 32 * r;
+      if (i < units) {
+        const int c = i >> 4, term = (i >> 3) & 1, u = i & 7;
+        *reinterpret_cast<uint4*>(blocks + (int64_t)c * bb + packed_unit_offset(2 * col + term, u)) = v[r];
+      }
+    }
+  }
+  const uint8_t* sf = a.ws.xsf + (int64_t)t * 2 * (dp / 32);
+  for (int i = lane; i < 2 * nb; i += 32) {
+    const int term = i / nb, b = i - term * nb;
+    blocks[(int64_t)(b / 4) * bb + packed_sf_offset(bt, 2 * col + term, b)] = __ldcg(sf + term * (dp / 32) + b);
+  }
+}
+
+constexpr int64_t kPackChunkTasksMax = 1 << 16;   // up to this many (pair, chunk) tasks: one warp each
+
+// Every pair's activation rows and scales into its token tile's packed blocks: one warp
+// per (pair, 128-chunk) for small batches, one warp per pair otherwise.
 __global__ void pack_kernel(FwdArgs a) {
   pdl_trigger();
   pdl_wait();
-  const int P = a.T * a.k, bt = a.ws.tile_tokens;
-  for (int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x >> 5)) {
+  const int P = a.T * a.k, bt = a.ws.tile_tokens, kc = a.ws.dp / kKChunk;
+  if ((int64_t)P * kc > kPackChunkTasksMax) {
+    for (int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x >> 5)) {
+      const int q = a.ws.perm[p];
+      const int e = a.ws.topk_idx[q];
+      const int j = p - a.ws.offsets[e];
+      pack_pair(a, q / a.k, a.ws.tile_base[e] + j / bt, j % bt);
+    }
+    return;
+  }
+  const int64_t tasks = (int64_t)P * kc;
+  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < tasks;
+       w += (int64_t)gridDim.x * (blockDim.x >> 5)) {
+    const int p = (int)(w / kc), c = (int)(w - (int64_t)p * kc);
     const int q = a.ws.perm[p];
     const int e = a.ws.topk_idx[q];
     const int j = p - a.ws.offsets[e];
-    pack_pair(a, q / a.k, a.ws.tile_base[e] + j / bt, j % bt);
+    pack_pair_chunk(a, q / a.k, a.ws.tile_base[e] + j / bt, j % bt, c);
   }
 }
 
@@ -670,11 +761,12 @@ int launch_route_nj(const FwdArgs& a) {
     ev_after(a);
     return 1;
   }
-  const int EP = 32 * NJ;
-  const size_t smem = sizeof(float) * (RT + RT * (RK + 1) + RK * (EP + 1) + RT * (EP + 1));
-  if (!ensure_smem_limit(route_kernel<NJ>, smem, tile_limits)) return -1;
+  constexpr int RKC = NJ <= 2 ? 64 : 32;   // chunk: router rows of a stage stay small
+  using C = RouteTilesCfg<NJ, RKC>;
+  const size_t smem = C::smem(a.d);
+  if (!ensure_smem_limit(route_tiles_kernel<NJ, RKC>, smem, tile_limits)) return -1;
   ev_before(a);
-  route_kernel<NJ><<<(a.T + RT - 1) / RT, 256, smem, a.stream>>>(a);
+  route_tiles_kernel<NJ, RKC><<<(a.T + kRT - 1) / kRT, 256, smem, a.stream>>>(a);
   ev_after(a);
   return 1;
 }
@@ -712,16 +804,18 @@ int launch_route(const FwdArgs& a_in) {
   else r = launch_route_nj<8>(a);
   if (r < 0) return -1;
   n += r;
-  if (a.fuse_group) return cudaGetLastError() == cudaSuccess ? n : -1;
+  if (!a.fuse_group) {
+    ev_before(a);
+    if (launch_kernel(group_kernel, dim3(a.E), dim3(1024), 0, a.stream, a.pdl != 0, a, tile_tokens) != cudaSuccess)
+      return -1;
+    ev_after(a);
+    ++n;
+  }
+  const int64_t P = (int64_t)a.T * a.k, tasks = P * (a.ws.dp / kKChunk);
+  const int64_t warps = tasks > kPackChunkTasksMax ? P : tasks;   // one warp per task (pack_kernel)
   ev_before(a);
-  if (launch_kernel(group_kernel, dim3(a.E), dim3(1024), 0, a.stream, a.pdl != 0, a, tile_tokens) != cudaSuccess)
-    return -1;
-  ev_after(a);
-  ++n;
-  const int P = a.T * a.k;
-  ev_before(a);
-  if (launch_kernel(pack_kernel, dim3(std::min((P + 7) / 8, 148 * 16)), dim3(256), 0, a.stream, a.pdl != 0, a) !=
-      cudaSuccess)
+  if (launch_kernel(pack_kernel, dim3((unsigned)std::min<int64_t>((warps + 7) / 8, 148 * 32)), dim3(256), 0, a.stream,
+                    a.pdl != 0, a) != cudaSuccess)
     return -1;
   ev_after(a);
   ++n;

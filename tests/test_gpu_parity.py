@@ -26,6 +26,9 @@ SMALL = {
     "wide_E": synth.MoEConfig("wide_E", T=16, d=256, I=128, E=256, k=8),
     "mid_ragged": synth.MoEConfig("mid_ragged", T=200, d=2880, I=2880, E=8, k=4),
     "clamp": synth.MoEConfig("clamp", T=32, d=2880, I=2880, E=4, k=2, w1_mul=8.0),
+    # more than 256 tokens: the tiled router (64- and 32-wide chunks)
+    "tiled_route": synth.MoEConfig("tiled_route", T=333, d=256, I=128, E=64, k=4),
+    "tiled_wide_E": synth.MoEConfig("tiled_wide_E", T=300, d=256, I=128, E=256, k=8),
 }
 PATHS = ["gemv", "gemm"]
 
@@ -310,8 +313,8 @@ def test_non_finite_input_is_reported():
 def test_launch_count_reported():
     c = case(SMALL["tiny"])
     cfg = c["cfg"]
-    for path, n in (("gemm", 6),   # route, group, gather, gate_up, down, combine
-                    ("gemv", 3)):  # route (+ grouping + gather), gate_up, down (+ combine)
+    for path, n in (("gemm", 6),   # route, group, pack, gate_up, down, combine
+                    ("gemv", 4)):  # route (+ grouping), pack, gate_up, down (+ combine)
         dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path=path)
         ws = moe.new_workspace(dims, cfg.T)
         moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws)
