@@ -196,8 +196,8 @@ int32_t moe_resolve_path(const moe_dims* dims, int32_t T);
  *     and 128-chunk: the tile's 2 * BN E4M3 rows (hi / lo term of each token) in the
  *     tensor cores' 128-byte-swizzled order, then their scales (BN = 8 on the GEMV path,
  *     96 on the GEMM path),
- * ys  [S][T*k][d] fp32 (weighted expert outputs, sorted order; S = 2 partial sums on the
- *     GEMV path, whose down GEMM splits its reduction axis in two, else 1);
+ * ys  [S][T*k][d] fp32 (weighted expert outputs, sorted order; S = 3 planes of partial sums
+ *     on the GEMV path, whose down GEMM splits its reduction axis in up to three, else 1);
  * offsets[MOE_WS_FIELDS-1] = total bytes.  Errors: MOE_ERR_INVALID_ARG,
  * MOE_ERR_UNSUPPORTED_SHAPE. */
 #define MOE_WS_FIELDS 17
@@ -223,7 +223,7 @@ int32_t moe_last_launch_count(void);
  * implicit synchronization once it is running -- use it instead of moe_forward.
  * Scratch: a fixed 16 MiB array in the library's own device memory, present on every GPU
  * that loads the library until the process exits.  T whose moe_workspace_bytes() exceed
- * 16 MiB is rejected with MOE_ERR_WORKSPACE (at d = I = 2880, E = 32, top-4: up to 119
+ * 16 MiB is rejected with MOE_ERR_WORKSPACE (at d = I = 2880, E = 32, top-4: up to 56
  * tokens).
  * The first call on a device looks up the array's device address for that device
  * (cudaGetSymbolAddress); make that first call before any stream capture.

@@ -60,7 +60,7 @@ struct MxParams {
   int32_t K;               // reduction length (d for gate_up, I for down)
   int32_t KC;              // 128-chunks of the reduction axis (K rounded up)
   int32_t n_rt;            // row tiles per token tile: I/64 (gate_up) or ceil(d/128) (down)
-  int32_t ksplit;          // reduction-axis splits per (token tile, row tile) (down only; >= 1)
+  int32_t ksplit_max;      // reduction-axis splits per (token tile, row tile) allowed (down only)
   int32_t P;               // pairs (rows of ys per split)
   int32_t* status;
   float limit;
@@ -111,7 +111,8 @@ struct MxCfg {
                                    : COLS_NEEDED <= 256 ? 256 : 512;
   static constexpr int EPI_GROUP_BYTES = TC * 64 * 4 + TC * 4;  // g / u exchange; token list (down)
   static constexpr int EPI_BYTES = EG * EPI_GROUP_BYTES;
-  static constexpr int BAR_BYTES = 8 * (2 * S + 5) + 16;
+  static constexpr int NISS = NPW;                      // copy issuers per stage, one barrier each
+  static constexpr int BAR_BYTES = 8 * ((NISS + 1) * S + 5) + 16;
   static constexpr int SMEM_BYTES = S * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024 /*align slack*/;
   static constexpr int EPI_THREADS = 128 * EG;
   static constexpr int MMA_WARP = NPW;                // warps 0..NPW-1 produce
@@ -122,7 +123,7 @@ struct MxCfg {
   static_assert(SMEM_BYTES * CPS <= 227 * 1024, "shared memory budget of CPS co-resident CTAs");
   static_assert(kBM * NP <= 256, "TMA box height");
   static_assert(EG == 1 || EG == 2, "one or two epilogue warpgroups");
-  static_assert(NPW >= 1 && NPW <= 4, "producer warps");
+  static_assert(NPW >= 1 && NPW <= 3, "producer warps: one per kind of copy at most");
 };
 
 // Work item i: token tile tt, row tile rt, and the chunk range [kc0, kc1) of split ks.
@@ -130,15 +131,23 @@ struct Item {
   int tt, rt, ks, kc0, kc1;
 };
 
-__device__ __forceinline__ Item item_of(const MxParams& p, int i) {
+__device__ __forceinline__ Item item_of(const MxParams& p, int i, int ksplit) {
   Item it;
-  const int r = i / p.ksplit;
-  it.ks = i - r * p.ksplit;
+  const int r = i / ksplit;
+  it.ks = i - r * ksplit;
   it.tt = r / p.n_rt;
   it.rt = r - it.tt * p.n_rt;
-  it.kc0 = it.ks * p.KC / p.ksplit;
-  it.kc1 = (it.ks + 1) * p.KC / p.ksplit;
+  it.kc0 = it.ks * p.KC / ksplit;
+  it.kc1 = (it.ks + 1) * p.KC / ksplit;
   return it;
+}
+
+// Splits of the reduction axis for n0 (token tile, row tile) units over `grid` CTAs: the
+// fewest (at most smax) that give every CTA two items, so that one item's epilogue runs
+// under the next item's loads (the accumulator is double-buffered).
+__device__ __forceinline__ int choose_ksplit(int n0, int grid, int smax) {
+  if (n0 <= 0) return 1;
+  return max(1, min(smax, (2 * grid + n0 - 1) / n0));
 }
 
 template <int BN, int NP, int S, int CPS, int EG, int NPW, int MODE>
@@ -150,8 +159,8 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* epi = smem + S * C::STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(epi + C::EPI_BYTES);
-  uint64_t* sfree = full + S;       // stage consumed (its MMAs done)
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi + C::EPI_BYTES);   // [S][NISS] copies landed
+  uint64_t* sfree = full + S * C::NISS;   // stage consumed (its MMAs done)
   uint64_t* accf = sfree + S;       // [2] accumulator ready
   uint64_t* acce = accf + 2;        // [2] accumulator drained by the epilogue
   uint64_t* drain = acce + 2;       // final MMA drain
@@ -163,7 +172,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      ptx::mbar_init(&full[s], 1);
+      for (int w = 0; w < C::NISS; ++w) ptx::mbar_init(&full[s * C::NISS + w], 1);
       ptx::mbar_init(&sfree[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -185,7 +194,9 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
   const uint32_t tmem = *s_tmem;
   // Everything above overlaps the previous kernel; the work list is its output.
   pdl_wait();
-  const int n_items = *p.ntiles * p.n_rt * p.ksplit;
+  const int n_units = *p.ntiles * p.n_rt;
+  const int ksplit = choose_ksplit(n_units, (int)gridDim.x, p.ksplit_max);   // same in every CTA
+  const int n_items = n_units * ksplit;
 
   auto a_s = [&](int s) { return smem + s * C::STAGE_BYTES; };
   auto b_s = [&](int s) { return smem + s * C::STAGE_BYTES + C::B_OFF; };
@@ -193,17 +204,18 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
 
   if (warp < NPW) {
     // ------------------------------------------------------------------ producers
-    // Producer warp w fills the stages g with g % NPW == w; the warp waits converged and
-    // lane 0 issues the three copies of a stage.
+    // Every stage takes three copies: the weight box (TMA), the activation block and the
+    // weight scale factors (bulk).  Producer warp w issues the kinds k with k % NPW == w on
+    // its own barrier full[s][w], so that one warp's copies do not queue behind another's;
+    // the warp waits converged and lane 0 issues.
     int64_t g = 0;  // global stage counter of this CTA
     bool stop = false, withheld = false;
     for (int i = blockIdx.x; i < n_items && !stop; i += gridDim.x) {
-      const Item it = item_of(p, i);
+      const Item it = item_of(p, i, ksplit);
       const int tt = it.tt, rt = it.rt;
       const int nst = (it.kc1 - it.kc0 + NP - 1) / NP;   // stages of this item
       const Tile tl = p.tiles[tt];
       for (int st = 0; st < nst; ++st, ++g) {
-        if ((int)(g % NPW) != warp) continue;
         const int s = (int)(g % S);
         bool ok = true;
         if (g >= S) ok = ptx::mbar_wait_bounded(&sfree[s], (uint32_t)((g / S) - 1) & 1, s_abort, kWaitLimitNs);
@@ -217,23 +229,28 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
         }
         const int c0 = it.kc0 + st * NP, nck = min(NP, it.kc1 - c0);
         if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(&full[s], C::A_TX + nck * (C::B_BLOCK + kSfGroupBytes));
-          ptx::tma_load_2d(a_s(s), &tm_w, 0, (int)(((int64_t)tl.e * p.NT + rt) * p.KC + c0) * kBM, &full[s]);
-          ptx::bulk_load(b_s(s), p.bp_in + ((int64_t)tt * p.KC + c0) * C::B_BLOCK, nck * C::B_BLOCK, &full[s]);
-          ptx::bulk_load(sfa_s(s), p.w_sf + ((int64_t)(tl.e * p.NT + rt) * p.KC + c0) * kSfGroupBytes,
-                         nck * kSfGroupBytes, &full[s]);
+          uint64_t* bar = &full[s * C::NISS + warp];
+          const bool do_w = (0 % NPW) == warp, do_b = (1 % NPW) == warp, do_f = (2 % NPW) == warp;
+          ptx::mbar_arrive_expect_tx(bar, (do_w ? C::A_TX : 0) + (do_b ? nck * C::B_BLOCK : 0) +
+                                              (do_f ? nck * kSfGroupBytes : 0));
+          if (do_w)
+            ptx::tma_load_2d(a_s(s), &tm_w, 0, (int)(((int64_t)tl.e * p.NT + rt) * p.KC + c0) * kBM, bar);
+          if (do_b) ptx::bulk_load(b_s(s), p.bp_in + ((int64_t)tt * p.KC + c0) * C::B_BLOCK, nck * C::B_BLOCK, bar);
+          if (do_f)
+            ptx::bulk_load(sfa_s(s), p.w_sf + ((int64_t)(tl.e * p.NT + rt) * p.KC + c0) * kSfGroupBytes,
+                           nck * kSfGroupBytes, bar);
         }
         __syncwarp();
       }
     }
     // Never leave copies in flight when the CTA exits (consumers may have aborted before
-    // waiting for them): wait, bounded, for the last fill of every slot.  On the normal
-    // path these have all landed already.
+    // waiting for them): wait, bounded, for this warp's last fill of every slot.  On the
+    // normal path these have all landed already.
     {
       volatile int local_abort = 0;
       for (int64_t q = (g > S ? g - S : 0); q < g; ++q) {
-        if ((int)(q % NPW) != warp || (withheld && q == 0)) continue;
-        ptx::mbar_wait_bounded(&full[q % S], (uint32_t)(q / S) & 1, &local_abort, kWaitLimitNs);
+        if (withheld && q == 0) continue;
+        ptx::mbar_wait_bounded(&full[(q % S) * C::NISS + warp], (uint32_t)(q / S) & 1, &local_abort, kWaitLimitNs);
       }
     }
     __syncwarp();
@@ -253,12 +270,14 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
           break;
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + b * C::ACC_COLS;
-        const Item it = item_of(p, i);
+        const Item it = item_of(p, i, ksplit);
         const int nst = (it.kc1 - it.kc0 + NP - 1) / NP;
         for (int st = 0; st < nst; ++st, ++g) {
           const int s = (int)(g % S);
-          if (!__all_sync(0xffffffffu,
-                          ptx::mbar_wait_bounded(&full[s], (uint32_t)(g / S) & 1, s_abort, kWaitLimitNs))) {
+          bool landed = true;
+          for (int w = 0; w < C::NISS && landed; ++w)
+            landed = ptx::mbar_wait_bounded(&full[s * C::NISS + w], (uint32_t)(g / S) & 1, s_abort, kWaitLimitNs);
+          if (!__all_sync(0xffffffffu, landed)) {
             stop = true;
             break;
           }
@@ -322,7 +341,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
       // role at any time; the barrier reduction freezes one answer for all).
       if (ptx::bar_or<3, C::EPI_THREADS>(!ready)) break;
       ptx::tc_fence_after();
-      const Item it = item_of(p, i);
+      const Item it = item_of(p, i, ksplit);
       const int tt = it.tt, rt = it.rt;
       const Tile tl = p.tiles[tt];
       const uint32_t acc = tmem + lane_addr + b * C::ACC_COLS;
@@ -424,7 +443,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
             if (et < nt) {
               const int tok = p.perm[tl.row0 + jbase + et] / p.k;
               const int prev = atomicAdd(p.arrivals + (int64_t)tok * p.n_rt + rt, 1);
-              s_tok[et] = (prev == p.k * p.ksplit - 1) ? tok : -1;
+              s_tok[et] = (prev == p.k * ksplit - 1) ? tok : -1;
             }
             group_sync();
             __threadfence();
@@ -436,7 +455,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
                 float accv = __uint_as_float((uint32_t)p.x[(int64_t)tok * p.d + gc] << 16);
                 for (int j = 0; j < p.k; ++j) {
                   const int srow = p.inv[(int64_t)tok * p.k + j];
-                  for (int sp = 0; sp < p.ksplit; ++sp)
+                  for (int sp = 0; sp < ksplit; ++sp)
                     accv += __ldcg(p.ys + ((int64_t)sp * p.P + srow) * p.d + gc);
                 }
                 uint32_t bb = __float_as_uint(accv);
@@ -532,7 +551,7 @@ int launch_one(const FwdArgs& a) {
   prm.K = K;
   prm.KC = KC;
   prm.n_rt = (MODE == MODE_GATE_UP) ? a.I / 64 : (a.d + kBM - 1) / kBM;
-  prm.ksplit = std::max(1, std::min(KSPLIT, KC));   // every split keeps at least one chunk
+  prm.ksplit_max = std::max(1, std::min(KSPLIT, KC));   // every split keeps at least one chunk
   prm.P = P;
   prm.status = a.ws.status;
   prm.limit = a.limit;
@@ -560,7 +579,7 @@ int launch_one(const FwdArgs& a) {
       return -1;
     attr_done.fetch_or(bit, std::memory_order_release);
   }
-  const int64_t max_items = (int64_t)((P + BN - 1) / BN + a.E) * prm.n_rt * prm.ksplit;
+  const int64_t max_items = (int64_t)((P + BN - 1) / BN + a.E) * prm.n_rt * prm.ksplit_max;
   const int grid = (int)std::min<int64_t>(max_items, (int64_t)sm_count() * CPS);
   ev_before(a);
   if (launch_kernel(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, a.stream, a.pdl != 0, m_w, prm) !=
@@ -590,7 +609,7 @@ int launch_one(const FwdArgs& a) {
 #define MOE_GEMV_NPW 1
 #endif
 #ifndef MOE_GEMV_DOWN_SPLIT
-#define MOE_GEMV_DOWN_SPLIT 2
+#define MOE_GEMV_DOWN_SPLIT 3
 #endif
 // Large batches: 96-token tiles (MMA N = 192).
 #ifndef MOE_GEMM_NP
@@ -608,6 +627,7 @@ int launch_one(const FwdArgs& a) {
 #ifndef MOE_GEMM_NPW
 #define MOE_GEMM_NPW 1
 #endif
+
 constexpr int kGemvBN = 8, kGemvNP = MOE_GEMV_NP, kGemvS = MOE_GEMV_S, kGemvCPS = MOE_GEMV_CPS,
               kGemvEG = MOE_GEMV_EG, kGemvNPW = MOE_GEMV_NPW, kGemvDownSplit = MOE_GEMV_DOWN_SPLIT;
 constexpr int kGemmBN = 96, kGemmNP = MOE_GEMM_NP, kGemmS = MOE_GEMM_S, kGemmCPS = MOE_GEMM_CPS,
