@@ -60,8 +60,14 @@ def lib():
             L.oracle_group.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
             L.oracle_group.restype = i32
             L.oracle_moe_forward.argtypes = [i32, i32, i32, i32, i32, dbl, dbl, vp, vp, vp, vp, vp, vp, vp, vp,
-                                             vp, i32, vp, vp, vp, vp, vp, i32]
+                                             vp, i32, vp, vp, vp, vp, vp, i32, i32]
             L.oracle_moe_forward.restype = i32
+            L.oracle_e4m3_nearest_code.argtypes = [dbl]
+            L.oracle_e4m3_nearest_code.restype = i32
+            L.oracle_e4m3_value.argtypes = [i32]
+            L.oracle_e4m3_value.restype = dbl
+            L.oracle_mxfp8_quantize.argtypes = [vp, i64, vp, vp]
+            L.oracle_mxfp8_quantize.restype = i32
             _lib = L
     return _lib
 
@@ -79,6 +85,29 @@ def e2m1_value(code: int) -> float:
 
 def round_bf16(v: float) -> float:
     return lib().oracle_round_bf16(float(v))
+
+
+# Activation formats of the expert GEMMs: bf16 (exact) or MXFP8 (E4M3 in 32-blocks).
+ACT_FORMATS = {"bf16": 0, "mxfp8": 1}
+
+
+def e4m3_nearest_code(a: float) -> int:
+    """E4M3 code (0..0x7E) of the value nearest to |a|; ties to the even code; saturating."""
+    return lib().oracle_e4m3_nearest_code(float(a))
+
+
+def e4m3_value(code: int) -> float:
+    return lib().oracle_e4m3_value(int(code))
+
+
+def mxfp8_quantize(v: np.ndarray):
+    """float64 [..., n] (n a multiple of 32) -> (quantized values, block exponents [..., n/32])."""
+    v = np.ascontiguousarray(v, np.float64)
+    out = np.empty_like(v)
+    exps = np.empty(v.shape[:-1] + (v.shape[-1] // 32,), np.int32)
+    if lib().oracle_mxfp8_quantize(_p(v), v.size, _p(out), _p(exps)):
+        raise ValueError("length is not a multiple of 32")
+    return out, exps
 
 
 def storage_bytes(rows: int, K: int) -> tuple[int, int]:
@@ -150,11 +179,13 @@ def group(idx: np.ndarray, E: int):
 
 
 def moe_forward(x_bf16, gamma, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales, *, I, k,
-                eps=1e-5, limit=7.0, tokens=None, want_h=False, nthreads=0):
+                eps=1e-5, limit=7.0, tokens=None, want_h=False, nthreads=0, act="bf16"):
     """The whole layer for ``tokens`` (default: all rows of x).
 
     Weights in the oracle layout with a leading expert axis:
     w1_codes [E, 2I, d/2], w1_scales [E, 2I, d/32], w2_codes [E, d, I/2], w2_scales [E, d, I/32].
+    act: "bf16" (exact bf16 activations) or "mxfp8" (the expert inputs and the SwiGLU outputs
+    quantized to E4M3 in 32-value blocks before each projection; h is then returned quantized).
     Returns dict(y bf16 bits [n,d], y_f64 [n,d], idx [n,k], w [n,k], h [n,k,I] bf16 bits or None).
     """
     x_bf16 = np.ascontiguousarray(x_bf16, np.uint16)
@@ -174,7 +205,7 @@ def moe_forward(x_bf16, gamma, router_w, router_b, w1_codes, w1_scales, w2_codes
         _p(np.ascontiguousarray(router_w, np.float32)), _p(rb),
         _p(np.ascontiguousarray(w1_codes, np.uint8)), _p(np.ascontiguousarray(w1_scales, np.uint8)),
         _p(np.ascontiguousarray(w2_codes, np.uint8)), _p(np.ascontiguousarray(w2_scales, np.uint8)),
-        _p(toks), n, _p(y), _p(y64), _p(idx), _p(w), _p(h), nthreads)
+        _p(toks), n, _p(y), _p(y64), _p(idx), _p(w), _p(h), nthreads, ACT_FORMATS[act])
     del args
     if st:
         raise ValueError(f"oracle_moe_forward status {st}")

@@ -41,6 +41,16 @@
 //  * SwiGLU clamp (swiglu_limit 7): h = silu(min(g, 7)) * clamp(u, -7, 7);
 //    W1 rows 0..I-1 are the gate, rows I..2I-1 the up projection.
 //  * Block: y = x + sum_j w_j * Expert_j(bf16(RMSNorm(x))), j in slot order.
+//  * Optional MXFP8 activations (act_format 1; the pages quantize only the expert
+//    weights, so this mode is an extension): the expert inputs xe and the SwiGLU
+//    outputs h are each cut into 32-value blocks along the expert's reduction
+//    axis, the block structure [ARCH] "量化" gives for the weights, with an 8-bit
+//    element: OCP FP8 E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa bits;
+//    subnormals below 2^-6; largest finite 448; the pattern with all exponent
+//    and mantissa bits set is NaN).  Block scale X = 2^s, s = floor(log2(amax))
+//    - 7 (amax / X lands in [128, 256)), clamped to [-122, 126], s = 0 for an
+//    all-zero block; element = X * (E4M3 value nearest to v / X, ties to the
+//    even code, saturating at 448).
 //
 // Oracle storage layout (its own, documented here): codes [rows][K/2], two codes
 // per byte, low nibble = even k; scale bytes [rows][K/32].
@@ -118,6 +128,47 @@ int nearest_e2m1_magnitude_code(double a) {
     }
   }
   return best;
+}
+
+// The finite non-negative E4M3 values in code order (codes 0x00..0x7E), from the
+// format's fields: exponent field e (bits 6..3, bias 7), mantissa m (bits 2..0);
+// e = 0 is subnormal, m/8 * 2^-6; otherwise (1 + m/8) * 2^(e-7).  0x7F is NaN.
+const std::vector<double>& e4m3_grid() {
+  static const std::vector<double> grid = [] {
+    std::vector<double> g;
+    for (int code = 0; code < 0x7F; ++code) {
+      const int e = code >> 3, m = code & 7;
+      g.push_back(e == 0 ? std::ldexp(m / 8.0, -6) : std::ldexp(1.0 + m / 8.0, e - 7));
+    }
+    return g;
+  }();
+  return grid;
+}
+
+// Nearest E4M3 magnitude to a >= 0, ties to the even code, saturating at 448.
+int nearest_e4m3_code(double a) {
+  const std::vector<double>& g = e4m3_grid();
+  if (!(a > 0.0)) return 0;
+  if (a >= g.back()) return (int)g.size() - 1;
+  const int hi = (int)(std::lower_bound(g.begin(), g.end(), a) - g.begin());   // g[hi] >= a > g[hi-1]
+  const int lo = hi - 1;
+  const double dlo = a - g[lo], dhi = g[hi] - a;
+  if (dlo < dhi) return lo;
+  if (dhi < dlo) return hi;
+  return (lo & 1) ? hi : lo;
+}
+
+// MXFP8 quantization of one block of n <= 32 values in place (see the header).
+void mxfp8_block(double* v, int n, int32_t* exp_out) {
+  double amax = 0.0;
+  for (int i = 0; i < n; ++i) amax = std::max(amax, std::fabs(v[i]));
+  const int s = amax > 0.0 ? std::min(126, std::max(-122, floor_log2(amax) - 7)) : 0;
+  for (int i = 0; i < n; ++i) {
+    const double q = e4m3_grid()[nearest_e4m3_code(std::ldexp(std::fabs(v[i]), -s))];
+    v[i] = std::copysign(std::ldexp(q, s), v[i]);
+    if (q == 0.0) v[i] = 0.0;
+  }
+  if (exp_out) *exp_out = s;
 }
 
 template <class F>
@@ -210,6 +261,21 @@ int32_t oracle_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t r
 // bf16 helpers exposed for the oracle's own pins.
 // ---------------------------------------------------------------------------
 double oracle_round_bf16(double v) { return round_to_bf16(v); }
+
+// E4M3 code (0..0x7E) of the value nearest to |a|, ties to the even code, saturating.
+int32_t oracle_e4m3_nearest_code(double a) { return nearest_e4m3_code(std::fabs(a)); }
+double oracle_e4m3_value(int32_t code) { return (code >= 0 && code < 0x7F) ? e4m3_grid()[code] : NAN; }
+
+// MXFP8 quantization of n values (n a multiple of 32) in 32-value blocks; exps[n/32]
+// receives the block scale exponents (nullable).  Returns 0, or 2 if n % 32 != 0.
+int32_t oracle_mxfp8_quantize(const double* v, int64_t n, double* out, int32_t* exps) {
+  if (n % 32) return 2;
+  for (int64_t b = 0; b < n / 32; ++b) {
+    std::memcpy(out + 32 * b, v + 32 * b, 32 * sizeof(double));
+    mxfp8_block(out + 32 * b, 32, exps ? exps + b : nullptr);
+  }
+  return 0;
+}
 
 // ---------------------------------------------------------------------------
 // RMSNorm ([R-zh] sec. 7; eps = rms_norm_eps from [ATLAS]):
@@ -310,7 +376,7 @@ int32_t oracle_group(int32_t T, int32_t k, int32_t E, const int32_t* idx, int32_
 // [d][I].  h is rounded to bf16; o is returned unrounded.
 // ---------------------------------------------------------------------------
 static void expert_mlp(int32_t d, int32_t I, const double* w1, const double* w2, const double* xe, double limit,
-                       double* h, double* o) {
+                       bool mx_h, double* h, double* o) {
   for (int32_t n = 0; n < I; ++n) {
     double g = 0.0, u = 0.0;
     for (int32_t i = 0; i < d; ++i) g += w1[(int64_t)n * d + i] * xe[i];
@@ -319,6 +385,8 @@ static void expert_mlp(int32_t d, int32_t I, const double* w1, const double* w2,
     const double uc = std::min(std::max(u, -limit), limit);
     h[n] = round_to_bf16(silu(gc) * uc);
   }
+  if (mx_h)   // MXFP8 activations: the down projection reads h in 32-blocks along I
+    for (int32_t b = 0; b < I / 32; ++b) mxfp8_block(h + 32 * b, 32, nullptr);
   for (int32_t m = 0; m < d; ++m) {
     double acc = 0.0;
     for (int32_t n = 0; n < I; ++n) acc += w2[(int64_t)m * I + n] * h[n];
@@ -335,15 +403,18 @@ static void expert_mlp(int32_t d, int32_t I, const double* w1, const double* w2,
 // tok: the token ids to compute (n_tok of them; NULL = all T in order).
 // Outputs per computed token (row r = position in tok): y_bf16 [n][d];
 // optional: y_f64 [n][d] (before the final rounding), idx [n][k], w [n][k],
-// h_bf16 [n][k][I] (the rounded SwiGLU outputs, slot order).
+// h_bf16 [n][k][I] (the rounded SwiGLU outputs as the down projection reads them, slot
+// order).  act_format 0: bf16 activations; 1: MXFP8 activations (xe and h quantized in
+// 32-blocks, see the header).
 // Returns 0, or nonzero on bad arguments / NaN scale bytes.
 // ---------------------------------------------------------------------------
 int32_t oracle_moe_forward(int32_t T, int32_t d, int32_t I, int32_t E, int32_t k, double eps, double limit,
                            const uint16_t* x, const float* gamma, const float* router_w, const float* router_b,
                            const uint8_t* w1_codes, const uint8_t* w1_scales, const uint8_t* w2_codes,
                            const uint8_t* w2_scales, const int32_t* tok, int32_t n_tok, uint16_t* y_bf16,
-                           double* y_f64, int32_t* idx_out, double* w_out, uint16_t* h_bf16, int32_t nthreads) {
-  if (d % 32 || I % 32 || k < 1 || k > E) return 2;
+                           double* y_f64, int32_t* idx_out, double* w_out, uint16_t* h_bf16, int32_t nthreads,
+                           int32_t act_format) {
+  if (d % 32 || I % 32 || k < 1 || k > E || act_format < 0 || act_format > 1) return 2;
   if (!tok) n_tok = T;
   std::vector<int32_t> ids(n_tok);
   for (int32_t r = 0; r < n_tok; ++r) ids[r] = tok ? tok[r] : r;
@@ -362,6 +433,8 @@ int32_t oracle_moe_forward(int32_t T, int32_t d, int32_t I, int32_t E, int32_t k
   std::vector<double> xe((size_t)n_tok * d);
   oracle_rmsnorm(n_tok, d, xs.data(), gamma, eps, xe.data());
   for (auto& v : xe) v = round_to_bf16(v);
+  if (act_format == 1)
+    for (int64_t b = 0; b < (int64_t)n_tok * (d / 32); ++b) mxfp8_block(&xe[(size_t)b * 32], 32, nullptr);
 
   // Per (token, slot) expert outputs, computed expert by expert so that each
   // expert's weights are decoded once.
@@ -383,7 +456,8 @@ int32_t oracle_moe_forward(int32_t T, int32_t d, int32_t I, int32_t E, int32_t k
       for (int64_t j = j0; j < j1; ++j) {
         const int64_t q = jobs[j];
         const int64_t r = q / k;
-        expert_mlp(d, I, w1.data(), w2.data(), &xe[(size_t)r * d], limit, h.data(), &o[(size_t)q * d]);
+        expert_mlp(d, I, w1.data(), w2.data(), &xe[(size_t)r * d], limit, act_format == 1, h.data(),
+                   &o[(size_t)q * d]);
         if (h_bf16)
           for (int32_t n = 0; n < I; ++n) h_bf16[(size_t)q * I + n] = bf16_bits_of(h[n]);
       }

@@ -370,3 +370,123 @@ def test_forward_token_subset_equals_full_rows():
     sub = _oracle_y(case, tokens=np.array([11, 0, 5], np.int32))
     np.testing.assert_array_equal(sub["y"], full["y"][[11, 0, 5]])
     np.testing.assert_array_equal(sub["idx"], full["idx"][[11, 0, 5]])
+
+
+# --------------------------------------------------------------------------- MXFP8 activations
+# The optional MXFP8 activation format (an extension: the pages quantize only the weights)
+# keeps the pages' block structure, one 8-bit power-of-two scale per 32 values, with OCP FP8
+# E4M3 elements.  Pinned against the format's bit fields, torch's float8_e4m3fn cast
+# (round to nearest even) and a dense layer written out here.
+
+def _torch_e4m3(a: np.ndarray) -> np.ndarray:
+    """|a| < 464 rounded to E4M3 by torch's cast (values >= 464 would not saturate there)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a, np.float32))
+    return t.to(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_e4m3_grid_matches_bit_fields_and_torch():
+    import torch
+    vals = np.array([oracle.e4m3_value(c) for c in range(0x7F)])
+    fields = []
+    for c in range(0x7F):
+        e, m = c >> 3, c & 7
+        fields.append(m / 8 * 2.0 ** -6 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+    np.testing.assert_array_equal(vals, np.array(fields))
+    lib_vals = torch.arange(0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(vals, lib_vals)
+    assert vals[-1] == 448.0 and vals[1] == 2.0 ** -9 and vals[8] == 2.0 ** -6
+    assert math.isnan(oracle.e4m3_value(0x7F))
+    assert np.all(np.diff(vals) > 0)
+
+
+def test_e4m3_nearest_ties_to_even_and_saturates():
+    vals = np.array([oracle.e4m3_value(c) for c in range(0x7F)])
+    mids = (vals[:-1] + vals[1:]) / 2            # exact in float64
+    for i, mid in enumerate(mids):               # between codes i and i+1: the even one wins
+        assert oracle.e4m3_nearest_code(mid) == (i if i % 2 == 0 else i + 1), (i, mid)
+        assert oracle.e4m3_nearest_code(np.nextafter(mid, 0)) == i
+        assert oracle.e4m3_nearest_code(np.nextafter(mid, 1e9)) == i + 1
+    for a in (448.0, 460.0, 464.0, 1e6, float("inf")):
+        assert oracle.e4m3_nearest_code(a) == 0x7E
+    assert oracle.e4m3_nearest_code(0.0) == 0 and oracle.e4m3_nearest_code(2.0 ** -10) == 0
+    rng = np.random.default_rng(5)
+    a = np.concatenate([np.exp(rng.uniform(np.log(2.0 ** -12), np.log(440.0), 4000)), mids[mids < 440]])
+    a = a.astype(np.float32).astype(np.float64)  # values torch's float32 cast keeps exactly
+    codes = np.array([oracle.e4m3_nearest_code(v) for v in a])
+    np.testing.assert_array_equal(vals[codes], _torch_e4m3(a))
+
+
+def test_mxfp8_block_scale_exponent():
+    blocks = []
+    for amax in (1.0, 255.9, 256.0, 2.0 ** -20, 3.0e38, 2.0 ** -121):
+        b = np.zeros(32)
+        b[7] = -amax
+        b[3] = amax / 3
+        blocks.append(b)
+    blocks.append(np.zeros(32))
+    q, exps = oracle.mxfp8_quantize(np.stack(blocks))
+    expect = [-7, 0, 1, -27, 120, -122, 0]
+    np.testing.assert_array_equal(exps[:, 0], expect)
+    assert np.all(q[-1] == 0.0)
+    for i, amax in enumerate((1.0, 255.9, 256.0, 2.0 ** -20, 3.0e38)):
+        assert 128.0 <= abs(q[i, 7]) / 2.0 ** expect[i] <= 256.0
+
+
+def test_mxfp8_error_bound_and_grid_membership():
+    rng = np.random.default_rng(6)
+    v = rng.standard_normal((200, 64)) * np.exp(rng.uniform(-8, 8, (200, 1)))
+    v[:, 5] = 0.0
+    q, exps = oracle.mxfp8_quantize(v)
+    s = np.repeat(exps, 32, axis=1).astype(np.float64)
+    r = np.abs(v) / 2.0 ** s
+    top = np.floor(np.log2(np.where(r > 0, r, 1.0)))
+    bound = np.where(r >= 2.0 ** -6, 2.0 ** (top - 4), 2.0 ** -10) * 2.0 ** s
+    assert np.all(np.abs(q - v) <= bound * (1 + 1e-12))
+    grid = {oracle.e4m3_value(c) for c in range(0x7F)}
+    assert all(abs(x) in grid for x in (q / 2.0 ** s).ravel())
+    assert np.all(np.sign(q) * np.sign(v) >= 0) and np.all(q[:, 5] == 0.0)
+    # idempotent: quantized values are their own quantization
+    q2, exps2 = oracle.mxfp8_quantize(q)
+    np.testing.assert_array_equal(q2, q)
+
+
+def _mx_ref(v: np.ndarray) -> np.ndarray:
+    """MXFP8 of rows of v written out here: blocks of 32 along the last axis, scale
+    2^(floor(log2 amax) - 7), elements through torch's E4M3 cast."""
+    out = np.empty_like(v)
+    for idx in np.ndindex(v.shape[:-1]):
+        for b in range(v.shape[-1] // 32):
+            blk = v[idx][32 * b: 32 * b + 32]
+            amax = np.abs(blk).max()
+            s = (np.frexp(amax)[1] - 1 - 7) if amax > 0 else 0
+            s = min(126, max(-122, s))
+            out[idx][32 * b: 32 * b + 32] = _torch_e4m3(blk / 2.0 ** s) * 2.0 ** s
+    return out
+
+
+def test_forward_mxfp8_single_expert_is_dense_layer_on_quantized_activations():
+    """E = 1, k = 1 with MXFP8 activations: xe and h quantized in 32-blocks along the
+    reduction axis of the projection that reads them."""
+    case = _small_case(7, 64, 96, 1, 1, seed=15)
+    cfg, x, gamma, rw, rb, W, dec1, dec2 = case
+    out = _oracle_y(case, want_h=True, act="mxfp8")
+    xv = bf16_bits_to_f64(x)
+    xn = xv / np.sqrt(np.mean(xv ** 2, axis=1, keepdims=True) + 1e-5) * gamma
+    xe = _mx_ref(round_bf16(xn))
+    gt, up = xe @ dec1[0][:cfg.I].T, xe @ dec1[0][cfg.I:].T
+    h = _mx_ref(round_bf16(silu(np.minimum(gt, 7.0)) * np.clip(up, -7.0, 7.0)))
+    np.testing.assert_array_equal(bf16_bits_to_f64(out["h"][:, 0, :]), h)
+    np.testing.assert_allclose(out["y_f64"], xv + h @ dec2[0].T, rtol=0, atol=1e-12)
+    base = _oracle_y(case)
+    assert not np.array_equal(base["y_f64"], out["y_f64"])   # the format is in effect
+
+
+def test_forward_mxfp8_stays_close_to_bf16():
+    """MXFP8 activations move the layer's output by the E4M3 rounding only (~2^-5 relative
+    per element): small against the output and far from it."""
+    case = _small_case(16, 128, 128, 4, 2, seed=16)
+    a, b = _oracle_y(case)["y_f64"], _oracle_y(case, act="mxfp8")["y_f64"]
+    x = bf16_bits_to_f64(case[1])
+    delta = np.linalg.norm(b - a) / np.linalg.norm(a - x)
+    assert 1e-3 < delta < 0.1, delta
