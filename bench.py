@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(synth.CONFIGS))
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
+    ap.add_argument("--act", default="bf16", choices=["bf16", "mxfp8"],
+                    help="activation format of the expert GEMMs: exact bf16 (the layer as stated) or MXFP8")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of "
                     "replaying a captured CUDA graph")
@@ -100,14 +102,15 @@ def file_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key, config_name):
-    """Per-launch DRAM bytes from a committed ncu capture, if it still matches the kernel source."""
+def ncu_traffic(kernel_key, config_name, act="bf16"):
+    """Per-launch DRAM bytes from a committed ncu capture, if it still matches the kernel source
+    (captures of the MXFP8 activation format are filed under "<config>/mxfp8")."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     try:
         d = json.load(open(p))
-        ent = d.get(config_name, {}).get(kernel_key)
+        ent = d.get(config_name if act == "bf16" else f"{config_name}/{act}", {}).get(kernel_key)
         if not ent:
             return None
         src = os.path.join(ROOT, "mxfp4_expert_gemm_b200", "csrc", ent["source"])
@@ -212,7 +215,7 @@ def device_inputs(cfg, rank, need_oracle_weights):
 # ------------------------------------------------------------------------------ CPU oracle timing
 
 
-def time_oracle(cfg, inp, budget_s, tokens_per_step=None, steps=None, warmup=0):
+def time_oracle(cfg, inp, budget_s, tokens_per_step=None, steps=None, warmup=0, act="bf16"):
     """Time the CPU oracle (as it stands) on samples of the workload's tokens.
 
     Returns (tokens/s, threads, sample description)."""
@@ -227,7 +230,7 @@ def time_oracle(cfg, inp, budget_s, tokens_per_step=None, steps=None, warmup=0):
         toks = order[(np.arange(n) + i * n) % T]
         t0 = time.perf_counter()
         oracle.moe_forward(inp["x"], inp["gamma"], inp["rw"], inp["rb"], *inp["oracle_W"], I=cfg.I, k=cfg.k,
-                           eps=cfg.rms_eps, limit=cfg.swiglu_limit, tokens=toks)
+                           eps=cfg.rms_eps, limit=cfg.swiglu_limit, tokens=toks, act=act)
         dt = time.perf_counter() - t0
         if i >= warmup:
             times.append(dt)
@@ -259,7 +262,7 @@ def run_ours(args, rank, world, local_rank):
     cfg = synth.CONFIGS[args.config]
     want_cpu = (rank == 0 and world == 1 and not args.no_cpu_baseline)
     inp = device_inputs(cfg, rank, need_oracle_weights=want_cpu)
-    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, cfg.rms_eps, cfg.swiglu_limit, path=args.path)
+    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, cfg.rms_eps, cfg.swiglu_limit, path=args.path, act=args.act)
     ws = moe.new_workspace(dims, cfg.T)
     y = torch.empty_like(inp["x_dev"])
     stream = torch.cuda.current_stream()
@@ -398,7 +401,8 @@ def run_ours(args, rank, world, local_rank):
         achieved = alg / (gu_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "kernel": "gate_up (mx_expert_kernel<GATE_UP>)", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": ncu_traffic("gate_up", cfg.name),
+                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "traffic": ncu_traffic("gate_up", cfg.name, args.act),
                 "algorithmic_bytes_per_launch": alg, "launch_ms": round(gu_ms, 5), "peak_source": f"hbm_gbs, {peak_src}"}
         layer_bytes = used * (w1_bytes + w2_bytes)
         layer_ms = total_ms / K
@@ -411,13 +415,16 @@ def run_ours(args, rank, world, local_rank):
         achieved = alg / (gu_ms * 1e-3) / 1e12
         # kind::mxf8f6f4 runs at the fp8 rate: nominal fp8 / bf16 = 2 (4.5 vs 2.25 PFLOP/s dense)
         peak = round(2.0 * peaks["bf16_tflops"], 1)
+        cols = 1 if args.act == "mxfp8" else 2   # E4M3 MMA columns per token
         roof = {"bound": "tensor", "kernel": "gate_up (mx_expert_kernel<GATE_UP>)", "achieved": round(achieved, 1),
                 "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": ncu_traffic("gate_up", cfg.name), "algorithmic_flops_per_launch": alg,
-                "mma_flops_per_launch": 2 * alg, "mma_frac": round(2 * achieved / peak, 4),
+                "traffic": ncu_traffic("gate_up", cfg.name, args.act), "algorithmic_flops_per_launch": alg,
+                "mma_flops_per_launch": cols * alg, "mma_frac": round(cols * achieved / peak, 4),
                 "launch_ms": round(gu_ms, 5),
                 "peak_source": f"2 x bf16_tflops burst ({peak_src}): the block-scaled E2M1 x E4M3 MMA runs at the "
-                               "fp8 rate; each activation is two E4M3 columns, so the MMA does 2x the algorithmic flops"}
+                               "fp8 rate; " + ("each activation is two E4M3 columns, so the MMA does 2x the "
+                                               "algorithmic flops" if cols == 2 else "MXFP8 activations: one "
+                                               "E4M3 column per token")}
         layer_flops = 6 * d * I * P
         layer_ms = total_ms / K
         roof["layer"] = {"flops": layer_flops, "achieved_TFLOPs": round(layer_flops / (layer_ms * 1e-3) / 1e12, 1),
@@ -430,6 +437,7 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "e2m1xe4m3", "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[cfg.name], "name": cfg.name, "tokens_per_gpu": cfg.T,
                    "global_batch": cfg.T * world, "path": path_used, "parallelism": f"dp{world}",
+                   "activations": "exact bf16" if args.act == "bf16" else "MXFP8 (E4M3, 32-value blocks)",
                    "l2": "flushed before every step (256 MiB write, outside the step events)",
                    "timing": "sum of per-step CUDA events on the launching stream; max over ranks",
                    "launch": "CUDA graph replay per step" if use_graph else "host launches per step",
@@ -442,7 +450,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
     }
     if want_cpu:
-        v, cores, sample = time_oracle(cfg, inp, args.cpu_seconds)
+        v, cores, sample = time_oracle(cfg, inp, args.cpu_seconds, act=args.act)
         line["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     if rank == 0:
@@ -478,7 +486,8 @@ def run_reference(args, rank, world):
     # one token per step keeps --steps K --warmup W within minutes on the host cores
     n = 1
     t0 = time.perf_counter()
-    v, cores, sample = time_oracle(cfg, inp, 0, tokens_per_step=n, steps=args.steps, warmup=args.warmup)
+    v, cores, sample = time_oracle(cfg, inp, 0, tokens_per_step=n, steps=args.steps, warmup=args.warmup,
+                                   act=args.act)
     wall = time.perf_counter() - t0
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(n / v * 1e3, 3),

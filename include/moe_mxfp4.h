@@ -65,9 +65,25 @@ typedef enum {
 
 typedef enum {
   MOE_PATH_AUTO = 0, /* GEMV when tokens per expert are few, else GEMM */
-  MOE_PATH_GEMV = 1, /* weight-streaming path: 8-token tiles (small batches) */
-  MOE_PATH_GEMM = 2  /* grouped GEMM: 96-token tiles (large batches) */
+  MOE_PATH_GEMV = 1, /* weight-streaming path: 8-token tiles (16 with MXFP8 activations) */
+  MOE_PATH_GEMM = 2  /* grouped GEMM: 96-token tiles (192 with MXFP8 activations) */
 } moe_path;
+
+/* Activation format of the expert GEMMs (the weights are MXFP4 in both).
+ * MOE_ACT_BF16: the expert inputs xe = bf16(RMSNorm(x)) and the SwiGLU outputs h are used
+ *   exactly as bf16 (each carried to the tensor cores as two E4M3 terms with their block
+ *   scales; exact for every value above 2^-13 of its 32-block's largest).  The layer as the
+ *   pages state it.
+ * MOE_ACT_MXFP8: xe and h are quantized to MXFP8 before each projection: in 32-value blocks
+ *   along the projection's reduction axis (the pages' block of one 8-bit scale per 32
+ *   values), scale 2^(floor(log2 amax) - 7) clamped to [2^-122, 2^126] (1 for an all-zero
+ *   block), elements rounded to the nearest OCP FP8 E4M3 value (ties to even).  Half the
+ *   activation bytes and tensor-core work; the output moves by the E4M3 rounding (about
+ *   1e-2 of the expert output's norm).  An extension: the pages quantize only the weights. */
+typedef enum {
+  MOE_ACT_BF16 = 0,
+  MOE_ACT_MXFP8 = 1
+} moe_act_format;
 
 /* Which projection a weight tensor is (sets its row order in storage). */
 typedef enum {
@@ -84,6 +100,7 @@ typedef struct {
   float rms_eps;        /* RMSNorm epsilon (gpt-oss: 1e-5)                              */
   float swiglu_limit;   /* SwiGLU clamp (gpt-oss: 7)                                    */
   int32_t path;         /* a moe_path value                                             */
+  int32_t act_format;   /* a moe_act_format value: the expert GEMMs' activation format  */
 } moe_dims;
 
 /* ---------------------------------------------------------------- MXFP4 storage

@@ -33,6 +33,10 @@ MOE_PATH_GEMV = 1
 MOE_PATH_GEMM = 2
 PATHS = {"auto": MOE_PATH_AUTO, "gemv": MOE_PATH_GEMV, "gemm": MOE_PATH_GEMM}
 
+MOE_ACT_BF16 = 0
+MOE_ACT_MXFP8 = 1
+ACT_FORMATS = {"bf16": MOE_ACT_BF16, "mxfp8": MOE_ACT_MXFP8}
+
 MOE_WEIGHT_PLAIN = 0
 MOE_WEIGHT_GATE_UP = 1
 ROLES = {"plain": MOE_WEIGHT_PLAIN, "down": MOE_WEIGHT_PLAIN, "gate_up": MOE_WEIGHT_GATE_UP}
@@ -47,14 +51,16 @@ class MoeError(RuntimeError):
 class moe_dims(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("I", ctypes.c_int32), ("E", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("block", ctypes.c_int32), ("rms_eps", ctypes.c_float), ("swiglu_limit", ctypes.c_float),
-                ("path", ctypes.c_int32)]
+                ("path", ctypes.c_int32), ("act_format", ctypes.c_int32)]
 
 
 def make_dims(d: int, I: int, E: int, top_k: int, rms_eps: float = 1e-5, swiglu_limit: float = 7.0,
-              path: int | str = MOE_PATH_AUTO, block: int = 32) -> moe_dims:
+              path: int | str = MOE_PATH_AUTO, block: int = 32, act: int | str = MOE_ACT_BF16) -> moe_dims:
     if isinstance(path, str):
         path = PATHS[path]
-    return moe_dims(d, I, E, top_k, block, rms_eps, swiglu_limit, path)
+    if isinstance(act, str):
+        act = ACT_FORMATS[act]
+    return moe_dims(d, I, E, top_k, block, rms_eps, swiglu_limit, path, act)
 
 
 _lib = None

@@ -34,21 +34,22 @@ __host__ __device__ __forceinline__ int sf_byte_in_group(int r, int b) {
   return (r & 31) * 16 + ((r & 127) >> 5) * 4 + (b & 3);
 }
 
-// Scale-factor groups of one token tile: tile_tokens tokens give 2 * tile_tokens MMA
-// columns (hi and lo term of each token), 128 columns per group.
-__host__ __device__ constexpr int sf_groups_of(int tile_tokens) { return (2 * tile_tokens + 127) / 128; }
+// A token tile feeds the MMA `rows` = terms * tile_tokens E4M3 rows (MMA columns): two
+// per token (hi and lo term, bf16 activations) or one (MXFP8 activations); row n belongs
+// to token n / terms.  Scale-factor groups: 128 rows each.
+__host__ __device__ constexpr int sf_groups_of(int rows) { return (rows + 127) / 128; }
 
 // Packed activation block of one token tile and one 128-chunk of the reduction axis: the
-// tile's 2 * tile_tokens E4M3 rows of 128 bytes (row n = MMA column n = hi / lo term of
-// token n / 2) in the 128-byte-swizzled order the MMA reads (16-byte unit u of row n at
-// unit u ^ (n % 8)), then the tile's scale-factor groups for the chunk's four 32-blocks,
-// padded to a multiple of 1 KB.  One contiguous copy brings a block into shared memory.
-__host__ __device__ constexpr int packed_block_bytes(int tile_tokens) {
-  return (2 * tile_tokens * kKChunk + sf_groups_of(tile_tokens) * kSfGroupBytes + 1023) / 1024 * 1024;
+// tile's `rows` E4M3 rows of 128 bytes in the 128-byte-swizzled order the MMA reads
+// (16-byte unit u of row n at unit u ^ (n % 8)), then the tile's scale-factor groups for
+// the chunk's four 32-blocks, padded to a multiple of 1 KB.  One contiguous copy brings a
+// block into shared memory.
+__host__ __device__ constexpr int packed_block_bytes(int rows) {
+  return (rows * kKChunk + sf_groups_of(rows) * kSfGroupBytes + 1023) / 1024 * 1024;
 }
 __host__ __device__ __forceinline__ int packed_unit_offset(int n, int u) { return n * kKChunk + ((u ^ (n & 7)) << 4); }
-__host__ __device__ __forceinline__ int packed_sf_offset(int tile_tokens, int n, int b) {
-  return 2 * tile_tokens * kKChunk + (n >> 7) * kSfGroupBytes + sf_byte_in_group(n & 127, b & 3);
+__host__ __device__ __forceinline__ int packed_sf_offset(int rows, int n, int b) {
+  return rows * kKChunk + (n >> 7) * kSfGroupBytes + sf_byte_in_group(n & 127, b & 3);
 }
 
 // ------------------------------------------------------------------ MXFP4 storage layout
@@ -96,17 +97,19 @@ struct WsLayout {
   size_t total;
   int64_t max_tiles;
   int32_t tile_tokens;
+  int32_t terms;     // E4M3 rows per token fed to the MMAs: 2 (bf16 activations) or 1 (MXFP8)
   int32_t ksplit;   // down GEMM reduction-axis splits (ys planes)
   int32_t dp, ip;   // d and I rounded up to 128
 };
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-inline WsLayout ws_layout(const moe_dims& dm, int64_t T, int tile_tokens, int ksplit) {
+inline WsLayout ws_layout(const moe_dims& dm, int64_t T, int tile_tokens, int ksplit, int terms) {
   WsLayout L{};
   const int64_t P = T * dm.top_k;
   L.tile_tokens = tile_tokens;
   L.ksplit = ksplit;
+  L.terms = terms;
   L.max_tiles = (P + tile_tokens - 1) / tile_tokens + dm.E;
   L.dp = (int32_t)kpad128(dm.d);
   L.ip = (int32_t)kpad128(dm.I);
@@ -129,8 +132,8 @@ inline WsLayout ws_layout(const moe_dims& dm, int64_t T, int tile_tokens, int ks
   L.w_sorted = take(4 * (size_t)P);
   L.xq = take(2 * (size_t)T * L.dp);
   L.xsf = take(2 * (size_t)T * (L.dp / 32));
-  L.bpx = take((size_t)L.max_tiles * (L.dp / kKChunk) * packed_block_bytes(tile_tokens));
-  L.bph = take((size_t)L.max_tiles * (L.ip / kKChunk) * packed_block_bytes(tile_tokens));
+  L.bpx = take((size_t)L.max_tiles * (L.dp / kKChunk) * packed_block_bytes(terms * tile_tokens));
+  L.bph = take((size_t)L.max_tiles * (L.ip / kKChunk) * packed_block_bytes(terms * tile_tokens));
   L.ys = take(4 * (size_t)ksplit * P * dm.d);
   L.total = o;
   return L;
@@ -158,6 +161,7 @@ struct Ws {
   float* ys;
   int64_t max_tiles;
   int32_t tile_tokens;
+  int32_t terms;
   int32_t ksplit;
   int32_t dp, ip;
 };
@@ -186,6 +190,7 @@ inline Ws ws_pointers(void* base, const WsLayout& L, int E) {
   w.max_tiles = L.max_tiles;
   w.tile_tokens = L.tile_tokens;
   w.ksplit = L.ksplit;
+  w.terms = L.terms;
   w.dp = L.dp;
   w.ip = L.ip;
   return w;
@@ -345,7 +350,7 @@ int launch_quantize(const float* w, int32_t E, int32_t N, int32_t K, int32_t rol
 int launch_route(const FwdArgs& a);     // norm + router + top-k + E4M3 split, grouping, packing
 int launch_combine(const FwdArgs& a);   // y = x + sum_j ys[inv]
 int launch_experts(const FwdArgs& a);   // block-scaled tcgen05 expert MLPs (gate_up, down)
-int expert_tile_tokens(int path);       // token tile of a path
+int expert_tile_tokens(int path, int terms);   // token tile of a path
 int expert_down_split(int path);        // reduction-axis splits of a path's down GEMM
 
 }  // namespace moe

@@ -88,19 +88,19 @@ struct MxParams {
 #endif
 constexpr int kSfSlots = MOE_SF_SLOTS;  // scale-factor TMEM slots, used stage after stage in turn
 
-template <int BN, int NP, int S, int CPS, int EG, int NPW>
+template <int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS>
 struct MxCfg {
-  static constexpr int N2 = 2 * BN;                     // MMA N: hi and lo column per token
+  static constexpr int N2 = TERMS * BN;                 // MMA N: hi (and lo) column per token
   static constexpr int G = (N2 + 127) / 128;            // scale-factor groups of the B operand
   static constexpr int A_PANEL = kBM * kKChunk;         // 128 rows x 128 codes, one byte each
   static constexpr int B_PANEL = N2 * kKChunk;          // N2 rows x 128 E4M3
-  static constexpr int B_BLOCK = packed_block_bytes(BN);  // B panel + its scale factors, padded
+  static constexpr int B_BLOCK = packed_block_bytes(N2);  // B panel + its scale factors, padded
   static constexpr int B_OFF = NP * A_PANEL;
   static constexpr int SFA_OFF = B_OFF + NP * B_BLOCK;
   static constexpr int STAGE_BYTES = ((SFA_OFF + NP * kSfGroupBytes + 1023) / 1024) * 1024;
   static constexpr int A_TX = NP * kBM * kKChunk / 2;   // the weight box counts packed bytes
   static constexpr int CW = N2 < 32 ? N2 : 32;          // accumulator columns per epilogue read
-  static constexpr int TC = CW / 2;                     // tokens per epilogue read
+  static constexpr int TC = CW / TERMS;                 // tokens per epilogue read
   static constexpr int HT = TC / 2;                     // tokens each side (gate / up) finishes
   static constexpr int ACC_COLS = N2 < 32 ? 32 : N2;    // one accumulator buffer
   static constexpr int SF_SLOT_COLS = 4 * NP * (1 + G);         // A then B scale factors of a stage
@@ -142,6 +142,14 @@ __device__ __forceinline__ Item item_of(const MxParams& p, int i, int ksplit) {
   return it;
 }
 
+// Accumulator of token j in a 32-column epilogue read: the sum of its hi and lo columns
+// (bf16 activations carried as two E4M3 terms) or its one column (MXFP8 activations).
+template <int TERMS>
+__device__ __forceinline__ float token_acc(const uint32_t (&v)[32], int j) {
+  if (TERMS == 2) return __uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]);
+  return __uint_as_float(v[j]);
+}
+
 // Splits of the reduction axis for n0 (token tile, row tile) units over `grid` CTAs: the
 // fewest (at most smax) that give every CTA two items, so that one item's epilogue runs
 // under the next item's loads (the accumulator is double-buffered).
@@ -150,10 +158,10 @@ __device__ __forceinline__ int choose_ksplit(int n0, int grid, int smax) {
   return max(1, min(smax, (2 * grid + n0 - 1) / n0));
 }
 
-template <int BN, int NP, int S, int CPS, int EG, int NPW, int MODE>
-__global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
+template <int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, int MODE>
+__global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>::THREADS, CPS)
     mx_expert_kernel(const __grid_constant__ CUtensorMap tm_w, const MxParams p) {
-  using C = MxCfg<BN, NP, S, CPS, EG, NPW>;
+  using C = MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>;
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
 
@@ -371,17 +379,14 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
 #pragma unroll
           for (int c = 0; c < C::HT; ++c) {
             const int jj = gate_side ? C::HT + c : c;  // token the other side finishes
-            const float val = gate_side ? __uint_as_float(v[2 * (C::HT + c)]) + __uint_as_float(v[2 * (C::HT + c) + 1])
-                                        : __uint_as_float(v[2 * c]) + __uint_as_float(v[2 * c + 1]);
+            const float val = gate_side ? token_acc<TERMS>(v, C::HT + c) : token_acc<TERMS>(v, c);
             s_x[jj * 64 + f] = val;
           }
           group_sync();
 #pragma unroll
           for (int c = 0; c < C::HT; ++c) {
             const int jj = gate_side ? c : C::HT + c;  // token this side finishes
-            const float mine = gate_side ? __uint_as_float(v[2 * c]) + __uint_as_float(v[2 * c + 1])
-                                         : __uint_as_float(v[2 * (C::HT + c)]) +
-                                               __uint_as_float(v[2 * (C::HT + c) + 1]);
+            const float mine = gate_side ? token_acc<TERMS>(v, c) : token_acc<TERMS>(v, C::HT + c);
             const float other = s_x[jj * 64 + f];
             const float gv = fminf(gate_side ? mine : other, L);
             const float uv = fminf(fmaxf(gate_side ? other : mine, -L), L);
@@ -392,17 +397,18 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
             const float vv[1] = {hv};
             uint32_t hi, lo, s1, s2;
             e4m3_split<1>(vv, hi, lo, s1, s2);
-            const int j = c0 / 2 + jj;                 // token within the tile
+            const int j = c0 / TERMS + jj;             // token within the tile
             if (j < tl.rows) {
               // the down GEMM's packed block: chunk kb / 4, rows 2j (hi) and 2j + 1 (lo),
               // byte f' = 32 (kb % 4) + lane of the 128-byte row
               uint8_t* blk = p.bp_out + ((int64_t)tt * p.KCo + kb / 4) * C::B_BLOCK;
               const int u = 2 * (kb & 3) + (lane >> 4);
-              blk[packed_unit_offset(2 * j, u) + (lane & 15)] = (uint8_t)hi;
-              blk[packed_unit_offset(2 * j + 1, u) + (lane & 15)] = (uint8_t)lo;
+              // (with MXFP8 activations only the hi term: h rounded to E4M3 in its block)
+              blk[packed_unit_offset(TERMS * j, u) + (lane & 15)] = (uint8_t)hi;
+              if (TERMS == 2) blk[packed_unit_offset(2 * j + 1, u) + (lane & 15)] = (uint8_t)lo;
               if (lane == 0) {
-                blk[packed_sf_offset(BN, 2 * j, kb)] = (uint8_t)s1;
-                blk[packed_sf_offset(BN, 2 * j + 1, kb)] = (uint8_t)s2;
+                blk[packed_sf_offset(C::N2, TERMS * j, kb)] = (uint8_t)s1;
+                if (TERMS == 2) blk[packed_sf_offset(C::N2, 2 * j + 1, kb)] = (uint8_t)s2;
               }
             }
           }
@@ -425,13 +431,13 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW>::THREADS, CPS)
             ptx::tc_fence_before();
             ptx::mbar_arrive(&acce[b]);
           }
-          const int jbase = c0 / 2;
+          const int jbase = c0 / TERMS;
           const int nt = min(C::TC, tl.rows - jbase);   // tokens of this read (may be <= 0)
 #pragma unroll
           for (int c = 0; c < C::TC; ++c) {
             if (c < nt && m < p.d) {
               const int64_t prow = tl.row0 + jbase + c;
-              const float o = __uint_as_float(v[2 * c]) + __uint_as_float(v[2 * c + 1]);
+              const float o = token_acc<TERMS>(v, c);
               ys[prow * p.d + m] = o * p.w_sorted[prow];
             }
           }
@@ -520,9 +526,9 @@ int sm_count() {
   return n;
 }
 
-template <int MODE, int BN, int NP, int S, int CPS, int EG, int NPW, int KSPLIT>
+template <int MODE, int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, int KSPLIT>
 int launch_one(const FwdArgs& a) {
-  using C = MxCfg<BN, NP, S, CPS, EG, NPW>;
+  using C = MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>;
   const int P = a.T * a.k;
   const int K = (MODE == MODE_GATE_UP) ? a.d : a.I;
   const int N = (MODE == MODE_GATE_UP) ? 2 * a.I : a.d;  // weight rows per expert
@@ -569,7 +575,7 @@ int launch_one(const FwdArgs& a) {
   prm.y = a.y;
   prm.arrivals = a.ws.arrivals;
 
-  auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, NPW, MODE>;
+  auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, NPW, TERMS, MODE>;
   static std::atomic<uint64_t> attr_done{0};   // per-device "attribute set" bits
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -636,23 +642,31 @@ static_assert(kGemvBN >= kMinTileTokens, "tile list sized for the smallest tile"
 
 }  // namespace
 
-int expert_tile_tokens(int path) { return path == MOE_PATH_GEMV ? kGemvBN : kGemmBN; }
+// With MXFP8 activations a token is one MMA column instead of two: tiles of twice the
+// tokens keep the same MMA shape.
+int expert_tile_tokens(int path, int terms) { return (path == MOE_PATH_GEMV ? kGemvBN : kGemmBN) * (2 / terms); }
 
 int expert_down_split(int path) { return path == MOE_PATH_GEMV ? kGemvDownSplit : 1; }
 
-int launch_experts(const FwdArgs& a) {
+namespace {
+template <int TERMS>
+int launch_pair(const FwdArgs& a) {
+  constexpr int gv = kGemvBN * 2 / TERMS, gm = kGemmBN * 2 / TERMS;
   int n1, n2;
-  if (a.ws.tile_tokens == kGemvBN) {
-    n1 = launch_one<MODE_GATE_UP, kGemvBN, kGemvNP, kGemvS, kGemvCPS, kGemvEG, kGemvNPW, 1>(a);
+  if (a.ws.tile_tokens == gv) {
+    n1 = launch_one<MODE_GATE_UP, gv, kGemvNP, kGemvS, kGemvCPS, kGemvEG, kGemvNPW, TERMS, 1>(a);
     if (n1 < 0) return -1;
-    n2 = launch_one<MODE_DOWN, kGemvBN, kGemvNP, kGemvS, kGemvCPS, kGemvEG, kGemvNPW, kGemvDownSplit>(a);
+    n2 = launch_one<MODE_DOWN, gv, kGemvNP, kGemvS, kGemvCPS, kGemvEG, kGemvNPW, TERMS, kGemvDownSplit>(a);
   } else {
-    n1 = launch_one<MODE_GATE_UP, kGemmBN, kGemmNP, kGemmS, kGemmCPS, kGemmEG, kGemmNPW, 1>(a);
+    n1 = launch_one<MODE_GATE_UP, gm, kGemmNP, kGemmS, kGemmCPS, kGemmEG, kGemmNPW, TERMS, 1>(a);
     if (n1 < 0) return -1;
-    n2 = launch_one<MODE_DOWN, kGemmBN, kGemmNP, kGemmS, kGemmCPS, kGemmEG, kGemmNPW, 1>(a);
+    n2 = launch_one<MODE_DOWN, gm, kGemmNP, kGemmS, kGemmCPS, kGemmEG, kGemmNPW, TERMS, 1>(a);
   }
   if (n2 < 0) return -1;
   return n1 + n2;
 }
+}  // namespace
+
+int launch_experts(const FwdArgs& a) { return a.ws.terms == 1 ? launch_pair<1>(a) : launch_pair<2>(a); }
 
 }  // namespace moe

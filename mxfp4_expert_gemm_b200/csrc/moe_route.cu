@@ -161,17 +161,20 @@ __device__ __forceinline__ void warp_topk_softmax(float (&l)[NJ], int E, int k, 
 // move the 16 16-byte units, lanes 16-23 the eight scale bytes.
 __device__ __forceinline__ void pack_pair_chunk(const FwdArgs& a, int t, int tile, int col, int c) {
   const int lane = threadIdx.x & 31;
-  const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk;
-  uint8_t* block = a.ws.bpx + ((int64_t)tile * kc + c) * packed_block_bytes(bt);
+  const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk, terms = a.ws.terms;
+  const int rows = terms * bt;
+  uint8_t* block = a.ws.bpx + ((int64_t)tile * kc + c) * packed_block_bytes(rows);
   if (lane < 16) {   // (units past d are never read by the MMAs)
     const int term = lane >> 3, u = lane & 7;
-    const uint4 v =
-        __ldcg(reinterpret_cast<const uint4*>(a.ws.xq + (int64_t)t * 2 * dp + term * dp + c * kKChunk) + u);
-    *reinterpret_cast<uint4*>(block + packed_unit_offset(2 * col + term, u)) = v;
+    if (term < terms) {
+      const uint4 v =
+          __ldcg(reinterpret_cast<const uint4*>(a.ws.xq + (int64_t)t * 2 * dp + term * dp + c * kKChunk) + u);
+      *reinterpret_cast<uint4*>(block + packed_unit_offset(terms * col + term, u)) = v;
+    }
   } else if (lane < 24) {
     const int term = (lane - 16) >> 2, b = 4 * c + ((lane - 16) & 3);
-    if (b < nb)
-      block[packed_sf_offset(bt, 2 * col + term, b)] =
+    if (term < terms && b < nb)
+      block[packed_sf_offset(rows, terms * col + term, b)] =
           __ldcg(a.ws.xsf + (int64_t)t * 2 * (dp / 32) + term * (dp / 32) + b);
   }
 }
@@ -648,18 +651,19 @@ __global__ void __launch_bounds__(1024) group_kernel(FwdArgs a, int tile_tokens)
 // warp; each lane keeps four 16-byte copies in flight.
 __device__ __forceinline__ void pack_pair(const FwdArgs& a, int t, int tile, int col) {
   const int lane = threadIdx.x & 31;
-  const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk;
-  const int bb = packed_block_bytes(bt);
+  const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk, terms = a.ws.terms;
+  const int rows_t = terms * bt;
+  const int bb = packed_block_bytes(rows_t);
   uint8_t* blocks = a.ws.bpx + (int64_t)tile * kc * bb;
   const uint8_t* rows = a.ws.xq + (int64_t)t * 2 * dp;
-  const int units = kc * 16;   // (chunk, term, unit); units past d are never read by the MMAs
+  const int units = kc * 8 * terms;   // (chunk, term, unit); units past d are never read by the MMAs
   for (int i0 = lane; i0 < units; i0 += 128) {
     uint4 v[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int i = i0 + 32 * r;
       if (i < units) {
-        const int c = i >> 4, term = (i >> 3) & 1, u = i & 7;
+        const int c = i / (8 * terms), term = (i >> 3) % terms, u = i & 7;
         v[r] = __ldcg(reinterpret_cast<const uint4*>(rows + term * dp + c * kKChunk) + u);
       }
     }
@@ -667,15 +671,15 @@ __device__ __forceinline__ void pack_pair(const FwdArgs& a, int t, int tile, int
     for (int r = 0; r < 4; ++r) {
       const int i = i0 + 32 * r;
       if (i < units) {
-        const int c = i >> 4, term = (i >> 3) & 1, u = i & 7;
-        *reinterpret_cast<uint4*>(blocks + (int64_t)c * bb + packed_unit_offset(2 * col + term, u)) = v[r];
+        const int c = i / (8 * terms), term = (i >> 3) % terms, u = i & 7;
+        *reinterpret_cast<uint4*>(blocks + (int64_t)c * bb + packed_unit_offset(terms * col + term, u)) = v[r];
       }
     }
   }
   const uint8_t* sf = a.ws.xsf + (int64_t)t * 2 * (dp / 32);
-  for (int i = lane; i < 2 * nb; i += 32) {
+  for (int i = lane; i < terms * nb; i += 32) {
     const int term = i / nb, b = i - term * nb;
-    blocks[(int64_t)(b / 4) * bb + packed_sf_offset(bt, 2 * col + term, b)] = __ldcg(sf + term * (dp / 32) + b);
+    blocks[(int64_t)(b / 4) * bb + packed_sf_offset(rows_t, terms * col + term, b)] = __ldcg(sf + term * (dp / 32) + b);
   }
 }
 

@@ -18,8 +18,13 @@ import synth
 from _inputs import routed_inputs
 
 
-# Token tile of each path (moe_mxfp4.h: "8-token tiles", "96-token tiles").
+# Token tile of each path (moe_mxfp4.h: "8-token tiles", "96-token tiles"; twice that with
+# MXFP8 activations, one MMA column per token).
 TILE_TOKENS = {"gemv": 8, "gemm": 96}
+
+
+def tile_tokens(path: str, act: str = "bf16") -> int:
+    return TILE_TOKENS[path] * (2 if act == "mxfp8" else 1)
 
 
 def decode_e4m3(b: np.ndarray) -> np.ndarray:
@@ -111,21 +116,21 @@ def case(cfg: synth.MoEConfig):
                 rb_dev=torch.from_numpy(rb).cuda())
 
 
-def run_gpu(c, path, T=None):
+def run_gpu(c, path, T=None, act="bf16"):
     cfg = c["cfg"]
-    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, cfg.rms_eps, cfg.swiglu_limit, path=path)
+    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, cfg.rms_eps, cfg.swiglu_limit, path=path, act=act)
     T = cfg.T
     ws = moe.new_workspace(dims, T)
     y, r = moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws,
                            want_routing=True)
     st = moe.moe_device_status(ws)
-    return dict(y=y, routing=r, ws=ws, dims=dims, status=st)
+    return dict(y=y, routing=r, ws=ws, dims=dims, status=st, act=act)
 
 
-def oracle_rows(c, tokens=None, want_h=False):
+def oracle_rows(c, tokens=None, want_h=False, act="bf16"):
     cfg = c["cfg"]
     return oracle.moe_forward(c["x"], c["gamma"], c["rw"], c["rb"], *c["W"]["oracle"], I=cfg.I, k=cfg.k,
-                              eps=cfg.rms_eps, limit=cfg.swiglu_limit, tokens=tokens, want_h=want_h)
+                              eps=cfg.rms_eps, limit=cfg.swiglu_limit, tokens=tokens, want_h=want_h, act=act)
 
 
 def parity_stats(y_gpu_u16, y_ref_u16, x_u16) -> dict:

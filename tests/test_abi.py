@@ -53,6 +53,10 @@ def test_workspace_size_and_layout(L):
     P = 4096 * 4
     assert lay["ys"] + 4 * P * 2880 <= n
     assert moe.moe_workspace_bytes(moe.make_dims(2880, 2880, 32, 4, block=16), 16) == 0
+    # MXFP8 activations: one E4M3 row per token, tiles of twice the tokens, same block size
+    mx = moe.moe_workspace_layout(moe.make_dims(2880, 2880, 32, 4, act="mxfp8"), 4096)
+    assert mx["status"] == 0 and mx["total"] <= n
+    assert moe.moe_workspace_bytes(moe.make_dims(2880, 2880, 32, 4, act=9), 16) == 0
 
 
 def _call_forward(L, dims, T, ptr=256, ws_bytes=1 << 40):
@@ -70,6 +74,7 @@ def test_argument_checks_before_device(L):
     assert _call_forward(L, moe.make_dims(2880, 2880, 4, 5), 4) == moe.MOE_ERR_UNSUPPORTED_SHAPE
     assert _call_forward(L, moe.make_dims(2880, 2880, 32, 4, path=9), 4) == moe.MOE_ERR_INVALID_ARG
     assert _call_forward(L, moe.make_dims(2880, 2880, 32, 4, rms_eps=-1.0), 4) == moe.MOE_ERR_INVALID_ARG
+    assert _call_forward(L, moe.make_dims(2880, 2880, 32, 4, act=7), 4) == moe.MOE_ERR_INVALID_ARG
     assert _call_forward(L, ok, -1) == moe.MOE_ERR_INVALID_ARG
     assert _call_forward(L, ok, 4, ptr=8) == moe.MOE_ERR_INVALID_ARG          # misaligned
     assert _call_forward(L, ok, 4, ptr=0) == moe.MOE_ERR_INVALID_ARG          # null

@@ -12,7 +12,7 @@ import mxfp4_expert_gemm_b200 as moe
 import oracle
 import synth
 from _gpu_case import (TILE_TOKENS, assert_parity, bf16_dev, bf16_host, case, decode_e4m3, oracle_rows, parity_stats, run_gpu,
-                       stored_row_of, stored_to_rowmajor, weights)
+                       stored_row_of, stored_to_rowmajor, tile_tokens, weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -154,16 +154,19 @@ def test_forward_parity(name, path):
 
 def _h_from_workspace(g, cfg):
     """h [P, I] (sorted pairs) rebuilt from the down GEMM's packed activation blocks: per
-    token tile and 128-chunk, 2*BN E4M3 rows (row n = hi / lo term of token n // 2, 16-byte
-    unit u stored at unit u ^ (n % 8)), then the scale-factor groups (byte
-    (n%32)*16 + ((n%128)//32)*4 + b%4 of group n // 128 for 32-block b)."""
+    token tile and 128-chunk, terms*BN E4M3 rows (row n = term n % terms of token
+    n // terms: hi / lo for bf16 activations, one row for MXFP8; 16-byte unit u stored at
+    unit u ^ (n % 8)), then the scale-factor groups (byte (n%32)*16 + ((n%128)//32)*4 + b%4
+    of group n // 128 for 32-block b)."""
     dims, ws, T = g["dims"], g["ws"], cfg.T
     P = T * cfg.k
     Ip = moe.kpad128(cfg.I)
     KC = Ip // 128
-    bt = TILE_TOKENS[moe.resolved_path(dims, T)]
-    G = (2 * bt + 127) // 128
-    BB = (2 * bt * 128 + G * 512 + 1023) // 1024 * 1024
+    nterms = 1 if g["act"] == "mxfp8" else 2
+    bt = tile_tokens(moe.resolved_path(dims, T), g["act"])
+    R = nterms * bt
+    G = (R + 127) // 128
+    BB = (R * 128 + G * 512 + 1023) // 1024 * 1024
     view = lambda f, dt, sh: moe.workspace_view(ws, dims, T, f, dt, sh).cpu().numpy()
     offsets = view("offsets", torch.int32, (cfg.E + 1,))
     tbase = view("tile_base", torch.int32, (cfg.E,))
@@ -177,14 +180,14 @@ def _h_from_workspace(g, cfg):
         j = p - offsets[e]
         tile, col = tbase[e] + j // bt, j % bt
         terms = []
-        for n in (2 * col, 2 * col + 1):
+        for n in range(nterms * col, nterms * col + nterms):
             phys = n * 128 + ((u ^ (n % 8)) << 4)                                    # [8]
             rows = bph[tile][:, (phys[:, None] + np.arange(16)[None, :]).ravel()]     # [KC, 128]
             codes = rows.reshape(-1)[: cfg.I]
-            sfo = 2 * bt * 128 + (n // 128) * 512 + (n % 32) * 16 + ((n % 128) // 32) * 4 + b % 4
+            sfo = R * 128 + (n // 128) * 512 + (n % 32) * 16 + ((n % 128) // 32) * 4 + b % 4
             sc = bph[tile, b // 4, sfo].astype(np.float64) - 127
             terms.append(decode_e4m3(codes) * np.repeat(np.exp2(sc), 32))
-        h[p] = terms[0] + terms[1]
+        h[p] = sum(terms)
     return h
 
 
@@ -239,6 +242,77 @@ def test_full_size_sampled(name, path, n_sample):
     y = bf16_host(g["y"])[toks]
     st = parity_stats(y, ref["y"], c["x"][toks])
     assert_parity(st, f"{name}/{path}")
+
+
+# ------------------------------------------------------------------------------ MXFP8 activations
+# MOE_ACT_MXFP8: the expert inputs and the SwiGLU outputs quantized to E4M3 in 32-value
+# blocks; the oracle models the same quantization (act="mxfp8").  Same bars as the bf16
+# format, plus the distance to the exact-bf16 layer, which the format is allowed to move.
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_parity_mxfp8(name, path):
+    c = case(SMALL[name])
+    cfg = c["cfg"]
+    g = run_gpu(c, path, act="mxfp8")
+    assert g["status"] == moe.MOE_OK, moe.status_string(g["status"])
+    ref = oracle_rows(c, act="mxfp8")
+    y = bf16_host(g["y"])
+    st = parity_stats(y, ref["y"], c["x"])
+    assert_parity(st, f"{name}/{path}/mxfp8")
+    assert st["delta_rel_fro"] <= 2.5e-2, st
+    np.testing.assert_array_equal(np.sort(g["routing"]["topk_idx"].cpu().numpy(), 1), np.sort(ref["idx"], 1))
+    # Against the exact layer (bf16 activations) the format still meets the layer's tolerance
+    # on y.  (Its distance relative to y - x is not bounded here: where the expert output is
+    # small next to x, that ratio mostly counts bf16 rounding flips of y.)
+    exact = parity_stats(y, oracle_rows(c)["y"], c["x"])
+    assert_parity(exact, f"{name}/{path}/mxfp8 vs bf16 layer")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_swiglu_output_h_mxfp8(path):
+    """h as the down GEMM reads it with MXFP8 activations: one E4M3 row per token with its
+    block scale, equal to the oracle's quantized h up to rare one-step rounding flips (h is
+    computed in fp32 here and in fp64 there before both round it)."""
+    c = case(SMALL["mid_ragged"])
+    cfg = c["cfg"]
+    g = run_gpu(c, path, act="mxfp8")
+    assert g["status"] == moe.MOE_OK
+    P = cfg.T * cfg.k
+    h = _h_from_workspace(g, cfg)
+    inv = moe.workspace_view(g["ws"], g["dims"], cfg.T, "inv", torch.int32, (P,)).cpu().numpy()
+    idx = g["routing"]["topk_idx"].cpu().numpy()
+    ref = oracle_rows(c, want_h=True, act="mxfp8")
+    href = synth.bf16_to_f32(ref["h"]).astype(np.float64)
+    same = total = 0
+    num = den = 0.0
+    for t in range(cfg.T):
+        for s in range(cfg.k):
+            so = int(np.nonzero(ref["idx"][t] == idx[t, s])[0][0])
+            a, b = h[inv[t * cfg.k + s]], href[t, so]
+            same += int(np.count_nonzero(a == b))
+            total += a.size
+            num += float((a - b) @ (a - b))
+            den += float(b @ b)
+    assert same / total >= 0.99, same / total
+    assert np.sqrt(num / den) <= 1e-2
+
+
+@pytest.mark.parametrize("name,path,n_sample", [("prefill_20b", "gemm", 32), ("moe_120b", "gemm", 32),
+                                                ("prefill_20b", "gemv", 8)])
+def test_full_size_sampled_mxfp8(name, path, n_sample):
+    c = case(C[name])
+    cfg = c["cfg"]
+    g = run_gpu(c, path, act="mxfp8")
+    assert g["status"] == moe.MOE_OK, moe.status_string(g["status"])
+    np.testing.assert_array_equal(np.sort(g["routing"]["topk_idx"].cpu().numpy(), 1), np.sort(c["route"]["idx"], 1))
+    rng = np.random.default_rng(1)
+    toks = np.sort(rng.choice(cfg.T, size=n_sample, replace=False)).astype(np.int32)
+    toks[0], toks[-1] = 0, cfg.T - 1
+    ref = oracle_rows(c, tokens=toks, act="mxfp8")
+    st = parity_stats(bf16_host(g["y"])[toks], ref["y"], c["x"][toks])
+    assert_parity(st, f"{name}/{path}/mxfp8")
 
 
 # ------------------------------------------------------------------------------ edge cases
