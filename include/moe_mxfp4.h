@@ -78,8 +78,9 @@ typedef enum {
  *   along the projection's reduction axis (the pages' block of one 8-bit scale per 32
  *   values), scale 2^(floor(log2 amax) - 7) clamped to [2^-122, 2^126] (1 for an all-zero
  *   block), elements rounded to the nearest OCP FP8 E4M3 value (ties to even).  Half the
- *   activation bytes and tensor-core work; the output moves by the E4M3 rounding (about
- *   1e-2 of the expert output's norm).  An extension: the pages quantize only the weights. */
+ *   activation bytes and tensor-core work; the E4M3 rounding moves the expert output
+ *   (y - x) by about 5% of its norm at gpt-oss width, more than the exact layer's parity
+ *   tolerance on y.  An extension: the pages quantize only the weights. */
 typedef enum {
   MOE_ACT_BF16 = 0,
   MOE_ACT_MXFP8 = 1
