@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
 
 // ----------------------------------------------------------------------------------
 // Large batches: fused RMSNorm + router + top-k + softmax, kRT tokens per CTA, 256
-// threads.  The reduction axis is walked in chunks of RK through a ring of kNS cp.async
+// threads.  The reduction axis is walked in chunks of RK through a ring of NS cp.async
 // stages, each holding the chunk's bf16 x rows of the CTA's tokens and the router rows
 // [E][RK] (fp32, rows padded by 4 floats so that the float4 reads of 32 consecutive
 // experts hit distinct banks).  Per chunk, warp w first normalizes tokens 2w and 2w + 1
@@ -389,7 +389,6 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
 // in warp order.  Outputs: xq / xsf, topk_idx, topk_w, expert histogram.
 // ----------------------------------------------------------------------------------
 constexpr int kRT = 16;                  // tokens per CTA
-constexpr int kNS = 4;                   // cp.async stages
 constexpr int kTokenKernelMaxT = 256;    // up to this many tokens: one CTA per token
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -401,14 +400,14 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int NJ, int RK>
+template <int NJ, int RK, int NS>
 struct RouteTilesCfg {
   static constexpr int EP = 32 * NJ;
   static constexpr int WST = RK + 4;                       // router row stride (floats)
   static constexpr int W_FLOATS = EP * WST;                // one stage of router rows
   static constexpr int X_HALVES = kRT * RK;                // one stage of x (bf16)
   static constexpr int KW = RK / 8;                        // columns of a chunk per warp
-  static constexpr size_t STAGES = sizeof(float) * (kNS * W_FLOATS + kRT * RK) + 2 * kNS * X_HALVES;
+  static constexpr size_t STAGES = sizeof(float) * (NS * W_FLOATS + kRT * RK) + 2 * NS * X_HALVES;
   // RMSNorm weights (d floats) follow the stages / partials
   static constexpr size_t PARTIALS = sizeof(float) * 8 * kRT * EP;   // final reduction (reuses the stages)
   static constexpr size_t MAIN = STAGES > PARTIALS ? STAGES : PARTIALS;
@@ -416,13 +415,13 @@ struct RouteTilesCfg {
   static_assert(KW % 4 == 0, "float4 columns per warp");
 };
 
-template <int NJ, int RK>
+template <int NJ, int RK, int NS>
 __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
-  using C = RouteTilesCfg<NJ, RK>;
+  using C = RouteTilesCfg<NJ, RK, NS>;
   extern __shared__ __align__(16) float smem[];
-  float* s_w = smem;                                        // [kNS][EP][WST]
-  float* s_xn = smem + kNS * C::W_FLOATS;                   // [kRT][RK]
-  uint16_t* s_x = reinterpret_cast<uint16_t*>(s_xn + kRT * RK);  // [kNS][kRT][RK]
+  float* s_w = smem;                                        // [NS][EP][WST]
+  float* s_xn = smem + NS * C::W_FLOATS;                   // [kRT][RK]
+  uint16_t* s_x = reinterpret_cast<uint16_t*>(s_xn + kRT * RK);  // [NS][kRT][RK]
   float* s_g = smem + C::MAIN / sizeof(float);             // [d] RMSNorm weights
   __shared__ float s_r[kRT];
   pdl_trigger();
@@ -433,8 +432,8 @@ __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
   const int nchunks = d / RK;
   const int dp = a.ws.dp;
 
-  auto issue = [&](int c) {   // chunk c into stage c % kNS
-    const int st = c % kNS, k0 = c * RK;
+  auto issue = [&](int c) {   // chunk c into stage c % NS
+    const int st = c % NS, k0 = c * RK;
     for (int i = tid; i < kRT * (RK / 8); i += 256) {   // x: 16-byte pieces
       const int tt = i / (RK / 8), q = i - tt * (RK / 8);
       if (tt < nt) cp_async16(s_x + (st * kRT + tt) * RK + q * 8, a.x + (int64_t)(t0 + tt) * d + k0 + q * 8);
@@ -444,7 +443,7 @@ __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
       cp_async16(s_w + (st * C::EP + e) * C::WST + q * 4, a.router_w + (int64_t)e * d + k0 + q * 4);
     }
   };
-  for (int c = 0; c < kNS - 1; ++c) {
+  for (int c = 0; c < NS - 1; ++c) {
     if (c < nchunks) issue(c);
     cp_async_commit();
   }
@@ -480,11 +479,11 @@ __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
     for (int j = 0; j < NJ; ++j) acc[t][j] = 0.f;
 
   for (int c = 0; c < nchunks; ++c) {
-    if (c + kNS - 1 < nchunks) issue(c + kNS - 1);
+    if (c + NS - 1 < nchunks) issue(c + NS - 1);
     cp_async_commit();
-    cp_async_wait<kNS - 1>();
+    cp_async_wait<NS - 1>();
     __syncthreads();
-    const int st = c % kNS, k0 = c * RK;
+    const int st = c % NS, k0 = c * RK;
     // normalize this warp's tokens, split into E4M3 terms (warp-private rows of s_xn)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -765,12 +764,16 @@ int launch_route_nj(const FwdArgs& a) {
     ev_after(a);
     return 1;
   }
-  constexpr int RKC = NJ <= 2 ? 64 : 32;   // chunk: router rows of a stage stay small
-  using C = RouteTilesCfg<NJ, RKC>;
+  // chunk width and stages: the router rows of a stage stay within shared memory (up to 128
+  // experts: 64-wide chunks; 128 experts take two stages of 34 KB, which measured faster
+  // than four stages of 32-wide chunks)
+  constexpr int RKC = NJ <= 4 ? 64 : 32;
+  constexpr int NSC = NJ == 4 ? 2 : 4;
+  using C = RouteTilesCfg<NJ, RKC, NSC>;
   const size_t smem = C::smem(a.d);
-  if (!ensure_smem_limit(route_tiles_kernel<NJ, RKC>, smem, tile_limits)) return -1;
+  if (!ensure_smem_limit(route_tiles_kernel<NJ, RKC, NSC>, smem, tile_limits)) return -1;
   ev_before(a);
-  route_tiles_kernel<NJ, RKC><<<(a.T + kRT - 1) / kRT, 256, smem, a.stream>>>(a);
+  route_tiles_kernel<NJ, RKC, NSC><<<(a.T + kRT - 1) / kRT, 256, smem, a.stream>>>(a);
   ev_after(a);
   return 1;
 }
