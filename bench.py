@@ -97,9 +97,18 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def code_sha(text: str) -> str:
+    """Hash of a CUDA/C++ source with its comments and whitespace removed: a capture stays
+    valid across comment edits and goes stale with any change to the code itself."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256("".join(text.split()).encode()).hexdigest()[:16]
+
+
 def file_sha(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(path, encoding="utf-8") as f:
+        return code_sha(f.read())
 
 
 def ncu_traffic(kernel_key, config_name, act="bf16"):

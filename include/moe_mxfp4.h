@@ -169,11 +169,12 @@ moe_status moe_route(const moe_dims* dims, int32_t T, const uint16_t* x, const f
  * counts_out [E].
  * y may not alias x.  T >= 1 (T = 0 returns MOE_OK and launches nothing).
  * Arithmetic: the expert projections run on the tensor cores' block-scaled MMA
- * (E2M1 weights with their E8M0 scales, as stored) with fp32 accumulation.  Each
- * activation (xe, then h) enters as two E4M3 terms with one E8M0 scale per 32 values
- * each: hi = RN(v / 2^s1), lo = RN((v - hi * 2^s1) / 2^s2), s1 and s2 set by the
- * largest |v| and the largest residual of the block.  hi + lo equals v whenever
- * |v| >= 2^-13 * max|block|; smaller values are off by at most 2^-20 * max|block|.
+ * (E2M1 weights with their E8M0 scales, as stored) with fp32 accumulation.  With
+ * MOE_ACT_BF16 each activation (xe, then h) enters as two E4M3 terms with one E8M0 scale
+ * per 32 values each: hi = RN(v / 2^s1), lo = RN((v - hi * 2^s1) / 2^s2), s1 and s2 set by
+ * the largest |v| and the largest residual of the block.  hi + lo equals v whenever
+ * |v| >= 2^-13 * max|block|; smaller values are off by at most 2^-20 * max|block|.  With
+ * MOE_ACT_MXFP8 the hi term alone enters (see moe_act_format).
  * Errors: as moe_route. */
 moe_status moe_forward(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
                        const float* router_w, const float* router_b, const uint8_t* w1_codes,
@@ -211,9 +212,10 @@ int32_t moe_resolve_path(const moe_dims* dims, int32_t T);
  * xq  [T][2][dp] E4M3 (hi and lo terms of xe = bf16(xn) per token; dp = d rounded up to
  *     a multiple of 128), xsf [T][2][dp/32] E8M0 (their scales),
  * bpx / bph: packed activation blocks of xe and of the SwiGLU output h, per token tile
- *     and 128-chunk: the tile's 2 * BN E4M3 rows (hi / lo term of each token) in the
- *     tensor cores' 128-byte-swizzled order, then their scales (BN = 8 on the GEMV path,
- *     96 on the GEMM path),
+ *     and 128-chunk: the tile's 2 * BN E4M3 rows (hi / lo term of each token; BN = 8 on
+ *     the GEMV path, 96 on the GEMM path) or, with MOE_ACT_MXFP8, its BN rows (one per
+ *     token; BN = 16 / 192), in the tensor cores' 128-byte-swizzled order, then their
+ *     scales,
  * ys  [S][T*k][d] fp32 (weighted expert outputs, sorted order; S = 3 planes of partial sums
  *     on the GEMV path, whose down GEMM splits its reduction axis in up to three, else 1);
  * offsets[MOE_WS_FIELDS-1] = total bytes.  Errors: MOE_ERR_INVALID_ARG,

@@ -8,9 +8,10 @@
 //
 // The tensor cores read the MXFP4 weights as stored: tcgen05.mma kind::mxf8f6f4 with an
 // E2M1 A operand (the weights, 128 rows per tile) scaled by its E8M0 block scales, and an
-// E4M3 B operand (the activations) scaled by theirs; fp32 accumulation in TMEM.  Each
-// activation vector is two B columns, its hi and lo E4M3 terms (see e4m3_split), so a
-// tile of BN tokens is an MMA of N = 2*BN and the epilogue adds column pairs.
+// E4M3 B operand (the activations) scaled by theirs; fp32 accumulation in TMEM.  With bf16
+// activations each activation vector is two B columns, its hi and lo E4M3 terms (see
+// e4m3_split), so a tile of BN tokens is an MMA of N = 2*BN and the epilogue adds column
+// pairs (TERMS = 2); with MXFP8 activations a token is one column (TERMS = 1).
 //
 // Persistent kernel, CPS CTAs per SM.  A work item is 128 weight rows x one token tile
 // over the whole reduction axis; CTA b takes items b, b + grid, ...  A pipeline stage
@@ -18,7 +19,7 @@
 //   warps 0..  producers: per stage one TMA load of the weight codes (NP consecutive
 //              8 KB tile blocks; E2M1, unpacked by the copy to one byte per code in
 //              shared memory, 128B swizzle), one bulk copy of the token tile's packed
-//              activation blocks (2*BN E4M3 rows per chunk, already in the swizzled order,
+//              activation blocks (TERMS*BN E4M3 rows per chunk, already in the swizzled order,
 //              followed by their scale factors) and one bulk copy of the weight scale
 //              factors (stored in the tensor cores' scale-factor layout);
 //   warp 1     TMEM allocation and the MMA issuer (one thread): per stage it copies the
@@ -357,7 +358,8 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>::THREADS
         // Per read of TC tokens the gate thread of feature f (lane row f < 64) and the up
         // thread of f (row f + 64) trade: the gate side finishes the first HT tokens, the
         // up side the rest.  Each warp then holds one 32-feature block of h per token and
-        // splits it into E4M3 hi / lo terms for the down GEMM.
+        // splits it into E4M3 hi / lo terms for the down GEMM (the hi term alone, h rounded
+        // to MXFP8, when TERMS = 1).
         float* s_x = reinterpret_cast<float*>(gepi);  // [TC tokens][64 features]
         const float L = p.limit;
         const bool gate_side = q < 2;
@@ -596,7 +598,8 @@ int launch_one(const FwdArgs& a) {
 }
 
 // Pipeline shapes (compile-time; overridable with -D for tuning builds).
-// Small batches (few tokens per expert): 8-token tiles (MMA N = 16), three independent
+// Small batches (few tokens per expert): 8-token tiles (MMA N = 16; 16 tokens with MXFP8
+// activations), three independent
 // pipelines (CTAs) per SM: each CTA's copies are served in order, so more CTAs keep
 // more of HBM's requests in flight.
 #ifndef MOE_GEMV_NP
