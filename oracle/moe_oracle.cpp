@@ -244,17 +244,20 @@ int32_t oracle_quantize(const float* w, int64_t rows, int32_t K, uint8_t* codes,
 // Decode rows to fp64: value = E2M1(code) * 2^(byte - 127).  Returns 1 if a
 // scale byte is 0xFF (the E8M0 NaN encoding), else 0.
 int32_t oracle_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int32_t K, double* out) {
-  int32_t status = 0;
+  std::atomic<int32_t> status{0};
   const int nb = K / 32;
-  for (int64_t r = 0; r < rows; ++r)
-    for (int32_t k = 0; k < K; ++k) {
-      const uint8_t byte = codes[r * (K / 2) + k / 2];
-      const int c = (k & 1) ? (byte >> 4) : (byte & 15);
-      const uint8_t sb = scales[r * nb + k / 32];
-      if (sb == 0xFF) status = 1;
-      out[r * K + k] = e2m1_value(c) * std::ldexp(1.0, (int)sb - 127);
-    }
-  return status;
+  // Every element is decoded on its own; rows are split over threads.
+  parallel_chunks(rows, 0, [&](int64_t r0, int64_t r1) {
+    for (int64_t r = r0; r < r1; ++r)
+      for (int32_t k = 0; k < K; ++k) {
+        const uint8_t byte = codes[r * (K / 2) + k / 2];
+        const int c = (k & 1) ? (byte >> 4) : (byte & 15);
+        const uint8_t sb = scales[r * nb + k / 32];
+        if (sb == 0xFF) status = 1;
+        out[r * K + k] = e2m1_value(c) * std::ldexp(1.0, (int)sb - 127);
+      }
+  });
+  return status.load();
 }
 
 // ---------------------------------------------------------------------------
