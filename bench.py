@@ -7,6 +7,12 @@ seeded synthetic tensors of the workload's shapes (``synth``) and are resident
 in HBM before the timed region; the L2 is flushed (256 MiB write) before every
 step, outside the step's events.
 
+The line is headlined by the largest single-GPU workload, the skewed-routing
+gpt-oss-120b batch (T = 16384, E = 128, tensor-bound: the "% of FP4 tensor peak"
+half of the metric).  The gpt-oss-20b decode batch (T = 16, E = 32, HBM-bound:
+the "% of HBM bandwidth" half) is measured in the same run and reported under
+``"decode"`` with its own timing, roofline and end-to-end figures.
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--path auto|gemv|gemm]
     python bench.py --impl reference ...   # the CPU oracle on the host cores, same metric
 
@@ -17,7 +23,6 @@ over ranks and ``value`` counts the tokens of all ranks.
 from __future__ import annotations
 
 import argparse
-import ctypes
 import hashlib
 import json
 import os
@@ -34,7 +39,8 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "MoE-layer tokens/s on 1 B200; % of FP4 tensor peak (prefill) / HBM BW (decode)"
-DEFAULT_CONFIG = "decode_20b"
+HEADLINE_CONFIG = "skew_120b"
+DECODE_CONFIG = "decode_20b"
 WORKLOAD_TEXT = {
     "tiny": "tiny MoE layer: T=32, d=128, I=128, E=4, top-2, MXFP4 block 32",
     "decode_20b": "gpt-oss-20b MoE layer, decode: T=16, d=2880, I=2880, E=32, top-4, MXFP4 experts",
@@ -43,25 +49,39 @@ WORKLOAD_TEXT = {
     "skew_120b": "skewed routing: T=16384, d=I=2880, E=128, top-4, Zipf(1.2) router bias, MXFP4 experts",
 }
 KERNELS = ["route", "group", "pack", "gate_up", "down", "combine"]
+KERNELS_FUSED = ["route", "pack", "gate_up", "down"]     # small batches: grouping and combine fused
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FP4_DENSE_NOMINAL_TFLOPS = 9000.0
+# dense tensor-core rate of each MMA kind relative to bf16 (NVIDIA's B200 figures:
+# bf16 2.25, fp8 4.5, fp4 9 PFLOP/s dense)
+RATE_VS_BF16 = {"fp8": 2.0, "fp4": 4.0}
+CSRC = os.path.join(ROOT, "mxfp4_expert_gemm_b200", "csrc")
+# source files whose code a kernel's counters depend on (the kernel's file and its headers)
+KERNEL_SOURCES = {
+    "gate_up": ["moe_mx.cu", "moe_internal.cuh", "sm100_ptx.cuh"],
+    "down": ["moe_mx.cu", "moe_internal.cuh", "sm100_ptx.cuh"],
+    "route": ["moe_route.cu", "moe_internal.cuh"],
+    "group": ["moe_route.cu", "moe_internal.cuh"],
+    "pack": ["moe_route.cu", "moe_internal.cuh"],
+    "combine": ["moe_route.cu", "moe_internal.cuh"],
+}
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(synth.CONFIGS))
+    ap.add_argument("--config", default=None, choices=list(synth.CONFIGS),
+                    help="measure this workload alone (default: the skewed 120b batch, plus the 20b decode batch)")
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
     ap.add_argument("--act", default="bf16", choices=["bf16", "mxfp8"],
                     help="activation format of the expert GEMMs: exact bf16 (the layer as stated) or MXFP8")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of "
                     "replaying a captured CUDA graph")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
-    return ap.parse_args()
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget per workload")
+    return ap.parse_args(argv)
 
 
 def dist_env():
@@ -111,19 +131,29 @@ def file_sha(path):
         return code_sha(f.read())
 
 
+def sources_sha(files) -> str:
+    """Hash of the code (without comments) of several source files, in the given order."""
+    text = "".join(open(os.path.join(CSRC, f), encoding="utf-8").read() + "\n" for f in files)
+    return code_sha(text)
+
+
+def traffic_key(config_name, act="bf16"):
+    return config_name if act == "bf16" else f"{config_name}/{act}"
+
+
 def ncu_traffic(kernel_key, config_name, act="bf16"):
-    """Per-launch DRAM bytes from a committed ncu capture, if it still matches the kernel source
-    (captures of the MXFP8 activation format are filed under "<config>/mxfp8")."""
+    """Per-launch DRAM bytes of a kernel from a committed ncu capture, while the capture still
+    matches the code of the kernel and its headers (captures of the MXFP8 activation format
+    are filed under "<config>/mxfp8"); None otherwise."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     try:
         d = json.load(open(p))
-        ent = d.get(config_name if act == "bf16" else f"{config_name}/{act}", {}).get(kernel_key)
+        ent = d.get(traffic_key(config_name, act), {}).get(kernel_key)
         if not ent:
             return None
-        src = os.path.join(ROOT, "mxfp4_expert_gemm_b200", "csrc", ent["source"])
-        if file_sha(src) != ent["source_sha"]:
+        if sources_sha(ent["sources"]) != ent["source_sha"]:
             return None
         return ent["dram_bytes_per_launch"]
     except Exception:
@@ -153,16 +183,19 @@ class ClockSampler:
             self.max_mhz = None
         self._stop = threading.Event()
 
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def __enter__(self):
@@ -186,7 +219,7 @@ class ClockSampler:
 # ------------------------------------------------------------------------------ inputs
 
 
-def device_inputs(cfg, rank, need_oracle_weights):
+def device_inputs(cfg, rank):
     """Hidden rows (this rank's tokens), router, and MXFP4 weights quantized on the GPU."""
     import torch
     import mxfp4_expert_gemm_b200 as moe
@@ -201,42 +234,48 @@ def device_inputs(cfg, rank, need_oracle_weights):
     w1s = torch.empty(s1s, dtype=torch.uint8, device=dev)
     w2c = torch.empty(s2c, dtype=torch.uint8, device=dev)
     w2s = torch.empty(s2s, dtype=torch.uint8, device=dev)
-    ow = None
-    if need_oracle_weights:
-        import oracle
-        ow = (np.empty((E, 2 * I, d // 2), np.uint8), np.empty((E, 2 * I, d // 32), np.uint8),
-              np.empty((E, d, I // 2), np.uint8), np.empty((E, d, I // 32), np.uint8))
     for e in range(E):
-        w1 = synth.w1_expert(cfg, e)
-        moe.moe_mxfp4_quantize(torch.from_numpy(w1).to(dev), w1c[e:e + 1], w1s[e:e + 1], role="gate_up")
-        w2 = synth.w2_expert(cfg, e)
-        moe.moe_mxfp4_quantize(torch.from_numpy(w2).to(dev), w2c[e:e + 1], w2s[e:e + 1], role="down")
-        if ow is not None:
-            ow[0][e], ow[1][e] = oracle.quantize(w1)
-            ow[2][e], ow[3][e] = oracle.quantize(w2)
+        moe.moe_mxfp4_quantize(torch.from_numpy(synth.w1_expert(cfg, e)).to(dev), w1c[e:e + 1], w1s[e:e + 1],
+                               role="gate_up")
+        moe.moe_mxfp4_quantize(torch.from_numpy(synth.w2_expert(cfg, e)).to(dev), w2c[e:e + 1], w2s[e:e + 1],
+                               role="down")
     torch.cuda.synchronize()
     xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
     return dict(x=x, gamma=gamma, rw=rw, rb=rb, x_dev=xt, gamma_dev=torch.from_numpy(gamma).to(dev),
                 rw_dev=torch.from_numpy(rw).to(dev), rb_dev=torch.from_numpy(rb).to(dev),
-                W=(w1c, w1s, w2c, w2s), oracle_W=ow)
+                W=(w1c, w1s, w2c, w2s))
 
 
 # ------------------------------------------------------------------------------ CPU oracle timing
 
 
-def time_oracle(cfg, inp, budget_s, tokens_per_step=None, steps=None, warmup=0, act="bf16"):
-    """Time the CPU oracle (as it stands) on samples of the workload's tokens.
+def oracle_inputs(cfg, x, tokens):
+    """The oracle's inputs for a sample of tokens: router tensors and the MXFP4 weights of the
+    experts the oracle's own routing picks for them (the other experts are never read)."""
+    import oracle
+    gamma, rw, rb = synth.norm_weight(cfg), synth.router_weight(cfg), synth.router_bias(cfg)
+    used = np.unique(oracle.route(x[tokens], gamma, rw, rb, cfg.k, cfg.rms_eps)["idx"])
+    E, d, I = cfg.E, cfg.d, cfg.I
+    ow = (np.zeros((E, 2 * I, d // 2), np.uint8), np.zeros((E, 2 * I, d // 32), np.uint8),
+          np.zeros((E, d, I // 2), np.uint8), np.zeros((E, d, I // 32), np.uint8))
+    for e in used.tolist():
+        ow[0][e], ow[1][e] = oracle.quantize(synth.w1_expert(cfg, e))
+        ow[2][e], ow[3][e] = oracle.quantize(synth.w2_expert(cfg, e))
+    return dict(x=x, gamma=gamma, rw=rw, rb=rb, oracle_W=ow)
 
-    Returns (tokens/s, threads, sample description)."""
+
+def time_oracle(cfg, inp, tokens_per_call, budget_s=None, steps=None, warmup=0, act="bf16", vary=True):
+    """Time the CPU oracle (as it stands) on calls of ``tokens_per_call`` consecutive tokens of
+    the workload (the next tokens each call, or with ``vary`` False the first ones every
+    call); run until ``budget_s`` seconds (after at least one call) or for ``warmup + steps``
+    calls.  Returns (tokens/s, threads, sample description)."""
     import oracle
     T = cfg.T
-    n = tokens_per_step or T
-    order = np.arange(T, dtype=np.int32)
-    times, done = [], 0
+    n = tokens_per_call
+    times, done, i = [], 0, 0
     t_start = time.perf_counter()
-    i = 0
     while True:
-        toks = order[(np.arange(n) + i * n) % T]
+        toks = ((np.arange(n) + (i if vary else 0) * n) % T).astype(np.int32)
         t0 = time.perf_counter()
         oracle.moe_forward(inp["x"], inp["gamma"], inp["rw"], inp["rb"], *inp["oracle_W"], I=cfg.I, k=cfg.k,
                            eps=cfg.rms_eps, limit=cfg.swiglu_limit, tokens=toks, act=act)
@@ -251,42 +290,39 @@ def time_oracle(cfg, inp, budget_s, tokens_per_step=None, steps=None, warmup=0, 
         elif time.perf_counter() - t_start >= budget_s and times:
             break
     total = sum(times)
-    sample = f"{len(times)} oracle forward(s) of {n} token(s) each from the {cfg.name} batch ({total:.1f} s)"
+    which = "consecutive tokens" if vary else "the batch's first tokens every time"
+    sample = (f"{len(times)} oracle forward(s) of {n} token(s) each ({which}) from the {cfg.name} batch "
+              f"({total:.1f} s, fp64, all host threads)")
     return done / total, os.cpu_count(), sample
+
+
+def cpu_tokens_per_call(cfg):
+    """A bounded oracle sample: one call is a few seconds of host work at gpt-oss width."""
+    return min(cfg.T, 256)
 
 
 # ------------------------------------------------------------------------------ our arm
 
 
-def run_ours(args, rank, world, local_rank):
+def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
+    """One workload: timed steps (graph replay), per-kernel times, roofline, end to end,
+    clocks and the CPU oracle baseline.  Returns the workload's record."""
     import torch
     import mxfp4_expert_gemm_b200 as moe
-    torch.cuda.set_device(local_rank)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        pg = dist
-    cfg = synth.CONFIGS[args.config]
-    want_cpu = (rank == 0 and world == 1 and not args.no_cpu_baseline)
-    inp = device_inputs(cfg, rank, need_oracle_weights=want_cpu)
+    inp = device_inputs(cfg, rank)
     dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, cfg.rms_eps, cfg.swiglu_limit, path=args.path, act=args.act)
     ws = moe.new_workspace(dims, cfg.T)
     y = torch.empty_like(inp["x_dev"])
-    stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    nk = len(KERNELS)
     W = inp["W"]
+    fwd = (dims, inp["x_dev"], inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws)
 
-    def step(events=None):
-        # the current stream: inside a graph capture this is the capturing stream
-        moe.moe_forward_timed(dims, inp["x_dev"], inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws, y=y,
-                              events=events)
+    def plain_step():
+        moe.moe_forward(*fwd, y=y)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
-        step()
+        plain_step()
     torch.cuda.synchronize()
     st = moe.moe_device_status(ws)
     if st != moe.MOE_OK:
@@ -296,14 +332,9 @@ def run_ours(args, rank, world, local_rank):
     K = args.steps
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)]]
-    for e in [*starts, *stops, *kev[0]]:
+    for e in [*starts, *stops]:
         e.record()  # creates the underlying CUDA events
     torch.cuda.synchronize()
-
-    def plain_step():
-        moe.moe_forward(dims, inp["x_dev"], inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws, y=y)
-
     use_graph = not args.no_graph
     graph = None
     if use_graph:
@@ -330,29 +361,40 @@ def run_ours(args, rank, world, local_rank):
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
-    total_ms = float(sum(step_ms))
+    total_ms = float(sum(a.elapsed_time(b) for a, b in zip(starts, stops)))
     plain_step()
     launches = moe.last_launch_count() * K   # kernels per forward x timed steps
+    del graph
+
     # ---- instrumented pass (outside the timed region): the same steps with a CUDA event
-    # pair around each of the library's launches, replayed from one graph per step
+    # pair around each of the library's launches, replayed from one graph
+    kev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(KERNELS))]
+    for e in kev:
+        e.record()
+    torch.cuda.synchronize()
+
+    def timed_step():
+        moe.moe_forward_timed(*fwd, y=y, events=kev)
+
     kgraph = None
     if use_graph:
         kgraph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(kgraph):
-            step(kev[0])
+            timed_step()
+    else:
+        timed_step()
     n_timed = moe.last_launch_count()
-    names = KERNELS if n_timed == len(KERNELS) else ["route", "pack", "gate_up", "down"]
+    names = KERNELS if n_timed == len(KERNELS) else KERNELS_FUSED
     per_kernel = {name: [] for name in names[:n_timed]}
     for i in range(K):
         flush.zero_()
         if use_graph:
             kgraph.replay()
         else:
-            step(kev[0])
+            timed_step()
         torch.cuda.synchronize()
         for j, name in enumerate(names[:n_timed]):
-            per_kernel[name].append(kev[0][2 * j].elapsed_time(kev[0][2 * j + 1]))
+            per_kernel[name].append(kev[2 * j].elapsed_time(kev[2 * j + 1]))
     del kgraph
     st = moe.moe_device_status(ws)
     if st != moe.MOE_OK:
@@ -360,13 +402,14 @@ def run_ours(args, rank, world, local_rank):
     kern_ms = {name: statistics.mean(v) for name, v in per_kernel.items()}
     total_ms = max_over_ranks(total_ms, pg)
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers (pinned)
     x_host = torch.empty(inp["x_dev"].shape, dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(inp["x_dev"].cpu())
     y_host = torch.empty_like(x_host, pin_memory=True)
     e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     e_stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     x_dev2 = torch.empty_like(inp["x_dev"])
+
     def e2e_step():
         x_dev2.copy_(x_host, non_blocking=True)
         moe.moe_forward(dims, x_dev2, inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws, y=y)
@@ -393,60 +436,62 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(e_starts, e_stops)))
     e2e_ms = max_over_ranks(e2e_ms, pg)
+    del e2e_graph
     assert moe.moe_device_status(ws) == moe.MOE_OK
 
-    # ---- roofline of the dominant kernel
+    # ---- roofline of the dominant kernel (gate_up) and of the layer
     peaks, peak_src = load_peaks()
-    counts = np.bincount(_routing(moe, dims, inp, ws, cfg).ravel(), minlength=cfg.E)
+    counts = np.bincount(moe.moe_route(dims, inp["x_dev"], inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"],
+                                       ws)["topk_idx"].cpu().numpy().ravel(), minlength=cfg.E)
     used = int(np.count_nonzero(counts))
     P = cfg.T * cfg.k
     d, I = cfg.d, cfg.I
     w1_bytes = 2 * I * d // 2 + (d // 32) * 2 * I
     w2_bytes = d * I // 2 + (I // 32) * d
-    decode_like = (P / cfg.E) <= 24
-    gu_ms = kern_ms.get("gate_up")
-    if decode_like:
-        alg = used * w1_bytes + P * d * 2 + P * I * 2   # expert weights streamed once + activations in/out
+    gu_ms = kern_ms["gate_up"]
+    layer_ms = total_ms / K
+    traffic = ncu_traffic("gate_up", cfg.name, args.act)
+    if (P / cfg.E) <= 24:   # few tokens per expert: the weight stream bounds the layer
+        alg = used * w1_bytes + P * d * 2 + P * I * 2   # expert weights streamed once + activations in / out
         achieved = alg / (gu_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "kernel": "gate_up (mx_expert_kernel<GATE_UP>)", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                "traffic": ncu_traffic("gate_up", cfg.name, args.act),
-                "algorithmic_bytes_per_launch": alg, "launch_ms": round(gu_ms, 5), "peak_source": f"hbm_gbs, {peak_src}"}
+                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                "algorithmic_bytes_per_launch": alg, "launch_ms": round(gu_ms, 5),
+                "peak_source": f"hbm_gbs, {peak_src}"}
         layer_bytes = used * (w1_bytes + w2_bytes)
-        layer_ms = total_ms / K
-        roof["layer"] = {"unique_expert_bytes": layer_bytes, "experts_used": used,
-                         "achieved_GBps": round(layer_bytes / (layer_ms * 1e-3) / 1e9, 1),
-                         "frac_of_measured_hbm": round(layer_bytes / (layer_ms * 1e-3) / 1e9 / peak, 4),
-                         "frac_of_8TBps": round(layer_bytes / (layer_ms * 1e-3) / 8e12, 4)}
-    else:
+        gbps = layer_bytes / (layer_ms * 1e-3) / 1e9
+        roof["layer"] = {"unique_expert_bytes": layer_bytes, "experts_used": used, "achieved_GBps": round(gbps, 1),
+                         "frac_of_peak": round(gbps / peak, 4), "frac_of_8TBps": round(gbps * 1e9 / 8e12, 4)}
+    else:                   # many tokens per expert: the tensor cores bound the layer
         alg = 4 * d * I * P
         achieved = alg / (gu_ms * 1e-3) / 1e12
-        # kind::mxf8f6f4 runs at the fp8 rate: nominal fp8 / bf16 = 2 (4.5 vs 2.25 PFLOP/s dense)
-        peak = round(2.0 * peaks["bf16_tflops"], 1)
+        fp8_peak = round(RATE_VS_BF16["fp8"] * peaks["bf16_tflops"], 1)
+        fp4_peak = round(RATE_VS_BF16["fp4"] * peaks["bf16_tflops"], 1)
         cols = 1 if args.act == "mxfp8" else 2   # E4M3 MMA columns per token
         roof = {"bound": "tensor", "kernel": "gate_up (mx_expert_kernel<GATE_UP>)", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": ncu_traffic("gate_up", cfg.name, args.act), "algorithmic_flops_per_launch": alg,
-                "mma_flops_per_launch": cols * alg, "mma_frac": round(cols * achieved / peak, 4),
-                "launch_ms": round(gu_ms, 5),
-                "peak_source": f"2 x bf16_tflops burst ({peak_src}): the block-scaled E2M1 x E4M3 MMA runs at the "
-                               "fp8 rate; " + ("each activation is two E4M3 columns, so the MMA does 2x the "
-                                               "algorithmic flops" if cols == 2 else "MXFP8 activations: one "
-                                               "E4M3 column per token")}
+                "peak": fp8_peak, "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4), "traffic": traffic,
+                "algorithmic_flops_per_launch": alg, "launch_ms": round(gu_ms, 5),
+                "peak_source": f"2 x bf16_tflops burst ({peak_src}): the block-scaled E2M1 x E4M3 MMA "
+                               "(kind::mxf8f6f4) runs at the fp8 rate",
+                "mma_flops_per_launch": cols * alg, "mma_frac": round(cols * achieved / fp8_peak, 4),
+                "mma_note": ("each bf16 activation enters the MMA as two E4M3 columns (hi and lo terms), so the "
+                             "MMA executes 2x the algorithmic flops" if cols == 2 else
+                             "MXFP8 activations: one E4M3 column per token"),
+                "frac_of_fp4_peak": round(achieved / fp4_peak, 4),
+                "fp4_peak": fp4_peak, "fp4_peak_source": f"4 x bf16_tflops burst ({peak_src})"}
         layer_flops = 6 * d * I * P
-        layer_ms = total_ms / K
-        roof["layer"] = {"flops": layer_flops, "achieved_TFLOPs": round(layer_flops / (layer_ms * 1e-3) / 1e12, 1),
-                         "frac_of_fp4_dense_nominal": round(layer_flops / (layer_ms * 1e-3) / 1e12 / FP4_DENSE_NOMINAL_TFLOPS, 4)}
+        tfl = layer_flops / (layer_ms * 1e-3) / 1e12
+        roof["layer"] = {"flops": layer_flops, "achieved_TFLOPs": round(tfl, 1),
+                         "frac_of_fp8_peak": round(tfl / fp8_peak, 4), "frac_of_fp4_peak": round(tfl / fp4_peak, 4)}
 
-    value = job_throughput(cfg.T, world, K, total_ms)
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
-        "warmup": max(3, args.warmup), "ms_per_step": round(total_ms / K, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "e2m1xe4m3", "data": "synthetic",
+    rec = {
+        "value": round(job_throughput(cfg.T, world, K, total_ms), 1), "unit": "tokens/s",
+        "ms_per_step": round(total_ms / K, 5),
         "config": {"workload": WORKLOAD_TEXT[cfg.name], "name": cfg.name, "tokens_per_gpu": cfg.T,
                    "global_batch": cfg.T * world, "path": path_used, "parallelism": f"dp{world}",
-                   "activations": "exact bf16" if args.act == "bf16" else "MXFP8 (E4M3, 32-value blocks)",
+                   "activations": ("bf16, exact (each value carried into the MMA as two E4M3 terms)"
+                                   if args.act == "bf16" else "MXFP8 (E4M3 in 32-value blocks)"),
                    "l2": "flushed before every step (256 MiB write, outside the step events)",
                    "timing": "sum of per-step CUDA events on the launching stream; max over ranks",
                    "launch": "CUDA graph replay per step" if use_graph else "host launches per step",
@@ -458,21 +503,48 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
+    del ws, flush, W, inp["W"]
     if want_cpu:
-        v, cores, sample = time_oracle(cfg, inp, args.cpu_seconds, act=args.act)
-        line["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                "sample": sample}
+        n = cpu_tokens_per_call(cfg)
+        v, cores, sample = time_oracle(cfg, oracle_inputs(cfg, inp["x"], np.arange(n)), n,
+                                       budget_s=args.cpu_seconds, act=args.act, vary=False)
+        rec["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": sample}
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    torch.cuda.set_device(local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    want_cpu = (rank == 0 and world == 1 and not args.no_cpu_baseline)
+    names = [args.config] if args.config else [HEADLINE_CONFIG, DECODE_CONFIG]
+    recs = [measure(synth.CONFIGS[n], args, rank, world, local_rank, pg, want_cpu) for n in names]
+    head = recs[0]
+    line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "mxfp4xbf16" if args.act == "bf16" else "mxfp4xmxfp8",
+            "dtype_note": ("MXFP4 (E2M1 + E8M0) weights x bf16 activations, each carried into the tensor cores "
+                           "as two E4M3 terms with their block scales; fp32 accumulation"
+                           if args.act == "bf16" else "MXFP4 weights x MXFP8 (E4M3) activations; fp32 accumulation"),
+            "data": "synthetic"}
+    for key in ("config", "kernel_ms", "roofline", "e2e", "gpu_launches", "clocks", "cpu_baseline"):
+        if key in head:
+            line[key] = head[key]
+    if len(recs) > 1:
+        line["decode"] = recs[1]
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, e2e_graph
     if pg:
         pg.barrier()
         pg.destroy_process_group()
-
-
-def _routing(moe, dims, inp, ws, cfg):
-    out = moe.moe_route(dims, inp["x_dev"], inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], ws)
-    return out["topk_idx"].cpu().numpy()
 
 
 # ------------------------------------------------------------------------------ reference arm
@@ -481,22 +553,14 @@ def _routing(moe, dims, inp, ws, cfg):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    cfg = synth.CONFIGS[args.config]
-    import oracle
+    cfg = synth.CONFIGS[args.config or HEADLINE_CONFIG]
     x = synth.hidden(cfg)
-    inp = dict(x=x, gamma=synth.norm_weight(cfg), rw=synth.router_weight(cfg), rb=synth.router_bias(cfg))
-    E, d, I = cfg.E, cfg.d, cfg.I
-    ow = (np.empty((E, 2 * I, d // 2), np.uint8), np.empty((E, 2 * I, d // 32), np.uint8),
-          np.empty((E, d, I // 2), np.uint8), np.empty((E, d, I // 32), np.uint8))
-    for e in range(E):
-        ow[0][e], ow[1][e] = oracle.quantize(synth.w1_expert(cfg, e))
-        ow[2][e], ow[3][e] = oracle.quantize(synth.w2_expert(cfg, e))
-    inp["oracle_W"] = ow
     # one token per step keeps --steps K --warmup W within minutes on the host cores
     n = 1
+    calls = args.warmup + args.steps
+    inp = oracle_inputs(cfg, x, (np.arange(calls * n)) % cfg.T)
     t0 = time.perf_counter()
-    v, cores, sample = time_oracle(cfg, inp, 0, tokens_per_step=n, steps=args.steps, warmup=args.warmup,
-                                   act=args.act)
+    v, cores, sample = time_oracle(cfg, inp, n, steps=args.steps, warmup=args.warmup, act=args.act)
     wall = time.perf_counter() - t0
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(n / v * 1e3, 3),

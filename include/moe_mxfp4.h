@@ -245,13 +245,18 @@ int32_t moe_last_launch_count(void);
  * that loads the library until the process exits.  T whose moe_workspace_bytes() exceed
  * 16 MiB is rejected with MOE_ERR_WORKSPACE (at d = I = 2880, E = 32, top-4: up to 56
  * tokens).
- * The first call on a device looks up the array's device address for that device
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * The first call in a CUDA context (normally a device's primary context) looks up the
+ * array's device address in that context (cudaGetSymbolAddress) and remembers it for that
+ * context; make that first call before any stream capture.  After cudaDeviceReset the
+ * next call in the new context looks the address up again.
  * All calls share the one array and it keeps the previous call's contents; the device
  * status word and the expert counters are cleared by every call.  Calls that overlap on
  * the GPU (unordered streams, or several host threads) race on the array.
- * Arguments as moe_forward; status_out (device int32, may be NULL) receives the call's
- * device status word (0 = MOE_OK) on `stream` once the call's kernels have run. */
+ * Arguments as moe_forward; status_out (device int32, 4-byte aligned, may be NULL)
+ * receives the call's device status word (0 = MOE_OK) on `stream` once the call's kernels
+ * have run (with T = 0: 0).  When the call returns an error, status_out is not written.
+ * Errors: as moe_forward (the same codes for the same argument errors), and
+ * MOE_ERR_WORKSPACE for T beyond the array. */
 moe_status moe_forward_no_alloc(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
                                 const float* router_w, const float* router_b, const uint8_t* w1_codes,
                                 const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,

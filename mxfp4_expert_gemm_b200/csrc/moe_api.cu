@@ -96,6 +96,10 @@ moe_status copy_out(void* dst, const void* src, size_t bytes, cudaStream_t st) {
 
 }  // namespace
 
+namespace moe {
+moe_status validate_dims(const moe_dims* dims, int32_t T) { return check_dims(dims, T); }
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_mxfp4_codes_bytes(int32_t E, int32_t N, int32_t K) {

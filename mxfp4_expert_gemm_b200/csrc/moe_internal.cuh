@@ -206,6 +206,15 @@ inline Ws ws_pointers(void* base, const WsLayout& L, int E) {
 // Hence hi * 2^s1 + lo * 2^s2 == v for every v of the block within a factor 2^13 of the
 // largest, and within 2^-20 of the largest otherwise.
 
+// fp32 -> bf16 bit pattern, round to nearest, ties to even.  A NaN stays a NaN (quiet,
+// sign kept); the rounding carry alone could turn a NaN whose payload sits in the low 16
+// bits into an infinity.
+__device__ __forceinline__ uint16_t bf16_bits_rne(float f) {
+  const uint32_t u = __float_as_uint(f);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x0040u);
+  return (uint16_t)((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+}
+
 // floor(log2(a)) for a finite a > 0 (normal or subnormal), exactly.
 __device__ __forceinline__ int floor_log2f(float a) {
   const uint32_t bits = __float_as_uint(a);
@@ -352,5 +361,6 @@ int launch_combine(const FwdArgs& a);   // y = x + sum_j ys[inv]
 int launch_experts(const FwdArgs& a);   // block-scaled tcgen05 expert MLPs (gate_up, down)
 int expert_tile_tokens(int path, int terms);   // token tile of a path
 int expert_down_split(int path);        // reduction-axis splits of a path's down GEMM
+moe_status validate_dims(const moe_dims* dims, int32_t T);   // the argument checks of every call
 
 }  // namespace moe

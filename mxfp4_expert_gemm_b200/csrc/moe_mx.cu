@@ -393,9 +393,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>::THREADS
             const float gv = fminf(gate_side ? mine : other, L);
             const float uv = fminf(fmaxf(gate_side ? other : mine, -L), L);
             float hv = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;   // silu(g) * u
-            uint32_t bits = __float_as_uint(hv);
-            bits = (bits + 0x7FFFu + ((bits >> 16) & 1u)) & 0xFFFF0000u;    // round to bf16
-            hv = __uint_as_float(bits);
+            hv = __uint_as_float((uint32_t)bf16_bits_rne(hv) << 16);   // h is stored as bf16
             const float vv[1] = {hv};
             uint32_t hi, lo, s1, s2;
             e4m3_split<1>(vv, hi, lo, s1, s2);
@@ -466,9 +464,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>::THREADS
                   for (int sp = 0; sp < ksplit; ++sp)
                     accv += __ldcg(p.ys + ((int64_t)sp * p.P + srow) * p.d + gc);
                 }
-                uint32_t bb = __float_as_uint(accv);
-                bb = (bb + 0x7FFFu + ((bb >> 16) & 1u)) >> 16;   // round to bf16
-                p.y[(int64_t)tok * p.d + gc] = (uint16_t)bb;
+                p.y[(int64_t)tok * p.d + gc] = bf16_bits_rne(accv);
               }
             }
             group_sync();

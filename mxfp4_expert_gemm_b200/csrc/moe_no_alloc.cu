@@ -12,6 +12,7 @@
 // without ordering) race on it.  It keeps the previous call's contents; the parts that
 // must start at zero (the device status word, the expert counters) are cleared on every
 // call.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <mutex>
 
@@ -20,26 +21,56 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
-constexpr int kMaxDevices = 64;
+constexpr int kMaxContexts = 64;
 
 __device__ __align__(256) uint8_t g_no_alloc_scratch[kNoAllocScratchBytes];
 
+// The array's address belongs to a CUDA context (the module is loaded once per context),
+// so the lookup is remembered per current context.
+struct ScratchEntry {
+  CUcontext ctx;
+  void* ptr;
+};
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+ScratchEntry g_scratch[kMaxContexts] = {};
+int g_scratch_n = 0;
 
-// Device address of the scratch array on the current device.  The array's name in host
-// code is only a host-side handle; the address must come from cudaGetSymbolAddress,
-// once per device, with that device current.
-moe_status scratch_for_current_device(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
+}
+
+// Device address of the scratch array in the current context.  In host code the array's
+// name is only a host-side handle; the address comes from cudaGetSymbolAddress with the
+// context current.
+moe_status scratch_for_current_context(void** out) {
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return MOE_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  for (int i = 0; ctx && i < g_scratch_n; ++i)
+    if (g_scratch[i].ctx == ctx) {
+      *out = g_scratch[i].ptr;
+      return MOE_OK;
+    }
+  // (the lookup also makes the current device's primary context current when no context
+  // was yet)
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+  if (!ctx && (get(&ctx) != CUDA_SUCCESS || !ctx)) return MOE_ERR_CUDA;
+  if (g_scratch_n < kMaxContexts) g_scratch[g_scratch_n++] = {ctx, p};
+  *out = p;
   return MOE_OK;
 }
 
@@ -51,14 +82,18 @@ moe_status moe_forward_no_alloc(const moe_dims* dims, int32_t T, const uint16_t*
                                 const float* router_w, const float* router_b, const uint8_t* w1_codes,
                                 const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
                                 uint16_t* y, int32_t* status_out, void* stream) {
-  const size_t need = moe_workspace_bytes(dims, T);
-  if (need == 0) return dims ? MOE_ERR_UNSUPPORTED_SHAPE : MOE_ERR_INVALID_ARG;
-  if (need > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
-  if (T == 0) return MOE_OK;
-  void* ws = nullptr;
-  moe_status st = scratch_for_current_device(&ws);
+  moe_status st = moe::validate_dims(dims, T);   // the same argument errors as moe_forward
   if (st != MOE_OK) return st;
+  if (status_out && (reinterpret_cast<uintptr_t>(status_out) & 3u)) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {   // nothing to compute; the call's status is OK
+    if (status_out && cudaMemsetAsync(status_out, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (moe_workspace_bytes(dims, T) > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
+  void* ws = nullptr;
+  st = scratch_for_current_context(&ws);
+  if (st != MOE_OK) return st;
   if (cudaMemsetAsync(ws, 0, moe::kStatusBytes, s) != cudaSuccess) return MOE_ERR_CUDA;
   st = moe_forward(dims, T, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales, y, nullptr,
                    nullptr, nullptr, ws, kNoAllocScratchBytes, stream);

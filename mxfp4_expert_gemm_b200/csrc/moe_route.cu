@@ -22,12 +22,6 @@ namespace {
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
-// Round fp32 to bf16 (nearest, ties to even); input finite.
-__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
-  uint32_t u = __float_as_uint(f);
-  u += 0x7FFFu + ((u >> 16) & 1u);
-  return (uint16_t)(u >> 16);
-}
 
 // ----------------------------------------------------------------------------------
 // Quantization: one warp per 32-value block, lane i holds element i.
@@ -316,7 +310,7 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
     uint8_t* xq = a.ws.xq + t * 2 * dp;
     uint8_t* sf = a.ws.xsf + t * 2 * (dp / 32);
     for (int b = warp; b < d / 32; b += kTokWarps) {
-      const float v[1] = {bf16_to_f32(f32_to_bf16_rne(s_xn[32 * b + lane]))};
+      const float v[1] = {bf16_to_f32(bf16_bits_rne(s_xn[32 * b + lane]))};
       uint32_t hi, lo, s1, s2;
       e4m3_split<1>(v, hi, lo, s1, s2);
       xq[32 * b + lane] = (uint8_t)hi;
@@ -499,7 +493,7 @@ __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
           const float v1 = __uint_as_float(pr & 0xFFFF0000u) * r * s_g[k0 + kk + 1];
           s_xn[tt * RK + kk] = v0;
           s_xn[tt * RK + kk + 1] = v1;
-          const float v[2] = {bf16_to_f32(f32_to_bf16_rne(v0)), bf16_to_f32(f32_to_bf16_rne(v1))};
+          const float v[2] = {bf16_to_f32(bf16_bits_rne(v0)), bf16_to_f32(bf16_bits_rne(v1))};
           uint32_t hi, lo, s1, s2;
           e4m3_split<2>(v, hi, lo, s1, s2);   // lanes 0-15: block k0/32, 16-31: the next
           *reinterpret_cast<uint16_t*>(xq + k0 + kk) = (uint16_t)hi;
@@ -511,7 +505,7 @@ __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
         } else {   // RK == 32: one 32-block per chunk, one value per lane
           const float v0 = bf16_to_f32(s_x[(st * kRT + tt) * RK + lane]) * r * s_g[k0 + lane];
           s_xn[tt * RK + lane] = v0;
-          const float v[1] = {bf16_to_f32(f32_to_bf16_rne(v0))};
+          const float v[1] = {bf16_to_f32(bf16_bits_rne(v0))};
           uint32_t hi, lo, s1, s2;
           e4m3_split<1>(v, hi, lo, s1, s2);
           xq[k0 + lane] = (uint8_t)hi;
@@ -732,8 +726,8 @@ __global__ void combine_kernel(FwdArgs a) {
     }
   }
   uint2 out;
-  out.x = (uint32_t)f32_to_bf16_rne(v[0]) | ((uint32_t)f32_to_bf16_rne(v[1]) << 16);
-  out.y = (uint32_t)f32_to_bf16_rne(v[2]) | ((uint32_t)f32_to_bf16_rne(v[3]) << 16);
+  out.x = (uint32_t)bf16_bits_rne(v[0]) | ((uint32_t)bf16_bits_rne(v[1]) << 16);
+  out.y = (uint32_t)bf16_bits_rne(v[2]) | ((uint32_t)bf16_bits_rne(v[3]) << 16);
   *reinterpret_cast<uint2*>(a.y + (int64_t)t * a.d + i4) = out;
   }
 }

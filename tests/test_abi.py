@@ -96,3 +96,20 @@ def test_no_device_is_an_error_not_a_fallback(L):
         pytest.skip("a GPU is present")
     st = _call_forward(L, moe.make_dims(128, 128, 4, 2), 4)
     assert st in (moe.MOE_ERR_CUDA, moe.MOE_ERR_DEVICE)
+
+
+def test_no_alloc_argument_checks_match_moe_forward(L):
+    """moe_forward_no_alloc answers argument errors with moe_forward's codes, before any
+    device work."""
+    p = ctypes.c_void_p(256)
+
+    def call(dims, T):
+        return L.moe_forward_no_alloc(ctypes.byref(dims) if dims is not None else None, T, p, p, p, p, p, p, p, p,
+                                      ctypes.c_void_p(256 + 4096), None, None)
+
+    for dims, T in ((moe.make_dims(2880, 2880, 32, 4, path=9), 4), (moe.make_dims(2880, 2880, 32, 4, act=3), 4),
+                    (moe.make_dims(2880, 2880, 32, 4), -1), (moe.make_dims(2880, 2880, 32, 4, block=16), 4),
+                    (moe.make_dims(2880 + 32, 2880, 32, 4), 4), (moe.make_dims(2880, 2880, 4, 5), 4)):
+        assert call(dims, T) == _call_forward(L, dims, T), (dims.path, dims.act_format, T)
+    assert call(None, 4) == moe.MOE_ERR_INVALID_ARG
+    assert call(moe.make_dims(2880, 2880, 32, 4), 4096) == moe.MOE_ERR_WORKSPACE   # beyond the 16 MiB scratch
