@@ -81,6 +81,9 @@ def parse(argv=None):
     ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of "
                     "replaying a captured CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget per workload")
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor parallelism over the intermediate features: every rank holds a slice of I "
+                         "for all experts and runs the whole batch; one all-reduce of the partial outputs")
     return ap.parse_args(argv)
 
 
@@ -217,6 +220,24 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------ inputs
+
+
+def slice_inputs(cfg, i0, i1):
+    """MXFP4 weights (quantized on the GPU) of the slice [i0, i1) of the intermediate features:
+    W1's gate rows [i0, i1) and up rows [I + i0, I + i1), W2's columns [i0, i1)."""
+    import torch
+    import mxfp4_expert_gemm_b200 as moe
+    E, d, I, Ir = cfg.E, cfg.d, cfg.I, i1 - i0
+    W = [torch.empty(sh, dtype=torch.uint8, device="cuda")
+         for sh in (*moe.mxfp4_shapes(E, 2 * Ir, d), *moe.mxfp4_shapes(E, d, Ir))]
+    for e in range(E):
+        w1 = synth.w1_expert(cfg, e)
+        w1s = np.ascontiguousarray(np.concatenate([w1[i0:i1], w1[I + i0:I + i1]]))
+        w2s = np.ascontiguousarray(synth.w2_expert(cfg, e)[:, i0:i1])
+        moe.moe_mxfp4_quantize(torch.from_numpy(w1s).cuda(), W[0][e:e + 1], W[1][e:e + 1], role="gate_up")
+        moe.moe_mxfp4_quantize(torch.from_numpy(w2s).cuda(), W[2][e:e + 1], W[3][e:e + 1], role="down")
+    torch.cuda.synchronize()
+    return W
 
 
 def device_inputs(cfg, rank):
@@ -514,6 +535,71 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
     return rec
 
 
+def measure_tp(cfg, args, rank, world, local_rank, pg):
+    """Tensor parallelism over I: the whole batch on every rank, each rank its slice of the
+    intermediate features; per step the slice's partial forward, one all-reduce of the fp32
+    partial outputs (NCCL), and the residual pass.  Host launches (no graph around the
+    collective); step time = max over ranks; total work fixed (strong scaling)."""
+    import torch
+    import mxfp4_expert_gemm_b200 as moe
+    i0, i1 = moe.intermediate_slices(cfg.I, world)[rank]
+    x = synth.hidden(cfg)
+    dev = "cuda"
+    x_dev = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    gamma = torch.from_numpy(synth.norm_weight(cfg)).to(dev)
+    rw, rb = torch.from_numpy(synth.router_weight(cfg)).to(dev), torch.from_numpy(synth.router_bias(cfg)).to(dev)
+    W = slice_inputs(cfg, i0, i1)
+    dims = moe.make_dims(cfg.d, i1 - i0, cfg.E, cfg.k, cfg.rms_eps, cfg.swiglu_limit, path=args.path, act=args.act)
+    ws = moe.new_workspace(dims, cfg.T)
+    part = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device=dev)
+    y = torch.empty_like(x_dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        moe.moe_forward_partial(dims, x_dev, gamma, rw, rb, *W, ws, y_partial=part)
+        n = moe.last_launch_count()
+        if pg:
+            pg.all_reduce(part)
+        moe.moe_residual_norm(x_dev, part, y=y)
+        return n + moe.last_launch_count()
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if moe.moe_device_status(ws) != moe.MOE_OK:
+        raise RuntimeError("device status after warm-up")
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    launches = 0
+    with ClockSampler(local_rank) as clk:
+        for i in range(K):
+            flush.zero_()
+            starts[i].record()
+            launches += step()
+            stops[i].record()
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    total_ms = max_over_ranks(float(sum(a.elapsed_time(b) for a, b in zip(starts, stops))), pg)
+    if moe.moe_device_status(ws) != moe.MOE_OK:
+        raise RuntimeError("device status after the timed steps")
+    return {"value": round(job_throughput(cfg.T, 1, K, total_ms), 1), "unit": "tokens/s",
+            "ms_per_step": round(total_ms / K, 5),
+            "config": {"workload": WORKLOAD_TEXT[cfg.name], "name": cfg.name, "global_batch": cfg.T,
+                       "parallelism": f"tp{world}", "slice": [i0, i1], "path": moe.resolved_path(dims, cfg.T),
+                       "collective": "NCCL all-reduce (sum) of the fp32 partial outputs [T, d] per step",
+                       "l2": "flushed before every step (256 MiB write, outside the step events)",
+                       "timing": "sum of per-step CUDA events on the launching stream; max over ranks",
+                       "launch": "host launches per step"},
+            "gpu_launches": launches, "clocks": clk.summary()}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     torch.cuda.set_device(local_rank)
@@ -524,6 +610,19 @@ def run_ours(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         pg = dist
     want_cpu = (rank == 0 and world == 1 and not args.no_cpu_baseline)
+    if args.tp:
+        rec = measure_tp(synth.CONFIGS[args.config or HEADLINE_CONFIG], args, rank, world, local_rank, pg)
+        line = {"metric": METRIC, "value": rec["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": max(3, args.warmup), "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None,
+                "dtype": "mxfp4xbf16" if args.act == "bf16" else "mxfp4xmxfp8", "data": "synthetic",
+                "config": rec["config"], "gpu_launches": rec["gpu_launches"], "clocks": rec["clocks"]}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if pg:
+            pg.barrier()
+            pg.destroy_process_group()
+        return
     names = [args.config] if args.config else [HEADLINE_CONFIG, DECODE_CONFIG]
     recs = [measure(synth.CONFIGS[n], args, rank, world, local_rank, pg, want_cpu) for n in names]
     head = recs[0]

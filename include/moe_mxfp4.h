@@ -199,6 +199,50 @@ moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x,
                              uint16_t* y, int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out,
                              void* ws, size_t ws_bytes, void* stream, void* const* events, int32_t n_events);
 
+/* moe_forward, and in the same pass the next block's first RMSNorm of the output
+ * (every block holds two RMSNorms and maps [N x d] to [N x d]: ewbang.com article, section
+ * Transformer 块):
+ *   y      [T][d] bf16 = x + MoE(RMSNorm(x))                    (as moe_forward)
+ *   y_norm [T][d] bf16 = bf16(y / sqrt(mean(y^2) + next_eps) * next_norm_w), on the bf16 y
+ * next_norm_w [d] fp32 (device), next_eps >= 0.  The routing-weighted sum of the k expert
+ * outputs, the residual add and the RMSNorm run in one pass over each token's row (on
+ * both paths; the small-batch path then does not fold the sum into the down GEMM).
+ * y and y_norm may not alias x or each other.  Errors: as moe_forward; MOE_ERR_INVALID_ARG
+ * for a null / misaligned next_norm_w or y_norm, or a negative or non-finite next_eps. */
+moe_status moe_forward_norm(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                            const float* router_w, const float* router_b, const uint8_t* w1_codes,
+                            const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                            const float* next_norm_w, float next_eps, uint16_t* y, uint16_t* y_norm, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* One slice of the intermediate features, for splitting a layer over G GPUs (tensor
+ * parallelism over I; the pages run the layer on one GPU, this is an extension).  The
+ * expert MLP is separable over its intermediate features: h's feature i depends only on
+ * W1's gate row i and up row I + i, and the down projection sums W2[:, i] * h_i over i.
+ * A rank holds, for every expert, the gate rows [i0, i1) and up rows [I + i0, I + i1) of
+ * W1 and the columns [i0, i1) of W2, quantized as the layer of intermediate size
+ * dims->I = i1 - i0 (a multiple of 64; W1 with role MOE_WEIGHT_GATE_UP, W2 plain; since i0
+ * is a multiple of 64 the slice's MXFP4 blocks are those of the whole matrix).  Every rank
+ * routes the same x with the same router and gets the same experts.  The call writes
+ *   y_partial [T][d] fp32 = sum_j w_j * W2[e_j][:, i0:i1] . h_j[i0:i1]   (no residual)
+ * The sum of y_partial over slices that cover [0, I) (one all-reduce) is the expert mix of
+ * the whole layer; moe_residual_norm then gives y = bf16(x + sum).
+ * y_partial may not alias x.  Errors: as moe_forward. */
+moe_status moe_forward_partial(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                               const float* router_w, const float* router_b, const uint8_t* w1_codes,
+                               const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                               float* y_partial, int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* y [T][d] bf16 = bf16(x + s) for s [T][d] fp32 (device; e.g. the all-reduced outputs of
+ * moe_forward_partial), and with norm_w non-NULL also the next block's RMSNorm
+ * y_norm = bf16(y / sqrt(mean(y^2) + eps) * norm_w) on the bf16 y.  One launch.
+ * d a positive multiple of 64; y and y_norm may not alias x or each other.
+ * Errors: MOE_ERR_INVALID_ARG (T < 0, d <= 0, null / misaligned pointer, bad eps),
+ * MOE_ERR_UNSUPPORTED_SHAPE (d not a multiple of 64), MOE_ERR_DEVICE, MOE_ERR_CUDA. */
+moe_status moe_residual_norm(int32_t T, int32_t d, const uint16_t* x, const float* s, const float* norm_w,
+                             float eps, uint16_t* y, uint16_t* y_norm, void* stream);
+
 /* The path moe_forward takes for these dims and T: dims->path, or for MOE_PATH_AUTO the
  * choice it makes (MOE_PATH_GEMV when T*top_k/E <= 24 tokens per expert, else
  * MOE_PATH_GEMM).  Returns -1 for invalid dims. */

@@ -100,6 +100,13 @@ def lib():
             L.moe_device_status.restype = ctypes.c_int
             L.moe_status_string.argtypes = [ctypes.c_int]
             L.moe_status_string.restype = ctypes.c_char_p
+            L.moe_forward_partial.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.moe_forward_partial.restype = ctypes.c_int
+            L.moe_forward_norm.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
+                                           vp, sz, vp]
+            L.moe_forward_norm.restype = ctypes.c_int
+            L.moe_residual_norm.argtypes = [i32, i32, vp, vp, vp, ctypes.c_float, vp, vp, vp]
+            L.moe_residual_norm.restype = ctypes.c_int
             L.moe_forward_no_alloc.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             L.moe_forward_no_alloc.restype = ctypes.c_int
             L.moe_debug_inject_timeout.argtypes = [i32]
@@ -237,6 +244,70 @@ def moe_forward(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scal
                              _ptr(r["counts"]) if r else None, _ptr(ws), ws.numel(), _stream(stream)),
            "moe_forward")
     return (y, r) if want_routing else y
+
+
+def moe_forward_partial(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales,
+                        ws, y_partial=None, want_routing=False, stream=None):
+    """One slice of the intermediate features (weights of the slice, dims.I = its width):
+    y_partial [T, d] fp32 = the slice's share of the expert mix, without the residual."""
+    T = x.shape[0]
+    _need(x, torch.bfloat16, "x")
+    dev = x.device
+    if y_partial is None:
+        y_partial = torch.empty((T, dims.d), dtype=torch.float32, device=dev)
+    r = None
+    if want_routing:
+        r = dict(topk_idx=torch.empty((T, dims.top_k), dtype=torch.int32, device=dev),
+                 topk_w=torch.empty((T, dims.top_k), dtype=torch.float32, device=dev),
+                 counts=torch.empty(dims.E, dtype=torch.int32, device=dev))
+    _check(lib().moe_forward_partial(ctypes.byref(dims), T, _ptr(x), _ptr(norm_w), _ptr(router_w), _ptr(router_b),
+                                     _ptr(w1_codes), _ptr(w1_scales), _ptr(w2_codes), _ptr(w2_scales), _ptr(y_partial),
+                                     _ptr(r["topk_idx"]) if r else None, _ptr(r["topk_w"]) if r else None,
+                                     _ptr(r["counts"]) if r else None, _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_forward_partial")
+    return (y_partial, r) if want_routing else y_partial
+
+
+def moe_forward_norm(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales, ws,
+                     next_norm_w, next_eps=1e-5, y=None, y_norm=None, stream=None):
+    """(y, y_norm): the layer's output and the next block's RMSNorm of it, in one pass."""
+    _need(x, torch.bfloat16, "x")
+    _need(next_norm_w, torch.float32, "next_norm_w", (dims.d,))
+    y = torch.empty_like(x) if y is None else y
+    y_norm = torch.empty_like(x) if y_norm is None else y_norm
+    _check(lib().moe_forward_norm(ctypes.byref(dims), x.shape[0], _ptr(x), _ptr(norm_w), _ptr(router_w),
+                                  _ptr(router_b), _ptr(w1_codes), _ptr(w1_scales), _ptr(w2_codes), _ptr(w2_scales),
+                                  _ptr(next_norm_w), float(next_eps), _ptr(y), _ptr(y_norm), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "moe_forward_norm")
+    return y, y_norm
+
+
+def moe_residual_norm(x, s, norm_w=None, eps=1e-5, y=None, y_norm=None, stream=None):
+    """y = bf16(x + s) for fp32 s [T, d]; with norm_w also y_norm = bf16(RMSNorm(y) * norm_w)."""
+    _need(x, torch.bfloat16, "x")
+    _need(s, torch.float32, "s", tuple(x.shape))
+    T, d = x.shape
+    y = torch.empty_like(x) if y is None else y
+    if norm_w is not None and y_norm is None:
+        y_norm = torch.empty_like(x)
+    _check(lib().moe_residual_norm(T, d, _ptr(x), _ptr(s), _ptr(norm_w), float(eps), _ptr(y),
+                                   _ptr(y_norm) if norm_w is not None else None, _stream(stream)),
+           "moe_residual_norm")
+    return (y, y_norm) if norm_w is not None else y
+
+
+def intermediate_slices(I: int, G: int) -> list[tuple[int, int]]:
+    """[i0, i1) of G slices of the intermediate features, each a multiple of 64 wide (the
+    64-feature blocks dealt out as evenly as they go: 2880 = 45 blocks -> 23 + 22 for G = 2)."""
+    if I % 64 or G < 1 or G > I // 64:
+        raise ValueError(f"cannot cut I = {I} into {G} slices of whole 64-feature blocks")
+    nb = I // 64
+    out, b0 = [], 0
+    for g in range(G):
+        nbg = nb // G + (1 if g < nb % G else 0)
+        out.append((64 * b0, 64 * (b0 + nbg)))
+        b0 += nbg
+    return out
 
 
 WS_FIELDS = ("status", "counts", "offsets", "ntiles", "tile_base", "tiles", "topk_idx", "topk_w", "perm", "inv",

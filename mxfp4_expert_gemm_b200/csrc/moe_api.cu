@@ -94,6 +94,91 @@ moe_status copy_out(void* dst, const void* src, size_t bytes, cudaStream_t st) {
   return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Where a forward call writes the layer's output.
+struct Outputs {
+  uint16_t* y = nullptr;               // bf16 [T][d]: x + the expert mix
+  float* y_partial = nullptr;          // fp32 [T][d]: the expert mix alone (instead of y)
+  const float* next_norm_w = nullptr;  // with y_norm: the next block's RMSNorm of y
+  float next_eps = 0.f;
+  uint16_t* y_norm = nullptr;
+  int32_t* topk_idx = nullptr;
+  float* topk_w = nullptr;
+  int32_t* counts = nullptr;
+};
+
+moe_status forward_impl(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                        const float* router_w, const float* router_b, const uint8_t* w1_codes,
+                        const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                        const Outputs& out, void* ws, size_t ws_bytes, void* stream, void* const* events,
+                        int32_t n_events) {
+  g_last_launches = 0;
+  if (n_events < 0 || (n_events > 0 && !events)) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_dims(dims, T);
+  if (st != MOE_OK) return st;
+  if (T > 0) {  // (argument errors come before any device query)
+    if (!w1_codes || !w1_scales || !w2_codes || !w2_scales) return MOE_ERR_INVALID_ARG;
+    if (!aligned32(w1_codes) || !aligned16(w1_scales) || !aligned32(w2_codes) || !aligned16(w2_scales))
+      return MOE_ERR_INVALID_ARG;
+    void* const dst = out.y_partial ? static_cast<void*>(out.y_partial) : static_cast<void*>(out.y);
+    if (!dst || !aligned16(dst) || (const void*)dst == (const void*)x) return MOE_ERR_INVALID_ARG;
+    if (out.next_norm_w) {
+      if (!out.y_norm || !aligned16(out.next_norm_w) || !aligned16(out.y_norm)) return MOE_ERR_INVALID_ARG;
+      if ((void*)out.y_norm == (void*)out.y || (const void*)out.y_norm == (const void*)x) return MOE_ERR_INVALID_ARG;
+      if (!(out.next_eps >= 0.f) || !std::isfinite(out.next_eps)) return MOE_ERR_INVALID_ARG;
+    }
+  }
+  moe::FwdArgs a;
+  moe::WsLayout L;
+  st = prepare(dims, T, x, norm_w, router_w, router_b, ws, ws_bytes, a, L);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  a.w1c = w1_codes;
+  a.w1s = w1_scales;
+  a.w2c = w2_codes;
+  a.w2s = w2_scales;
+  a.y = out.y;
+  a.y_partial = out.y_partial;
+  a.next_norm_w = out.next_norm_w;
+  a.next_eps = out.next_eps;
+  a.y_norm = out.y_norm;
+  a.stream = static_cast<cudaStream_t>(stream);
+  moe::EventRec rec;
+  rec.events = events;
+  rec.n = n_events;
+  if (n_events > 0) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(a.stream, &cs) != cudaSuccess) return MOE_ERR_CUDA;
+    rec.capturing = cs == cudaStreamCaptureStatusActive;
+  }
+  a.ev = &rec;
+  a.inject_timeout = g_inject_timeout;
+  g_inject_timeout = 0;
+  const int path = resolve_path(*dims, T);
+  // Small-batch path: fewer, fused kernels (routing + grouping + tile scales; down + combine).
+  // The next block's RMSNorm needs whole rows, which the separate combine pass holds.
+  a.fuse_group = (path == MOE_PATH_GEMV && T <= moe::kFusedGroupMaxT) ? 1 : 0;
+  a.fuse_combine = (path == MOE_PATH_GEMV && !a.next_norm_w) ? 1 : 0;
+  // Overlap each kernel's launch and prologue with its predecessor, except when per-kernel
+  // events are recorded between the kernels.
+  a.pdl = (n_events == 0) ? 1 : 0;
+  int n = moe::launch_route(a);
+  if (n < 0) return MOE_ERR_CUDA;
+  const int ne = moe::launch_experts(a);
+  if (ne < 0) return MOE_ERR_CUDA;
+  n += ne;
+  if (!a.fuse_combine) {
+    const int nc = moe::launch_combine(a);
+    if (nc < 0) return MOE_ERR_CUDA;
+    n += nc;
+  }
+  const size_t P = (size_t)T * dims->top_k;
+  if ((st = copy_out(out.topk_idx, a.ws.topk_idx, 4 * P, a.stream)) != MOE_OK) return st;
+  if ((st = copy_out(out.topk_w, a.ws.topk_w, 4 * P, a.stream)) != MOE_OK) return st;
+  if ((st = copy_out(out.counts, a.ws.counts, 4 * (size_t)dims->E, a.stream)) != MOE_OK) return st;
+  g_last_launches = n;
+  return MOE_OK;
+}
+
 }  // namespace
 
 namespace moe {
@@ -169,61 +254,61 @@ moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x,
                              const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
                              uint16_t* y, int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, void* ws,
                              size_t ws_bytes, void* stream, void* const* events, int32_t n_events) {
+  Outputs out;
+  out.y = y;
+  out.topk_idx = topk_idx_out;
+  out.topk_w = topk_w_out;
+  out.counts = counts_out;
+  return forward_impl(dims, T, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales, out, ws,
+                      ws_bytes, stream, events, n_events);
+}
+
+moe_status moe_forward_partial(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                               const float* router_w, const float* router_b, const uint8_t* w1_codes,
+                               const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                               float* y_partial, int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out,
+                               void* ws, size_t ws_bytes, void* stream) {
+  Outputs out;
+  out.y_partial = y_partial;
+  out.topk_idx = topk_idx_out;
+  out.topk_w = topk_w_out;
+  out.counts = counts_out;
+  return forward_impl(dims, T, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales, out, ws,
+                      ws_bytes, stream, nullptr, 0);
+}
+
+moe_status moe_forward_norm(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
+                            const float* router_w, const float* router_b, const uint8_t* w1_codes,
+                            const uint8_t* w1_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                            const float* next_norm_w, float next_eps, uint16_t* y, uint16_t* y_norm, void* ws,
+                            size_t ws_bytes, void* stream) {
+  Outputs out;
+  out.y = y;
+  out.next_norm_w = next_norm_w;
+  out.next_eps = next_eps;
+  out.y_norm = y_norm;
+  return forward_impl(dims, T, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales, out, ws,
+                      ws_bytes, stream, nullptr, 0);
+}
+
+moe_status moe_residual_norm(int32_t T, int32_t d, const uint16_t* x, const float* s, const float* norm_w,
+                             float eps, uint16_t* y, uint16_t* y_norm, void* stream) {
   g_last_launches = 0;
-  if (n_events < 0 || (n_events > 0 && !events)) return MOE_ERR_INVALID_ARG;
-  moe_status st = check_dims(dims, T);
-  if (st != MOE_OK) return st;
-  if (T > 0) {  // (argument errors come before any device query)
-    if (!w1_codes || !w1_scales || !w2_codes || !w2_scales || !y) return MOE_ERR_INVALID_ARG;
-    if (!aligned32(w1_codes) || !aligned16(w1_scales) || !aligned32(w2_codes) || !aligned16(w2_scales) ||
-        !aligned16(y))
-      return MOE_ERR_INVALID_ARG;
-    if ((const void*)y == (const void*)x) return MOE_ERR_INVALID_ARG;
-  }
-  moe::FwdArgs a;
-  moe::WsLayout L;
-  st = prepare(dims, T, x, norm_w, router_w, router_b, ws, ws_bytes, a, L);
-  if (st != MOE_OK) return st;
+  if (T < 0 || d <= 0 || d % 64 || d > (1 << 16)) return T < 0 || d <= 0 ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return MOE_OK;
-  a.w1c = w1_codes;
-  a.w1s = w1_scales;
-  a.w2c = w2_codes;
-  a.w2s = w2_scales;
-  a.y = y;
-  a.stream = static_cast<cudaStream_t>(stream);
-  moe::EventRec rec;
-  rec.events = events;
-  rec.n = n_events;
-  if (n_events > 0) {
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(a.stream, &cs) != cudaSuccess) return MOE_ERR_CUDA;
-    rec.capturing = cs == cudaStreamCaptureStatusActive;
+  if (!x || !s || !y || !aligned16(x) || !aligned16(s) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if ((const void*)y == (const void*)x) return MOE_ERR_INVALID_ARG;
+  if (norm_w) {
+    if (!y_norm || !aligned16(norm_w) || !aligned16(y_norm) || y_norm == y || (const void*)y_norm == (const void*)x)
+      return MOE_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return MOE_ERR_INVALID_ARG;
   }
-  a.ev = &rec;
-  a.inject_timeout = g_inject_timeout;
-  g_inject_timeout = 0;
-  const int path = resolve_path(*dims, T);
-  // Small-batch path: fewer, fused kernels (routing + grouping + tile scales; down + combine).
-  a.fuse_group = (path == MOE_PATH_GEMV && T <= moe::kFusedGroupMaxT) ? 1 : 0;
-  a.fuse_combine = (path == MOE_PATH_GEMV) ? 1 : 0;
-  // Overlap each kernel's launch and prologue with its predecessor, except when per-kernel
-  // events are recorded between the kernels.
-  a.pdl = (n_events == 0) ? 1 : 0;
-  int n = moe::launch_route(a);
-  if (n < 0) return MOE_ERR_CUDA;
-  const int ne = moe::launch_experts(a);
-  if (ne < 0) return MOE_ERR_CUDA;
-  n += ne;
-  if (!a.fuse_combine) {
-    const int nc = moe::launch_combine(a);
-    if (nc < 0) return MOE_ERR_CUDA;
-    n += nc;
-  }
-  const size_t P = (size_t)T * dims->top_k;
-  if ((st = copy_out(topk_idx_out, a.ws.topk_idx, 4 * P, a.stream)) != MOE_OK) return st;
-  if ((st = copy_out(topk_w_out, a.ws.topk_w, 4 * P, a.stream)) != MOE_OK) return st;
-  if ((st = copy_out(counts_out, a.ws.counts, 4 * (size_t)dims->E, a.stream)) != MOE_OK) return st;
-  g_last_launches = n;
+  const moe_status st = check_device();
+  if (st != MOE_OK) return st;
+  if (moe::launch_residual_norm(T, d, x, s, norm_w, eps, y, norm_w ? y_norm : nullptr,
+                                static_cast<cudaStream_t>(stream)) < 0)
+    return MOE_ERR_CUDA;
+  g_last_launches = 1;
   return MOE_OK;
 }
 

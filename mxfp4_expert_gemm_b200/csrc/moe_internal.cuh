@@ -302,6 +302,11 @@ struct FwdArgs {
   const uint8_t* w2c;
   const uint8_t* w2s;
   uint16_t* y;
+  // Optional outputs in place of (or beside) y:
+  float* y_partial;          // [T][d] fp32 sum_j w_j o_j without the residual (a slice of I)
+  const float* next_norm_w;  // [d]: also write y_norm = bf16(RMSNorm(y) * next_norm_w)
+  float next_eps;
+  uint16_t* y_norm;          // [T][d] bf16
   Ws ws;
   cudaStream_t stream;
   EventRec* ev;
@@ -357,7 +362,10 @@ __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
 int launch_quantize(const float* w, int32_t E, int32_t N, int32_t K, int32_t role, uint8_t* codes,
                     uint8_t* scales, int32_t* status, cudaStream_t st);
 int launch_route(const FwdArgs& a);     // norm + router + top-k + E4M3 split, grouping, packing
-int launch_combine(const FwdArgs& a);   // y = x + sum_j ys[inv]
+int launch_combine(const FwdArgs& a);   // y = x + sum_j ys[inv] (or the partial sum, or y and y_norm)
+// y = bf16(x + s) for a dense fp32 s [T][d], and optionally y_norm (one pass per row)
+int launch_residual_norm(int32_t T, int32_t d, const uint16_t* x, const float* s, const float* norm_w, float eps,
+                         uint16_t* y, uint16_t* y_norm, cudaStream_t st);
 int launch_experts(const FwdArgs& a);   // block-scaled tcgen05 expert MLPs (gate_up, down)
 int expert_tile_tokens(int path, int terms);   // token tile of a path
 int expert_down_split(int path);        // reduction-axis splits of a path's down GEMM

@@ -81,6 +81,7 @@ struct MxParams {
   const int32_t* inv;
   const uint16_t* x;
   uint16_t* y;
+  float* y_partial;        // instead of y: the fp32 sum without the residual (a slice of I)
   int32_t* arrivals;
 };
 
@@ -458,13 +459,14 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>::THREADS
               if (tok < 0) continue;
               for (int col = et; col < ncol; col += 128) {
                 const int64_t gc = kBM * rt + col;
-                float accv = __uint_as_float((uint32_t)p.x[(int64_t)tok * p.d + gc] << 16);
+                float accv = p.y_partial ? 0.f : __uint_as_float((uint32_t)p.x[(int64_t)tok * p.d + gc] << 16);
                 for (int j = 0; j < p.k; ++j) {
                   const int srow = p.inv[(int64_t)tok * p.k + j];
                   for (int sp = 0; sp < ksplit; ++sp)
                     accv += __ldcg(p.ys + ((int64_t)sp * p.P + srow) * p.d + gc);
                 }
-                p.y[(int64_t)tok * p.d + gc] = bf16_bits_rne(accv);
+                if (p.y_partial) p.y_partial[(int64_t)tok * p.d + gc] = accv;
+                else p.y[(int64_t)tok * p.d + gc] = bf16_bits_rne(accv);
               }
             }
             group_sync();
@@ -571,6 +573,7 @@ int launch_one(const FwdArgs& a) {
   prm.inv = a.ws.inv;
   prm.x = a.x;
   prm.y = a.y;
+  prm.y_partial = a.y_partial;
   prm.arrivals = a.ws.arrivals;
 
   auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, NPW, TERMS, MODE>;

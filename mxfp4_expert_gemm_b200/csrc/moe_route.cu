@@ -704,31 +704,131 @@ __global__ void pack_kernel(FwdArgs a) {
   }
 }
 
-// y[t] = bf16(x[t] + sum_j sum_s ys[s][inv[t*k + j]]), j in slot order, then split order.
+// y[t] = bf16(x[t] + sum_j sum_s ys[s][inv[t*k + j]]), j in slot order, then split order;
+// with y_partial the fp32 sum alone (no residual: one rank's slice of the intermediate
+// features, summed over the ranks afterwards).
 __global__ void combine_kernel(FwdArgs a) {
   pdl_trigger();
   pdl_wait();
   const int i4 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i4 >= a.d) return;
-  for (int t = blockIdx.y; t < a.T; t += gridDim.y) {
-  const uint2 xr = *reinterpret_cast<const uint2*>(a.x + (int64_t)t * a.d + i4);
-  float v[4] = {__uint_as_float(xr.x << 16), __uint_as_float(xr.x & 0xFFFF0000u), __uint_as_float(xr.y << 16),
-                __uint_as_float(xr.y & 0xFFFF0000u)};
   const int64_t P = (int64_t)a.T * a.k;
-  for (int j = 0; j < a.k; ++j) {
-    const int p = a.ws.inv[(int64_t)t * a.k + j];
-    for (int sp = 0; sp < a.ws.ksplit; ++sp) {   // partial sums of a split down GEMM
-      const float4 o = *reinterpret_cast<const float4*>(a.ws.ys + (sp * P + p) * a.d + i4);
-      v[0] += o.x;
-      v[1] += o.y;
-      v[2] += o.z;
-      v[3] += o.w;
+  for (int t = blockIdx.y; t < a.T; t += gridDim.y) {
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (!a.y_partial) {
+      const uint2 xr = *reinterpret_cast<const uint2*>(a.x + (int64_t)t * a.d + i4);
+      v[0] = __uint_as_float(xr.x << 16);
+      v[1] = __uint_as_float(xr.x & 0xFFFF0000u);
+      v[2] = __uint_as_float(xr.y << 16);
+      v[3] = __uint_as_float(xr.y & 0xFFFF0000u);
+    }
+    for (int j = 0; j < a.k; ++j) {
+      const int p = a.ws.inv[(int64_t)t * a.k + j];
+      for (int sp = 0; sp < a.ws.ksplit; ++sp) {   // partial sums of a split down GEMM
+        const float4 o = *reinterpret_cast<const float4*>(a.ws.ys + (sp * P + p) * a.d + i4);
+        v[0] += o.x;
+        v[1] += o.y;
+        v[2] += o.z;
+        v[3] += o.w;
+      }
+    }
+    if (a.y_partial) {
+      *reinterpret_cast<float4*>(a.y_partial + (int64_t)t * a.d + i4) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+      uint2 out;
+      out.x = (uint32_t)bf16_bits_rne(v[0]) | ((uint32_t)bf16_bits_rne(v[1]) << 16);
+      out.y = (uint32_t)bf16_bits_rne(v[2]) | ((uint32_t)bf16_bits_rne(v[3]) << 16);
+      *reinterpret_cast<uint2*>(a.y + (int64_t)t * a.d + i4) = out;
     }
   }
-  uint2 out;
-  out.x = (uint32_t)bf16_bits_rne(v[0]) | ((uint32_t)bf16_bits_rne(v[1]) << 16);
-  out.y = (uint32_t)bf16_bits_rne(v[2]) | ((uint32_t)bf16_bits_rne(v[3]) << 16);
-  *reinterpret_cast<uint2*>(a.y + (int64_t)t * a.d + i4) = out;
+}
+
+// ----------------------------------------------------------------------------------
+// Rows that finish a block: y = bf16(x + s) and, with norm_w, the next block's RMSNorm of
+// it, y_norm = bf16(y / sqrt(mean(y^2) + eps) * norm_w) on the bf16 y (each block holds two
+// RMSNorms: "Transformer 块" of the ewbang.com GPT-OSS article).  s is either the sum of the
+// token's k expert outputs (ys through inv, slot order then split order, as combine_kernel)
+// or a dense fp32 row (the all-reduced partial outputs of the ranks that hold slices of the
+// intermediate features).  One CTA of 256 threads per row; the row's sum of squares is a
+// block reduction in fixed order.
+// ----------------------------------------------------------------------------------
+struct FinishArgs {
+  int32_t T, d, k, ksplit;
+  int64_t P;
+  const uint16_t* x;
+  const float* ys;        // pair outputs [ksplit][P][d] (or NULL)
+  const int32_t* inv;
+  const float* s;         // dense fp32 [T][d] (or NULL)
+  const float* norm_w;    // NULL: y only
+  float eps;
+  uint16_t* y;
+  uint16_t* y_norm;
+};
+
+constexpr int kFinishThreads = 256;
+
+__global__ void __launch_bounds__(kFinishThreads) finish_rows_kernel(FinishArgs f) {
+  __shared__ float s_red[kFinishThreads / 32];
+  pdl_trigger();
+  pdl_wait();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int t = blockIdx.x; t < f.T; t += gridDim.x) {
+    float ss = 0.f;
+    for (int i4 = tid * 4; i4 < f.d; i4 += kFinishThreads * 4) {
+      const uint2 xr = *reinterpret_cast<const uint2*>(f.x + (int64_t)t * f.d + i4);
+      float v[4] = {__uint_as_float(xr.x << 16), __uint_as_float(xr.x & 0xFFFF0000u), __uint_as_float(xr.y << 16),
+                    __uint_as_float(xr.y & 0xFFFF0000u)};
+      if (f.ys) {
+        for (int j = 0; j < f.k; ++j) {
+          const int p = f.inv[(int64_t)t * f.k + j];
+          for (int sp = 0; sp < f.ksplit; ++sp) {
+            const float4 o = *reinterpret_cast<const float4*>(f.ys + (sp * f.P + p) * f.d + i4);
+            v[0] += o.x;
+            v[1] += o.y;
+            v[2] += o.z;
+            v[3] += o.w;
+          }
+        }
+      } else {
+        const float4 o = *reinterpret_cast<const float4*>(f.s + (int64_t)t * f.d + i4);
+        v[0] += o.x;
+        v[1] += o.y;
+        v[2] += o.z;
+        v[3] += o.w;
+      }
+      uint16_t b[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        b[q] = bf16_bits_rne(v[q]);
+        const float yb = bf16_to_f32(b[q]);
+        ss = fmaf(yb, yb, ss);
+      }
+      uint2 out;
+      out.x = (uint32_t)b[0] | ((uint32_t)b[1] << 16);
+      out.y = (uint32_t)b[2] | ((uint32_t)b[3] << 16);
+      *reinterpret_cast<uint2*>(f.y + (int64_t)t * f.d + i4) = out;
+    }
+    if (f.norm_w) {
+#pragma unroll
+      for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) s_red[warp] = ss;
+      __syncthreads();
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < kFinishThreads / 32; ++w) tot += s_red[w];
+      const float r = 1.0f / sqrtf(tot / (float)f.d + f.eps);
+      for (int i4 = tid * 4; i4 < f.d; i4 += kFinishThreads * 4) {   // this thread's own y values
+        const uint2 yr = *reinterpret_cast<const uint2*>(f.y + (int64_t)t * f.d + i4);
+        const float4 g = *reinterpret_cast<const float4*>(f.norm_w + i4);
+        const float v0 = __uint_as_float(yr.x << 16) * r * g.x, v1 = __uint_as_float(yr.x & 0xFFFF0000u) * r * g.y;
+        const float v2 = __uint_as_float(yr.y << 16) * r * g.z, v3 = __uint_as_float(yr.y & 0xFFFF0000u) * r * g.w;
+        uint2 out;
+        out.x = (uint32_t)bf16_bits_rne(v0) | ((uint32_t)bf16_bits_rne(v1) << 16);
+        out.y = (uint32_t)bf16_bits_rne(v2) | ((uint32_t)bf16_bits_rne(v3) << 16);
+        *reinterpret_cast<uint2*>(f.y_norm + (int64_t)t * f.d + i4) = out;
+      }
+      __syncthreads();   // s_red is reused by the next row
+    }
   }
 }
 
@@ -824,10 +924,48 @@ int launch_route(const FwdArgs& a_in) {
 }
 
 int launch_combine(const FwdArgs& a) {
+  if (a.next_norm_w) {   // y and the next block's RMSNorm of it: whole rows per CTA
+    FinishArgs f{};
+    f.T = a.T;
+    f.d = a.d;
+    f.k = a.k;
+    f.ksplit = a.ws.ksplit;
+    f.P = (int64_t)a.T * a.k;
+    f.x = a.x;
+    f.ys = a.ws.ys;
+    f.inv = a.ws.inv;
+    f.norm_w = a.next_norm_w;
+    f.eps = a.next_eps;
+    f.y = a.y;
+    f.y_norm = a.y_norm;
+    ev_before(a);
+    if (launch_kernel(finish_rows_kernel, dim3((unsigned)std::min(a.T, 148 * 8)), dim3(kFinishThreads), 0, a.stream,
+                      a.pdl != 0, f) != cudaSuccess)
+      return -1;
+    ev_after(a);
+    return cudaGetLastError() == cudaSuccess ? 1 : -1;
+  }
   dim3 grid((a.d / 4 + 127) / 128, std::min(a.T, 65535));
   ev_before(a);
   if (launch_kernel(combine_kernel, grid, dim3(128), 0, a.stream, a.pdl != 0, a) != cudaSuccess) return -1;
   ev_after(a);
+  return cudaGetLastError() == cudaSuccess ? 1 : -1;
+}
+
+int launch_residual_norm(int32_t T, int32_t d, const uint16_t* x, const float* s, const float* norm_w, float eps,
+                         uint16_t* y, uint16_t* y_norm, cudaStream_t st) {
+  FinishArgs f{};
+  f.T = T;
+  f.d = d;
+  f.x = x;
+  f.s = s;
+  f.norm_w = norm_w;
+  f.eps = eps;
+  f.y = y;
+  f.y_norm = y_norm;
+  if (launch_kernel(finish_rows_kernel, dim3((unsigned)std::min(T, 148 * 8)), dim3(kFinishThreads), 0, st, false,
+                    f) != cudaSuccess)
+    return -1;
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 

@@ -53,6 +53,8 @@ def lib():
             L.oracle_dequantize.restype = i32
             L.oracle_round_bf16.argtypes = [dbl]
             L.oracle_round_bf16.restype = dbl
+            L.oracle_to_bf16.argtypes = [vp, i64, vp]
+            L.oracle_to_bf16.restype = None
             L.oracle_rmsnorm.argtypes = [i32, i32, vp, vp, dbl, vp]
             L.oracle_rmsnorm.restype = None
             L.oracle_route.argtypes = [i32, i32, i32, i32, vp, vp, dbl, vp, vp, vp, vp, vp, vp, i32]
@@ -66,6 +68,8 @@ def lib():
             L.oracle_e4m3_nearest_code.restype = i32
             L.oracle_e4m3_value.argtypes = [i32]
             L.oracle_e4m3_value.restype = dbl
+            L.oracle_mxfp4_quantize_values.argtypes = [vp, i64, vp]
+            L.oracle_mxfp4_quantize_values.restype = i32
             L.oracle_mxfp8_quantize.argtypes = [vp, i64, vp, vp]
             L.oracle_mxfp8_quantize.restype = i32
             _lib = L
@@ -87,8 +91,9 @@ def round_bf16(v: float) -> float:
     return lib().oracle_round_bf16(float(v))
 
 
-# Activation formats of the expert GEMMs: bf16 (exact) or MXFP8 (E4M3 in 32-blocks).
-ACT_FORMATS = {"bf16": 0, "mxfp8": 1}
+# Activation formats of the expert GEMMs: bf16 (exact), MXFP8 (E4M3 in 32-blocks) or MXFP4
+# (E2M1 in 32-blocks, the weights' own format).
+ACT_FORMATS = {"bf16": 0, "mxfp8": 1, "mxfp4": 2}
 
 
 def e4m3_nearest_code(a: float) -> int:
@@ -108,6 +113,16 @@ def mxfp8_quantize(v: np.ndarray):
     if lib().oracle_mxfp8_quantize(_p(v), v.size, _p(out), _p(exps)):
         raise ValueError("length is not a multiple of 32")
     return out, exps
+
+
+def mxfp4_quantize_values(v: np.ndarray) -> np.ndarray:
+    """float64 [..., n] (n a multiple of 32) -> the values after MXFP4 quantization in
+    32-value blocks, by the rule the expert weights are quantized with."""
+    v = np.ascontiguousarray(v, np.float64)
+    out = np.empty_like(v)
+    if lib().oracle_mxfp4_quantize_values(_p(v), v.size, _p(out)):
+        raise ValueError("length is not a multiple of 32")
+    return out
 
 
 def storage_bytes(rows: int, K: int) -> tuple[int, int]:
@@ -147,6 +162,20 @@ def rmsnorm(x_bf16: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
     return out
 
 
+def to_bf16(v: np.ndarray) -> np.ndarray:
+    """float64 array -> bf16 bit patterns (uint16), round to nearest, ties to even."""
+    v = np.ascontiguousarray(v, np.float64)
+    out = np.empty(v.shape, np.uint16)
+    lib().oracle_to_bf16(_p(v), v.size, _p(out))
+    return out
+
+
+def next_block_norm(y_bf16: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
+    """The next block's first RMSNorm of a block's bf16 output, rounded to bf16 (every block
+    holds two RMSNorms; ewbang.com GPT-OSS article, section Transformer 块)."""
+    return to_bf16(rmsnorm(y_bf16, gamma, eps))
+
+
 def route(x_bf16, gamma, router_w, router_b, k, eps, nthreads=0):
     """-> dict(idx [T,k] i32, w [T,k] f64, logits [T,E] f64, gap [T] f64)."""
     x_bf16 = np.ascontiguousarray(x_bf16, np.uint16)
@@ -184,8 +213,9 @@ def moe_forward(x_bf16, gamma, router_w, router_b, w1_codes, w1_scales, w2_codes
 
     Weights in the oracle layout with a leading expert axis:
     w1_codes [E, 2I, d/2], w1_scales [E, 2I, d/32], w2_codes [E, d, I/2], w2_scales [E, d, I/32].
-    act: "bf16" (exact bf16 activations) or "mxfp8" (the expert inputs and the SwiGLU outputs
-    quantized to E4M3 in 32-value blocks before each projection; h is then returned quantized).
+    act: "bf16" (exact bf16 activations), "mxfp8" or "mxfp4" (the expert inputs and the SwiGLU
+    outputs quantized to E4M3 / E2M1 in 32-value blocks before each projection; h is then
+    returned quantized).
     Returns dict(y bf16 bits [n,d], y_f64 [n,d], idx [n,k], w [n,k], h [n,k,I] bf16 bits or None).
     """
     x_bf16 = np.ascontiguousarray(x_bf16, np.uint16)

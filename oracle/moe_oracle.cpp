@@ -51,6 +51,11 @@
 //    - 7 (amax / X lands in [128, 256)), clamped to [-122, 126], s = 0 for an
 //    all-zero block; element = X * (E4M3 value nearest to v / X, ties to the
 //    even code, saturating at 448).
+//  * Optional MXFP4 activations (act_format 2; also an extension): the same points and
+//    blocks, with the expert weights' own format ([ARCH] "量化": 4-bit values, one
+//    8-bit scale per 32): E2M1 elements and the weights' scale rule, s = floor(log2
+//    amax) - 2 clamped to [-127, 127] (s = 0 for an all-zero block), element =
+//    2^s * (E2M1 value nearest to v / 2^s, ties to the even code, saturating at 6).
 //
 // Oracle storage layout (its own, documented here): codes [rows][K/2], two codes
 // per byte, low nibble = even k; scale bytes [rows][K/32].
@@ -171,6 +176,24 @@ void mxfp8_block(double* v, int n, int32_t* exp_out) {
   if (exp_out) *exp_out = s;
 }
 
+// MXFP4 quantization of one block of n <= 32 values in place, by the rule the expert
+// weights are quantized with (oracle_quantize): 2^s * nearest E2M1 value of v / 2^s.
+void mxfp4_block(double* v, int n) {
+  double amax = 0.0;
+  for (int i = 0; i < n; ++i) amax = std::max(amax, std::fabs(v[i]));
+  const int s = amax > 0.0 ? std::clamp(floor_log2(amax) - 2, -127, 127) : 0;
+  for (int i = 0; i < n; ++i) {
+    const int c = nearest_e2m1_magnitude_code(std::fabs(std::ldexp(v[i], -s)));
+    v[i] = c == 0 ? 0.0 : std::copysign(std::ldexp(kE2M1[c], s), v[i]);
+  }
+}
+
+// The activation format's quantization of one 32-block (act_format 1: MXFP8, 2: MXFP4).
+void quantize_activation_block(double* v, int32_t act_format) {
+  if (act_format == 1) mxfp8_block(v, 32, nullptr);
+  else if (act_format == 2) mxfp4_block(v, 32);
+}
+
 template <class F>
 void parallel_chunks(int64_t n, int nthreads, F&& body) {
   if (nthreads <= 0) nthreads = (int)std::max(1u, std::thread::hardware_concurrency());
@@ -265,9 +288,25 @@ int32_t oracle_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t r
 // ---------------------------------------------------------------------------
 double oracle_round_bf16(double v) { return round_to_bf16(v); }
 
+// bf16 bit patterns of n doubles, each rounded to nearest (ties to even) as above.
+void oracle_to_bf16(const double* v, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = bf16_bits_of(round_to_bf16(v[i]));
+}
+
 // E4M3 code (0..0x7E) of the value nearest to |a|, ties to the even code, saturating.
 int32_t oracle_e4m3_nearest_code(double a) { return nearest_e4m3_code(std::fabs(a)); }
 double oracle_e4m3_value(int32_t code) { return (code >= 0 && code < 0x7F) ? e4m3_grid()[code] : NAN; }
+
+// MXFP4 quantization (the weights' rule) of n values (n a multiple of 32) in 32-value
+// blocks.  Returns 0, or 2 if n % 32 != 0.
+int32_t oracle_mxfp4_quantize_values(const double* v, int64_t n, double* out) {
+  if (n % 32) return 2;
+  for (int64_t b = 0; b < n / 32; ++b) {
+    std::memcpy(out + 32 * b, v + 32 * b, 32 * sizeof(double));
+    mxfp4_block(out + 32 * b, 32);
+  }
+  return 0;
+}
 
 // MXFP8 quantization of n values (n a multiple of 32) in 32-value blocks; exps[n/32]
 // receives the block scale exponents (nullable).  Returns 0, or 2 if n % 32 != 0.
@@ -379,7 +418,7 @@ int32_t oracle_group(int32_t T, int32_t k, int32_t E, const int32_t* idx, int32_
 // [d][I].  h is rounded to bf16; o is returned unrounded.
 // ---------------------------------------------------------------------------
 static void expert_mlp(int32_t d, int32_t I, const double* w1, const double* w2, const double* xe, double limit,
-                       bool mx_h, double* h, double* o) {
+                       int32_t act_format, double* h, double* o) {
   for (int32_t n = 0; n < I; ++n) {
     double g = 0.0, u = 0.0;
     for (int32_t i = 0; i < d; ++i) g += w1[(int64_t)n * d + i] * xe[i];
@@ -388,8 +427,8 @@ static void expert_mlp(int32_t d, int32_t I, const double* w1, const double* w2,
     const double uc = std::min(std::max(u, -limit), limit);
     h[n] = round_to_bf16(silu(gc) * uc);
   }
-  if (mx_h)   // MXFP8 activations: the down projection reads h in 32-blocks along I
-    for (int32_t b = 0; b < I / 32; ++b) mxfp8_block(h + 32 * b, 32, nullptr);
+  if (act_format)   // low-precision activations: the down projection reads h in 32-blocks along I
+    for (int32_t b = 0; b < I / 32; ++b) quantize_activation_block(h + 32 * b, act_format);
   for (int32_t m = 0; m < d; ++m) {
     double acc = 0.0;
     for (int32_t n = 0; n < I; ++n) acc += w2[(int64_t)m * I + n] * h[n];
@@ -407,7 +446,7 @@ static void expert_mlp(int32_t d, int32_t I, const double* w1, const double* w2,
 // Outputs per computed token (row r = position in tok): y_bf16 [n][d];
 // optional: y_f64 [n][d] (before the final rounding), idx [n][k], w [n][k],
 // h_bf16 [n][k][I] (the rounded SwiGLU outputs as the down projection reads them, slot
-// order).  act_format 0: bf16 activations; 1: MXFP8 activations (xe and h quantized in
+// order).  act_format 0: bf16 activations; 1: MXFP8, 2: MXFP4 activations (xe and h quantized in
 // 32-blocks, see the header).
 // Returns 0, or nonzero on bad arguments / NaN scale bytes.
 // ---------------------------------------------------------------------------
@@ -417,7 +456,7 @@ int32_t oracle_moe_forward(int32_t T, int32_t d, int32_t I, int32_t E, int32_t k
                            const uint8_t* w2_scales, const int32_t* tok, int32_t n_tok, uint16_t* y_bf16,
                            double* y_f64, int32_t* idx_out, double* w_out, uint16_t* h_bf16, int32_t nthreads,
                            int32_t act_format) {
-  if (d % 32 || I % 32 || k < 1 || k > E || act_format < 0 || act_format > 1) return 2;
+  if (d % 32 || I % 32 || k < 1 || k > E || act_format < 0 || act_format > 2) return 2;
   if (!tok) n_tok = T;
   std::vector<int32_t> ids(n_tok);
   for (int32_t r = 0; r < n_tok; ++r) ids[r] = tok ? tok[r] : r;
@@ -436,8 +475,8 @@ int32_t oracle_moe_forward(int32_t T, int32_t d, int32_t I, int32_t E, int32_t k
   std::vector<double> xe((size_t)n_tok * d);
   oracle_rmsnorm(n_tok, d, xs.data(), gamma, eps, xe.data());
   for (auto& v : xe) v = round_to_bf16(v);
-  if (act_format == 1)
-    for (int64_t b = 0; b < (int64_t)n_tok * (d / 32); ++b) mxfp8_block(&xe[(size_t)b * 32], 32, nullptr);
+  if (act_format)
+    for (int64_t b = 0; b < (int64_t)n_tok * (d / 32); ++b) quantize_activation_block(&xe[(size_t)b * 32], act_format);
 
   // Per (token, slot) expert outputs, computed expert by expert so that each
   // expert's weights are decoded once.
@@ -459,7 +498,7 @@ int32_t oracle_moe_forward(int32_t T, int32_t d, int32_t I, int32_t E, int32_t k
       for (int64_t j = j0; j < j1; ++j) {
         const int64_t q = jobs[j];
         const int64_t r = q / k;
-        expert_mlp(d, I, w1.data(), w2.data(), &xe[(size_t)r * d], limit, act_format == 1, h.data(),
+        expert_mlp(d, I, w1.data(), w2.data(), &xe[(size_t)r * d], limit, act_format, h.data(),
                    &o[(size_t)q * d]);
         if (h_bf16)
           for (int32_t n = 0; n < I; ++n) h_bf16[(size_t)q * I + n] = bf16_bits_of(h[n]);

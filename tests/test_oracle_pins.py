@@ -187,6 +187,20 @@ def test_round_bf16_midpoints_and_against_float32_bits():
     np.testing.assert_array_equal(got, ref.astype(np.float64))
 
 
+def test_to_bf16_array_matches_scalar_rounding_and_float32_bits():
+    rng = np.random.default_rng(5)
+    v = rng.standard_normal(3000) * np.exp2(rng.integers(-40, 40, 3000))
+    v[:4] = [1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8 + 2 ** -30), 0.0]
+    bits = oracle.to_bf16(v)
+    assert bits[0] == 0x3F80 and bits[1] == 0x3F82 and bits[2] == 0xBF81 and bits[3] == 0
+    got = synth.bf16_to_f32(bits).astype(np.float64)
+    np.testing.assert_array_equal(got, [oracle.round_bf16(float(a)) for a in v])
+    f = v.astype(np.float32)   # float32 inputs: rounding their bit patterns gives the same bf16
+    u = f.view(np.uint32).astype(np.uint64)
+    np.testing.assert_array_equal(oracle.to_bf16(f.astype(np.float64)),
+                                  ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16))
+
+
 # --------------------------------------------------------------------------- RMSNorm
 
 
@@ -211,6 +225,19 @@ def test_rmsnorm_closed_forms():
 
 
 # --------------------------------------------------------------------------- routing
+
+
+def test_next_block_norm_closed_form():
+    """A row of equal magnitudes c normalizes to +-gamma * c / sqrt(c^2 + eps), rounded to bf16."""
+    d = 128
+    c = 3.0
+    row = np.full(d, 0x4040, np.uint16)                 # 3.0
+    row[1::2] = 0xC040                                  # -3.0
+    gamma = np.linspace(0.25, 4.0, d).astype(np.float32)
+    got = synth.bf16_to_f32(oracle.next_block_norm(row[None, :], gamma, 1e-5)[0]).astype(np.float64)
+    want = np.where(np.arange(d) % 2, -1.0, 1.0) * gamma.astype(np.float64) * c / math.sqrt(c * c + 1e-5)
+    np.testing.assert_array_equal(got, [oracle.round_bf16(w) for w in want])
+    assert np.all(np.abs(got - want) <= np.abs(want) * 2.0 ** -8)
 
 
 def test_route_mixture_example_0p7_0p3():
@@ -490,3 +517,68 @@ def test_forward_mxfp8_stays_close_to_bf16():
     x = bf16_bits_to_f64(case[1])
     delta = np.linalg.norm(b - a) / np.linalg.norm(a - x)
     assert 1e-3 < delta < 0.1, delta
+
+
+# --------------------------------------------------------------------------- MXFP4 activations
+# The optional MXFP4 activation format (an extension, like MXFP8) quantizes the expert inputs
+# and the SwiGLU outputs with the weights' own format and rule (ewbang.com article, 量化:
+# 4-bit values, one 8-bit scale per 32).  Pinned against the already pinned weight quantizer
+# and against the E2M1 bit fields written out here.
+
+_E2M1_GRID = np.array([e2m1_from_bits(c) for c in range(8)])   # magnitudes, codes 0..7
+
+
+def _mx4_ref(v: np.ndarray) -> np.ndarray:
+    """MXFP4 of rows of v written out here: scale 2^(floor(log2 amax) - 2) per 32-block,
+    each |v| / scale to the nearest E2M1 magnitude (the even code on a tie, 6 above 6)."""
+    out = np.empty_like(v)
+    for idx in np.ndindex(v.shape[:-1]):
+        for b in range(v.shape[-1] // 32):
+            blk = v[idx][32 * b: 32 * b + 32]
+            amax = np.abs(blk).max()
+            s = min(127, max(-127, np.frexp(amax)[1] - 1 - 2)) if amax > 0 else 0
+            r = np.abs(blk) / 2.0 ** s
+            err = np.abs(r[:, None] - _E2M1_GRID[None, :])
+            best = err.min(axis=1, keepdims=True)
+            cand = np.where(err == best, np.arange(8)[None, :], 99)
+            even = np.where(cand % 2 == 0, cand, 99).min(axis=1)
+            code = np.where(even < 99, even, cand.min(axis=1))
+            code = np.where(r >= 6.0, 7, code)
+            out[idx][32 * b: 32 * b + 32] = np.where(code == 0, 0.0, np.sign(blk) * _E2M1_GRID[code] * 2.0 ** s)
+    return out
+
+
+def test_mxfp4_activations_match_the_weight_quantizer_and_bit_fields():
+    rng = np.random.default_rng(21)
+    v = rng.standard_normal((64, 96)) * np.exp(rng.uniform(-6, 6, (64, 1)))
+    v[0, :32] = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0] * 4) * np.where(np.arange(32) % 3, 1, -1)
+    v[1, :32] = 0.0
+    v = v.astype(np.float32).astype(np.float64)            # float32 values: the weight quantizer's input type
+    q = oracle.mxfp4_quantize_values(v)
+    np.testing.assert_array_equal(q, _mx4_ref(v))
+    codes, scales = oracle.quantize(v.astype(np.float32))
+    np.testing.assert_array_equal(q, oracle.dequantize(codes, scales))
+    assert np.all(q[1, :32] == 0.0)
+    np.testing.assert_array_equal(oracle.mxfp4_quantize_values(q), q)   # idempotent
+
+
+def test_forward_mxfp4_single_expert_is_dense_layer_on_quantized_activations():
+    case = _small_case(7, 64, 96, 1, 1, seed=17)
+    cfg, x, gamma, rw, rb, W, dec1, dec2 = case
+    out = _oracle_y(case, want_h=True, act="mxfp4")
+    xv = bf16_bits_to_f64(x)
+    xn = xv / np.sqrt(np.mean(xv ** 2, axis=1, keepdims=True) + 1e-5) * gamma
+    xe = _mx4_ref(round_bf16(xn))
+    gt, up = xe @ dec1[0][:cfg.I].T, xe @ dec1[0][cfg.I:].T
+    h = _mx4_ref(round_bf16(silu(np.minimum(gt, 7.0)) * np.clip(up, -7.0, 7.0)))
+    np.testing.assert_array_equal(bf16_bits_to_f64(out["h"][:, 0, :]), h)
+    np.testing.assert_allclose(out["y_f64"], xv + h @ dec2[0].T, rtol=0, atol=1e-12)
+
+
+def test_forward_mxfp4_moves_the_layer_more_than_mxfp8():
+    case = _small_case(16, 128, 128, 4, 2, seed=18)
+    a = _oracle_y(case)["y_f64"]
+    x = bf16_bits_to_f64(case[1])
+    d8 = np.linalg.norm(_oracle_y(case, act="mxfp8")["y_f64"] - a) / np.linalg.norm(a - x)
+    d4 = np.linalg.norm(_oracle_y(case, act="mxfp4")["y_f64"] - a) / np.linalg.norm(a - x)
+    assert d8 < d4 < 0.5, (d8, d4)
