@@ -75,8 +75,8 @@ def parse(argv=None):
     ap.add_argument("--config", default=None, choices=list(synth.CONFIGS),
                     help="measure this workload alone (default: the skewed 120b batch, plus the 20b decode batch)")
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
-    ap.add_argument("--act", default="bf16", choices=["bf16", "mxfp8"],
-                    help="activation format of the expert GEMMs: exact bf16 (the layer as stated) or MXFP8")
+    ap.add_argument("--act", default="bf16", choices=["bf16", "mxfp8", "mxfp4"],
+                    help="activation format of the expert GEMMs: exact bf16 (the layer as stated), MXFP8 or MXFP4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of "
                     "replaying a captured CUDA graph")

@@ -80,10 +80,19 @@ typedef enum {
  *   block), elements rounded to the nearest OCP FP8 E4M3 value (ties to even).  Half the
  *   activation bytes and tensor-core work; the E4M3 rounding moves the expert output
  *   (y - x) by about 5% of its norm at gpt-oss width, more than the exact layer's parity
- *   tolerance on y.  An extension: the pages quantize only the weights. */
+ *   tolerance on y.  An extension: the pages quantize only the weights.
+ * MOE_ACT_MXFP4: xe and h are quantized to MXFP4, the expert weights' own format and rule
+ *   (E2M1 elements, one E8M0 scale per 32 values along the projection's reduction axis,
+ *   scale 2^(floor(log2 amax) - 2) clamped to [2^-127, 2^127], elements rounded to the
+ *   nearest E2M1 value, ties to even, saturating at 6).  The expert GEMMs then run the
+ *   FP4 x FP4 block-scaled MMA (the FP4 rate) on the weight codes as stored; a quarter of
+ *   the bf16 activation bytes.  The E2M1 rounding moves the expert output far more than
+ *   MXFP8's (about 22% of y - x at gpt-oss width, against MXFP8's 5%); also an
+ *   extension. */
 typedef enum {
   MOE_ACT_BF16 = 0,
-  MOE_ACT_MXFP8 = 1
+  MOE_ACT_MXFP8 = 1,
+  MOE_ACT_MXFP4 = 2
 } moe_act_format;
 
 /* Which projection a weight tensor is (sets its row order in storage). */

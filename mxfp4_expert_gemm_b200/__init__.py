@@ -35,7 +35,8 @@ PATHS = {"auto": MOE_PATH_AUTO, "gemv": MOE_PATH_GEMV, "gemm": MOE_PATH_GEMM}
 
 MOE_ACT_BF16 = 0
 MOE_ACT_MXFP8 = 1
-ACT_FORMATS = {"bf16": MOE_ACT_BF16, "mxfp8": MOE_ACT_MXFP8}
+MOE_ACT_MXFP4 = 2
+ACT_FORMATS = {"bf16": MOE_ACT_BF16, "mxfp8": MOE_ACT_MXFP8, "mxfp4": MOE_ACT_MXFP4}
 
 MOE_WEIGHT_PLAIN = 0
 MOE_WEIGHT_GATE_UP = 1

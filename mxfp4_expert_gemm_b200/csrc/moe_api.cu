@@ -34,7 +34,8 @@ moe_status check_device() {
 moe_status check_dims(const moe_dims* dm, int32_t T) {
   if (!dm || T < 0) return MOE_ERR_INVALID_ARG;
   if (dm->path < MOE_PATH_AUTO || dm->path > MOE_PATH_GEMM) return MOE_ERR_INVALID_ARG;
-  if (dm->act_format != MOE_ACT_BF16 && dm->act_format != MOE_ACT_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (dm->act_format != MOE_ACT_BF16 && dm->act_format != MOE_ACT_MXFP8 && dm->act_format != MOE_ACT_MXFP4)
+    return MOE_ERR_INVALID_ARG;
   if (!(dm->rms_eps >= 0.f) || !std::isfinite(dm->rms_eps)) return MOE_ERR_INVALID_ARG;
   if (!(dm->swiglu_limit > 0.f) || !std::isfinite(dm->swiglu_limit)) return MOE_ERR_INVALID_ARG;
   if (dm->block != 32) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -53,12 +54,14 @@ int resolve_path(const moe_dims& dm, int32_t T) {
   return per_expert <= 24.0 ? MOE_PATH_GEMV : MOE_PATH_GEMM;
 }
 
-// E4M3 rows per token fed to the expert GEMMs: bf16 activations travel as two terms.
-int terms_of(const moe_dims& dm) { return dm.act_format == MOE_ACT_MXFP8 ? 1 : 2; }
+// Activation rows per token fed to the expert GEMMs: bf16 activations travel as two E4M3
+// terms; MXFP8 as one E4M3 row, MXFP4 as one row of packed E2M1 codes.
+int terms_of(const moe_dims& dm) { return dm.act_format == MOE_ACT_BF16 ? 2 : 1; }
 
 moe::WsLayout layout_for(const moe_dims& dm, int32_t T) {
   const int path = resolve_path(dm, T), terms = terms_of(dm);
-  return moe::ws_layout(dm, T, moe::expert_tile_tokens(path, terms), moe::expert_down_split(path), terms);
+  return moe::ws_layout(dm, T, moe::expert_tile_tokens(path, terms), moe::expert_down_split(path), terms,
+                        dm.act_format == MOE_ACT_MXFP4 ? 1 : 0);
 }
 
 moe_status prepare(const moe_dims* dm, int32_t T, const uint16_t* x, const float* norm_w, const float* router_w,

@@ -40,16 +40,44 @@ __host__ __device__ __forceinline__ int sf_byte_in_group(int r, int b) {
 __host__ __device__ constexpr int sf_groups_of(int rows) { return (rows + 127) / 128; }
 
 // Packed activation block of one token tile and one 128-chunk of the reduction axis: the
-// tile's `rows` E4M3 rows of 128 bytes in the 128-byte-swizzled order the MMA reads
-// (16-byte unit u of row n at unit u ^ (n % 8)), then the tile's scale-factor groups for
-// the chunk's four 32-blocks, padded to a multiple of 1 KB.  One contiguous copy brings a
-// block into shared memory.
-__host__ __device__ constexpr int packed_block_bytes(int rows) {
-  return (rows * kKChunk + sf_groups_of(rows) * kSfGroupBytes + 1023) / 1024 * 1024;
+// tile's `rows` rows in the swizzled order the MMA reads, then the tile's scale-factor
+// groups for the chunk's four 32-blocks, padded to a multiple of 1 KB.  One contiguous copy
+// brings a block into shared memory.  A row holds the chunk's 128 activations:
+//  - E4M3 (bf16 as two terms, or MXFP8): 128 bytes, 128-byte swizzle (16-byte unit u of
+//    row n at unit u ^ (n % 8));
+//  - E2M1 (MXFP4): 64 bytes of packed codes (element 2i in the low nibble of byte i),
+//    64-byte swizzle (unit u of row n at unit u ^ ((n / 2) % 4)).
+__host__ __device__ constexpr int packed_block_bytes(int rows, int row_bytes = kKChunk) {
+  return (rows * row_bytes + sf_groups_of(rows) * kSfGroupBytes + 1023) / 1024 * 1024;
 }
 __host__ __device__ __forceinline__ int packed_unit_offset(int n, int u) { return n * kKChunk + ((u ^ (n & 7)) << 4); }
-__host__ __device__ __forceinline__ int packed_sf_offset(int rows, int n, int b) {
-  return rows * kKChunk + (n >> 7) * kSfGroupBytes + sf_byte_in_group(n & 127, b & 3);
+__host__ __device__ __forceinline__ int packed_unit_offset64(int n, int u) {
+  return n * (kKChunk / 2) + ((u ^ ((n >> 1) & 3)) << 4);
+}
+__host__ __device__ __forceinline__ int packed_sf_offset(int rows, int n, int b, int row_bytes = kKChunk) {
+  return rows * row_bytes + (n >> 7) * kSfGroupBytes + sf_byte_in_group(n & 127, b & 3);
+}
+
+// ---------------------------------------------------------------- MXFP4 (E2M1 + E8M0)
+// The format of the pages (ewbang.com GPT-OSS article, section 量化: 4-bit values, one
+// 8-bit scale per 32): block scale 2^s with s = floor(log2 amax) - 2 clamped to [-127, 127]
+// (0 for an all-zero block), element = nearest E2M1 value of v / 2^s (ties to the even
+// code), saturating at 6.  Used for the weights and, with MXFP4 activations, for the
+// expert inputs and the SwiGLU outputs.
+
+// E2M1 magnitude code (0..7) of a >= 0 (already divided by the block scale): the number of
+// rounding thresholds between grid neighbours (0 .5 1 1.5 2 3 4 6) that a passes; ">" where
+// a tie belongs to the lower (even) code, ">=" where it belongs to the upper one.
+__device__ __forceinline__ int e2m1_code_of(float a) {
+  int c = 0;
+  c += a > 0.25f;   // tie -> 0
+  c += a >= 0.75f;  // tie -> 1.0
+  c += a > 1.25f;   // tie -> 1.0
+  c += a >= 1.75f;  // tie -> 2.0
+  c += a > 2.5f;    // tie -> 2.0
+  c += a >= 3.5f;   // tie -> 4.0
+  c += a > 5.0f;    // tie -> 4.0
+  return c;
 }
 
 // ------------------------------------------------------------------ MXFP4 storage layout
@@ -88,7 +116,8 @@ struct WsLayout {
   size_t perm;      // int32 [P]   sorted position -> t*k + slot
   size_t inv;       // int32 [P]   t*k + slot -> sorted position
   size_t w_sorted;  // f32 [P]     routing weight of each sorted pair
-  size_t xq;        // E4M3 [T][2][dp]   hi / lo terms of xe = bf16(RMSNorm(x))
+  size_t xq;        // E4M3 [T][2][dp]   hi / lo terms of xe = bf16(RMSNorm(x)) (MXFP4: packed
+                    // E2M1 codes in the first dp/2 bytes of each token's row)
   size_t xsf;       // E8M0 [T][2][dp/32] their scales
   size_t bpx;       // packed blocks [max_tiles][dp/128] of xe per token tile (gate_up's B)
   size_t bph;       // packed blocks [max_tiles][ip/128] of h per token tile (down's B)
@@ -97,19 +126,22 @@ struct WsLayout {
   size_t total;
   int64_t max_tiles;
   int32_t tile_tokens;
-  int32_t terms;     // E4M3 rows per token fed to the MMAs: 2 (bf16 activations) or 1 (MXFP8)
+  int32_t terms;     // rows per token fed to the MMAs: 2 (bf16 activations) or 1 (MXFP8, MXFP4)
+  int32_t fp4;       // activations are MXFP4 (E2M1 rows of 64 bytes per chunk)
   int32_t ksplit;   // down GEMM reduction-axis splits (ys planes)
   int32_t dp, ip;   // d and I rounded up to 128
 };
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-inline WsLayout ws_layout(const moe_dims& dm, int64_t T, int tile_tokens, int ksplit, int terms) {
+inline WsLayout ws_layout(const moe_dims& dm, int64_t T, int tile_tokens, int ksplit, int terms, int fp4) {
   WsLayout L{};
   const int64_t P = T * dm.top_k;
+  const int row_bytes = fp4 ? kKChunk / 2 : kKChunk;
   L.tile_tokens = tile_tokens;
   L.ksplit = ksplit;
   L.terms = terms;
+  L.fp4 = fp4;
   L.max_tiles = (P + tile_tokens - 1) / tile_tokens + dm.E;
   L.dp = (int32_t)kpad128(dm.d);
   L.ip = (int32_t)kpad128(dm.I);
@@ -132,8 +164,8 @@ inline WsLayout ws_layout(const moe_dims& dm, int64_t T, int tile_tokens, int ks
   L.w_sorted = take(4 * (size_t)P);
   L.xq = take(2 * (size_t)T * L.dp);
   L.xsf = take(2 * (size_t)T * (L.dp / 32));
-  L.bpx = take((size_t)L.max_tiles * (L.dp / kKChunk) * packed_block_bytes(terms * tile_tokens));
-  L.bph = take((size_t)L.max_tiles * (L.ip / kKChunk) * packed_block_bytes(terms * tile_tokens));
+  L.bpx = take((size_t)L.max_tiles * (L.dp / kKChunk) * packed_block_bytes(terms * tile_tokens, row_bytes));
+  L.bph = take((size_t)L.max_tiles * (L.ip / kKChunk) * packed_block_bytes(terms * tile_tokens, row_bytes));
   L.ys = take(4 * (size_t)ksplit * P * dm.d);
   L.total = o;
   return L;
@@ -162,6 +194,7 @@ struct Ws {
   int64_t max_tiles;
   int32_t tile_tokens;
   int32_t terms;
+  int32_t fp4;
   int32_t ksplit;
   int32_t dp, ip;
 };
@@ -191,6 +224,7 @@ inline Ws ws_pointers(void* base, const WsLayout& L, int E) {
   w.tile_tokens = L.tile_tokens;
   w.ksplit = L.ksplit;
   w.terms = L.terms;
+  w.fp4 = L.fp4;
   w.dp = L.dp;
   w.ip = L.ip;
   return w;
@@ -272,6 +306,30 @@ __device__ __forceinline__ void e4m3_split(const float (&v)[V], uint32_t& hi, ui
   }
   sf_hi = (uint32_t)(s1 + 127);
   sf_lo = (uint32_t)(s2 + 127);
+}
+
+// Warp-cooperative MXFP4 quantization of 32-value blocks, in the lane layout of e4m3_split
+// (each lane holds V consecutive values of a block spread over 32/V lanes), by the rule of
+// the weights (see e2m1_code_of).  Returns this lane's E2M1 codes (value i in bits 4i..4i+3;
+// bit 3 of a code is the sign, set only on non-zero codes) and the block's scale byte.
+template <int V>
+__device__ __forceinline__ void e2m1_quant(const float (&v)[V], uint32_t& codes, uint32_t& sf) {
+  constexpr int kLanes = 32 / V;
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < V; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+  for (int o = kLanes / 2; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  int s = 0;
+  if (amax > 0.f && amax < INFINITY) s = max(-127, min(127, floor_log2f(amax) - 2));
+  codes = 0u;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    int c = e2m1_code_of(ldexpf(fabsf(v[i]), -s));   // exact power-of-two scaling
+    if (v[i] < 0.f && c != 0) c |= 8;
+    codes |= (uint32_t)c << (4 * i);
+  }
+  sf = (uint32_t)(s + 127);
 }
 
 // Optional per-kernel CUDA events supplied by the caller: event 2i is recorded just

@@ -90,13 +90,16 @@ struct MxParams {
 #endif
 constexpr int kSfSlots = MOE_SF_SLOTS;  // scale-factor TMEM slots, used stage after stage in turn
 
-template <int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS>
+template <int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, bool FP4>
 struct MxCfg {
   static constexpr int N2 = TERMS * BN;                 // MMA N: hi (and lo) column per token
   static constexpr int G = (N2 + 127) / 128;            // scale-factor groups of the B operand
-  static constexpr int A_PANEL = kBM * kKChunk;         // 128 rows x 128 codes, one byte each
-  static constexpr int B_PANEL = N2 * kKChunk;          // N2 rows x 128 E4M3
-  static constexpr int B_BLOCK = packed_block_bytes(N2);  // B panel + its scale factors, padded
+  // Bytes of one operand row of a 128-chunk: E2M1 unpacked to a byte per code (A) or E4M3
+  // (B), 128; with MXFP4 activations both operands are packed E2M1, 64.
+  static constexpr int RB = FP4 ? kKChunk / 2 : kKChunk;
+  static constexpr int A_PANEL = kBM * RB;              // 128 weight rows
+  static constexpr int B_PANEL = N2 * RB;               // N2 activation rows
+  static constexpr int B_BLOCK = packed_block_bytes(N2, RB);  // B panel + its scale factors, padded
   static constexpr int B_OFF = NP * A_PANEL;
   static constexpr int SFA_OFF = B_OFF + NP * B_BLOCK;
   static constexpr int STAGE_BYTES = ((SFA_OFF + NP * kSfGroupBytes + 1023) / 1024) * 1024;
@@ -160,10 +163,10 @@ __device__ __forceinline__ int choose_ksplit(int n0, int grid, int smax) {
   return max(1, min(smax, (2 * grid + n0 - 1) / n0));
 }
 
-template <int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, int MODE>
-__global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>::THREADS, CPS)
+template <int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, bool FP4, int MODE>
+__global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::THREADS, CPS)
     mx_expert_kernel(const __grid_constant__ CUtensorMap tm_w, const MxParams p) {
-  using C = MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>;
+  using C = MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>;
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
 
@@ -307,14 +310,26 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>::THREADS
                                       ptx::smem_desc_k_rows16(b_s(s) + c * C::B_BLOCK + C::B_PANEL + gg * kSfGroupBytes));
             }
             for (int c = 0; c < nck; ++c) {
-              const int nkb = min(4, kblocks - 4 * (c0 + c));
-              const uint64_t adesc = ptx::smem_desc_k_sw128(a_s(s) + c * C::A_PANEL);
-              const uint64_t bdesc = ptx::smem_desc_k_sw128(b_s(s) + c * C::B_BLOCK);
+              const int nkb = min(4, kblocks - 4 * (c0 + c));   // 32-blocks of this chunk (K % 64 == 0: even)
               const uint32_t sfa = sf_slot + C::SFA_COL + 4 * c, sfb = sf_slot + C::SFB_COL + 4 * c * C::G;
-              for (int kk = 0; kk < nkb; ++kk)
-                ptx::mma_mx_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
-                               ptx::idesc_mx_e2m1_e4m3(kBM, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
-                               (st | c | kk) != 0);
+              if (FP4) {
+                // FP4 x FP4: one MMA per 64 k (32 bytes of each packed row); it takes the scale
+                // bytes 2kk and 2kk + 1 of each row's scale-factor word
+                const uint64_t adesc = ptx::smem_desc_k_sw64(a_s(s) + c * C::A_PANEL);
+                const uint64_t bdesc = ptx::smem_desc_k_sw64(b_s(s) + c * C::B_BLOCK);
+                for (int kk = 0; kk < nkb / 2; ++kk)
+                  ptx::mma_mxf4_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
+                                   ptx::idesc_mxf4(kBM, C::N2, (uint32_t)(2 * kk), (uint32_t)(2 * kk)), sfa, sfb,
+                                   (st | c | kk) != 0);
+              } else {
+                // E2M1 x E4M3: one MMA per 32 k (32 bytes of each row), scale byte kk
+                const uint64_t adesc = ptx::smem_desc_k_sw128(a_s(s) + c * C::A_PANEL);
+                const uint64_t bdesc = ptx::smem_desc_k_sw128(b_s(s) + c * C::B_BLOCK);
+                for (int kk = 0; kk < nkb; ++kk)
+                  ptx::mma_mx_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
+                                 ptx::idesc_mx_e2m1_e4m3(kBM, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
+                                 (st | c | kk) != 0);
+              }
             }
             ptx::tc_commit(&sfree[s]);
           }
@@ -396,9 +411,22 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>::THREADS
             float hv = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;   // silu(g) * u
             hv = __uint_as_float((uint32_t)bf16_bits_rne(hv) << 16);   // h is stored as bf16
             const float vv[1] = {hv};
+            const int j = c0 / TERMS + jj;             // token within the tile
+            if (FP4) {
+              // MXFP4 activations: h's 32-block as E2M1 codes (two per byte) and its scale,
+              // into the down GEMM's packed block: chunk kb / 4, 16-byte unit kb % 4 of row j
+              uint32_t code, sf4;
+              e2m1_quant<1>(vv, code, sf4);
+              const uint32_t code_hi = __shfl_down_sync(0xffffffffu, code, 1);
+              if (j < tl.rows) {
+                uint8_t* blk = p.bp_out + ((int64_t)tt * p.KCo + kb / 4) * C::B_BLOCK;
+                if ((lane & 1) == 0) blk[packed_unit_offset64(j, kb & 3) + lane / 2] = (uint8_t)(code | (code_hi << 4));
+                if (lane == 0) blk[packed_sf_offset(C::N2, j, kb, C::RB)] = (uint8_t)sf4;
+              }
+              continue;
+            }
             uint32_t hi, lo, s1, s2;
             e4m3_split<1>(vv, hi, lo, s1, s2);
-            const int j = c0 / TERMS + jj;             // token within the tile
             if (j < tl.rows) {
               // the down GEMM's packed block: chunk kb / 4, rows 2j (hi) and 2j + 1 (lo),
               // byte f' = 32 (kb % 4) + lane of the 128-byte row
@@ -503,7 +531,7 @@ EncodeTiledFn encode_fn() {
 }
 
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box) {
+              const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[4], gs[3];
@@ -514,7 +542,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
   return fn(m, dt, rank, const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -526,9 +554,9 @@ int sm_count() {
   return n;
 }
 
-template <int MODE, int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, int KSPLIT>
+template <int MODE, int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, bool FP4, int KSPLIT>
 int launch_one(const FwdArgs& a) {
-  using C = MxCfg<BN, NP, S, CPS, EG, NPW, TERMS>;
+  using C = MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>;
   const int P = a.T * a.k;
   const int K = (MODE == MODE_GATE_UP) ? a.d : a.I;
   const int N = (MODE == MODE_GATE_UP) ? 2 * a.I : a.d;  // weight rows per expert
@@ -537,16 +565,26 @@ int launch_one(const FwdArgs& a) {
   const uint8_t* codes = (MODE == MODE_GATE_UP) ? a.w1c : a.w2c;
   const uint8_t* scales = (MODE == MODE_GATE_UP) ? a.w1s : a.w2s;
 
-  // Weight codes [E][NT][KC][128][64] viewed as rows of 128 codes (E2M1, unpacked by the
-  // copy): one box brings NP consecutive tile blocks (NP x 128 rows), each a
-  // 128B-swizzled [128][128] panel in shared memory.
+  // Weight codes [E][NT][KC][128][64] viewed as rows of 64 bytes: one box brings NP
+  // consecutive tile blocks (NP x 128 rows).  E2M1 x E4M3: the rows are 128 codes, unpacked
+  // by the copy to a byte each, 128B-swizzled [128][128] panels in shared memory; FP4 x FP4:
+  // the packed bytes as stored, 64B-swizzled [128][64] panels.
   CUtensorMap m_w;
   {
     const int NT = (N + kBM - 1) / kBM;
-    const uint64_t dims[2] = {(uint64_t)kKChunk, (uint64_t)a.E * NT * KC * kBM};
+    const uint64_t rows = (uint64_t)a.E * NT * KC * kBM;
     const uint64_t str[1] = {(uint64_t)kKChunk / 2};
-    const uint32_t box[2] = {kKChunk, (uint32_t)(kBM * NP)};
-    if (!make_map(&m_w, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, codes, dims, str, box)) return -1;
+    if (FP4) {
+      const uint64_t dims[2] = {(uint64_t)kKChunk / 2, rows};
+      const uint32_t box[2] = {kKChunk / 2, (uint32_t)(kBM * NP)};
+      if (!make_map(&m_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
+        return -1;
+    } else {
+      const uint64_t dims[2] = {(uint64_t)kKChunk, rows};
+      const uint32_t box[2] = {kKChunk, (uint32_t)(kBM * NP)};
+      if (!make_map(&m_w, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, codes, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+        return -1;
+    }
   }
   MxParams prm;
   prm.tiles = a.ws.tiles;
@@ -576,7 +614,7 @@ int launch_one(const FwdArgs& a) {
   prm.y_partial = a.y_partial;
   prm.arrivals = a.ws.arrivals;
 
-  auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, NPW, TERMS, MODE>;
+  auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, NPW, TERMS, FP4, MODE>;
   static std::atomic<uint64_t> attr_done{0};   // per-device "attribute set" bits
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -636,6 +674,15 @@ int launch_one(const FwdArgs& a) {
 #define MOE_GEMM_NPW 1
 #endif
 
+// With MXFP4 activations the packed E2M1 operands take half the shared memory per stage:
+// more stages in flight.
+#ifndef MOE_GEMV_S_FP4
+#define MOE_GEMV_S_FP4 6
+#endif
+#ifndef MOE_GEMM_S_FP4
+#define MOE_GEMM_S_FP4 4
+#endif
+
 constexpr int kGemvBN = 8, kGemvNP = MOE_GEMV_NP, kGemvS = MOE_GEMV_S, kGemvCPS = MOE_GEMV_CPS,
               kGemvEG = MOE_GEMV_EG, kGemvNPW = MOE_GEMV_NPW, kGemvDownSplit = MOE_GEMV_DOWN_SPLIT;
 constexpr int kGemmBN = 96, kGemmNP = MOE_GEMM_NP, kGemmS = MOE_GEMM_S, kGemmCPS = MOE_GEMM_CPS,
@@ -644,31 +691,35 @@ static_assert(kGemvBN >= kMinTileTokens, "tile list sized for the smallest tile"
 
 }  // namespace
 
-// With MXFP8 activations a token is one MMA column instead of two: tiles of twice the
-// tokens keep the same MMA shape.
+// With MXFP8 or MXFP4 activations a token is one MMA column instead of two: tiles of twice
+// the tokens keep the same MMA shape.
 int expert_tile_tokens(int path, int terms) { return (path == MOE_PATH_GEMV ? kGemvBN : kGemmBN) * (2 / terms); }
 
 int expert_down_split(int path) { return path == MOE_PATH_GEMV ? kGemvDownSplit : 1; }
 
 namespace {
-template <int TERMS>
+template <int TERMS, bool FP4>
 int launch_pair(const FwdArgs& a) {
   constexpr int gv = kGemvBN * 2 / TERMS, gm = kGemmBN * 2 / TERMS;
+  constexpr int sv = FP4 ? MOE_GEMV_S_FP4 : kGemvS, sm = FP4 ? MOE_GEMM_S_FP4 : kGemmS;
   int n1, n2;
   if (a.ws.tile_tokens == gv) {
-    n1 = launch_one<MODE_GATE_UP, gv, kGemvNP, kGemvS, kGemvCPS, kGemvEG, kGemvNPW, TERMS, 1>(a);
+    n1 = launch_one<MODE_GATE_UP, gv, kGemvNP, sv, kGemvCPS, kGemvEG, kGemvNPW, TERMS, FP4, 1>(a);
     if (n1 < 0) return -1;
-    n2 = launch_one<MODE_DOWN, gv, kGemvNP, kGemvS, kGemvCPS, kGemvEG, kGemvNPW, TERMS, kGemvDownSplit>(a);
+    n2 = launch_one<MODE_DOWN, gv, kGemvNP, sv, kGemvCPS, kGemvEG, kGemvNPW, TERMS, FP4, kGemvDownSplit>(a);
   } else {
-    n1 = launch_one<MODE_GATE_UP, gm, kGemmNP, kGemmS, kGemmCPS, kGemmEG, kGemmNPW, TERMS, 1>(a);
+    n1 = launch_one<MODE_GATE_UP, gm, kGemmNP, sm, kGemmCPS, kGemmEG, kGemmNPW, TERMS, FP4, 1>(a);
     if (n1 < 0) return -1;
-    n2 = launch_one<MODE_DOWN, gm, kGemmNP, kGemmS, kGemmCPS, kGemmEG, kGemmNPW, TERMS, 1>(a);
+    n2 = launch_one<MODE_DOWN, gm, kGemmNP, sm, kGemmCPS, kGemmEG, kGemmNPW, TERMS, FP4, 1>(a);
   }
   if (n2 < 0) return -1;
   return n1 + n2;
 }
 }  // namespace
 
-int launch_experts(const FwdArgs& a) { return a.ws.terms == 1 ? launch_pair<1>(a) : launch_pair<2>(a); }
+int launch_experts(const FwdArgs& a) {
+  if (a.ws.fp4) return launch_pair<1, true>(a);
+  return a.ws.terms == 1 ? launch_pair<1, false>(a) : launch_pair<2, false>(a);
+}
 
 }  // namespace moe

@@ -29,20 +29,6 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_floa
 // the E2M1 code of |x| * 2^-s is the number of rounding thresholds it passes,
 // each threshold taking ties toward the even code.
 // ----------------------------------------------------------------------------------
-__device__ __forceinline__ int e2m1_code_of(float a) {
-  // grid 0 .5 1 1.5 2 3 4 6; thresholds between neighbours, "<" where the tie
-  // belongs to the upper (even) code, "<=" where it belongs to the lower one.
-  int c = 0;
-  c += a > 0.25f;   // tie -> 0
-  c += a >= 0.75f;  // tie -> 1.0
-  c += a > 1.25f;   // tie -> 1.0
-  c += a >= 1.75f;  // tie -> 2.0
-  c += a > 2.5f;    // tie -> 2.0
-  c += a >= 3.5f;   // tie -> 4.0
-  c += a > 5.0f;    // tie -> 4.0
-  return c;
-}
-
 __global__ void quantize_kernel(const float* __restrict__ w, int64_t nblocks, int32_t N, int32_t K, int32_t role,
                                 uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int32_t* status) {
   const int lane = threadIdx.x & 31;
@@ -157,6 +143,17 @@ __device__ __forceinline__ void pack_pair_chunk(const FwdArgs& a, int t, int til
   const int lane = threadIdx.x & 31;
   const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk, terms = a.ws.terms;
   const int rows = terms * bt;
+  if (a.ws.fp4) {   // MXFP4: one 64-byte row of packed codes; lanes 0-3 move it, 16-19 the scales
+    uint8_t* block = a.ws.bpx + ((int64_t)tile * kc + c) * packed_block_bytes(rows, kKChunk / 2);
+    if (lane < 4) {
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.ws.xq + (int64_t)t * 2 * dp + c * (kKChunk / 2)) + lane);
+      *reinterpret_cast<uint4*>(block + packed_unit_offset64(col, lane)) = v;
+    } else if (lane >= 16 && lane < 20) {
+      const int b = 4 * c + (lane - 16);
+      if (b < nb) block[packed_sf_offset(rows, col, b, kKChunk / 2)] = __ldcg(a.ws.xsf + (int64_t)t * 2 * (dp / 32) + b);
+    }
+    return;
+  }
   uint8_t* block = a.ws.bpx + ((int64_t)tile * kc + c) * packed_block_bytes(rows);
   if (lane < 16) {   // (units past d are never read by the MMAs)
     const int term = lane >> 3, u = lane & 7;
@@ -311,6 +308,14 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
     uint8_t* sf = a.ws.xsf + t * 2 * (dp / 32);
     for (int b = warp; b < d / 32; b += kTokWarps) {
       const float v[1] = {bf16_to_f32(bf16_bits_rne(s_xn[32 * b + lane]))};
+      if (a.ws.fp4) {   // MXFP4 activations: packed E2M1 codes, two per byte
+        uint32_t c, s1;
+        e2m1_quant<1>(v, c, s1);
+        const uint32_t c_hi = __shfl_down_sync(0xffffffffu, c, 1);
+        if ((lane & 1) == 0) xq[16 * b + lane / 2] = (uint8_t)(c | (c_hi << 4));
+        if (lane == 0) sf[b] = (uint8_t)s1;
+        continue;
+      }
       uint32_t hi, lo, s1, s2;
       e4m3_split<1>(v, hi, lo, s1, s2);
       xq[32 * b + lane] = (uint8_t)hi;
@@ -494,6 +499,13 @@ __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
           s_xn[tt * RK + kk] = v0;
           s_xn[tt * RK + kk + 1] = v1;
           const float v[2] = {bf16_to_f32(bf16_bits_rne(v0)), bf16_to_f32(bf16_bits_rne(v1))};
+          if (a.ws.fp4) {   // MXFP4 activations: this lane's two codes are one byte
+            uint32_t c, s1;
+            e2m1_quant<2>(v, c, s1);
+            xq[(k0 + kk) / 2] = (uint8_t)c;
+            if ((lane & 15) == 0) sf[(k0 + kk) / 32] = (uint8_t)s1;
+            continue;
+          }
           uint32_t hi, lo, s1, s2;
           e4m3_split<2>(v, hi, lo, s1, s2);   // lanes 0-15: block k0/32, 16-31: the next
           *reinterpret_cast<uint16_t*>(xq + k0 + kk) = (uint16_t)hi;
@@ -506,6 +518,14 @@ __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
           const float v0 = bf16_to_f32(s_x[(st * kRT + tt) * RK + lane]) * r * s_g[k0 + lane];
           s_xn[tt * RK + lane] = v0;
           const float v[1] = {bf16_to_f32(bf16_bits_rne(v0))};
+          if (a.ws.fp4) {
+            uint32_t c, s1;
+            e2m1_quant<1>(v, c, s1);
+            const uint32_t c_hi = __shfl_down_sync(0xffffffffu, c, 1);
+            if ((lane & 1) == 0) xq[(k0 + lane) / 2] = (uint8_t)(c | (c_hi << 4));
+            if (lane == 0) sf[k0 / 32] = (uint8_t)s1;
+            continue;
+          }
           uint32_t hi, lo, s1, s2;
           e4m3_split<1>(v, hi, lo, s1, s2);
           xq[k0 + lane] = (uint8_t)hi;
@@ -646,6 +666,20 @@ __device__ __forceinline__ void pack_pair(const FwdArgs& a, int t, int tile, int
   const int lane = threadIdx.x & 31;
   const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk, terms = a.ws.terms;
   const int rows_t = terms * bt;
+  if (a.ws.fp4) {   // MXFP4: per chunk one 64-byte row of packed codes (4 units) and 4 scales
+    const int bb = packed_block_bytes(rows_t, kKChunk / 2);
+    uint8_t* blocks = a.ws.bpx + (int64_t)tile * kc * bb;
+    const uint8_t* row = a.ws.xq + (int64_t)t * 2 * dp;
+    for (int i = lane; i < kc * 4; i += 32) {
+      const int c = i >> 2, u = i & 3;
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(row + c * (kKChunk / 2)) + u);
+      *reinterpret_cast<uint4*>(blocks + (int64_t)c * bb + packed_unit_offset64(col, u)) = v;
+    }
+    const uint8_t* sf = a.ws.xsf + (int64_t)t * 2 * (dp / 32);
+    for (int b = lane; b < nb; b += 32)
+      blocks[(int64_t)(b / 4) * bb + packed_sf_offset(rows_t, col, b, kKChunk / 2)] = __ldcg(sf + b);
+    return;
+  }
   const int bb = packed_block_bytes(rows_t);
   uint8_t* blocks = a.ws.bpx + (int64_t)tile * kc * bb;
   const uint8_t* rows = a.ws.xq + (int64_t)t * 2 * dp;

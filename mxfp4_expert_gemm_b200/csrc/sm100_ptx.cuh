@@ -188,6 +188,44 @@ __device__ __forceinline__ void mma_mx_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// SMEM descriptor of a K-major operand tile laid out by a 64-byte-swizzled load: rows of 64
+// bytes, 8-row groups 512 bytes apart (the tile starts on a 512-byte boundary).
+__device__ __forceinline__ uint64_t smem_desc_k_sw64(const void* tile) {
+  const uint64_t addr = smem_u32(tile);
+  uint64_t d = (addr & 0x3FFFFull) >> 4;   // start address (16-byte units)
+  d |= 1ull << 16;                          // leading byte offset (unused by swizzled K-major)
+  d |= (uint64_t)(512 >> 4) << 32;          // stride byte offset: next 8-row group
+  d |= 1ull << 46;                          // descriptor version (sm_100)
+  d |= 4ull << 61;                          // 64-byte swizzle
+  return d;
+}
+
+// Instruction descriptor of kind::mxf4.block_scale: E2M1 A and B (packed, K-major), fp32 D,
+// E8M0 scale factors, K = 64 per MMA.  With one scale per 32 values an MMA uses two scale
+// bytes of each 32-bit scale-factor word: bytes sf_id and sf_id + 1 (sf_id 0 or 2).
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t sfa_id, uint32_t sfb_id) {
+  return ((sfb_id & 3u) << 4)            // B scale-factor byte
+         | (1u << 7)                     // A format: E2M1
+         | (1u << 10)                    // B format: E2M1
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | (1u << 23)                    // scale format: E8M0
+         | ((uint32_t)(M >> 4) << 24)    // M / 16
+         | ((sfa_id & 3u) << 29);        // A scale-factor byte
+}
+
+// D[tmem] (+)= (A * SFA) * (B * SFB)^T over one 64-wide K block, kind::mxf4 (FP4 x FP4, one
+// E8M0 scale per 32 values), one CTA.
+__device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // SMEM descriptor of an unswizzled K-major source of 16-byte rows: 8-row core matrices
 // stored back to back (128 bytes apart).
 __device__ __forceinline__ uint64_t smem_desc_k_rows16(const void* p) {

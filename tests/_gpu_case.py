@@ -24,7 +24,16 @@ TILE_TOKENS = {"gemv": 8, "gemm": 96}
 
 
 def tile_tokens(path: str, act: str = "bf16") -> int:
-    return TILE_TOKENS[path] * (2 if act == "mxfp8" else 1)
+    return TILE_TOKENS[path] * (1 if act == "bf16" else 2)
+
+
+_E2M1_LUT = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6])
+
+
+def decode_e2m1_packed(b: np.ndarray) -> np.ndarray:
+    """Packed E2M1 bytes -> float64 values, two per byte (element 2i in the low nibble)."""
+    b = b.astype(np.int64)
+    return np.stack([_E2M1_LUT[b & 15], _E2M1_LUT[b >> 4]], axis=-1).reshape(*b.shape[:-1], -1)
 
 
 def decode_e4m3(b: np.ndarray) -> np.ndarray:

@@ -5,8 +5,8 @@ T = 8192, E = 128; the Zipf-skewed 120b batch, T = 16384) run through the C ABI 
 are compared with the oracle on every token, on the exact (bf16-activation) layer.
 The routing and the grouping (counts, offsets, the (expert, token)-sorted pair list,
 the token tiles of both paths) are compared bit for bit.  The MXFP8 activation format
-is checked on a deterministic token set that holds the first and the last token of
-every token tile of every expert.
+and the MXFP4 activation formats are checked on a deterministic token set that holds the
+first and the last token of every token tile of every expert.
 
 The oracle is computed once per workload (all host cores, about a minute for the
 20b prefill batch and a few minutes for the skewed batch) and shared by the paths.
@@ -123,16 +123,18 @@ def test_full_size_every_row(name, path):
     assert row_err.max() <= 1e-2, (int(row_err.argmax()), float(row_err.max()))
 
 
-@pytest.mark.parametrize("name,path", [("prefill_20b", "gemm"), ("moe_120b", "gemm"), ("prefill_20b", "gemv")])
-def test_full_size_mxfp8_tile_cover(name, path):
-    """MXFP8 activations at full size, on the first and last token of every token tile."""
+@pytest.mark.parametrize("name,path,act", [("prefill_20b", "gemm", "mxfp8"), ("moe_120b", "gemm", "mxfp8"),
+                                           ("prefill_20b", "gemv", "mxfp8"), ("prefill_20b", "gemm", "mxfp4"),
+                                           ("skew_120b", "gemm", "mxfp4"), ("prefill_20b", "gemv", "mxfp4")])
+def test_full_size_low_precision_tile_cover(name, path, act):
+    """MXFP8 / MXFP4 activations at full size, on the first and last token of every token tile."""
     c = case(C[name])
     cfg = c["cfg"]
-    g = run_gpu(c, path, act="mxfp8")
+    g = run_gpu(c, path, act=act)
     assert g["status"] == moe.MOE_OK, moe.status_string(g["status"])
     np.testing.assert_array_equal(np.sort(g["routing"]["topk_idx"].cpu().numpy(), 1),
                                   np.sort(c["route"]["idx"], 1))
-    toks = tile_cover_tokens(c["route"]["idx"], cfg.E, tile_tokens(path, "mxfp8"))
-    ref = oracle_rows(c, tokens=toks, act="mxfp8")
+    toks = tile_cover_tokens(c["route"]["idx"], cfg.E, tile_tokens(path, act))
+    ref = oracle_rows(c, tokens=toks, act=act)
     st = parity_stats(bf16_host(g["y"])[toks], ref["y"], c["x"][toks])
-    assert_parity(st, f"{name}/{path}/mxfp8")
+    assert_parity(st, f"{name}/{path}/{act}")

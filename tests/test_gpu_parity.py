@@ -11,8 +11,8 @@ import torch
 import mxfp4_expert_gemm_b200 as moe
 import oracle
 import synth
-from _gpu_case import (TILE_TOKENS, assert_parity, bf16_dev, bf16_host, case, decode_e4m3, oracle_rows, parity_stats, run_gpu,
-                       stored_row_of, stored_to_rowmajor, tile_tokens, weights)
+from _gpu_case import (TILE_TOKENS, assert_parity, bf16_dev, bf16_host, case, decode_e2m1_packed, decode_e4m3,
+                       oracle_rows, parity_stats, run_gpu, stored_row_of, stored_to_rowmajor, tile_tokens, weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -152,6 +152,37 @@ def test_forward_parity(name, path):
     np.testing.assert_array_equal(np.sort(g["routing"]["topk_idx"].cpu().numpy(), 1), np.sort(ref["idx"], 1))
 
 
+def _h_from_workspace_fp4(g, cfg):
+    """h [P, I] from the down GEMM's packed MXFP4 blocks: per token tile and 128-chunk, one
+    row of 64 bytes per token (16-byte unit u of row n stored at unit u ^ ((n // 2) % 4);
+    element 2i in the low nibble of byte i), then the scale-factor groups."""
+    dims, ws, T = g["dims"], g["ws"], cfg.T
+    P = T * cfg.k
+    KC = moe.kpad128(cfg.I) // 128
+    bt = tile_tokens(moe.resolved_path(dims, T), "mxfp4")
+    G = (bt + 127) // 128
+    BB = (bt * 64 + G * 512 + 1023) // 1024 * 1024
+    view = lambda f, dt, sh: moe.workspace_view(ws, dims, T, f, dt, sh).cpu().numpy()
+    offsets = view("offsets", torch.int32, (cfg.E + 1,))
+    tbase = view("tile_base", torch.int32, (cfg.E,))
+    n_tiles = (P + bt - 1) // bt + cfg.E
+    bph = view("bph", torch.uint8, (n_tiles, KC, BB))
+    h = np.empty((P, cfg.I))
+    b = np.arange(cfg.I // 32)
+    u = np.arange(4)
+    for p in range(P):
+        e = int(np.searchsorted(offsets, p, side="right") - 1)
+        j = p - offsets[e]
+        tile, n = tbase[e] + j // bt, j % bt
+        phys = n * 64 + ((u ^ ((n >> 1) % 4)) << 4)
+        rows = bph[tile][:, (phys[:, None] + np.arange(16)[None, :]).ravel()]      # [KC, 64]
+        vals = decode_e2m1_packed(rows).reshape(-1)[: cfg.I]
+        sfo = bt * 64 + (n // 128) * 512 + (n % 32) * 16 + ((n % 128) // 32) * 4 + b % 4
+        sc = bph[tile, b // 4, sfo].astype(np.float64) - 127
+        h[p] = vals * np.repeat(np.exp2(sc), 32)
+    return h
+
+
 def _h_from_workspace(g, cfg):
     """h [P, I] (sorted pairs) rebuilt from the down GEMM's packed activation blocks: per
     token tile and 128-chunk, terms*BN E4M3 rows (row n = term n % terms of token
@@ -262,6 +293,54 @@ def test_swiglu_output_h_mxfp8(path):
     inv = moe.workspace_view(g["ws"], g["dims"], cfg.T, "inv", torch.int32, (P,)).cpu().numpy()
     idx = g["routing"]["topk_idx"].cpu().numpy()
     ref = oracle_rows(c, want_h=True, act="mxfp8")
+    href = synth.bf16_to_f32(ref["h"]).astype(np.float64)
+    same = total = 0
+    num = den = 0.0
+    for t in range(cfg.T):
+        for s in range(cfg.k):
+            so = int(np.nonzero(ref["idx"][t] == idx[t, s])[0][0])
+            a, b = h[inv[t * cfg.k + s]], href[t, so]
+            same += int(np.count_nonzero(a == b))
+            total += a.size
+            num += float((a - b) @ (a - b))
+            den += float(b @ b)
+    assert same / total >= 0.99, same / total
+    assert np.sqrt(num / den) <= 1e-2
+
+
+# ------------------------------------------------------------------------------ MXFP4 activations
+# MOE_ACT_MXFP4: the expert inputs and the SwiGLU outputs quantized with the weights' own
+# format (E2M1 in 32-value blocks); the FP4 x FP4 MMA.  The oracle models the same
+# quantization (act="mxfp4").  Same bars as the other formats, against that oracle.
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_parity_mxfp4(name, path):
+    c = case(SMALL[name])
+    g = run_gpu(c, path, act="mxfp4")
+    assert g["status"] == moe.MOE_OK, moe.status_string(g["status"])
+    ref = oracle_rows(c, act="mxfp4")
+    st = parity_stats(bf16_host(g["y"]), ref["y"], c["x"])
+    assert_parity(st, f"{name}/{path}/mxfp4")
+    assert st["delta_rel_fro"] <= 2.5e-2, st
+    np.testing.assert_array_equal(np.sort(g["routing"]["topk_idx"].cpu().numpy(), 1), np.sort(ref["idx"], 1))
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_swiglu_output_h_mxfp4(path):
+    """h as the down GEMM reads it with MXFP4 activations: one row of packed E2M1 codes per
+    token with its block scales, equal to the oracle's quantized h up to rare one-step
+    rounding flips (h is computed in fp32 here and in fp64 there before both round it)."""
+    c = case(SMALL["mid_ragged"])
+    cfg = c["cfg"]
+    g = run_gpu(c, path, act="mxfp4")
+    assert g["status"] == moe.MOE_OK
+    P = cfg.T * cfg.k
+    h = _h_from_workspace_fp4(g, cfg)
+    inv = moe.workspace_view(g["ws"], g["dims"], cfg.T, "inv", torch.int32, (P,)).cpu().numpy()
+    idx = g["routing"]["topk_idx"].cpu().numpy()
+    ref = oracle_rows(c, want_h=True, act="mxfp4")
     href = synth.bf16_to_f32(ref["h"]).astype(np.float64)
     same = total = 0
     num = den = 0.0
