@@ -59,7 +59,9 @@ typedef enum {
   MOE_ERR_CUDA = 4,              /* a CUDA runtime error at launch */
   MOE_ERR_TIMEOUT = 5,           /* (device) a pipeline wait gave up; the kernel exited cleanly */
   MOE_ERR_NONFINITE = 6,         /* (device) Inf/NaN in the input or the weights */
-                                 /* 7 is not used */
+  MOE_ERR_BOUNDS = 7,            /* (device; bounds-checking builds only, see build.py) a kernel
+                                    computed a store address outside its buffer; the store was
+                                    skipped */
   MOE_ERR_DEVICE = 8             /* the current device is not sm_100 */
 } moe_status;
 

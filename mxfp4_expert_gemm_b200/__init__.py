@@ -8,6 +8,7 @@ sm_100, the calls raise.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import re
@@ -26,6 +27,7 @@ MOE_ERR_WORKSPACE = 3
 MOE_ERR_CUDA = 4
 MOE_ERR_TIMEOUT = 5
 MOE_ERR_NONFINITE = 6
+MOE_ERR_BOUNDS = 7
 MOE_ERR_DEVICE = 8
 
 MOE_PATH_AUTO = 0
@@ -75,47 +77,70 @@ def lib():
         if _lib is None:
             if not os.path.exists(LIB_PATH):
                 raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m mxfp4_expert_gemm_b200.build`")
-            L = ctypes.CDLL(LIB_PATH)
-            vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
-            dp = ctypes.POINTER(moe_dims)
-            L.moe_mxfp4_codes_bytes.argtypes = [i32, i32, i32]
-            L.moe_mxfp4_codes_bytes.restype = sz
-            L.moe_mxfp4_scales_bytes.argtypes = [i32, i32, i32]
-            L.moe_mxfp4_scales_bytes.restype = sz
-            L.moe_mxfp4_quantize.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
-            L.moe_mxfp4_quantize.restype = ctypes.c_int
-            L.moe_workspace_bytes.argtypes = [dp, i32]
-            L.moe_workspace_bytes.restype = sz
-            L.moe_route.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
-            L.moe_route.restype = ctypes.c_int
-            L.moe_forward.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
-            L.moe_forward.restype = ctypes.c_int
-            L.moe_forward_timed.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
-                                            vp, i32]
-            L.moe_forward_timed.restype = ctypes.c_int
-            L.moe_resolve_path.argtypes = [dp, i32]
-            L.moe_resolve_path.restype = i32
-            L.moe_workspace_layout.argtypes = [dp, i32, vp]
-            L.moe_workspace_layout.restype = ctypes.c_int
-            L.moe_device_status.argtypes = [vp, vp]
-            L.moe_device_status.restype = ctypes.c_int
-            L.moe_status_string.argtypes = [ctypes.c_int]
-            L.moe_status_string.restype = ctypes.c_char_p
-            L.moe_forward_partial.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
-            L.moe_forward_partial.restype = ctypes.c_int
-            L.moe_forward_norm.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
-                                           vp, sz, vp]
-            L.moe_forward_norm.restype = ctypes.c_int
-            L.moe_residual_norm.argtypes = [i32, i32, vp, vp, vp, ctypes.c_float, vp, vp, vp]
-            L.moe_residual_norm.restype = ctypes.c_int
-            L.moe_forward_no_alloc.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
-            L.moe_forward_no_alloc.restype = ctypes.c_int
-            L.moe_debug_inject_timeout.argtypes = [i32]
-            L.moe_debug_inject_timeout.restype = None
-            L.moe_last_launch_count.argtypes = []
-            L.moe_last_launch_count.restype = i32
-            _lib = L
+            _lib = load_library(LIB_PATH)
     return _lib
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Run the calls inside the block on another build of the library (for example the
+    bounds-checking build, libmoe_mxfp4_bounds.so), then switch back."""
+    global _lib
+    other = load_library(path)
+    prev = lib()
+    with _lock:
+        _lib = other
+    try:
+        yield other
+    finally:
+        with _lock:
+            _lib = prev
+
+
+def load_library(path: str):
+    """Load a build of the library and declare its functions' argument types."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing")
+    L = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    dp = ctypes.POINTER(moe_dims)
+    L.moe_mxfp4_codes_bytes.argtypes = [i32, i32, i32]
+    L.moe_mxfp4_codes_bytes.restype = sz
+    L.moe_mxfp4_scales_bytes.argtypes = [i32, i32, i32]
+    L.moe_mxfp4_scales_bytes.restype = sz
+    L.moe_mxfp4_quantize.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
+    L.moe_mxfp4_quantize.restype = ctypes.c_int
+    L.moe_workspace_bytes.argtypes = [dp, i32]
+    L.moe_workspace_bytes.restype = sz
+    L.moe_route.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_route.restype = ctypes.c_int
+    L.moe_forward.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_forward.restype = ctypes.c_int
+    L.moe_forward_timed.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                    vp, i32]
+    L.moe_forward_timed.restype = ctypes.c_int
+    L.moe_resolve_path.argtypes = [dp, i32]
+    L.moe_resolve_path.restype = i32
+    L.moe_workspace_layout.argtypes = [dp, i32, vp]
+    L.moe_workspace_layout.restype = ctypes.c_int
+    L.moe_device_status.argtypes = [vp, vp]
+    L.moe_device_status.restype = ctypes.c_int
+    L.moe_status_string.argtypes = [ctypes.c_int]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_forward_partial.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_forward_partial.restype = ctypes.c_int
+    L.moe_forward_norm.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
+                                   vp, sz, vp]
+    L.moe_forward_norm.restype = ctypes.c_int
+    L.moe_residual_norm.argtypes = [i32, i32, vp, vp, vp, ctypes.c_float, vp, vp, vp]
+    L.moe_residual_norm.restype = ctypes.c_int
+    L.moe_forward_no_alloc.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.moe_forward_no_alloc.restype = ctypes.c_int
+    L.moe_debug_inject_timeout.argtypes = [i32]
+    L.moe_debug_inject_timeout.restype = None
+    L.moe_last_launch_count.argtypes = []
+    L.moe_last_launch_count.restype = i32
+    return L
 
 
 def header_functions() -> list[str]:

@@ -354,6 +354,7 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_TIMEOUT: return "device wait timed out";
     case MOE_ERR_NONFINITE: return "non-finite value";
+    case MOE_ERR_BOUNDS: return "store outside its buffer (bounds-checking build)";
     case MOE_ERR_DEVICE: return "device is not sm_100";
   }
   return "unknown status";

@@ -191,6 +191,9 @@ struct Ws {
   uint8_t* bpx;
   uint8_t* bph;
   float* ys;
+  uint8_t* bpx_end;    // ends of the buffers written at computed offsets (bounds checks)
+  uint8_t* bph_end;
+  float* ys_end;
   int64_t max_tiles;
   int32_t tile_tokens;
   int32_t terms;
@@ -218,6 +221,9 @@ inline Ws ws_pointers(void* base, const WsLayout& L, int E) {
   w.bpx = reinterpret_cast<uint8_t*>(b + L.bpx);
   w.bph = reinterpret_cast<uint8_t*>(b + L.bph);
   w.ys = reinterpret_cast<float*>(b + L.ys);
+  w.bpx_end = w.bph;
+  w.bph_end = reinterpret_cast<uint8_t*>(b + L.ys);
+  w.ys_end = reinterpret_cast<float*>(b + L.total);
   w.ticket = w.counts + E;
   w.arrivals = w.counts + E + 4;
   w.max_tiles = L.max_tiles;
@@ -413,6 +419,23 @@ inline void ev_after(const FwdArgs& a) {
 // Record the first device-side error in the status word.
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
+}
+
+// Stores at computed offsets (packed blocks, expert outputs, outputs, quantized weights) go
+// through in_bounds(p, lo, hi, status): with MOE_DEBUG_BOUNDS defined (the bounds-checking
+// build) a store outside [lo, hi) is skipped and MOE_ERR_BOUNDS recorded; otherwise the
+// check compiles away.
+template <class T, class U>
+__device__ __forceinline__ bool in_bounds(const T* p, const U* lo, const U* hi, int32_t* status) {
+#ifdef MOE_DEBUG_BOUNDS
+  const char* c = reinterpret_cast<const char*>(p);
+  if (c >= reinterpret_cast<const char*>(lo) && c + sizeof(T) <= reinterpret_cast<const char*>(hi)) return true;
+  set_status(status, MOE_ERR_BOUNDS);
+  return false;
+#else
+  (void)p; (void)lo; (void)hi; (void)status;
+  return true;
+#endif
 }
 
 // --------------------------------------------------------------------------- launchers

@@ -83,6 +83,11 @@ struct MxParams {
   uint16_t* y;
   float* y_partial;        // instead of y: the fp32 sum without the residual (a slice of I)
   int32_t* arrivals;
+  // buffer ends for the stores at computed offsets (bounds-checking builds)
+  const uint8_t* bp_out_end;
+  const float* ys_end;
+  const uint16_t* y_end;
+  const float* y_partial_end;
 };
 
 #ifndef MOE_SF_SLOTS
@@ -420,8 +425,10 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
               const uint32_t code_hi = __shfl_down_sync(0xffffffffu, code, 1);
               if (j < tl.rows) {
                 uint8_t* blk = p.bp_out + ((int64_t)tt * p.KCo + kb / 4) * C::B_BLOCK;
-                if ((lane & 1) == 0) blk[packed_unit_offset64(j, kb & 3) + lane / 2] = (uint8_t)(code | (code_hi << 4));
-                if (lane == 0) blk[packed_sf_offset(C::N2, j, kb, C::RB)] = (uint8_t)sf4;
+                uint8_t* q = blk + packed_unit_offset64(j, kb & 3) + lane / 2;
+                if ((lane & 1) == 0 && in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)(code | (code_hi << 4));
+                q = blk + packed_sf_offset(C::N2, j, kb, C::RB);
+                if (lane == 0 && in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)sf4;
               }
               continue;
             }
@@ -433,11 +440,15 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
               uint8_t* blk = p.bp_out + ((int64_t)tt * p.KCo + kb / 4) * C::B_BLOCK;
               const int u = 2 * (kb & 3) + (lane >> 4);
               // (with MXFP8 activations only the hi term: h rounded to E4M3 in its block)
-              blk[packed_unit_offset(TERMS * j, u) + (lane & 15)] = (uint8_t)hi;
-              if (TERMS == 2) blk[packed_unit_offset(2 * j + 1, u) + (lane & 15)] = (uint8_t)lo;
+              uint8_t* q = blk + packed_unit_offset(TERMS * j, u) + (lane & 15);
+              if (in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)hi;
+              q = blk + packed_unit_offset(2 * j + 1, u) + (lane & 15);
+              if (TERMS == 2 && in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)lo;
               if (lane == 0) {
-                blk[packed_sf_offset(C::N2, TERMS * j, kb)] = (uint8_t)s1;
-                if (TERMS == 2) blk[packed_sf_offset(C::N2, 2 * j + 1, kb)] = (uint8_t)s2;
+                q = blk + packed_sf_offset(C::N2, TERMS * j, kb);
+                if (in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)s1;
+                q = blk + packed_sf_offset(C::N2, 2 * j + 1, kb);
+                if (TERMS == 2 && in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)s2;
               }
             }
           }
@@ -467,7 +478,8 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
             if (c < nt && m < p.d) {
               const int64_t prow = tl.row0 + jbase + c;
               const float o = token_acc<TERMS>(v, c);
-              ys[prow * p.d + m] = o * p.w_sorted[prow];
+              float* q = ys + prow * p.d + m;
+              if (in_bounds(q, p.ys, p.ys_end, p.status)) *q = o * p.w_sorted[prow];
             }
           }
           if (p.fuse_combine) {
@@ -493,8 +505,13 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
                   for (int sp = 0; sp < ksplit; ++sp)
                     accv += __ldcg(p.ys + ((int64_t)sp * p.P + srow) * p.d + gc);
                 }
-                if (p.y_partial) p.y_partial[(int64_t)tok * p.d + gc] = accv;
-                else p.y[(int64_t)tok * p.d + gc] = bf16_bits_rne(accv);
+                if (p.y_partial) {
+                  float* q = p.y_partial + (int64_t)tok * p.d + gc;
+                  if (in_bounds(q, p.y_partial, p.y_partial_end, p.status)) *q = accv;
+                } else {
+                  uint16_t* q = p.y + (int64_t)tok * p.d + gc;
+                  if (in_bounds(q, p.y, p.y_end, p.status)) *q = bf16_bits_rne(accv);
+                }
               }
             }
             group_sync();
@@ -612,6 +629,10 @@ int launch_one(const FwdArgs& a) {
   prm.x = a.x;
   prm.y = a.y;
   prm.y_partial = a.y_partial;
+  prm.bp_out_end = a.ws.bph_end;
+  prm.ys_end = a.ws.ys_end;
+  prm.y_end = a.y ? a.y + (int64_t)a.T * a.d : nullptr;
+  prm.y_partial_end = a.y_partial ? a.y_partial + (int64_t)a.T * a.d : nullptr;
   prm.arrivals = a.ws.arrivals;
 
   auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, NPW, TERMS, FP4, MODE>;

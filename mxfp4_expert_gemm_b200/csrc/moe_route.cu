@@ -30,7 +30,8 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_floa
 // each threshold taking ties toward the even code.
 // ----------------------------------------------------------------------------------
 __global__ void quantize_kernel(const float* __restrict__ w, int64_t nblocks, int32_t N, int32_t K, int32_t role,
-                                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int32_t* status) {
+                                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int32_t* status,
+                                const uint8_t* codes_end, const uint8_t* scales_end) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -63,9 +64,11 @@ __global__ void quantize_kernel(const float* __restrict__ w, int64_t nblocks, in
     const int64_t e_idx = row / N;
     const int64_t n = row - e_idx * N;
     const int64_t srow = role == MOE_WEIGHT_GATE_UP ? gate_up_stored_row(n, N / 2) : n;
-    if ((lane & 1) == 0) codes[mx_code_offset(e_idx, srow, 32 * kb + lane, N, K)] = (uint8_t)(c | (hi << 4));
+    uint8_t* qc = codes + mx_code_offset(e_idx, srow, 32 * kb + lane, N, K);
+    if ((lane & 1) == 0 && in_bounds(qc, codes, codes_end, status)) *qc = (uint8_t)(c | (hi << 4));
     if (lane == 0) {
-      scales[mx_scale_offset(e_idx, srow, kb, N, K)] = all_finite ? (uint8_t)(s + 127) : (uint8_t)0xFF;
+      uint8_t* qs = scales + mx_scale_offset(e_idx, srow, kb, N, K);
+      if (in_bounds(qs, scales, scales_end, status)) *qs = all_finite ? (uint8_t)(s + 127) : (uint8_t)0xFF;
       if (!all_finite) set_status(status, MOE_ERR_NONFINITE);
     }
   }
@@ -147,10 +150,13 @@ __device__ __forceinline__ void pack_pair_chunk(const FwdArgs& a, int t, int til
     uint8_t* block = a.ws.bpx + ((int64_t)tile * kc + c) * packed_block_bytes(rows, kKChunk / 2);
     if (lane < 4) {
       const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.ws.xq + (int64_t)t * 2 * dp + c * (kKChunk / 2)) + lane);
-      *reinterpret_cast<uint4*>(block + packed_unit_offset64(col, lane)) = v;
+      uint4* q = reinterpret_cast<uint4*>(block + packed_unit_offset64(col, lane));
+      if (in_bounds(q, a.ws.bpx, a.ws.bpx_end, a.ws.status)) *q = v;
     } else if (lane >= 16 && lane < 20) {
       const int b = 4 * c + (lane - 16);
-      if (b < nb) block[packed_sf_offset(rows, col, b, kKChunk / 2)] = __ldcg(a.ws.xsf + (int64_t)t * 2 * (dp / 32) + b);
+      uint8_t* q = block + packed_sf_offset(rows, col, b, kKChunk / 2);
+      if (b < nb && in_bounds(q, a.ws.bpx, a.ws.bpx_end, a.ws.status))
+        *q = __ldcg(a.ws.xsf + (int64_t)t * 2 * (dp / 32) + b);
     }
     return;
   }
@@ -160,13 +166,14 @@ __device__ __forceinline__ void pack_pair_chunk(const FwdArgs& a, int t, int til
     if (term < terms) {
       const uint4 v =
           __ldcg(reinterpret_cast<const uint4*>(a.ws.xq + (int64_t)t * 2 * dp + term * dp + c * kKChunk) + u);
-      *reinterpret_cast<uint4*>(block + packed_unit_offset(terms * col + term, u)) = v;
+      uint4* q = reinterpret_cast<uint4*>(block + packed_unit_offset(terms * col + term, u));
+      if (in_bounds(q, a.ws.bpx, a.ws.bpx_end, a.ws.status)) *q = v;
     }
   } else if (lane < 24) {
     const int term = (lane - 16) >> 2, b = 4 * c + ((lane - 16) & 3);
-    if (term < terms && b < nb)
-      block[packed_sf_offset(rows, terms * col + term, b)] =
-          __ldcg(a.ws.xsf + (int64_t)t * 2 * (dp / 32) + term * (dp / 32) + b);
+    uint8_t* q = block + packed_sf_offset(rows, terms * col + term, b);
+    if (term < terms && b < nb && in_bounds(q, a.ws.bpx, a.ws.bpx_end, a.ws.status))
+      *q = __ldcg(a.ws.xsf + (int64_t)t * 2 * (dp / 32) + term * (dp / 32) + b);
   }
 }
 
@@ -673,11 +680,14 @@ __device__ __forceinline__ void pack_pair(const FwdArgs& a, int t, int tile, int
     for (int i = lane; i < kc * 4; i += 32) {
       const int c = i >> 2, u = i & 3;
       const uint4 v = __ldcg(reinterpret_cast<const uint4*>(row + c * (kKChunk / 2)) + u);
-      *reinterpret_cast<uint4*>(blocks + (int64_t)c * bb + packed_unit_offset64(col, u)) = v;
+      uint4* q = reinterpret_cast<uint4*>(blocks + (int64_t)c * bb + packed_unit_offset64(col, u));
+      if (in_bounds(q, a.ws.bpx, a.ws.bpx_end, a.ws.status)) *q = v;
     }
     const uint8_t* sf = a.ws.xsf + (int64_t)t * 2 * (dp / 32);
-    for (int b = lane; b < nb; b += 32)
-      blocks[(int64_t)(b / 4) * bb + packed_sf_offset(rows_t, col, b, kKChunk / 2)] = __ldcg(sf + b);
+    for (int b = lane; b < nb; b += 32) {
+      uint8_t* q = blocks + (int64_t)(b / 4) * bb + packed_sf_offset(rows_t, col, b, kKChunk / 2);
+      if (in_bounds(q, a.ws.bpx, a.ws.bpx_end, a.ws.status)) *q = __ldcg(sf + b);
+    }
     return;
   }
   const int bb = packed_block_bytes(rows_t);
@@ -699,14 +709,16 @@ __device__ __forceinline__ void pack_pair(const FwdArgs& a, int t, int tile, int
       const int i = i0 + 32 * r;
       if (i < units) {
         const int c = i / (8 * terms), term = (i >> 3) % terms, u = i & 7;
-        *reinterpret_cast<uint4*>(blocks + (int64_t)c * bb + packed_unit_offset(terms * col + term, u)) = v[r];
+        uint4* q = reinterpret_cast<uint4*>(blocks + (int64_t)c * bb + packed_unit_offset(terms * col + term, u));
+        if (in_bounds(q, a.ws.bpx, a.ws.bpx_end, a.ws.status)) *q = v[r];
       }
     }
   }
   const uint8_t* sf = a.ws.xsf + (int64_t)t * 2 * (dp / 32);
   for (int i = lane; i < terms * nb; i += 32) {
     const int term = i / nb, b = i - term * nb;
-    blocks[(int64_t)(b / 4) * bb + packed_sf_offset(rows_t, terms * col + term, b)] = __ldcg(sf + term * (dp / 32) + b);
+    uint8_t* q = blocks + (int64_t)(b / 4) * bb + packed_sf_offset(rows_t, terms * col + term, b);
+    if (in_bounds(q, a.ws.bpx, a.ws.bpx_end, a.ws.status)) *q = __ldcg(sf + term * (dp / 32) + b);
   }
 }
 
@@ -920,7 +932,8 @@ int launch_quantize(const float* w, int32_t E, int32_t N, int32_t K, int32_t rol
   const int64_t nblocks = (int64_t)E * N * (K / 32);
   const int64_t want = (nblocks + 7) / 8;
   const int grid = (int)std::min<int64_t>(want, 148 * 64);
-  quantize_kernel<<<grid, 256, 0, st>>>(w, nblocks, N, K, role, codes, scales, status);
+  quantize_kernel<<<grid, 256, 0, st>>>(w, nblocks, N, K, role, codes, scales, status,
+                                        codes + blocks * kCodeBlockBytes, scales + blocks * kSfGroupBytes);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 

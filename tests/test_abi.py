@@ -38,7 +38,7 @@ def test_storage_sizes(L):
 
 
 def test_status_strings(L):
-    for s in (0, 1, 2, 3, 4, 5, 6, 8):
+    for s in (0, 1, 2, 3, 4, 5, 6, 7, 8):
         assert moe.status_string(s) and moe.status_string(s) != "unknown status"
     assert moe.status_string(99) == "unknown status"
 
