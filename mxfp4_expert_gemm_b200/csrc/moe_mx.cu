@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
           continue;
         }
         const int c0 = it.kc0 + st * NP, nck = min(NP, it.kc1 - c0);
-        if (lane == 0) {
+        if (ptx::elect_one()) {
           uint64_t* bar = &full[s * C::NISS + warp];
           const bool do_w = (0 % NPW) == warp, do_b = (1 % NPW) == warp, do_f = (2 % NPW) == warp;
           ptx::mbar_arrive_expect_tx(bar, (do_w ? C::A_TX : 0) + (do_b ? nck * C::B_BLOCK : 0) +
@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
           }
           ptx::tc_fence_after();
           const int c0 = it.kc0 + st * NP, nck = min(NP, it.kc1 - c0);
-          if (lane == 0) {
+          if (ptx::elect_one()) {
             // scale factors of this stage into their TMEM slot (the tensor pipe runs one
             // thread's copies and MMAs in issue order; with two slots a copy does not
             // overwrite columns the previous stage's MMAs still read)
@@ -340,11 +340,11 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
           }
           __syncwarp();
         }
-        if (!stop && lane == 0) ptx::tc_commit(&accf[b]);
+        if (!stop && ptx::elect_one()) ptx::tc_commit(&accf[b]);
         __syncwarp();
       }
       // Every MMA issued above completes before the drain barrier fires.
-      if (lane == 0) ptx::tc_commit(drain);
+      if (ptx::elect_one()) ptx::tc_commit(drain);
       __syncwarp();
       volatile int local_abort = 0;
       ptx::mbar_wait_bounded(drain, 0, &local_abort, kWaitLimitNs);
@@ -500,10 +500,28 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
               for (int col = et; col < ncol; col += 128) {
                 const int64_t gc = kBM * rt + col;
                 float accv = p.y_partial ? 0.f : __uint_as_float((uint32_t)p.x[(int64_t)tok * p.d + gc] << 16);
-                for (int j = 0; j < p.k; ++j) {
-                  const int srow = p.inv[(int64_t)tok * p.k + j];
-                  for (int sp = 0; sp < ksplit; ++sp)
-                    accv += __ldcg(p.ys + ((int64_t)sp * p.P + srow) * p.d + gc);
+                constexpr int kMaxParts = 24;   // k x splits loaded together (else one after another)
+                if (p.k * ksplit <= kMaxParts) {
+                  // every partial row's position first, then all their loads in flight at once;
+                  // the sum keeps the order slot, then split
+                  int srow[kMaxParts];
+                  float part[kMaxParts];
+#pragma unroll
+                  for (int q = 0; q < kMaxParts; ++q)   // part q: slot q / ksplit, split q % ksplit
+                    if (q < p.k * ksplit) srow[q] = p.inv[(int64_t)tok * p.k + q / ksplit];
+#pragma unroll
+                  for (int q = 0; q < kMaxParts; ++q)
+                    if (q < p.k * ksplit)
+                      part[q] = __ldcg(p.ys + ((int64_t)(q % ksplit) * p.P + srow[q]) * p.d + gc);
+#pragma unroll
+                  for (int q = 0; q < kMaxParts; ++q)
+                    if (q < p.k * ksplit) accv += part[q];
+                } else {
+                  for (int j = 0; j < p.k; ++j) {
+                    const int srow1 = p.inv[(int64_t)tok * p.k + j];
+                    for (int sp = 0; sp < ksplit; ++sp)
+                      accv += __ldcg(p.ys + ((int64_t)sp * p.P + srow1) * p.d + gc);
+                  }
                 }
                 if (p.y_partial) {
                   float* q = p.y_partial + (int64_t)tok * p.d + gc;

@@ -20,6 +20,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// One lane of the converged warp, chosen by the hardware (elect.sync).  Issuing tcgen05
+// and TMA instructions from such a branch lets the compiler keep their operands in the
+// warp's uniform registers; an `if (lane == 0)` branch made each tcgen05 issue several
+// times slower (the MMA issuer then could not keep the tensor pipe busy).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}" : "=r"(pred));
+  return pred != 0;
+}
+
 // ----------------------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
