@@ -142,11 +142,12 @@ __device__ __forceinline__ void warp_topk_softmax(float (&l)[NJ], int E, int k, 
 // Chunk c of token t's E4M3 rows (hi, lo) and their scales into the packed block of
 // token tile `tile`, MMA columns 2*col (hi) and 2*col + 1 (lo).  One warp: lanes 0-15
 // move the 16 16-byte units, lanes 16-23 the eight scale bytes.
+template <bool FP4>
 __device__ __forceinline__ void pack_pair_chunk(const FwdArgs& a, int t, int tile, int col, int c) {
   const int lane = threadIdx.x & 31;
   const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk, terms = a.ws.terms;
   const int rows = terms * bt;
-  if (a.ws.fp4) {   // MXFP4: one 64-byte row of packed codes; lanes 0-3 move it, 16-19 the scales
+  if (FP4) {   // MXFP4: one 64-byte row of packed codes; lanes 0-3 move it, 16-19 the scales
     uint8_t* block = a.ws.bpx + ((int64_t)tile * kc + c) * packed_block_bytes(rows, kKChunk / 2);
     if (lane < 4) {
       const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.ws.xq + (int64_t)t * 2 * dp + c * (kKChunk / 2)) + lane);
@@ -421,7 +422,7 @@ struct RouteTilesCfg {
   static_assert(KW % 4 == 0, "float4 columns per warp");
 };
 
-template <int NJ, int RK, int NS>
+template <int NJ, int RK, int NS, bool FP4>
 __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
   using C = RouteTilesCfg<NJ, RK, NS>;
   extern __shared__ __align__(16) float smem[];
@@ -506,7 +507,7 @@ __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
           s_xn[tt * RK + kk] = v0;
           s_xn[tt * RK + kk + 1] = v1;
           const float v[2] = {bf16_to_f32(bf16_bits_rne(v0)), bf16_to_f32(bf16_bits_rne(v1))};
-          if (a.ws.fp4) {   // MXFP4 activations: this lane's two codes are one byte
+          if (FP4) {   // MXFP4 activations: this lane's two codes are one byte
             uint32_t c, s1;
             e2m1_quant<2>(v, c, s1);
             xq[(k0 + kk) / 2] = (uint8_t)c;
@@ -525,7 +526,7 @@ __global__ void __launch_bounds__(256) route_tiles_kernel(FwdArgs a) {
           const float v0 = bf16_to_f32(s_x[(st * kRT + tt) * RK + lane]) * r * s_g[k0 + lane];
           s_xn[tt * RK + lane] = v0;
           const float v[1] = {bf16_to_f32(bf16_bits_rne(v0))};
-          if (a.ws.fp4) {
+          if (FP4) {
             uint32_t c, s1;
             e2m1_quant<1>(v, c, s1);
             const uint32_t c_hi = __shfl_down_sync(0xffffffffu, c, 1);
@@ -669,11 +670,12 @@ __global__ void __launch_bounds__(1024) group_kernel(FwdArgs a, int tile_tokens)
 
 // All chunks of token t's rows and scales into token tile `tile`'s packed blocks.  One
 // warp; each lane keeps four 16-byte copies in flight.
+template <bool FP4>
 __device__ __forceinline__ void pack_pair(const FwdArgs& a, int t, int tile, int col) {
   const int lane = threadIdx.x & 31;
   const int dp = a.ws.dp, nb = a.d / 32, bt = a.ws.tile_tokens, kc = dp / kKChunk, terms = a.ws.terms;
   const int rows_t = terms * bt;
-  if (a.ws.fp4) {   // MXFP4: per chunk one 64-byte row of packed codes (4 units) and 4 scales
+  if (FP4) {   // MXFP4: per chunk one 64-byte row of packed codes (4 units) and 4 scales
     const int bb = packed_block_bytes(rows_t, kKChunk / 2);
     uint8_t* blocks = a.ws.bpx + (int64_t)tile * kc * bb;
     const uint8_t* row = a.ws.xq + (int64_t)t * 2 * dp;
@@ -725,7 +727,9 @@ __device__ __forceinline__ void pack_pair(const FwdArgs& a, int t, int tile, int
 constexpr int64_t kPackChunkTasksMax = 1 << 16;   // up to this many (pair, chunk) tasks: one warp each
 
 // Every pair's activation rows and scales into its token tile's packed blocks: one warp
-// per (pair, 128-chunk) for small batches, one warp per pair otherwise.
+// per (pair, 128-chunk) for small batches, one warp per pair otherwise.  FP4: MXFP4
+// activations (64-byte rows of packed codes), a separate instantiation.
+template <bool FP4>
 __global__ void pack_kernel(FwdArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -735,7 +739,7 @@ __global__ void pack_kernel(FwdArgs a) {
       const int q = a.ws.perm[p];
       const int e = a.ws.topk_idx[q];
       const int j = p - a.ws.offsets[e];
-      pack_pair(a, q / a.k, a.ws.tile_base[e] + j / bt, j % bt);
+      pack_pair<FP4>(a, q / a.k, a.ws.tile_base[e] + j / bt, j % bt);
     }
     return;
   }
@@ -746,7 +750,7 @@ __global__ void pack_kernel(FwdArgs a) {
     const int q = a.ws.perm[p];
     const int e = a.ws.topk_idx[q];
     const int j = p - a.ws.offsets[e];
-    pack_pair_chunk(a, q / a.k, a.ws.tile_base[e] + j / bt, j % bt, c);
+    pack_pair_chunk<FP4>(a, q / a.k, a.ws.tile_base[e] + j / bt, j % bt, c);
   }
 }
 
@@ -895,7 +899,7 @@ bool ensure_smem_limit(K kern, size_t bytes, std::atomic<int>* limits /*[64]*/) 
 
 template <int NJ>
 int launch_route_nj(const FwdArgs& a) {
-  static std::atomic<int> tok_limits[64], tile_limits[64];
+  static std::atomic<int> tok_limits[64], tile_limits[64], tile_limits_fp4[64];
   if (a.T <= kTokenKernelMaxT) {
     const size_t smem = sizeof(float) * (a.d + 32 * NJ);
     if (!ensure_smem_limit(route_token_kernel<NJ>, smem, tok_limits)) return -1;
@@ -911,9 +915,10 @@ int launch_route_nj(const FwdArgs& a) {
   constexpr int NSC = NJ == 4 ? 2 : 4;
   using C = RouteTilesCfg<NJ, RKC, NSC>;
   const size_t smem = C::smem(a.d);
-  if (!ensure_smem_limit(route_tiles_kernel<NJ, RKC, NSC>, smem, tile_limits)) return -1;
+  auto kern = a.ws.fp4 ? route_tiles_kernel<NJ, RKC, NSC, true> : route_tiles_kernel<NJ, RKC, NSC, false>;
+  if (!ensure_smem_limit(kern, smem, a.ws.fp4 ? tile_limits_fp4 : tile_limits)) return -1;
   ev_before(a);
-  route_tiles_kernel<NJ, RKC, NSC><<<(a.T + kRT - 1) / kRT, 256, smem, a.stream>>>(a);
+  kern<<<(a.T + kRT - 1) / kRT, 256, smem, a.stream>>>(a);
   ev_after(a);
   return 1;
 }
@@ -962,8 +967,9 @@ int launch_route(const FwdArgs& a_in) {
   const int64_t P = (int64_t)a.T * a.k, tasks = P * (a.ws.dp / kKChunk);
   const int64_t warps = tasks > kPackChunkTasksMax ? P : tasks;   // one warp per task (pack_kernel)
   ev_before(a);
-  if (launch_kernel(pack_kernel, dim3((unsigned)std::min<int64_t>((warps + 7) / 8, 148 * 32)), dim3(256), 0, a.stream,
-                    a.pdl != 0, a) != cudaSuccess)
+  if (launch_kernel(a.ws.fp4 ? pack_kernel<true> : pack_kernel<false>,
+                    dim3((unsigned)std::min<int64_t>((warps + 7) / 8, 148 * 32)), dim3(256), 0, a.stream, a.pdl != 0,
+                    a) != cudaSuccess)
     return -1;
   ev_after(a);
   ++n;

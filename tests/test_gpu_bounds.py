@@ -106,4 +106,4 @@ def test_bounds_checking_build_runs_clean(bounds_lib, name, path, act):
         assert int(status.item()) == moe.MOE_OK
     for got, want in zip(w, c["W"]["gpu"]):
         assert torch.equal(got, want)   # the checked build quantizes bit for bit like the normal one
-    assert_parity(parity_stats(bf16_host(y), ref["y"], c["x"]), f"{name}/{path}/{act} (bounds build)")
+    assert_parity(parity_stats(bf16_host(y), ref["y"], c["x"]), f"{name}/{path}/{act} (bounds build)", act)

@@ -137,4 +137,4 @@ def test_full_size_low_precision_tile_cover(name, path, act):
     toks = tile_cover_tokens(c["route"]["idx"], cfg.E, tile_tokens(path, act))
     ref = oracle_rows(c, tokens=toks, act=act)
     st = parity_stats(bf16_host(g["y"])[toks], ref["y"], c["x"][toks])
-    assert_parity(st, f"{name}/{path}/{act}")
+    assert_parity(st, f"{name}/{path}/{act}", act)

@@ -322,7 +322,7 @@ def test_forward_parity_mxfp4(name, path):
     assert g["status"] == moe.MOE_OK, moe.status_string(g["status"])
     ref = oracle_rows(c, act="mxfp4")
     st = parity_stats(bf16_host(g["y"]), ref["y"], c["x"])
-    assert_parity(st, f"{name}/{path}/mxfp4")
+    assert_parity(st, f"{name}/{path}/mxfp4", "mxfp4")
     assert st["delta_rel_fro"] <= 2.5e-2, st
     np.testing.assert_array_equal(np.sort(g["routing"]["topk_idx"].cpu().numpy(), 1), np.sort(ref["idx"], 1))
 
