@@ -438,11 +438,71 @@ __device__ __forceinline__ bool in_bounds(const T* p, const U* lo, const U* hi, 
 #endif
 }
 
+// ----------------------------------------------------------------------------------
+// Top-k (value desc, index asc) + softmax over the selected logits for one token, by one
+// warp; the lane holding logit e is lane e % 32.  Writes the outputs and the histogram.
+// ----------------------------------------------------------------------------------
+template <int NJ>
+__device__ __forceinline__ void warp_topk_softmax(float (&l)[NJ], int E, int k, int64_t t, const FwdArgs& a) {
+  const int lane = threadIdx.x & 31;
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    if (lane + 32 * j < E && !isfinite(l[j])) {
+      bad = true;
+      l[j] = -INFINITY;
+    }
+    if (lane + 32 * j >= E) l[j] = -INFINITY;
+  }
+  if (__any_sync(0xffffffffu, bad)) set_status(a.ws.status, MOE_ERR_NONFINITE);
+  float lsel = 0.f, lmax = 0.f, z = 0.f;
+  int esel = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int jj = 0; jj < NJ; ++jj) {
+      const int e = lane + 32 * jj;
+      if (e < E && (l[jj] > bv || (l[jj] == bv && e < be))) {
+        bv = l[jj];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if (be >= E) be = j;  // only when every logit was non-finite; the status already says so
+    if (j == 0) lmax = bv;
+#pragma unroll
+    for (int jj = 0; jj < NJ; ++jj)
+      if (lane + 32 * jj == be) l[jj] = -INFINITY;
+    const float ex = expf(bv - lmax);
+    z += ex;
+    if (lane == j) {
+      lsel = ex;
+      esel = be;
+    }
+  }
+  if (lane < k) {
+    a.ws.topk_idx[t * k + lane] = esel;
+    a.ws.topk_w[t * k + lane] = lsel / z;
+    atomicAdd(&a.ws.counts[esel], 1);
+  }
+}
+
 // --------------------------------------------------------------------------- launchers
 // Each returns the number of kernels it launched (>= 0) or -1 on a launch error.
 int launch_quantize(const float* w, int32_t E, int32_t N, int32_t K, int32_t role, uint8_t* codes,
                     uint8_t* scales, int32_t* status, cudaStream_t st);
 int launch_route(const FwdArgs& a);     // norm + router + top-k + E4M3 split, grouping, packing
+int launch_route_mma(const FwdArgs& a); // the same first step for large batches, logits on the tensor cores
+bool route_mma_fits(int E, int d);      // its shared memory fits
 int launch_combine(const FwdArgs& a);   // y = x + sum_j ys[inv] (or the partial sum, or y and y_norm)
 // y = bf16(x + s) for a dense fp32 s [T][d], and optionally y_norm (one pass per row)
 int launch_residual_norm(int32_t T, int32_t d, const uint16_t* x, const float* s, const float* norm_w, float eps,

@@ -236,6 +236,38 @@ __device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// Instruction descriptor of kind::tf32: TF32 A and B (32-bit containers, K-major), fp32 D.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+  return (1u << 4)                       // D format: f32
+         | (2u << 7) | (2u << 10)        // A, B format: TF32
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T over one 8-wide K block, kind::tf32, one CTA.
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Order this thread's generic-proxy shared-memory writes before later async-proxy reads
+// (the tensor cores reading operands the threads wrote).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// fp32 -> TF32 (10 mantissa bits, round to nearest, ties away), in a 32-bit container.
+__device__ __forceinline__ float to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
 // SMEM descriptor of an unswizzled K-major source of 16-byte rows: 8-row core matrices
 // stored back to back (128 bytes apart).
 __device__ __forceinline__ uint64_t smem_desc_k_rows16(const void* p) {
