@@ -59,7 +59,7 @@ CSRC = os.path.join(ROOT, "mxfp4_expert_gemm_b200", "csrc")
 KERNEL_SOURCES = {
     "gate_up": ["moe_mx.cu", "moe_internal.cuh", "sm100_ptx.cuh"],
     "down": ["moe_mx.cu", "moe_internal.cuh", "sm100_ptx.cuh"],
-    "route": ["moe_route.cu", "moe_internal.cuh"],
+    "route": ["moe_route.cu", "moe_route_mma.cu", "moe_internal.cuh", "sm100_ptx.cuh"],
     "group": ["moe_route.cu", "moe_internal.cuh"],
     "pack": ["moe_route.cu", "moe_internal.cuh"],
     "combine": ["moe_route.cu", "moe_internal.cuh"],

@@ -111,7 +111,7 @@ struct MxCfg {
   static constexpr int A_TX = NP * kBM * kKChunk / 2;   // the weight box counts packed bytes
   static constexpr int CW = N2 < 32 ? N2 : 32;          // accumulator columns per epilogue read
   static constexpr int TC = CW / TERMS;                 // tokens per epilogue read
-  static constexpr int HT = TC / 2;                     // tokens each side (gate / up) finishes
+  static constexpr int SB = 8;                          // tokens per g / u exchange round (gate_up)
   static constexpr int ACC_COLS = N2 < 32 ? 32 : N2;    // one accumulator buffer
   static constexpr int SF_SLOT_COLS = 4 * NP * (1 + G);         // A then B scale factors of a stage
   static constexpr int SFA_COL = 2 * ACC_COLS;                   // + slot * SF_SLOT_COLS
@@ -119,7 +119,7 @@ struct MxCfg {
   static constexpr int COLS_NEEDED = 2 * ACC_COLS + kSfSlots * SF_SLOT_COLS;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 : COLS_NEEDED <= 128 ? 128
                                    : COLS_NEEDED <= 256 ? 256 : 512;
-  static constexpr int EPI_GROUP_BYTES = TC * 64 * 4 + TC * 4;  // g / u exchange; token list (down)
+  static constexpr int EPI_GROUP_BYTES = 2 * SB * 64 * 4 + TC * 4;  // g and u of SB tokens; token list (down)
   static constexpr int EPI_BYTES = EG * EPI_GROUP_BYTES;
   static constexpr int NISS = NPW;                      // copy issuers per stage, one barrier each
   static constexpr int BAR_BYTES = 8 * ((NISS + 1) * S + 5) + 16;
@@ -133,6 +133,7 @@ struct MxCfg {
   static_assert(SMEM_BYTES * CPS <= 227 * 1024, "shared memory budget of CPS co-resident CTAs");
   static_assert(kBM * NP <= 256, "TMA box height");
   static_assert(EG == 1 || EG == 2, "one or two epilogue warpgroups");
+  static_assert(TC % SB == 0, "an epilogue read holds whole exchange rounds");
   static_assert(NPW >= 1 && NPW <= 3, "producer warps: one per kind of copy at most");
 };
 
@@ -306,34 +307,61 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
             // thread's copies and MMAs in issue order; with two slots a copy does not
             // overwrite columns the previous stage's MMAs still read)
             const uint32_t sf_slot = tmem + (uint32_t)((g % kSfSlots) * C::SF_SLOT_COLS);
-            for (int c = 0; c < nck; ++c) {
-              ptx::tc_cp_32x128b_x4(sf_slot + C::SFA_COL + 4 * c,
-                                    ptx::smem_desc_k_rows16(sfa_s(s) + c * kSfGroupBytes));
+            const uint64_t a0 = FP4 ? ptx::smem_desc_k_sw64(a_s(s)) : ptx::smem_desc_k_sw128(a_s(s));
+            const uint64_t b0 = FP4 ? ptx::smem_desc_k_sw64(b_s(s)) : ptx::smem_desc_k_sw128(b_s(s));
+            const uint64_t f0 = ptx::smem_desc_k_rows16(sfa_s(s)), fb0 = ptx::smem_desc_k_rows16(b_s(s) + C::B_PANEL);
+            // (descriptor start addresses count 16-byte units: offsets within shared memory add)
+            constexpr uint64_t kA = C::A_PANEL >> 4, kB = C::B_BLOCK >> 4, kF = kSfGroupBytes >> 4;
+            if (nck == NP && 4 * (c0 + NP) <= kblocks) {
+              // a full stage: NP chunks of 4 blocks of 32, every index a compile-time constant
 #pragma unroll
-              for (int gg = 0; gg < C::G; ++gg)
-                ptx::tc_cp_32x128b_x4(sf_slot + C::SFB_COL + 4 * (c * C::G + gg),
-                                      ptx::smem_desc_k_rows16(b_s(s) + c * C::B_BLOCK + C::B_PANEL + gg * kSfGroupBytes));
-            }
-            for (int c = 0; c < nck; ++c) {
-              const int nkb = min(4, kblocks - 4 * (c0 + c));   // 32-blocks of this chunk (K % 64 == 0: even)
-              const uint32_t sfa = sf_slot + C::SFA_COL + 4 * c, sfb = sf_slot + C::SFB_COL + 4 * c * C::G;
-              if (FP4) {
-                // FP4 x FP4: one MMA per 64 k (32 bytes of each packed row); it takes the scale
-                // bytes 2kk and 2kk + 1 of each row's scale-factor word
-                const uint64_t adesc = ptx::smem_desc_k_sw64(a_s(s) + c * C::A_PANEL);
-                const uint64_t bdesc = ptx::smem_desc_k_sw64(b_s(s) + c * C::B_BLOCK);
-                for (int kk = 0; kk < nkb / 2; ++kk)
-                  ptx::mma_mxf4_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
-                                   ptx::idesc_mxf4(kBM, C::N2, (uint32_t)(2 * kk), (uint32_t)(2 * kk)), sfa, sfb,
+              for (int c = 0; c < NP; ++c) {
+                ptx::tc_cp_32x128b_x4(sf_slot + C::SFA_COL + 4 * c, f0 + c * kF);
+#pragma unroll
+                for (int gg = 0; gg < C::G; ++gg)
+                  ptx::tc_cp_32x128b_x4(sf_slot + C::SFB_COL + 4 * (c * C::G + gg), fb0 + c * kB + gg * kF);
+              }
+#pragma unroll
+              for (int c = 0; c < NP; ++c) {
+                const uint32_t sfa = sf_slot + C::SFA_COL + 4 * c, sfb = sf_slot + C::SFB_COL + 4 * c * C::G;
+                if (FP4) {
+#pragma unroll
+                  for (int kk = 0; kk < 2; ++kk)
+                    ptx::mma_mxf4_ss(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
+                                     ptx::idesc_mxf4(kBM, C::N2, (uint32_t)(2 * kk), (uint32_t)(2 * kk)), sfa, sfb,
+                                     (st | c | kk) != 0);
+                } else {
+#pragma unroll
+                  for (int kk = 0; kk < 4; ++kk)
+                    ptx::mma_mx_ss(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
+                                   ptx::idesc_mx_e2m1_e4m3(kBM, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
                                    (st | c | kk) != 0);
-              } else {
-                // E2M1 x E4M3: one MMA per 32 k (32 bytes of each row), scale byte kk
-                const uint64_t adesc = ptx::smem_desc_k_sw128(a_s(s) + c * C::A_PANEL);
-                const uint64_t bdesc = ptx::smem_desc_k_sw128(b_s(s) + c * C::B_BLOCK);
-                for (int kk = 0; kk < nkb; ++kk)
-                  ptx::mma_mx_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
-                                 ptx::idesc_mx_e2m1_e4m3(kBM, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
-                                 (st | c | kk) != 0);
+                }
+              }
+            } else {
+              for (int c = 0; c < nck; ++c) {
+                ptx::tc_cp_32x128b_x4(sf_slot + C::SFA_COL + 4 * c, f0 + c * kF);
+#pragma unroll
+                for (int gg = 0; gg < C::G; ++gg)
+                  ptx::tc_cp_32x128b_x4(sf_slot + C::SFB_COL + 4 * (c * C::G + gg), fb0 + c * kB + gg * kF);
+              }
+              for (int c = 0; c < nck; ++c) {
+                const int nkb = min(4, kblocks - 4 * (c0 + c));   // 32-blocks of this chunk (K % 64 == 0: even)
+                const uint32_t sfa = sf_slot + C::SFA_COL + 4 * c, sfb = sf_slot + C::SFB_COL + 4 * c * C::G;
+                if (FP4) {
+                  // FP4 x FP4: one MMA per 64 k (32 bytes of each packed row); it takes the scale
+                  // bytes 2kk and 2kk + 1 of each row's scale-factor word
+                  for (int kk = 0; kk < nkb / 2; ++kk)
+                    ptx::mma_mxf4_ss(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
+                                     ptx::idesc_mxf4(kBM, C::N2, (uint32_t)(2 * kk), (uint32_t)(2 * kk)), sfa, sfb,
+                                     (st | c | kk) != 0);
+                } else {
+                  // E2M1 x E4M3: one MMA per 32 k (32 bytes of each row), scale byte kk
+                  for (int kk = 0; kk < nkb; ++kk)
+                    ptx::mma_mx_ss(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
+                                   ptx::idesc_mx_e2m1_e4m3(kBM, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
+                                   (st | c | kk) != 0);
+                }
               }
             }
             ptx::tc_commit(&sfree[s]);
@@ -376,16 +404,20 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
       const Tile tl = p.tiles[tt];
       const uint32_t acc = tmem + lane_addr + b * C::ACC_COLS;
       if (MODE == MODE_GATE_UP) {
-        // Per read of TC tokens the gate thread of feature f (lane row f < 64) and the up
-        // thread of f (row f + 64) trade: the gate side finishes the first HT tokens, the
-        // up side the rest.  Each warp then holds one 32-feature block of h per token and
-        // splits it into E4M3 hi / lo terms for the down GEMM (the hi term alone, h rounded
-        // to MXFP8, when TERMS = 1).
-        float* s_x = reinterpret_cast<float*>(gepi);  // [TC tokens][64 features]
+        // Per read of TC tokens, in rounds of SB tokens: the gate threads (lane rows 0..63)
+        // put g, the up threads (rows 64..127) put u into shared memory; then each thread
+        // finishes 4 consecutive features of one token: h = bf16(silu(g) * u) and its share
+        // of the down GEMM's activation block (8 threads per 32-feature block: E4M3 hi / lo
+        // terms and their scales, the hi term alone with MXFP8 activations, or E2M1 codes).
+        float* s_g = reinterpret_cast<float*>(gepi);  // [SB tokens][64 features]
+        float* s_u = s_g + C::SB * 64;
         const float L = p.limit;
-        const bool gate_side = q < 2;
+        float* s_mine = (q < 2) ? s_g : s_u;
         const int f = 32 * (q & 1) + lane;           // feature within the item's 64
-        const int kb = 2 * rt + (q & 1);             // its 32-block along the down GEMM's K
+        const int jj = et >> 4;                      // token of the round this thread finishes
+        const int bq = (et >> 3) & 1;                // its 32-feature block (of the item's two)
+        const int u = et & 7;                        // features 32 bq + 4 u .. + 3
+        const int kb = 2 * rt + bq;                  // the block along the down GEMM's K
         if (eg * C::CW >= C::N2) {  // nothing for this group to read
           ptx::tc_fence_before();
           ptx::mbar_arrive(&acce[b]);
@@ -398,64 +430,59 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
             ptx::tc_fence_before();
             ptx::mbar_arrive(&acce[b]);
           }
-          // (register indices stay compile-time constants: select values, not indices)
 #pragma unroll
-          for (int c = 0; c < C::HT; ++c) {
-            const int jj = gate_side ? C::HT + c : c;  // token the other side finishes
-            const float val = gate_side ? token_acc<TERMS>(v, C::HT + c) : token_acc<TERMS>(v, c);
-            s_x[jj * 64 + f] = val;
-          }
-          group_sync();
+          for (int sb = 0; sb < C::TC; sb += C::SB) {
+            // (register indices stay compile-time constants)
 #pragma unroll
-          for (int c = 0; c < C::HT; ++c) {
-            const int jj = gate_side ? c : C::HT + c;  // token this side finishes
-            const float mine = gate_side ? token_acc<TERMS>(v, c) : token_acc<TERMS>(v, C::HT + c);
-            const float other = s_x[jj * 64 + f];
-            const float gv = fminf(gate_side ? mine : other, L);
-            const float uv = fminf(fmaxf(gate_side ? other : mine, -L), L);
-            float hv = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;   // silu(g) * u
-            hv = __uint_as_float((uint32_t)bf16_bits_rne(hv) << 16);   // h is stored as bf16
-            const float vv[1] = {hv};
-            const int j = c0 / TERMS + jj;             // token within the tile
+            for (int c = 0; c < C::SB; ++c) s_mine[c * 64 + f] = token_acc<TERMS>(v, sb + c);
+            group_sync();
+            const float4 g4 = *reinterpret_cast<const float4*>(s_g + jj * 64 + 32 * bq + 4 * u);
+            const float4 u4 = *reinterpret_cast<const float4*>(s_u + jj * 64 + 32 * bq + 4 * u);
+            const float gs[4] = {g4.x, g4.y, g4.z, g4.w}, us[4] = {u4.x, u4.y, u4.z, u4.w};
+            float hv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float gv = fminf(gs[i], L);
+              const float uv = fminf(fmaxf(us[i], -L), L);
+              const float h = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;   // silu(g) * u
+              hv[i] = __uint_as_float((uint32_t)bf16_bits_rne(h) << 16);   // h is stored as bf16
+            }
+            const int j = c0 / TERMS + sb + jj;   // token within the tile
+            uint8_t* blk = p.bp_out + ((int64_t)tt * p.KCo + kb / 4) * C::B_BLOCK;
             if (FP4) {
-              // MXFP4 activations: h's 32-block as E2M1 codes (two per byte) and its scale,
-              // into the down GEMM's packed block: chunk kb / 4, 16-byte unit kb % 4 of row j
-              uint32_t code, sf4;
-              e2m1_quant<1>(vv, code, sf4);
-              const uint32_t code_hi = __shfl_down_sync(0xffffffffu, code, 1);
+              // MXFP4 activations: 4 E2M1 codes (2 bytes) of row j's 64-byte row, unit kb % 4
+              uint32_t codes, sf4;
+              e2m1_quant<4>(hv, codes, sf4);
               if (j < tl.rows) {
-                uint8_t* blk = p.bp_out + ((int64_t)tt * p.KCo + kb / 4) * C::B_BLOCK;
-                uint8_t* q = blk + packed_unit_offset64(j, kb & 3) + lane / 2;
-                if ((lane & 1) == 0 && in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)(code | (code_hi << 4));
-                q = blk + packed_sf_offset(C::N2, j, kb, C::RB);
-                if (lane == 0 && in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)sf4;
+                uint16_t* q2 = reinterpret_cast<uint16_t*>(blk + packed_unit_offset64(j, kb & 3) + 2 * u);
+                if (in_bounds(q2, p.bp_out, p.bp_out_end, p.status)) *q2 = (uint16_t)codes;
+                uint8_t* qs = blk + packed_sf_offset(C::N2, j, kb, C::RB);
+                if (u == 0 && in_bounds(qs, p.bp_out, p.bp_out_end, p.status)) *qs = (uint8_t)sf4;
               }
-              continue;
-            }
-            uint32_t hi, lo, s1, s2;
-            e4m3_split<1>(vv, hi, lo, s1, s2);
-            if (j < tl.rows) {
-              // the down GEMM's packed block: chunk kb / 4, rows 2j (hi) and 2j + 1 (lo),
-              // byte f' = 32 (kb % 4) + lane of the 128-byte row
-              uint8_t* blk = p.bp_out + ((int64_t)tt * p.KCo + kb / 4) * C::B_BLOCK;
-              const int u = 2 * (kb & 3) + (lane >> 4);
-              // (with MXFP8 activations only the hi term: h rounded to E4M3 in its block)
-              uint8_t* q = blk + packed_unit_offset(TERMS * j, u) + (lane & 15);
-              if (in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)hi;
-              q = blk + packed_unit_offset(2 * j + 1, u) + (lane & 15);
-              if (TERMS == 2 && in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)lo;
-              if (lane == 0) {
-                q = blk + packed_sf_offset(C::N2, TERMS * j, kb);
-                if (in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)s1;
-                q = blk + packed_sf_offset(C::N2, 2 * j + 1, kb);
-                if (TERMS == 2 && in_bounds(q, p.bp_out, p.bp_out_end, p.status)) *q = (uint8_t)s2;
+            } else {
+              uint32_t hi, lo, s1, s2;
+              e4m3_split<4>(hv, hi, lo, s1, s2);
+              if (j < tl.rows) {
+                // the down GEMM's packed block: chunk kb / 4, rows TERMS j (hi) and 2 j + 1 (lo),
+                // bytes 32 (kb % 4) + 4 u .. + 3 of the 128-byte row
+                const int unit = 2 * (kb & 3) + (u >> 2);
+                uint32_t* qh = reinterpret_cast<uint32_t*>(blk + packed_unit_offset(TERMS * j, unit) + 4 * (u & 3));
+                if (in_bounds(qh, p.bp_out, p.bp_out_end, p.status)) *qh = hi;
+                uint32_t* ql = reinterpret_cast<uint32_t*>(blk + packed_unit_offset(2 * j + 1, unit) + 4 * (u & 3));
+                if (TERMS == 2 && in_bounds(ql, p.bp_out, p.bp_out_end, p.status)) *ql = lo;
+                if (u == 0) {
+                  uint8_t* qs = blk + packed_sf_offset(C::N2, TERMS * j, kb);
+                  if (in_bounds(qs, p.bp_out, p.bp_out_end, p.status)) *qs = (uint8_t)s1;
+                  qs = blk + packed_sf_offset(C::N2, 2 * j + 1, kb);
+                  if (TERMS == 2 && in_bounds(qs, p.bp_out, p.bp_out_end, p.status)) *qs = (uint8_t)s2;
+                }
               }
             }
+            group_sync();  // the exchange buffers are reused by the next round
           }
-          group_sync();  // s_x is reused by the next read
         }
       } else {
-        int* s_tok = reinterpret_cast<int*>(gepi + C::TC * 64 * 4);  // [TC]
+        int* s_tok = reinterpret_cast<int*>(gepi + 2 * C::SB * 64 * 4);  // [TC]
         float* ys = p.ys + (int64_t)it.ks * p.P * p.d;               // this split's partial sums
         const int m = kBM * rt + row;                                // output feature
         const int ncol = min(kBM, p.d - kBM * rt);
@@ -696,12 +723,14 @@ int launch_one(const FwdArgs& a) {
 #ifndef MOE_GEMV_DOWN_SPLIT
 #define MOE_GEMV_DOWN_SPLIT 3
 #endif
-// Large batches: 96-token tiles (MMA N = 192).
+// Large batches: 96-token tiles (MMA N = 192), one 128-chunk per stage and four stages:
+// three stages of copies in flight while one is consumed (16384 tokens x 128 experts:
+// gate_up 2.30 ms, down 1.15 ms, against 2.43 / 1.32 ms with two stages of two chunks).
 #ifndef MOE_GEMM_NP
-#define MOE_GEMM_NP 2
+#define MOE_GEMM_NP 1
 #endif
 #ifndef MOE_GEMM_S
-#define MOE_GEMM_S 2
+#define MOE_GEMM_S 4
 #endif
 #ifndef MOE_GEMM_CPS
 #define MOE_GEMM_CPS 1
@@ -719,7 +748,11 @@ int launch_one(const FwdArgs& a) {
 #define MOE_GEMV_S_FP4 6
 #endif
 #ifndef MOE_GEMM_S_FP4
-#define MOE_GEMM_S_FP4 4
+#define MOE_GEMM_S_FP4 8
+#endif
+// MXFP8 activations: a 32-column epilogue read holds 32 tokens (twice the exchange buffer)
+#ifndef MOE_GEMM_S_MXFP8
+#define MOE_GEMM_S_MXFP8 MOE_GEMM_S
 #endif
 
 constexpr int kGemvBN = 8, kGemvNP = MOE_GEMV_NP, kGemvS = MOE_GEMV_S, kGemvCPS = MOE_GEMV_CPS,
@@ -740,7 +773,7 @@ namespace {
 template <int TERMS, bool FP4>
 int launch_pair(const FwdArgs& a) {
   constexpr int gv = kGemvBN * 2 / TERMS, gm = kGemmBN * 2 / TERMS;
-  constexpr int sv = FP4 ? MOE_GEMV_S_FP4 : kGemvS, sm = FP4 ? MOE_GEMM_S_FP4 : kGemmS;
+  constexpr int sv = FP4 ? MOE_GEMV_S_FP4 : kGemvS, sm = FP4 ? MOE_GEMM_S_FP4 : TERMS == 1 ? MOE_GEMM_S_MXFP8 : kGemmS;
   int n1, n2;
   if (a.ws.tile_tokens == gv) {
     n1 = launch_one<MODE_GATE_UP, gv, kGemvNP, sv, kGemvCPS, kGemvEG, kGemvNPW, TERMS, FP4, 1>(a);
