@@ -61,6 +61,7 @@ struct MxParams {
   int32_t K;               // reduction length (d for gate_up, I for down)
   int32_t KC;              // 128-chunks of the reduction axis (K rounded up)
   int32_t n_rt;            // row tiles per token tile: I/64 (gate_up) or ceil(d/128) (down)
+  int32_t n_ru;            // row units per token tile: n_rt, or ceil(n_rt / 2) for CTA pairs
   int32_t ksplit_max;      // reduction-axis splits per (token tile, row tile) allowed (down only)
   int32_t P;               // pairs (rows of ys per split)
   int32_t* status;
@@ -95,7 +96,7 @@ struct MxParams {
 #endif
 constexpr int kSfSlots = MOE_SF_SLOTS;  // scale-factor TMEM slots, used stage after stage in turn
 
-template <int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, bool FP4>
+template <int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, bool FP4, int CG>
 struct MxCfg {
   static constexpr int N2 = TERMS * BN;                 // MMA N: hi (and lo) column per token
   static constexpr int G = (N2 + 127) / 128;            // scale-factor groups of the B operand
@@ -105,10 +106,16 @@ struct MxCfg {
   static constexpr int A_PANEL = kBM * RB;              // 128 weight rows
   static constexpr int B_PANEL = N2 * RB;               // N2 activation rows
   static constexpr int B_BLOCK = packed_block_bytes(N2, RB);  // B panel + its scale factors, padded
+  // A CTA pair (CG = 2) shares one MMA of M = 256: each CTA holds its 128 weight rows, half
+  // of the B rows and all of B's scale factors; one chunk per stage.
+  static constexpr int B_ROWS = N2 / CG;                // B rows in this CTA's shared memory
+  static constexpr int B_SF_OFF = B_ROWS * RB;          // B's scale factors within a chunk's B region
+  static constexpr int B_SMEM = CG == 1 ? B_BLOCK : ((B_SF_OFF + G * kSfGroupBytes + 1023) / 1024) * 1024;
   static constexpr int B_OFF = NP * A_PANEL;
-  static constexpr int SFA_OFF = B_OFF + NP * B_BLOCK;
+  static constexpr int SFA_OFF = B_OFF + NP * B_SMEM;
   static constexpr int STAGE_BYTES = ((SFA_OFF + NP * kSfGroupBytes + 1023) / 1024) * 1024;
   static constexpr int A_TX = NP * kBM * kKChunk / 2;   // the weight box counts packed bytes
+  static constexpr int PAIR_TX = A_TX + B_SF_OFF + G * kSfGroupBytes + kSfGroupBytes;  // one CTA's stage (pairs)
   static constexpr int CW = N2 < 32 ? N2 : 32;          // accumulator columns per epilogue read
   static constexpr int TC = CW / TERMS;                 // tokens per epilogue read
   static constexpr int SB = 8;                          // tokens per g / u exchange round (gate_up)
@@ -133,6 +140,8 @@ struct MxCfg {
   static_assert(SMEM_BYTES * CPS <= 227 * 1024, "shared memory budget of CPS co-resident CTAs");
   static_assert(kBM * NP <= 256, "TMA box height");
   static_assert(EG == 1 || EG == 2, "one or two epilogue warpgroups");
+  static_assert(CG == 1 || (CG == 2 && NP == 1 && NPW == 1 && CPS == 1 && B_ROWS % 8 == 0),
+                "CTA pairs: one chunk and one copy issuer per stage, one CTA per SM");
   static_assert(TC % SB == 0, "an epilogue read holds whole exchange rounds");
   static_assert(NPW >= 1 && NPW <= 3, "producer warps: one per kind of copy at most");
 };
@@ -142,12 +151,12 @@ struct Item {
   int tt, rt, ks, kc0, kc1;
 };
 
-__device__ __forceinline__ Item item_of(const MxParams& p, int i, int ksplit) {
+__device__ __forceinline__ Item item_of(const MxParams& p, int i, int ksplit, int cg, int rank) {
   Item it;
   const int r = i / ksplit;
   it.ks = i - r * ksplit;
-  it.tt = r / p.n_rt;
-  it.rt = r - it.tt * p.n_rt;
+  it.tt = r / p.n_ru;
+  it.rt = cg * (r - it.tt * p.n_ru) + rank;   // a pair's CTAs take consecutive row tiles
   it.kc0 = it.ks * p.KC / ksplit;
   it.kc1 = (it.ks + 1) * p.KC / ksplit;
   return it;
@@ -169,10 +178,37 @@ __device__ __forceinline__ int choose_ksplit(int n0, int grid, int smax) {
   return max(1, min(smax, (2 * grid + n0 - 1) / n0));
 }
 
-template <int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, bool FP4, int MODE>
-__global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::THREADS, CPS)
-    mx_expert_kernel(const __grid_constant__ CUtensorMap tm_w, const MxParams p) {
-  using C = MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>;
+// The tcgen05 operations of one CTA (CG = 1) or of a CTA pair issued by its leader (CG = 2).
+template <int CG>
+__device__ __forceinline__ void cp_sf(uint32_t taddr, uint64_t desc) {
+  if (CG == 2) ptx::tc_cp_32x128b_x4_pair(taddr, desc);
+  else ptx::tc_cp_32x128b_x4(taddr, desc);
+}
+template <int CG>
+__device__ __forceinline__ void mma_f8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                       uint32_t acc) {
+  if (CG == 2) ptx::mma_mx_ss_pair(d, a, b, idesc, sfa, sfb, acc);
+  else ptx::mma_mx_ss(d, a, b, idesc, sfa, sfb, acc);
+}
+template <int CG>
+__device__ __forceinline__ void mma_f4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                       uint32_t acc) {
+  if (CG == 2) ptx::mma_mxf4_ss_pair(d, a, b, idesc, sfa, sfb, acc);
+  else ptx::mma_mxf4_ss(d, a, b, idesc, sfa, sfb, acc);
+}
+// Arrive on `bar` (in both CTAs of a pair) when the issued tcgen05 operations are done.
+template <int CG>
+__device__ __forceinline__ void commit_to(uint64_t* bar) {
+  if (CG == 2) ptx::tc_commit_pair(bar, (uint16_t)0x3);
+  else ptx::tc_commit(bar);
+}
+
+template <int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, bool FP4, int CG, int MODE>
+__global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>::THREADS, CPS)
+    mx_expert_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_bsf, const __grid_constant__ CUtensorMap tm_sfa,
+                     const MxParams p) {
+  using C = MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>;
   extern __shared__ uint8_t smem_raw[];
   pdl_trigger();
 
@@ -188,6 +224,10 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kblocks = p.K / 32;
+  // CTA pairs: rank 0 (the leader) issues the MMAs; both CTAs walk the same items
+  const int rank = CG == 2 ? (int)ptx::cluster_ctarank() : 0;
+  const int unit0 = CG == 2 ? (int)blockIdx.x / 2 : (int)blockIdx.x;
+  const int unit_stride = CG == 2 ? (int)gridDim.x / 2 : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -196,25 +236,38 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&accf[b], 1);
-      ptx::mbar_init(&acce[b], C::EPI_THREADS);
+      // drained by every epilogue thread; with pairs, by one lane per epilogue warp of each CTA
+      ptx::mbar_init(&acce[b], CG == 2 ? CG * (C::EPI_THREADS / 32) : C::EPI_THREADS);
     }
     ptx::mbar_init(drain, 1);
     *s_abort = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tm_w);
+    if (CG == 2) {
+      ptx::prefetch_tensormap(&tm_b);
+      ptx::prefetch_tensormap(&tm_bsf);
+      ptx::prefetch_tensormap(&tm_sfa);
+    }
   }
   if (warp == C::MMA_WARP) {
-    ptx::tmem_alloc(s_tmem, C::TMEM_COLS);
-    ptx::tmem_relinquish();
+    if (CG == 2) {
+      ptx::tmem_alloc_pair(s_tmem, C::TMEM_COLS);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(s_tmem, C::TMEM_COLS);
+      ptx::tmem_relinquish();
+    }
     ptx::tc_fence_before();
   }
-  __syncthreads();
+  // (pairs: the peer's copies, commits and arrivals find initialized barriers)
+  if (CG == 2) ptx::cluster_sync();
+  else __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *s_tmem;
   // Everything above overlaps the previous kernel; the work list is its output.
   pdl_wait();
-  const int n_units = *p.ntiles * p.n_rt;
-  const int ksplit = choose_ksplit(n_units, (int)gridDim.x, p.ksplit_max);   // same in every CTA
+  const int n_units = *p.ntiles * p.n_ru;
+  const int ksplit = choose_ksplit(n_units, unit_stride, p.ksplit_max);   // same in every CTA
   const int n_items = n_units * ksplit;
 
   auto a_s = [&](int s) { return smem + s * C::STAGE_BYTES; };
@@ -229,8 +282,8 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
     // the warp waits converged and lane 0 issues.
     int64_t g = 0;  // global stage counter of this CTA
     bool stop = false, withheld = false;
-    for (int i = blockIdx.x; i < n_items && !stop; i += gridDim.x) {
-      const Item it = item_of(p, i, ksplit);
+    for (int i = unit0; i < n_items && !stop; i += unit_stride) {
+      const Item it = item_of(p, i, ksplit, CG, rank);
       const int tt = it.tt, rt = it.rt;
       const int nst = (it.kc1 - it.kc0 + NP - 1) / NP;   // stages of this item
       const Tile tl = p.tiles[tt];
@@ -247,6 +300,25 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
           continue;
         }
         const int c0 = it.kc0 + st * NP, nck = min(NP, it.kc1 - c0);
+        if (CG == 2) {
+          // Pairs: this CTA's weight rows (row tile rt; a pair's tile past the last re-reads
+          // the last, its results are not stored), its half of the token tile's B rows, all
+          // of B's scale factors and its weight scale factors, completing on the leader's
+          // barrier, which expects both CTAs' bytes.
+          if (ptx::elect_one()) {
+            const uint32_t bar = ptx::mapa_shared(&full[s * C::NISS], 0);
+            if (rank == 0) ptx::mbar_arrive_expect_tx(&full[s * C::NISS], CG * C::PAIR_TX);
+            const int rt_ld = min(rt, p.NT - 1);
+            const int64_t wrow = (((int64_t)tl.e * p.NT + rt_ld) * p.KC + c0);
+            const int64_t brow = ((int64_t)tt * p.KC + c0) * (C::B_BLOCK / C::RB);   // rows of RB bytes
+            ptx::tma_load_2d_pair(a_s(s), &tm_w, 0, (int)(wrow * kBM), bar);
+            ptx::tma_load_2d_pair(b_s(s), &tm_b, 0, (int)(brow + rank * C::B_ROWS), bar);
+            ptx::tma_load_2d_pair(b_s(s) + C::B_SF_OFF, &tm_bsf, 0, (int)(brow + C::N2), bar);
+            ptx::tma_load_2d_pair(sfa_s(s), &tm_sfa, 0, (int)(wrow * (kSfGroupBytes / 128)), bar);
+          }
+          __syncwarp();
+          continue;
+        }
         if (ptx::elect_one()) {
           uint64_t* bar = &full[s * C::NISS + warp];
           const bool do_w = (0 % NPW) == warp, do_b = (1 % NPW) == warp, do_f = (2 % NPW) == warp;
@@ -265,7 +337,9 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
     // Never leave copies in flight when the CTA exits (consumers may have aborted before
     // waiting for them): wait, bounded, for this warp's last fill of every slot.  On the
     // normal path these have all landed already.
-    {
+    // (pairs: both CTAs' copies complete on the leader's barriers; the leader waits for
+    // them here and the cluster barrier at the end holds the peer until it has)
+    if (CG == 1 || rank == 0) {
       volatile int local_abort = 0;
       for (int64_t q = (g > S ? g - S : 0); q < g; ++q) {
         if (withheld && q == 0) continue;
@@ -275,21 +349,26 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
     __syncwarp();
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------------ MMA issuer
-    // The warp waits converged; lane 0 issues the copies into TMEM, the MMAs and the
-    // commits.
-    {
+    // The warp waits converged; one elected lane issues the copies into TMEM, the MMAs and
+    // the commits.  With CTA pairs only the leader's issuer runs the loop; the commits reach
+    // the barriers of both CTAs.
+    if (CG == 1 || rank == 0) {
       int64_t g = 0;
       int li = 0;
       bool stop = false;
-      for (int i = blockIdx.x; i < n_items && !stop; i += gridDim.x, ++li) {
+      for (int i = unit0; i < n_items && !stop; i += unit_stride, ++li) {
         const int b = li & 1;
+        // (pairs: the drain arrivals come from the epilogues of both CTAs)
         if (li >= 2 &&
             !__all_sync(0xffffffffu,
-                        ptx::mbar_wait_bounded(&acce[b], (uint32_t)((li >> 1) - 1) & 1, s_abort, kWaitLimitNs)))
+                        CG == 2 ? ptx::mbar_wait_cluster_bounded(&acce[b], (uint32_t)((li >> 1) - 1) & 1, s_abort,
+                                                                 kWaitLimitNs)
+                                : ptx::mbar_wait_bounded(&acce[b], (uint32_t)((li >> 1) - 1) & 1, s_abort,
+                                                         kWaitLimitNs)))
           break;
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + b * C::ACC_COLS;
-        const Item it = item_of(p, i, ksplit);
+        const Item it = item_of(p, i, ksplit, CG, rank);
         const int nst = (it.kc1 - it.kc0 + NP - 1) / NP;
         for (int st = 0; st < nst; ++st, ++g) {
           const int s = (int)(g % S);
@@ -309,17 +388,17 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
             const uint32_t sf_slot = tmem + (uint32_t)((g % kSfSlots) * C::SF_SLOT_COLS);
             const uint64_t a0 = FP4 ? ptx::smem_desc_k_sw64(a_s(s)) : ptx::smem_desc_k_sw128(a_s(s));
             const uint64_t b0 = FP4 ? ptx::smem_desc_k_sw64(b_s(s)) : ptx::smem_desc_k_sw128(b_s(s));
-            const uint64_t f0 = ptx::smem_desc_k_rows16(sfa_s(s)), fb0 = ptx::smem_desc_k_rows16(b_s(s) + C::B_PANEL);
+            const uint64_t f0 = ptx::smem_desc_k_rows16(sfa_s(s)), fb0 = ptx::smem_desc_k_rows16(b_s(s) + C::B_SF_OFF);
             // (descriptor start addresses count 16-byte units: offsets within shared memory add)
-            constexpr uint64_t kA = C::A_PANEL >> 4, kB = C::B_BLOCK >> 4, kF = kSfGroupBytes >> 4;
+            constexpr uint64_t kA = C::A_PANEL >> 4, kB = C::B_SMEM >> 4, kF = kSfGroupBytes >> 4;
             if (nck == NP && 4 * (c0 + NP) <= kblocks) {
               // a full stage: NP chunks of 4 blocks of 32, every index a compile-time constant
 #pragma unroll
               for (int c = 0; c < NP; ++c) {
-                ptx::tc_cp_32x128b_x4(sf_slot + C::SFA_COL + 4 * c, f0 + c * kF);
+                cp_sf<CG>(sf_slot + C::SFA_COL + 4 * c, f0 + c * kF);
 #pragma unroll
                 for (int gg = 0; gg < C::G; ++gg)
-                  ptx::tc_cp_32x128b_x4(sf_slot + C::SFB_COL + 4 * (c * C::G + gg), fb0 + c * kB + gg * kF);
+                  cp_sf<CG>(sf_slot + C::SFB_COL + 4 * (c * C::G + gg), fb0 + c * kB + gg * kF);
               }
 #pragma unroll
               for (int c = 0; c < NP; ++c) {
@@ -327,23 +406,23 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
                 if (FP4) {
 #pragma unroll
                   for (int kk = 0; kk < 2; ++kk)
-                    ptx::mma_mxf4_ss(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
-                                     ptx::idesc_mxf4(kBM, C::N2, (uint32_t)(2 * kk), (uint32_t)(2 * kk)), sfa, sfb,
+                    mma_f4<CG>(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
+                                     ptx::idesc_mxf4(kBM * CG, C::N2, (uint32_t)(2 * kk), (uint32_t)(2 * kk)), sfa, sfb,
                                      (st | c | kk) != 0);
                 } else {
 #pragma unroll
                   for (int kk = 0; kk < 4; ++kk)
-                    ptx::mma_mx_ss(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
-                                   ptx::idesc_mx_e2m1_e4m3(kBM, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
+                    mma_f8<CG>(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
+                                   ptx::idesc_mx_e2m1_e4m3(kBM * CG, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
                                    (st | c | kk) != 0);
                 }
               }
             } else {
               for (int c = 0; c < nck; ++c) {
-                ptx::tc_cp_32x128b_x4(sf_slot + C::SFA_COL + 4 * c, f0 + c * kF);
+                cp_sf<CG>(sf_slot + C::SFA_COL + 4 * c, f0 + c * kF);
 #pragma unroll
                 for (int gg = 0; gg < C::G; ++gg)
-                  ptx::tc_cp_32x128b_x4(sf_slot + C::SFB_COL + 4 * (c * C::G + gg), fb0 + c * kB + gg * kF);
+                  cp_sf<CG>(sf_slot + C::SFB_COL + 4 * (c * C::G + gg), fb0 + c * kB + gg * kF);
               }
               for (int c = 0; c < nck; ++c) {
                 const int nkb = min(4, kblocks - 4 * (c0 + c));   // 32-blocks of this chunk (K % 64 == 0: even)
@@ -352,28 +431,30 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
                   // FP4 x FP4: one MMA per 64 k (32 bytes of each packed row); it takes the scale
                   // bytes 2kk and 2kk + 1 of each row's scale-factor word
                   for (int kk = 0; kk < nkb / 2; ++kk)
-                    ptx::mma_mxf4_ss(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
-                                     ptx::idesc_mxf4(kBM, C::N2, (uint32_t)(2 * kk), (uint32_t)(2 * kk)), sfa, sfb,
+                    mma_f4<CG>(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
+                                     ptx::idesc_mxf4(kBM * CG, C::N2, (uint32_t)(2 * kk), (uint32_t)(2 * kk)), sfa, sfb,
                                      (st | c | kk) != 0);
                 } else {
                   // E2M1 x E4M3: one MMA per 32 k (32 bytes of each row), scale byte kk
                   for (int kk = 0; kk < nkb; ++kk)
-                    ptx::mma_mx_ss(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
-                                   ptx::idesc_mx_e2m1_e4m3(kBM, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
+                    mma_f8<CG>(d_tmem, a0 + c * kA + 2 * kk, b0 + c * kB + 2 * kk,
+                                   ptx::idesc_mx_e2m1_e4m3(kBM * CG, C::N2, (uint32_t)kk, (uint32_t)kk), sfa, sfb,
                                    (st | c | kk) != 0);
                 }
               }
             }
-            ptx::tc_commit(&sfree[s]);
+            commit_to<CG>(&sfree[s]);
           }
           __syncwarp();
         }
-        if (!stop && ptx::elect_one()) ptx::tc_commit(&accf[b]);
+        if (!stop && ptx::elect_one()) commit_to<CG>(&accf[b]);
         __syncwarp();
       }
-      // Every MMA issued above completes before the drain barrier fires.
-      if (ptx::elect_one()) ptx::tc_commit(drain);
+      // Every MMA issued above completes before the drain barrier fires (in both CTAs).
+      if (ptx::elect_one()) commit_to<CG>(drain);
       __syncwarp();
+    }
+    {
       volatile int local_abort = 0;
       ptx::mbar_wait_bounded(drain, 0, &local_abort, kWaitLimitNs);
     }
@@ -386,12 +467,23 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
     const int et = threadIdx.x - 32 * C::EPI_WARP0 - 128 * eg;  // 0..127 within the group
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     uint8_t* gepi = epi + eg * C::EPI_GROUP_BYTES;
+    // The accumulator buffer goes back to the MMA issuer (pairs: one arrival per warp on the
+    // leader's barrier, after every lane's TMEM reads)
+    auto release_acc = [&](int b) {
+      ptx::tc_fence_before();
+      if (CG == 2) {
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(&acce[b], 0));
+      } else {
+        ptx::mbar_arrive(&acce[b]);
+      }
+    };
     auto group_sync = [&]() {            // the group's named barrier (128 threads)
       if (eg == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
       else asm volatile("bar.sync 2, 128;" ::: "memory");
     };
     int li = 0;
-    for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++li) {
+    for (int i = unit0; i < n_items; i += unit_stride, ++li) {
       const int b = li & 1;
       const bool ready = !*s_abort && ptx::mbar_wait_bounded(&accf[b], (uint32_t)(li >> 1) & 1, s_abort,
                                                              kWaitLimitNs);
@@ -399,7 +491,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
       // role at any time; the barrier reduction freezes one answer for all).
       if (ptx::bar_or<3, C::EPI_THREADS>(!ready)) break;
       ptx::tc_fence_after();
-      const Item it = item_of(p, i, ksplit);
+      const Item it = item_of(p, i, ksplit, CG, rank);
       const int tt = it.tt, rt = it.rt;
       const Tile tl = p.tiles[tt];
       const uint32_t acc = tmem + lane_addr + b * C::ACC_COLS;
@@ -419,16 +511,14 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
         const int u = et & 7;                        // features 32 bq + 4 u .. + 3
         const int kb = 2 * rt + bq;                  // the block along the down GEMM's K
         if (eg * C::CW >= C::N2) {  // nothing for this group to read
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(&acce[b]);
+          release_acc(b);
         }
         for (int c0 = eg * C::CW; c0 < C::N2; c0 += EG * C::CW) {
           uint32_t v[32];
           ptx::tmem_ld32(acc + c0, v);
           ptx::tmem_wait_ld();
           if (c0 + EG * C::CW >= C::N2) {  // last read: the accumulator goes back to the MMA issuer
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&acce[b]);
+            release_acc(b);
           }
 #pragma unroll
           for (int sb = 0; sb < C::TC; sb += C::SB) {
@@ -453,7 +543,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
               // MXFP4 activations: 4 E2M1 codes (2 bytes) of row j's 64-byte row, unit kb % 4
               uint32_t codes, sf4;
               e2m1_quant<4>(hv, codes, sf4);
-              if (j < tl.rows) {
+              if (j < tl.rows && rt < p.n_rt) {
                 uint16_t* q2 = reinterpret_cast<uint16_t*>(blk + packed_unit_offset64(j, kb & 3) + 2 * u);
                 if (in_bounds(q2, p.bp_out, p.bp_out_end, p.status)) *q2 = (uint16_t)codes;
                 uint8_t* qs = blk + packed_sf_offset(C::N2, j, kb, C::RB);
@@ -462,7 +552,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
             } else {
               uint32_t hi, lo, s1, s2;
               e4m3_split<4>(hv, hi, lo, s1, s2);
-              if (j < tl.rows) {
+              if (j < tl.rows && rt < p.n_rt) {
                 // the down GEMM's packed block: chunk kb / 4, rows TERMS j (hi) and 2 j + 1 (lo),
                 // bytes 32 (kb % 4) + 4 u .. + 3 of the 128-byte row
                 const int unit = 2 * (kb & 3) + (u >> 2);
@@ -487,16 +577,14 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
         const int m = kBM * rt + row;                                // output feature
         const int ncol = min(kBM, p.d - kBM * rt);
         if (eg * C::CW >= C::N2) {
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(&acce[b]);
+          release_acc(b);
         }
         for (int c0 = eg * C::CW; c0 < C::N2; c0 += EG * C::CW) {
           uint32_t v[32];
           ptx::tmem_ld32(acc + c0, v);
           ptx::tmem_wait_ld();
           if (c0 + EG * C::CW >= C::N2) {
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&acce[b]);
+            release_acc(b);
           }
           const int jbase = c0 / TERMS;
           const int nt = min(C::TC, tl.rows - jbase);   // tokens of this read (may be <= 0)
@@ -509,7 +597,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
               if (in_bounds(q, p.ys, p.ys_end, p.status)) *q = o * p.w_sorted[prow];
             }
           }
-          if (p.fuse_combine) {
+          if (CG == 1 && p.fuse_combine) {
             // Publish this read's outputs, count them per (token, column block); the writer of
             // a token's k-th contribution adds the k outputs in slot order plus the residual.
             __threadfence();
@@ -568,9 +656,13 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>::TH
 
   __syncthreads();
   if (*s_abort && threadIdx.x == 0) set_status(p.status, MOE_ERR_TIMEOUT);
+  // (pairs: the leader has seen every copy of both CTAs land and the MMAs into both TMEMs
+  // complete before either CTA frees its TMEM and exits)
+  if (CG == 2) ptx::cluster_sync();
   if (warp == C::MMA_WARP) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+    if (CG == 2) ptx::tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else ptx::tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -616,9 +708,31 @@ int sm_count() {
   return n;
 }
 
-template <int MODE, int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, bool FP4, int KSPLIT>
+// Clusters of two CTAs of `kern` that fit on the device at once (0 if none or on error).
+template <class K>
+int max_pair_clusters(K kern, int threads, int smem) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * sm_count());
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+template <int MODE, int BN, int NP, int S, int CPS, int EG, int NPW, int TERMS, bool FP4, int KSPLIT, int CG = 1>
 int launch_one(const FwdArgs& a) {
-  using C = MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4>;
+  using C = MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>;
   const int P = a.T * a.k;
   const int K = (MODE == MODE_GATE_UP) ? a.d : a.I;
   const int N = (MODE == MODE_GATE_UP) ? 2 * a.I : a.d;  // weight rows per expert
@@ -648,6 +762,25 @@ int launch_one(const FwdArgs& a) {
         return -1;
     }
   }
+  // CTA pairs load everything by tile copies that complete on the leader's barrier: the
+  // token tile's packed activation blocks viewed as rows of RB bytes (a CTA's half of the B
+  // rows; the scale-factor rows after them), and the weight scale factors as 128-byte rows
+  // (one 512-byte group per chunk).  The blocks are already in the order the MMA reads.
+  CUtensorMap m_b = m_w, m_bsf = m_w, m_sfa = m_w;
+  if (CG == 2) {
+    const int NT = (N + kBM - 1) / kBM;
+    const uint8_t* bp = (MODE == MODE_GATE_UP) ? a.ws.bpx : a.ws.bph;
+    const uint64_t brows = (uint64_t)a.ws.max_tiles * KC * (C::B_BLOCK / C::RB);
+    const uint64_t bdims[2] = {(uint64_t)C::RB, brows}, bstr[1] = {(uint64_t)C::RB};
+    const uint32_t bbox[2] = {(uint32_t)C::RB, (uint32_t)C::B_ROWS};
+    const uint32_t sbox[2] = {(uint32_t)C::RB, (uint32_t)(C::G * kSfGroupBytes / C::RB)};
+    const uint64_t fdims[2] = {128, (uint64_t)a.E * NT * KC * (kSfGroupBytes / 128)}, fstr[1] = {128};
+    const uint32_t fbox[2] = {128, kSfGroupBytes / 128};
+    if (!make_map(&m_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, bp, bdims, bstr, bbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&m_bsf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, bp, bdims, bstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&m_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, scales, fdims, fstr, fbox, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return -1;
+  }
   MxParams prm;
   prm.tiles = a.ws.tiles;
   prm.ntiles = a.ws.ntiles;
@@ -657,6 +790,7 @@ int launch_one(const FwdArgs& a) {
   prm.K = K;
   prm.KC = KC;
   prm.n_rt = (MODE == MODE_GATE_UP) ? a.I / 64 : (a.d + kBM - 1) / kBM;
+  prm.n_ru = (prm.n_rt + CG - 1) / CG;
   prm.ksplit_max = std::max(1, std::min(KSPLIT, KC));   // every split keeps at least one chunk
   prm.P = P;
   prm.status = a.ws.status;
@@ -680,7 +814,7 @@ int launch_one(const FwdArgs& a) {
   prm.y_partial_end = a.y_partial ? a.y_partial + (int64_t)a.T * a.d : nullptr;
   prm.arrivals = a.ws.arrivals;
 
-  auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, NPW, TERMS, FP4, MODE>;
+  auto kern = mx_expert_kernel<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG, MODE>;
   static std::atomic<uint64_t> attr_done{0};   // per-device "attribute set" bits
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -690,11 +824,28 @@ int launch_one(const FwdArgs& a) {
       return -1;
     attr_done.fetch_or(bit, std::memory_order_release);
   }
-  const int64_t max_items = (int64_t)((P + BN - 1) / BN + a.E) * prm.n_rt * prm.ksplit_max;
+  const int64_t max_items = (int64_t)((P + BN - 1) / BN + a.E) * prm.n_ru * prm.ksplit_max;
+  if (CG == 2) {
+    // persistent pairs: as many clusters of two as fit at once
+    static std::atomic<int> pair_limit[64];
+    int lim = pair_limit[dev & 63].load(std::memory_order_acquire);
+    if (lim <= 0) {
+      lim = max_pair_clusters(kern, C::THREADS, C::SMEM_BYTES);
+      if (lim <= 0) return -1;
+      pair_limit[dev & 63].store(lim, std::memory_order_release);
+    }
+    const int pairs = (int)std::min<int64_t>(max_items, (int64_t)lim);
+    ev_before(a);
+    if (launch_kernel_pairs(kern, dim3(2 * pairs), dim3(C::THREADS), C::SMEM_BYTES, a.stream, a.pdl != 0, m_w, m_b,
+                            m_bsf, m_sfa, prm) != cudaSuccess)
+      return -1;
+    ev_after(a);
+    return 1;
+  }
   const int grid = (int)std::min<int64_t>(max_items, (int64_t)sm_count() * CPS);
   ev_before(a);
-  if (launch_kernel(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, a.stream, a.pdl != 0, m_w, prm) !=
-      cudaSuccess)
+  if (launch_kernel(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, a.stream, a.pdl != 0, m_w, m_b, m_bsf, m_sfa,
+                    prm) != cudaSuccess)
     return -1;
   ev_after(a);
   return 1;
@@ -742,6 +893,19 @@ int launch_one(const FwdArgs& a) {
 #define MOE_GEMM_NPW 1
 #endif
 
+// Large batches run on CTA pairs (one MMA of M = 256 over two SMs, each SM holding half of
+// the token tile's B rows): per SM, half the activation bytes into shared memory and half
+// the operand reads of the MMA, and with the smaller stages more of them in flight.
+#ifndef MOE_GEMM_CG
+#define MOE_GEMM_CG 2
+#endif
+#ifndef MOE_GEMM_S2
+#define MOE_GEMM_S2 6
+#endif
+#ifndef MOE_GEMM_S2_FP4
+#define MOE_GEMM_S2_FP4 12
+#endif
+
 // With MXFP4 activations the packed E2M1 operands take half the shared memory per stage:
 // more stages in flight.
 #ifndef MOE_GEMV_S_FP4
@@ -779,6 +943,11 @@ int launch_pair(const FwdArgs& a) {
     n1 = launch_one<MODE_GATE_UP, gv, kGemvNP, sv, kGemvCPS, kGemvEG, kGemvNPW, TERMS, FP4, 1>(a);
     if (n1 < 0) return -1;
     n2 = launch_one<MODE_DOWN, gv, kGemvNP, sv, kGemvCPS, kGemvEG, kGemvNPW, TERMS, FP4, kGemvDownSplit>(a);
+  } else if (MOE_GEMM_CG == 2) {
+    constexpr int s2 = FP4 ? MOE_GEMM_S2_FP4 : MOE_GEMM_S2;
+    n1 = launch_one<MODE_GATE_UP, gm, 1, s2, 1, kGemmEG, 1, TERMS, FP4, 1, 2>(a);
+    if (n1 < 0) return -1;
+    n2 = launch_one<MODE_DOWN, gm, 1, s2, 1, kGemmEG, 1, TERMS, FP4, 1, 2>(a);
   } else {
     n1 = launch_one<MODE_GATE_UP, gm, kGemmNP, sm, kGemmCPS, kGemmEG, kGemmNPW, TERMS, FP4, 1>(a);
     if (n1 < 0) return -1;
