@@ -128,7 +128,8 @@ struct MxCfg {
                                    : COLS_NEEDED <= 256 ? 256 : 512;
   static constexpr int EPI_GROUP_BYTES = 2 * SB * 64 * 4 + TC * 4;  // g and u of SB tokens; token list (down)
   static constexpr int EPI_BYTES = EG * EPI_GROUP_BYTES;
-  static constexpr int NISS = NPW;                      // copy issuers per stage, one barrier each
+  // barriers per stage: one per copy issuer (pairs: one, the leader's, for all copies)
+  static constexpr int NISS = CG == 2 ? 1 : NPW;
   static constexpr int BAR_BYTES = 8 * ((NISS + 1) * S + 5) + 16;
   static constexpr int SMEM_BYTES = S * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024 /*align slack*/;
   static constexpr int EPI_THREADS = 128 * EG;
@@ -139,11 +140,11 @@ struct MxCfg {
   static_assert(COLS_NEEDED <= 512 && TMEM_COLS * CPS <= 512, "TMEM budget of CPS co-resident CTAs");
   static_assert(SMEM_BYTES * CPS <= 227 * 1024, "shared memory budget of CPS co-resident CTAs");
   static_assert(kBM * NP <= 256, "TMA box height");
-  static_assert(EG == 1 || EG == 2, "one or two epilogue warpgroups");
-  static_assert(CG == 1 || (CG == 2 && NP == 1 && NPW == 1 && CPS == 1 && B_ROWS % 8 == 0),
-                "CTA pairs: one chunk and one copy issuer per stage, one CTA per SM");
+  static_assert(EG >= 1 && EG <= 3, "one to three epilogue warpgroups");
+  static_assert(CG == 1 || (CG == 2 && NP == 1 && CPS == 1 && B_ROWS % 8 == 0),
+                "CTA pairs: one chunk per stage, one CTA per SM");
   static_assert(TC % SB == 0, "an epilogue read holds whole exchange rounds");
-  static_assert(NPW >= 1 && NPW <= 3, "producer warps: one per kind of copy at most");
+  static_assert(NPW >= 1 && NPW <= (CG == 2 ? 4 : 3), "producer warps: one per kind of copy at most");
 };
 
 // Work item i: token tile tt, row tile rt, and the chunk range [kc0, kc1) of split ks.
@@ -305,16 +306,19 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
           // the last, its results are not stored), its half of the token tile's B rows, all
           // of B's scale factors and its weight scale factors, completing on the leader's
           // barrier, which expects both CTAs' bytes.
+          // (several producer warps: warp w issues the copies k with k % NPW == w; the
+          // leader's warp 0 posts the byte count of all of them)
           if (ptx::elect_one()) {
-            const uint32_t bar = ptx::mapa_shared(&full[s * C::NISS], 0);
-            if (rank == 0) ptx::mbar_arrive_expect_tx(&full[s * C::NISS], CG * C::PAIR_TX);
+            const uint32_t bar = ptx::mapa_shared(&full[s], 0);
+            if (rank == 0 && warp == 0) ptx::mbar_arrive_expect_tx(&full[s], CG * C::PAIR_TX);
             const int rt_ld = min(rt, p.NT - 1);
             const int64_t wrow = (((int64_t)tl.e * p.NT + rt_ld) * p.KC + c0);
             const int64_t brow = ((int64_t)tt * p.KC + c0) * (C::B_BLOCK / C::RB);   // rows of RB bytes
-            ptx::tma_load_2d_pair(a_s(s), &tm_w, 0, (int)(wrow * kBM), bar);
-            ptx::tma_load_2d_pair(b_s(s), &tm_b, 0, (int)(brow + rank * C::B_ROWS), bar);
-            ptx::tma_load_2d_pair(b_s(s) + C::B_SF_OFF, &tm_bsf, 0, (int)(brow + C::N2), bar);
-            ptx::tma_load_2d_pair(sfa_s(s), &tm_sfa, 0, (int)(wrow * (kSfGroupBytes / 128)), bar);
+            if (0 % NPW == warp) ptx::tma_load_2d_pair(a_s(s), &tm_w, 0, (int)(wrow * kBM), bar);
+            if (1 % NPW == warp) ptx::tma_load_2d_pair(b_s(s), &tm_b, 0, (int)(brow + rank * C::B_ROWS), bar);
+            if (2 % NPW == warp) ptx::tma_load_2d_pair(b_s(s) + C::B_SF_OFF, &tm_bsf, 0, (int)(brow + C::N2), bar);
+            if (3 % NPW == warp)
+              ptx::tma_load_2d_pair(sfa_s(s), &tm_sfa, 0, (int)(wrow * (kSfGroupBytes / 128)), bar);
           }
           __syncwarp();
           continue;
@@ -339,7 +343,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
     // normal path these have all landed already.
     // (pairs: both CTAs' copies complete on the leader's barriers; the leader waits for
     // them here and the cluster barrier at the end holds the peer until it has)
-    if (CG == 1 || rank == 0) {
+    if (CG == 1 || (rank == 0 && warp == 0)) {
       volatile int local_abort = 0;
       for (int64_t q = (g > S ? g - S : 0); q < g; ++q) {
         if (withheld && q == 0) continue;
@@ -478,9 +482,10 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
         ptx::mbar_arrive(&acce[b]);
       }
     };
-    auto group_sync = [&]() {            // the group's named barrier (128 threads)
+    auto group_sync = [&]() {            // the group's named barrier (128 threads; 3 is the epilogue-wide vote)
       if (eg == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
-      else asm volatile("bar.sync 2, 128;" ::: "memory");
+      else if (eg == 1) asm volatile("bar.sync 2, 128;" ::: "memory");
+      else asm volatile("bar.sync 4, 128;" ::: "memory");
     };
     int li = 0;
     for (int i = unit0; i < n_items; i += unit_stride, ++li) {
@@ -534,7 +539,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
             for (int i = 0; i < 4; ++i) {
               const float gv = fminf(gs[i], L);
               const float uv = fminf(fmaxf(us[i], -L), L);
-              const float h = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;   // silu(g) * u
+              const float h = __fdividef(gv, 1.0f + __expf(-gv)) * uv;   // silu(g) * u
               hv[i] = __uint_as_float((uint32_t)bf16_bits_rne(h) << 16);   // h is stored as bf16
             }
             const int j = c0 / TERMS + sb + jj;   // token within the tile
@@ -895,15 +900,23 @@ int launch_one(const FwdArgs& a) {
 
 // Large batches run on CTA pairs (one MMA of M = 256 over two SMs, each SM holding half of
 // the token tile's B rows): per SM, half the activation bytes into shared memory and half
-// the operand reads of the MMA, and with the smaller stages more of them in flight.
+// the operand reads of the MMA.  Four stages (16384 tokens x 128 experts: gate_up 2.00 ms,
+// against 2.07 / 2.04 ms with six / seven; one copy-issuing warp, which measured faster than
+// two or four).
 #ifndef MOE_GEMM_CG
 #define MOE_GEMM_CG 2
 #endif
 #ifndef MOE_GEMM_S2
-#define MOE_GEMM_S2 6
+#define MOE_GEMM_S2 4
 #endif
 #ifndef MOE_GEMM_S2_FP4
 #define MOE_GEMM_S2_FP4 12
+#endif
+#ifndef MOE_GEMM_NPW2
+#define MOE_GEMM_NPW2 1
+#endif
+#ifndef MOE_GEMM_EG_GU
+#define MOE_GEMM_EG_GU MOE_GEMM_EG
 #endif
 
 // With MXFP4 activations the packed E2M1 operands take half the shared memory per stage:
@@ -945,9 +958,9 @@ int launch_pair(const FwdArgs& a) {
     n2 = launch_one<MODE_DOWN, gv, kGemvNP, sv, kGemvCPS, kGemvEG, kGemvNPW, TERMS, FP4, kGemvDownSplit>(a);
   } else if (MOE_GEMM_CG == 2) {
     constexpr int s2 = FP4 ? MOE_GEMM_S2_FP4 : MOE_GEMM_S2;
-    n1 = launch_one<MODE_GATE_UP, gm, 1, s2, 1, kGemmEG, 1, TERMS, FP4, 1, 2>(a);
+    n1 = launch_one<MODE_GATE_UP, gm, 1, s2, 1, MOE_GEMM_EG_GU, MOE_GEMM_NPW2, TERMS, FP4, 1, 2>(a);
     if (n1 < 0) return -1;
-    n2 = launch_one<MODE_DOWN, gm, 1, s2, 1, kGemmEG, 1, TERMS, FP4, 1, 2>(a);
+    n2 = launch_one<MODE_DOWN, gm, 1, s2, 1, kGemmEG, MOE_GEMM_NPW2, TERMS, FP4, 1, 2>(a);
   } else {
     n1 = launch_one<MODE_GATE_UP, gm, kGemmNP, sm, kGemmCPS, kGemmEG, kGemmNPW, TERMS, FP4, 1>(a);
     if (n1 < 0) return -1;
