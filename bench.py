@@ -49,7 +49,8 @@ WORKLOAD_TEXT = {
     "skew_120b": "skewed routing: T=16384, d=I=2880, E=128, top-4, Zipf(1.2) router bias, MXFP4 experts",
 }
 KERNELS = ["route", "group", "pack", "gate_up", "down", "combine"]
-KERNELS_FUSED = ["route", "pack", "gate_up", "down"]     # small batches: grouping and combine fused
+KERNELS_FUSED_GROUP = ["route", "pack", "gate_up", "down", "combine"]   # small batches: grouping in the router
+KERNELS_FUSED = ["route", "pack", "gate_up", "down"]     # ... and the combine in the down GEMM
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dense tensor-core rate of each MMA kind relative to bf16 (NVIDIA's B200 figures:
 # bf16 2.25, fp8 4.5, fp4 9 PFLOP/s dense)
@@ -405,7 +406,7 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
     else:
         timed_step()
     n_timed = moe.last_launch_count()
-    names = KERNELS if n_timed == len(KERNELS) else KERNELS_FUSED
+    names = {len(KERNELS): KERNELS, len(KERNELS_FUSED_GROUP): KERNELS_FUSED_GROUP}.get(n_timed, KERNELS_FUSED)
     per_kernel = {name: [] for name in names[:n_timed]}
     for i in range(K):
         flush.zero_()

@@ -47,6 +47,10 @@ moe_status check_dims(const moe_dims* dm, int32_t T) {
   return MOE_OK;
 }
 
+#ifndef MOE_GEMV_FUSE_COMBINE
+#define MOE_GEMV_FUSE_COMBINE 0
+#endif
+
 int resolve_path(const moe_dims& dm, int32_t T) {
   if (dm.path != MOE_PATH_AUTO) return dm.path;
   // Few tokens per expert: stream the weights with narrow token tiles.
@@ -160,7 +164,11 @@ moe_status forward_impl(const moe_dims* dims, int32_t T, const uint16_t* x, cons
   // Small-batch path: fewer, fused kernels (routing + grouping + tile scales; down + combine).
   // The next block's RMSNorm needs whole rows, which the separate combine pass holds.
   a.fuse_group = (path == MOE_PATH_GEMV && T <= moe::kFusedGroupMaxT) ? 1 : 0;
-  a.fuse_combine = (path == MOE_PATH_GEMV && !a.next_norm_w) ? 1 : 0;
+  // The combine runs as its own pass after the down GEMM, so that the down GEMM can split
+  // its reduction axis as finely as balances the CTAs without a combining epilogue per
+  // split.  MOE_GEMV_FUSE_COMBINE=1 builds the fused form (the last writer of each token's
+  // 128 columns combines).
+  a.fuse_combine = (MOE_GEMV_FUSE_COMBINE && path == MOE_PATH_GEMV && !a.next_norm_w) ? 1 : 0;
   // Overlap each kernel's launch and prologue with its predecessor, except when per-kernel
   // events are recorded between the kernels.
   a.pdl = (n_events == 0) ? 1 : 0;

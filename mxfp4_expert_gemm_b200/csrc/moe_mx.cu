@@ -63,6 +63,7 @@ struct MxParams {
   int32_t n_rt;            // row tiles per token tile: I/64 (gate_up) or ceil(d/128) (down)
   int32_t n_ru;            // row units per token tile: n_rt, or ceil(n_rt / 2) for CTA pairs
   int32_t ksplit_max;      // reduction-axis splits per (token tile, row tile) allowed (down only)
+  int32_t* ksplit_out;     // down: the number of splits used (the planes of ys the combine adds)
   int32_t P;               // pairs (rows of ys per split)
   int32_t* status;
   float limit;
@@ -104,7 +105,6 @@ struct MxCfg {
   // (B), 128; with MXFP4 activations both operands are packed E2M1, 64.
   static constexpr int RB = FP4 ? kKChunk / 2 : kKChunk;
   static constexpr int A_PANEL = kBM * RB;              // 128 weight rows
-  static constexpr int B_PANEL = N2 * RB;               // N2 activation rows
   static constexpr int B_BLOCK = packed_block_bytes(N2, RB);  // B panel + its scale factors, padded
   // A CTA pair (CG = 2) shares one MMA of M = 256: each CTA holds its 128 weight rows, half
   // of the B rows and all of B's scale factors; one chunk per stage.
@@ -172,11 +172,24 @@ __device__ __forceinline__ float token_acc(const uint32_t (&v)[32], int j) {
 }
 
 // Splits of the reduction axis for n0 (token tile, row tile) units over `grid` CTAs: the
-// fewest (at most smax) that give every CTA two items, so that one item's epilogue runs
-// under the next item's loads (the accumulator is double-buffered).
+// count (at most smax) that minimises the busiest CTA's work, ceil(n0 ks / grid) items of
+// 1 / ks of a unit each plus a fixed cost per item (its epilogue and pipeline turn-around,
+// taken as 1/16 of a whole unit); a CTA with a single item has no next item's loads to
+// hide that item's epilogue under (the accumulator is double-buffered), which counts as
+// one more unit.  Ties go to fewer splits.
 __device__ __forceinline__ int choose_ksplit(int n0, int grid, int smax) {
-  if (n0 <= 0) return 1;
-  return max(1, min(smax, (2 * grid + n0 - 1) / n0));
+  if (n0 <= 0 || smax <= 1) return 1;
+  int best = 1;
+  float best_t = 3.4e38f;
+  for (int ks = 1; ks <= smax; ++ks) {
+    const int per_cta = (n0 * ks + grid - 1) / grid;
+    const float t = (float)per_cta * (1.0f / (float)ks + 0.0625f) + (per_cta < 2 ? 1.0f : 0.f);
+    if (t < best_t - 1e-6f) {
+      best_t = t;
+      best = ks;
+    }
+  }
+  return best;
 }
 
 // The tcgen05 operations of one CTA (CG = 1) or of a CTA pair issued by its leader (CG = 2).
@@ -270,6 +283,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
   const int n_units = *p.ntiles * p.n_ru;
   const int ksplit = choose_ksplit(n_units, unit_stride, p.ksplit_max);   // same in every CTA
   const int n_items = n_units * ksplit;
+  if (MODE == MODE_DOWN && blockIdx.x == 0 && threadIdx.x == 0) *p.ksplit_out = ksplit;
 
   auto a_s = [&](int s) { return smem + s * C::STAGE_BYTES; };
   auto b_s = [&](int s) { return smem + s * C::STAGE_BYTES + C::B_OFF; };
@@ -797,6 +811,7 @@ int launch_one(const FwdArgs& a) {
   prm.n_rt = (MODE == MODE_GATE_UP) ? a.I / 64 : (a.d + kBM - 1) / kBM;
   prm.n_ru = (prm.n_rt + CG - 1) / CG;
   prm.ksplit_max = std::max(1, std::min(KSPLIT, KC));   // every split keeps at least one chunk
+  prm.ksplit_out = a.ws.ntiles + 1;
   prm.P = P;
   prm.status = a.ws.status;
   prm.limit = a.limit;
@@ -841,8 +856,8 @@ int launch_one(const FwdArgs& a) {
     }
     const int pairs = (int)std::min<int64_t>(max_items, (int64_t)lim);
     ev_before(a);
-    if (launch_kernel_pairs(kern, dim3(2 * pairs), dim3(C::THREADS), C::SMEM_BYTES, a.stream, a.pdl != 0, m_w, m_b,
-                            m_bsf, m_sfa, prm) != cudaSuccess)
+    if (launch_kernel_cluster(kern, dim3(2 * pairs), dim3(C::THREADS), C::SMEM_BYTES, a.stream, a.pdl != 0, 2u, m_w,
+                              m_b, m_bsf, m_sfa, prm) != cudaSuccess)
       return -1;
     ev_after(a);
     return 1;
@@ -877,7 +892,7 @@ int launch_one(const FwdArgs& a) {
 #define MOE_GEMV_NPW 1
 #endif
 #ifndef MOE_GEMV_DOWN_SPLIT
-#define MOE_GEMV_DOWN_SPLIT 3
+#define MOE_GEMV_DOWN_SPLIT 6
 #endif
 // Large batches: 96-token tiles (MMA N = 192), one 128-chunk per stage and four stages:
 // three stages of copies in flight while one is consumed (16384 tokens x 128 experts:

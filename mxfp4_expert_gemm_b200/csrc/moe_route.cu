@@ -15,6 +15,7 @@
 #include <cfloat>
 
 #include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 
@@ -169,7 +170,7 @@ __device__ void group_block(const FwdArgs& a, int tile_tokens) {
   }
   __syncthreads();
   // token tiles of every expert
-  for (int e = warp; e < E; e += 32) {
+  for (int e = warp; e < E; e += (int)(blockDim.x >> 5)) {
     const int base = s_tb[e];
     const int c_e = (e + 1 < E ? s_off[e + 1] : P) - s_off[e];
     for (int i = lane; i * tile_tokens < c_e; i += 32) {
@@ -205,12 +206,17 @@ __device__ void group_block(const FwdArgs& a, int tile_tokens) {
 }
 
 // ----------------------------------------------------------------------------------
-// Small batches: one CTA of 1024 threads per token.  The token's normalized row stays
-// in shared memory (fp32); warp w computes the logits of experts w, w+32, ..., each
-// lane issuing all of its 16-byte loads of the router row before the FMAs; warp 0 then
-// selects the top-k.
+// Small batches: one cluster of kTokCluster CTAs (256 threads each) per token.  Every CTA
+// of the cluster normalizes the token's row into shared memory (fp32; the row is small,
+// each CTA reads it), writes the activation format of its share of the 32-blocks, and
+// computes the logits of its share of the experts (warp w: experts first + w, + 8, ...,
+// each lane issuing all of its 16-byte loads of the router row before the FMAs); the
+// logits go into the shared memory of the cluster's first CTA, which after the cluster
+// barrier selects the top-k.  Spreading a token's experts over the cluster spreads the
+// router rows' bytes over four SMs.
 // ----------------------------------------------------------------------------------
-constexpr int kTokThreads = 1024;
+constexpr int kTokCluster = 4;
+constexpr int kTokThreads = 256;
 constexpr int kTokWarps = kTokThreads / 32;
 constexpr int kTokBatch = 12;   // router-row loads in flight per lane
 
@@ -220,10 +226,11 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
   pdl_trigger();
   const int d = a.d, E = a.E;
   float* s_xn = smem;          // [d]
-  float* s_l = smem + d;       // [32*NJ]
+  float* s_l = smem + d;       // [32*NJ] logits (in the cluster's first CTA)
   __shared__ float s_red[kTokWarps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t t = blockIdx.x;
+  const int rank = (int)ptx::cluster_ctarank();
+  const int64_t t = blockIdx.x / kTokCluster;
   const uint16_t* xr = a.x + t * d;
   float ss = 0.f;
   for (int i = tid * 8; i < d; i += kTokThreads * 8) {
@@ -252,11 +259,12 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
   }
   __syncthreads();
   {
-    // xe = bf16(xn) as E4M3 hi / lo terms: warp w splits 32-blocks w, w + 32, ...
-    const int dp = a.ws.dp;
+    // xe = bf16(xn) as E4M3 hi / lo terms (or one MXFP8 term, or MXFP4 codes): this CTA's
+    // 32-blocks, one per warp at a time
+    const int dp = a.ws.dp, nb = d / 32;
     uint8_t* xq = a.ws.xq + t * 2 * dp;
     uint8_t* sf = a.ws.xsf + t * 2 * (dp / 32);
-    for (int b = warp; b < d / 32; b += kTokWarps) {
+    for (int b = rank * nb / kTokCluster + warp; b < (rank + 1) * nb / kTokCluster; b += kTokWarps) {
       const float v[1] = {bf16_to_f32(bf16_bits_rne(s_xn[32 * b + lane]))};
       if (a.ws.fp4) {   // MXFP4 activations: packed E2M1 codes, two per byte
         uint32_t c, s1;
@@ -277,7 +285,7 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
     }
   }
   const int n4 = d / 4;
-  for (int e = warp; e < E; e += kTokWarps) {
+  for (int e = rank * E / kTokCluster + warp; e < (rank + 1) * E / kTokCluster; e += kTokWarps) {
     const float4* wr = reinterpret_cast<const float4*>(a.router_w + (int64_t)e * d);
     float acc = 0.f;
     // batches of kTokBatch 16-byte loads per lane, all issued before their FMAs
@@ -302,9 +310,10 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) s_l[e] = acc + (a.router_b ? a.router_b[e] : 0.f);
+    if (lane == 0) ptx::st_cluster_f32(ptx::mapa_shared(&s_l[e], 0), acc + (a.router_b ? a.router_b[e] : 0.f));
   }
-  __syncthreads();
+  ptx::cluster_sync();   // every logit of the token is in the first CTA's shared memory
+  if (rank != 0) return;
   if (warp == 0) {
     float l[NJ];
 #pragma unroll
@@ -312,11 +321,12 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
     warp_topk_softmax<NJ>(l, E, a.k, t, a);
   }
   if (a.fuse_group) {
-    // Publish this token (top-k, counts, xq rows), then take a ticket; the last CTA groups.
+    // Publish this token (top-k, counts, xq rows: the other CTAs of the cluster wrote
+    // theirs before the cluster barrier), then take a ticket; the last token's CTA groups.
     __shared__ int s_last;
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(a.ws.ticket, 1) == (int)gridDim.x - 1;
+    if (tid == 0) s_last = atomicAdd(a.ws.ticket, 1) == a.T - 1;
     __syncthreads();
     if (s_last) {
       __threadfence();
@@ -706,6 +716,7 @@ __global__ void combine_kernel(FwdArgs a) {
   const int i4 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i4 >= a.d) return;
   const int64_t P = (int64_t)a.T * a.k;
+  const int ksplit = a.ws.ntiles[1];   // the splits the down GEMM of this call used
   for (int t = blockIdx.y; t < a.T; t += gridDim.y) {
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (!a.y_partial) {
@@ -717,7 +728,7 @@ __global__ void combine_kernel(FwdArgs a) {
     }
     for (int j = 0; j < a.k; ++j) {
       const int p = a.ws.inv[(int64_t)t * a.k + j];
-      for (int sp = 0; sp < a.ws.ksplit; ++sp) {   // partial sums of a split down GEMM
+      for (int sp = 0; sp < ksplit; ++sp) {   // partial sums of a split down GEMM
         const float4 o = *reinterpret_cast<const float4*>(a.ws.ys + (sp * P + p) * a.d + i4);
         v[0] += o.x;
         v[1] += o.y;
@@ -746,7 +757,8 @@ __global__ void combine_kernel(FwdArgs a) {
 // block reduction in fixed order.
 // ----------------------------------------------------------------------------------
 struct FinishArgs {
-  int32_t T, d, k, ksplit;
+  int32_t T, d, k;
+  const int32_t* ksplit;  // the splits the down GEMM of this call used (device)
   int64_t P;
   const uint16_t* x;
   const float* ys;        // pair outputs [ksplit][P][d] (or NULL)
@@ -765,6 +777,7 @@ __global__ void __launch_bounds__(kFinishThreads) finish_rows_kernel(FinishArgs 
   pdl_trigger();
   pdl_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ks = f.ys ? *f.ksplit : 0;
   for (int t = blockIdx.x; t < f.T; t += gridDim.x) {
     float ss = 0.f;
     for (int i4 = tid * 4; i4 < f.d; i4 += kFinishThreads * 4) {
@@ -774,7 +787,7 @@ __global__ void __launch_bounds__(kFinishThreads) finish_rows_kernel(FinishArgs 
       if (f.ys) {
         for (int j = 0; j < f.k; ++j) {
           const int p = f.inv[(int64_t)t * f.k + j];
-          for (int sp = 0; sp < f.ksplit; ++sp) {
+          for (int sp = 0; sp < ks; ++sp) {
             const float4 o = *reinterpret_cast<const float4*>(f.ys + (sp * f.P + p) * f.d + i4);
             v[0] += o.x;
             v[1] += o.y;
@@ -847,7 +860,9 @@ int launch_route_nj(const FwdArgs& a) {
     const size_t smem = sizeof(float) * (a.d + 32 * NJ);
     if (!ensure_smem_limit(route_token_kernel<NJ>, smem, tok_limits)) return -1;
     ev_before(a);
-    route_token_kernel<NJ><<<a.T, kTokThreads, smem, a.stream>>>(a);
+    if (launch_kernel_cluster(route_token_kernel<NJ>, dim3(a.T * kTokCluster), dim3(kTokThreads), smem, a.stream,
+                              false, (unsigned)kTokCluster, a) != cudaSuccess)
+      return -1;
     ev_after(a);
     return 1;
   }
@@ -929,7 +944,7 @@ int launch_combine(const FwdArgs& a) {
     f.T = a.T;
     f.d = a.d;
     f.k = a.k;
-    f.ksplit = a.ws.ksplit;
+    f.ksplit = a.ws.ntiles + 1;
     f.P = (int64_t)a.T * a.k;
     f.x = a.x;
     f.ys = a.ws.ys;

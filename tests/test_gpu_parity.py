@@ -133,6 +133,15 @@ def test_route_bit_exact(name):
     np.testing.assert_allclose(wg.sum(1), 1.0, atol=2e-6)
     lg = ref["logits"][np.arange(cfg.T)[:, None], idx]
     assert np.all(np.diff(lg, axis=1) <= 1e-5)
+    # the token tiles: every expert's sorted pairs cut into tiles of the path's size, in
+    # expert order (written by the grouping kernel, or by the router's last CTA)
+    tt = TILE_TOKENS[moe.resolved_path(dims, cfg.T)]
+    want = [(e, int(gr["offsets"][e]) + i * tt, min(tt, int(gr["counts"][e]) - i * tt))
+            for e in range(cfg.E) for i in range(-(-int(gr["counts"][e]) // tt))]
+    n = int(moe.workspace_view(ws, dims, cfg.T, "ntiles", torch.int32, (1,)).item())
+    assert n == len(want)
+    got = moe.workspace_view(ws, dims, cfg.T, "tiles", torch.int32, (n, 4)).cpu().numpy()[:, :3]
+    np.testing.assert_array_equal(got, np.array(want, dtype=np.int32).reshape(-1, 3))
 
 
 # ------------------------------------------------------------------------------ whole layer
@@ -429,7 +438,7 @@ def test_launch_count_reported():
     c = case(SMALL["tiny"])
     cfg = c["cfg"]
     for path, n in (("gemm", 6),   # route, group, pack, gate_up, down, combine
-                    ("gemv", 4)):  # route (+ grouping), pack, gate_up, down (+ combine)
+                    ("gemv", 5)):  # route (+ grouping), pack, gate_up, down, combine
         dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, path=path)
         ws = moe.new_workspace(dims, cfg.T)
         moe.moe_forward(dims, c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"], ws)

@@ -116,3 +116,26 @@ def test_residual_norm_alone():
     # y alone, no norm
     y_only = moe.moe_residual_norm(bf16_dev(x), torch.from_numpy(s).cuda())
     np.testing.assert_array_equal(bf16_host(y_only), got_y)
+
+
+@pytest.mark.parametrize("path", ["gemv", "gemm"])
+def test_combine_adds_only_the_splits_of_this_call(path):
+    """The down GEMM chooses its reduction-axis splits per call; the combine and the
+    next-norm pass must add exactly those partial-sum planes.  Planes past them (left by an
+    earlier call that split further, or never written) hold garbage here and must not
+    enter y."""
+    c = case(SMALL["decode_20b"])
+    cfg = c["cfg"]
+    dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, cfg.rms_eps, cfg.swiglu_limit, path=path)
+    ws = moe.new_workspace(dims, cfg.T)
+    lay = moe.moe_workspace_layout(dims, cfg.T)
+    args = (c["x_dev"], c["gamma_dev"], c["rw_dev"], c["rb_dev"], *c["W"]["gpu"])
+    ws[lay["ys"]:lay["total"]].fill_(0x4B)   # every plane: about 1.3e7 per value
+    y = moe.moe_forward(dims, *args, ws)
+    assert moe.moe_device_status(ws) == moe.MOE_OK
+    assert_parity(parity_stats(bf16_host(y), oracle_rows(c)["y"], c["x"]), f"garbage planes/{path}")
+    ws[lay["ys"]:lay["total"]].fill_(0x4B)
+    g2 = torch.ones(cfg.d, dtype=torch.float32, device="cuda")
+    y2, _ = moe.moe_forward_norm(dims, *args, ws, g2, 1e-5)
+    assert moe.moe_device_status(ws) == moe.MOE_OK
+    np.testing.assert_array_equal(bf16_host(y2), bf16_host(y))
