@@ -303,12 +303,27 @@ __device__ __forceinline__ void e4m3_split(const float (&v)[V], uint32_t& hi, ui
   const float inv1 = pow2f(-s1), sc1 = pow2f(s1), inv2 = pow2f(-s2);
   hi = 0u;
   lo = 0u;
+  if constexpr (V % 2 == 0) {
+    // two values per conversion (each rounded on its own, as below)
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const uint32_t q = e4m3x2(v[i] * inv1, 0.f) & 0xFFu;
-    hi |= q << (8 * i);
-    const float r = v[i] - e4m3_to_f32(q) * sc1;   // exact
-    lo |= (e4m3x2(r * inv2, 0.f) & 0xFFu) << (8 * i);
+    for (int i = 0; i < V; i += 2) {
+      const uint32_t q2 = e4m3x2(v[i] * inv1, v[i + 1] * inv1);
+      hi |= q2 << (8 * i);
+      uint32_t h2;
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)q2));
+      const float d0 = __half2float(__ushort_as_half((uint16_t)(h2 & 0xFFFFu)));
+      const float d1 = __half2float(__ushort_as_half((uint16_t)(h2 >> 16)));
+      const float r0 = v[i] - d0 * sc1, r1 = v[i + 1] - d1 * sc1;   // exact
+      lo |= e4m3x2(r0 * inv2, r1 * inv2) << (8 * i);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      const uint32_t q = e4m3x2(v[i] * inv1, 0.f) & 0xFFu;
+      hi |= q << (8 * i);
+      const float r = v[i] - e4m3_to_f32(q) * sc1;   // exact
+      lo |= (e4m3x2(r * inv2, 0.f) & 0xFFu) << (8 * i);
+    }
   }
   sf_hi = (uint32_t)(s1 + 127);
   sf_lo = (uint32_t)(s2 + 127);

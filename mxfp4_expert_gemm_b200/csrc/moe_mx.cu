@@ -37,6 +37,7 @@
 // flag, every role leaves its loop, in-flight copies and MMAs are drained (bounded),
 // TMEM is freed and MOE_ERR_TIMEOUT is recorded.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -126,7 +127,8 @@ struct MxCfg {
   static constexpr int COLS_NEEDED = 2 * ACC_COLS + kSfSlots * SF_SLOT_COLS;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 32 ? 32 : COLS_NEEDED <= 64 ? 64 : COLS_NEEDED <= 128 ? 128
                                    : COLS_NEEDED <= 256 ? 256 : 512;
-  static constexpr int EPI_GROUP_BYTES = 2 * SB * 64 * 4 + TC * 4;  // g and u of SB tokens; token list (down)
+  // two buffers of g and u of SB tokens (gate_up), then the token list (down)
+  static constexpr int EPI_GROUP_BYTES = 4 * SB * 64 * 4 + TC * 4;
   static constexpr int EPI_BYTES = EG * EPI_GROUP_BYTES;
   // barriers per stage: one per copy issuer (pairs: one, the leader's, for all copies)
   static constexpr int NISS = CG == 2 ? 1 : NPW;
@@ -502,6 +504,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
       else asm volatile("bar.sync 4, 128;" ::: "memory");
     };
     int li = 0;
+    int rnd = 0;   // g / u exchange rounds so far (gate_up)
     for (int i = unit0; i < n_items; i += unit_stride, ++li) {
       const int b = li & 1;
       const bool ready = !*s_abort && ptx::mbar_wait_bounded(&accf[b], (uint32_t)(li >> 1) & 1, s_abort,
@@ -520,10 +523,10 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
         // finishes 4 consecutive features of one token: h = bf16(silu(g) * u) and its share
         // of the down GEMM's activation block (8 threads per 32-feature block: E4M3 hi / lo
         // terms and their scales, the hi term alone with MXFP8 activations, or E2M1 codes).
-        float* s_g = reinterpret_cast<float*>(gepi);  // [SB tokens][64 features]
-        float* s_u = s_g + C::SB * 64;
+        // (two exchange buffers used round after round: a round's writes go to the buffer
+        // last read two rounds before, which the previous round's barrier has released)
+        float* const s_gu = reinterpret_cast<float*>(gepi);  // [2][g, u][SB tokens][64 features]
         const float L = p.limit;
-        float* s_mine = (q < 2) ? s_g : s_u;
         const int f = 32 * (q & 1) + lane;           // feature within the item's 64
         const int jj = et >> 4;                      // token of the round this thread finishes
         const int bq = (et >> 3) & 1;                // its 32-feature block (of the item's two)
@@ -542,6 +545,10 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
 #pragma unroll
           for (int sb = 0; sb < C::TC; sb += C::SB) {
             // (register indices stay compile-time constants)
+            float* s_g = s_gu + (rnd & 1) * 2 * C::SB * 64;
+            float* s_u = s_g + C::SB * 64;
+            float* s_mine = (q < 2) ? s_g : s_u;
+            ++rnd;
 #pragma unroll
             for (int c = 0; c < C::SB; ++c) s_mine[c * 64 + f] = token_acc<TERMS>(v, sb + c);
             group_sync();
@@ -554,7 +561,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
               const float gv = fminf(gs[i], L);
               const float uv = fminf(fmaxf(us[i], -L), L);
               const float h = __fdividef(gv, 1.0f + __expf(-gv)) * uv;   // silu(g) * u
-              hv[i] = __uint_as_float((uint32_t)bf16_bits_rne(h) << 16);   // h is stored as bf16
+              hv[i] = __bfloat162float(__float2bfloat16_rn(h));   // h is stored as bf16 (round to nearest even)
             }
             const int j = c0 / TERMS + sb + jj;   // token within the tile
             uint8_t* blk = p.bp_out + ((int64_t)tt * p.KCo + kb / 4) * C::B_BLOCK;
@@ -587,11 +594,10 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
                 }
               }
             }
-            group_sync();  // the exchange buffers are reused by the next round
           }
         }
       } else {
-        int* s_tok = reinterpret_cast<int*>(gepi + 2 * C::SB * 64 * 4);  // [TC]
+        int* s_tok = reinterpret_cast<int*>(gepi + 4 * C::SB * 64 * 4);  // [TC]
         float* ys = p.ys + (int64_t)it.ks * p.P * p.d;               // this split's partial sums
         const int m = kBM * rt + row;                                // output feature
         const int ncol = min(kBM, p.d - kBM * rt);
