@@ -201,7 +201,7 @@ moe_status moe_forward(const moe_dims* dims, int32_t T, const uint16_t* x, const
  * that every replay records them.  The kernels of a call are, in order: route
  * (RMSNorm + router + top-k + E4M3 split of xe), group, pack (the token tiles' packed
  * activation blocks), gate_up, down, combine; on the GEMV path with T <= 64, route (which
- * then also groups), pack, gate_up and down (which then also combines).
+ * then also groups), pack, gate_up, down and combine.
  * Errors: as moe_forward; MOE_ERR_INVALID_ARG if n_events < 0 or events is NULL with
  * n_events > 0. */
 moe_status moe_forward_timed(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,

@@ -360,7 +360,8 @@ def workspace_view(ws: torch.Tensor, dims: moe_dims, T: int, field: str, dtype, 
 def moe_forward_timed(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales, ws,
                       y=None, events=None, stream=None):
     """moe_forward that records ``events`` (torch.cuda.Event, timing enabled) around each kernel:
-    event 2i before kernel i and 2i+1 after it (kernels: route, group, gather, gate_up, down, combine)."""
+    event 2i before kernel i and 2i+1 after it (kernels: route, group, pack, gate_up, down, combine;
+    small batches: route with the grouping, pack, gate_up, down, combine)."""
     _need(x, torch.bfloat16, "x")
     if y is None:
         y = torch.empty_like(x)

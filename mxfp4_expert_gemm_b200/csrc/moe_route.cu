@@ -349,7 +349,10 @@ __global__ void __launch_bounds__(kTokThreads) route_token_kernel(FwdArgs a) {
 // ----------------------------------------------------------------------------------
 constexpr int kRT = 16;                  // tokens per CTA
 constexpr int kTokenKernelMaxT = 256;    // up to this many tokens: one CTA per token
-constexpr int kRouteMmaMinCtas = 96;     // the tensor-core router from this many 128-token CTAs
+#ifndef MOE_ROUTE_MMA_MIN_CTAS
+#define MOE_ROUTE_MMA_MIN_CTAS 64
+#endif
+constexpr int kRouteMmaMinCtas = MOE_ROUTE_MMA_MIN_CTAS;   // the tensor-core router from this many 128-token CTAs
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
@@ -867,8 +870,9 @@ int launch_route_nj(const FwdArgs& a) {
     return 1;
   }
   // the tensor-core router keeps one CTA per 128 tokens busy for the whole reduction axis:
-  // it wins once the batch fills most of the SMs (16384 tokens: 0.33 ms against 0.55 ms);
-  // below that the 16-token tiles spread further (4096 tokens: 0.093 ms against 0.26 ms)
+  // it wins from about half the SMs (8192 tokens x 128 experts: 0.27 ms against 0.32 ms;
+  // 16384: 0.30 against 0.55); below that the 16-token tiles spread further (4096 tokens
+  // x 32 experts: 0.09 ms against 0.23 ms)
   if ((a.T + 127) / 128 >= kRouteMmaMinCtas && route_mma_fits(a.E, a.d)) return launch_route_mma(a);
   // chunk width and stages: the router rows of a stage stay within shared memory (up to 128
   // experts: 64-wide chunks; 128 experts take two stages of 34 KB, which measured faster

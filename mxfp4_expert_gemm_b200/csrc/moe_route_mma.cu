@@ -33,7 +33,8 @@ namespace {
 
 constexpr int kRM = 128;          // tokens per CTA (MMA M)
 constexpr int kRK = 32;           // reduction chunk: 32 fp32 per row, one 32-value block
-constexpr int kRThreads = 256;
+constexpr int kRThreads = 512;   // 16 warps: the per-chunk conversions are latency-bound chains
+constexpr int kXItems = kRM * 4 / kRThreads;   // activation items (8 values) per thread and chunk
 constexpr uint64_t kRWaitNs = 2000000000ull;
 
 __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
@@ -102,25 +103,41 @@ __global__ void __launch_bounds__(kRThreads, 1) route_mma_kernel(FwdArgs a, Rout
   }
   for (int i = tid * 4; i < d; i += kRThreads * 4)
     *reinterpret_cast<float4*>(s_g + i) = *reinterpret_cast<const float4*>(a.norm_w + i);
-  // 1 / rms of the CTA's tokens: warp w takes tokens 16w .. 16w + 15
-  for (int m = 16 * warp; m < 16 * warp + 16; ++m) {
-    float ss = 0.f;
-    if (m < nt) {
-      const uint16_t* xr = a.x + (int64_t)(t0 + m) * d;
-      for (int i = lane * 8; i < d; i += 256) {
-        const uint4 q = *reinterpret_cast<const uint4*>(xr + i);
-        const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+  // 1 / rms of the CTA's tokens: warp w takes tokens kRows w .. kRows w + kRows - 1, the
+  // loads of all its rows at one column step in flight together (each token's sum keeps its order: lane
+  // partial sums over the row, then the warp reduction)
+  {
+    constexpr int kRows = kRM / (kRThreads / 32);   // tokens per warp
+    float ss[kRows];
+#pragma unroll
+    for (int q = 0; q < kRows; ++q) ss[q] = 0.f;
+    for (int i = lane * 8; i < d; i += 256) {
+      uint4 v[kRows];
+#pragma unroll
+      for (int q = 0; q < kRows; ++q) {
+        const int m = kRows * warp + q;
+        v[q] = (m < nt) ? __ldg(reinterpret_cast<const uint4*>(a.x + (int64_t)(t0 + m) * d + i))
+                        : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int q = 0; q < kRows; ++q) {
+        const uint32_t wv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float lo = __uint_as_float(wv[j] << 16), hi = __uint_as_float(wv[j] & 0xFFFF0000u);
-          ss = fmaf(lo, lo, ss);
-          ss = fmaf(hi, hi, ss);
+          ss[q] = fmaf(lo, lo, ss[q]);
+          ss[q] = fmaf(hi, hi, ss[q]);
         }
       }
     }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) s_r[m] = m < nt ? 1.0f / sqrtf(ss / (float)d + a.eps) : 0.f;
+    for (int q = 0; q < kRows; ++q) {
+      float t = ss[q];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      const int m = kRows * warp + q;
+      if (lane == 0) s_r[m] = m < nt ? 1.0f / sqrtf(t / (float)d + a.eps) : 0.f;
+    }
   }
   ptx::fence_proxy_async_smem();
   __syncthreads();
@@ -128,23 +145,28 @@ __global__ void __launch_bounds__(kRThreads, 1) route_mma_kernel(FwdArgs a, Rout
   const uint32_t tmem = s_tmem;
   const uint32_t idesc = ptx::idesc_tf32(kRM, L.N);
 
-  // Raw loads of one chunk: x items (token m = i / 4, 8 values at 8 (i % 4)) for i = tid and
-  // tid + 256; W_r units (row e = j / 8, 4 values at 4 (j % 8)) for j = tid + 256 r.
+  // Raw loads of one chunk: x items (token m = i / 4, 8 values at 8 (i % 4)) for
+  // i = tid + kRThreads p; W_r units (row e = j / 8, 4 values at 4 (j % 8)) for
+  // j = tid + kRThreads r.
   constexpr int kWU = NJ * 32 * 8 / kRThreads > 0 ? NJ * 32 * 8 / kRThreads : 1;   // W units per thread
-  uint4 xraw[2];
-  float4 wraw[kWU];
-  auto load_chunk = [&](int c) {
+  // Three register buffers of raw loads, two chunks in flight while one is converted
+  // (the loop is unrolled by three so that every buffer keeps a fixed register name)
+  struct Raw {
+    uint4 x[kXItems];
+    float4 w[kWU];
+  };
+  auto load_chunk = [&](Raw& rb, int c) {
     const int k0 = c * kRK;
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
+    for (int p = 0; p < kXItems; ++p) {
       const int i = tid + kRThreads * p, m = i >> 2, g = i & 3;
-      xraw[p] = (m < nt) ? __ldg(reinterpret_cast<const uint4*>(a.x + (int64_t)(t0 + m) * d + k0 + 8 * g))
+      rb.x[p] = (m < nt) ? __ldg(reinterpret_cast<const uint4*>(a.x + (int64_t)(t0 + m) * d + k0 + 8 * g))
                          : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int r = 0; r < kWU; ++r) {
       const int j = tid + kRThreads * r, e = j >> 3, u = j & 7;
-      wraw[r] = (e < E) ? __ldg(reinterpret_cast<const float4*>(a.router_w + (int64_t)e * d + k0 + 4 * u))
+      rb.w[r] = (e < E) ? __ldg(reinterpret_cast<const float4*>(a.router_w + (int64_t)e * d + k0 + 4 * u))
                         : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
@@ -152,23 +174,18 @@ __global__ void __launch_bounds__(kRThreads, 1) route_mma_kernel(FwdArgs a, Rout
   bool ok = true;
   volatile int no_abort = 0;   // (the bounded waits' abort flag: unused here)
   int issued = -1;             // the last chunk whose MMAs were committed
-  load_chunk(0);
-  for (int c = 0; c < nch; ++c) {
+  // One chunk: convert it into stage c % 2 and issue its MMAs.  False when a wait gave up.
+  auto process = [&](int c, const Raw& cur) -> bool {
     const int s = c & 1, k0 = c * kRK;
     // the MMAs that read this stage two chunks ago are done
     if (c >= 2) ok = ptx::mbar_wait_bounded(&mma_done[s], (uint32_t)((c - 2) >> 1) & 1, &no_abort, kRWaitNs);
-    if (!__syncthreads_and(ok)) break;
-    uint4 xcur[2] = {xraw[0], xraw[1]};
-    float4 wcur[kWU];
-#pragma unroll
-    for (int r = 0; r < kWU; ++r) wcur[r] = wraw[r];
-    if (c + 1 < nch) load_chunk(c + 1);   // in flight while this chunk is converted
+    if (!__syncthreads_and(ok)) return false;
     // ---- activations: TF32 parts into A, the activation format into xq / xsf
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
+    for (int p = 0; p < kXItems; ++p) {
       const int i = tid + kRThreads * p, m = i >> 2, g = i & 3;
       const float r = s_r[m];
-      const uint32_t w4[4] = {xcur[p].x, xcur[p].y, xcur[p].z, xcur[p].w};
+      const uint32_t w4[4] = {cur.x[p].x, cur.x[p].y, cur.x[p].z, cur.x[p].w};
       float xn[8], hi[8], lo[8], xe[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -237,7 +254,7 @@ __global__ void __launch_bounds__(kRThreads, 1) route_mma_kernel(FwdArgs a, Rout
     for (int r = 0; r < kWU; ++r) {
       const int j = tid + kRThreads * r, e = j >> 3, u = j & 7;
       if (e < E) {
-        const float4 w = wcur[r];
+        const float4 w = cur.w[r];
         const float4 h = make_float4(ptx::to_tf32(w.x), ptx::to_tf32(w.y), ptx::to_tf32(w.z), ptx::to_tf32(w.w));
         const float4 l = make_float4(ptx::to_tf32(w.x - h.x), ptx::to_tf32(w.y - h.y), ptx::to_tf32(w.z - h.z),
                                      ptx::to_tf32(w.w - h.w));
@@ -263,6 +280,18 @@ __global__ void __launch_bounds__(kRThreads, 1) route_mma_kernel(FwdArgs a, Rout
       __syncwarp();
     }
     issued = c;
+    return true;
+  };
+  Raw r0, r1, r2;
+  load_chunk(r0, 0);
+  if (nch > 1) load_chunk(r1, 1);
+  for (int c = 0; c < nch; c += 3) {
+    if (c + 2 < nch) load_chunk(r2, c + 2);
+    if (!process(c, r0) || c + 1 >= nch) break;
+    if (c + 3 < nch) load_chunk(r0, c + 3);
+    if (!process(c + 1, r1) || c + 2 >= nch) break;
+    if (c + 4 < nch) load_chunk(r1, c + 4);
+    if (!process(c + 2, r2)) break;
   }
   // the last committed chunk's MMAs (and with them all earlier ones) are done
   if (issued >= 0) {
@@ -287,8 +316,9 @@ __global__ void __launch_bounds__(kRThreads, 1) route_mma_kernel(FwdArgs a, Rout
       }
     }
     __syncthreads();
-    // ---- top-k + softmax: warp w takes tokens 16w .. 16w + 15
-    for (int m = 16 * warp; m < 16 * warp + 16 && m < nt; ++m) {
+    // ---- top-k + softmax: warp w takes tokens kTokPerWarp w .. kTokPerWarp (w + 1) - 1
+    constexpr int kTokPerWarp = kRM / (kRThreads / 32);
+    for (int m = kTokPerWarp * warp; m < kTokPerWarp * (warp + 1) && m < nt; ++m) {
       float l[NJ];
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
