@@ -271,7 +271,7 @@ int32_t moe_resolve_path(const moe_dims* dims, int32_t T);
  *     the GEMV path, 96 on the GEMM path) or, with MOE_ACT_MXFP8, its BN rows (one per
  *     token; BN = 16 / 192), in the tensor cores' 128-byte-swizzled order, then their
  *     scales,
- * ys  [S][T*k][d] fp32 (weighted expert outputs, sorted order; S = 6 planes of partial sums
+ * ys  [S][T*k][d] fp32 (weighted expert outputs, row t*k + slot; S = 6 planes of partial sums
  *     on the GEMV path, whose down GEMM splits its reduction axis in up to six, else 1);
  * offsets[MOE_WS_FIELDS-1] = total bytes.  Errors: MOE_ERR_INVALID_ARG,
  * MOE_ERR_UNSUPPORTED_SHAPE. */

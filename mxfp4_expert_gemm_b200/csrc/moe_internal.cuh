@@ -122,7 +122,7 @@ struct WsLayout {
   size_t bpx;       // packed blocks [max_tiles][dp/128] of xe per token tile (gate_up's B)
   size_t bph;       // packed blocks [max_tiles][ip/128] of h per token tile (down's B)
   size_t ys;        // f32 [ksplit][P][d]  routing-weighted expert outputs (partial sums per
-                    // reduction-axis split of the down GEMM), sorted order
+                    // reduction-axis split of the down GEMM), row t * k + slot of pair (t, slot)
   size_t total;
   int64_t max_tiles;
   int32_t tile_tokens;

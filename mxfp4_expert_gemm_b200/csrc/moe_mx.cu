@@ -72,8 +72,8 @@ struct MxParams {
   // gate_up output: h as packed activation blocks of the down GEMM [tiles][KCo][block]
   uint8_t* bp_out;
   int32_t KCo;             // 128-chunks of I
-  // down output: ys [ksplit][P][d] fp32 = w * (partial) o; optionally
-  // y = bf16(x + sum_j sum_s ys[s][inv[t*k + j]]) by the last writer of each (token,
+  // down output: ys [ksplit][P][d] fp32 = w * (partial) o, row t * k + slot; optionally
+  // y = bf16(x + sum_j sum_s ys[s][t*k + j]) by the last writer of each (token,
   // 128-column) block
   float* ys;
   int32_t d;
@@ -618,7 +618,8 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
             if (c < nt && m < p.d) {
               const int64_t prow = tl.row0 + jbase + c;
               const float o = token_acc<TERMS>(v, c);
-              float* q = ys + prow * p.d + m;
+              // the row of pair t * k + slot: each token's k outputs are consecutive rows
+              float* q = ys + (int64_t)__ldg(p.perm + prow) * p.d + m;
               if (in_bounds(q, p.ys, p.ys_end, p.status)) *q = o * p.w_sorted[prow];
             }
           }
@@ -648,7 +649,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
                   float part[kMaxParts];
 #pragma unroll
                   for (int q = 0; q < kMaxParts; ++q)   // part q: slot q / ksplit, split q % ksplit
-                    if (q < p.k * ksplit) srow[q] = p.inv[(int64_t)tok * p.k + q / ksplit];
+                    if (q < p.k * ksplit) srow[q] = tok * p.k + q / ksplit;
 #pragma unroll
                   for (int q = 0; q < kMaxParts; ++q)
                     if (q < p.k * ksplit)
@@ -658,7 +659,7 @@ __global__ void __launch_bounds__(MxCfg<BN, NP, S, CPS, EG, NPW, TERMS, FP4, CG>
                     if (q < p.k * ksplit) accv += part[q];
                 } else {
                   for (int j = 0; j < p.k; ++j) {
-                    const int srow1 = p.inv[(int64_t)tok * p.k + j];
+                    const int srow1 = tok * p.k + j;
                     for (int sp = 0; sp < ksplit; ++sp)
                       accv += __ldcg(p.ys + ((int64_t)sp * p.P + srow1) * p.d + gc);
                   }

@@ -710,7 +710,7 @@ __global__ void pack_kernel(FwdArgs a) {
   }
 }
 
-// y[t] = bf16(x[t] + sum_j sum_s ys[s][inv[t*k + j]]), j in slot order, then split order;
+// y[t] = bf16(x[t] + sum_j sum_s ys[s][t*k + j]), j in slot order, then split order;
 // with y_partial the fp32 sum alone (no residual: one rank's slice of the intermediate
 // features, summed over the ranks afterwards).
 __global__ void combine_kernel(FwdArgs a) {
@@ -730,7 +730,7 @@ __global__ void combine_kernel(FwdArgs a) {
       v[3] = __uint_as_float(xr.y & 0xFFFF0000u);
     }
     for (int j = 0; j < a.k; ++j) {
-      const int p = a.ws.inv[(int64_t)t * a.k + j];
+      const int64_t p = (int64_t)t * a.k + j;   // the down GEMM writes pair t * k + j's row there
       for (int sp = 0; sp < ksplit; ++sp) {   // partial sums of a split down GEMM
         const float4 o = *reinterpret_cast<const float4*>(a.ws.ys + (sp * P + p) * a.d + i4);
         v[0] += o.x;
@@ -754,7 +754,7 @@ __global__ void combine_kernel(FwdArgs a) {
 // Rows that finish a block: y = bf16(x + s) and, with norm_w, the next block's RMSNorm of
 // it, y_norm = bf16(y / sqrt(mean(y^2) + eps) * norm_w) on the bf16 y (each block holds two
 // RMSNorms: "Transformer 块" of the ewbang.com GPT-OSS article).  s is either the sum of the
-// token's k expert outputs (ys through inv, slot order then split order, as combine_kernel)
+// token's k expert outputs (its k consecutive rows of ys, slot order then split order, as combine_kernel)
 // or a dense fp32 row (the all-reduced partial outputs of the ranks that hold slices of the
 // intermediate features).  One CTA of 256 threads per row; the row's sum of squares is a
 // block reduction in fixed order.
@@ -789,7 +789,7 @@ __global__ void __launch_bounds__(kFinishThreads) finish_rows_kernel(FinishArgs 
                     __uint_as_float(xr.y & 0xFFFF0000u)};
       if (f.ys) {
         for (int j = 0; j < f.k; ++j) {
-          const int p = f.inv[(int64_t)t * f.k + j];
+          const int64_t p = (int64_t)t * f.k + j;
           for (int sp = 0; sp < ks; ++sp) {
             const float4 o = *reinterpret_cast<const float4*>(f.ys + (sp * f.P + p) * f.d + i4);
             v[0] += o.x;
