@@ -14,22 +14,27 @@
 // pairs (TERMS = 2); with MXFP8 activations a token is one column (TERMS = 1).
 //
 // Persistent kernel, CPS CTAs per SM.  A work item is 128 weight rows x one token tile
-// over the whole reduction axis; CTA b takes items b, b + grid, ...  A pipeline stage
-// covers NP chunks of 128 along the reduction axis:
+// over the whole reduction axis (or a split of it); CTA b takes items b, b + grid, ...
+// With CG = 2 (large batches) two CTAs of a cluster share each MMA of M = 256: a pair
+// takes two consecutive row tiles of an item, each CTA holding its weight rows and half
+// of the token tile's activation rows (the CG == 2 branches below).  A pipeline stage covers NP
+// chunks of 128 along the reduction axis:
 //   warps 0..  producers: per stage one TMA load of the weight codes (NP consecutive
 //              8 KB tile blocks; E2M1, unpacked by the copy to one byte per code in
 //              shared memory, 128B swizzle), one bulk copy of the token tile's packed
 //              activation blocks (TERMS*BN E4M3 rows per chunk, already in the swizzled order,
 //              followed by their scale factors) and one bulk copy of the weight scale
-//              factors (stored in the tensor cores' scale-factor layout);
-//   warp 1     TMEM allocation and the MMA issuer (one thread): per stage it copies the
-//              scale factors into TMEM (tcgen05.cp) and issues one block-scaled MMA
-//              per 32-wide block of the reduction axis;
-//   warps 2.. epilogue, EG warpgroups taking alternate 32-column reads: read the fp32
+//              factors (stored in the tensor cores' scale-factor layout); pairs load the
+//              same by tile copies that complete on the leader's barrier;
+//   warp NPW   TMEM allocation and the MMA issuer (one elected thread): per stage it
+//              copies the scale factors into TMEM (tcgen05.cp) and issues one block-scaled
+//              MMA per 32-wide block of the reduction axis (pairs: the leader's only);
+//   then       epilogue, EG warpgroups taking alternate 32-column reads: read the fp32
 //              accumulator (double-buffered in TMEM so that it overlaps the next item's
-//              main loop), gate_up: SwiGLU and the E4M3 split of h for the down GEMM;
-//              down: routing weight, and for small batches the combine
-//              y = x + sum_j w_j o_j.
+//              main loop), gate_up: SwiGLU and the activation split of h for the down
+//              GEMM; down: the routing weight, into the pair's row of ys (a build with
+//              MOE_GEMV_FUSE_COMBINE=1 also combines y = x + sum_j w_j o_j there for
+//              small batches; by default the combine is its own pass).
 // Gate_up weights are stored in 128-row tiles of 64 gate rows (TMEM lanes 0..63) and the
 // 64 matching up rows (lanes 64..127), so g and u of one feature meet in the epilogue.
 //
