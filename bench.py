@@ -4,7 +4,7 @@
 A step is one ``moe_forward`` over one batch of tokens (RMSNorm, router, top-k,
 grouping, gate_up + SwiGLU, down + weighted combine + residual).  Inputs are
 seeded synthetic tensors of the workload's shapes (``synth``) and are resident
-in HBM before the timed region; the L2 is flushed (256 MiB write) before every
+in HBM before the timed region; the L2 is flushed (256 MiB write, then a 256 MiB read) before every
 step, outside the step's events.
 
 The line is headlined by the largest single-GPU workload, the skewed-routing
@@ -326,6 +326,27 @@ def cpu_tokens_per_call(cfg):
 # ------------------------------------------------------------------------------ our arm
 
 
+class L2Flush:
+    """Before every step: write a 256 MiB buffer (twice the L2), then read another one.
+    The write evicts everything the previous step left in L2; the read evicts the write's
+    own dirty lines (written back here, outside the step's events) so that the step does
+    not pay for the flush's write-backs.  The step starts with nothing of its own in L2."""
+
+    def __init__(self, device="cuda"):
+        import torch
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        self.r = torch.zeros(256 << 20, dtype=torch.uint8, device=device)
+
+    def __call__(self):
+        import torch
+        self.w.zero_()
+        torch.sum(self.r, dtype=torch.int32)
+
+
+L2_TEXT = ("flushed before every step: a 256 MiB write, then a 256 MiB read that writes the "
+           "dirty lines back (both outside the step events)")
+
+
 def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
     """One workload: timed steps (graph replay), per-kernel times, roofline, end to end,
     clocks and the CPU oracle baseline.  Returns the workload's record."""
@@ -335,7 +356,7 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
     dims = moe.make_dims(cfg.d, cfg.I, cfg.E, cfg.k, cfg.rms_eps, cfg.swiglu_limit, path=args.path, act=args.act)
     ws = moe.new_workspace(dims, cfg.T)
     y = torch.empty_like(inp["x_dev"])
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     W = inp["W"]
     fwd = (dims, inp["x_dev"], inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws)
 
@@ -343,7 +364,7 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
         moe.moe_forward(*fwd, y=y)
 
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush()
         plain_step()
     torch.cuda.synchronize()
     st = moe.moe_device_status(ws)
@@ -372,7 +393,7 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
     # ---- timed region: the layer as a user runs it (one graph replay per step)
     with ClockSampler(local_rank) as clk:
         for i in range(K):
-            flush.zero_()
+            flush()
             starts[i].record()
             if use_graph:
                 graph.replay()
@@ -409,7 +430,7 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
     names = {len(KERNELS): KERNELS, len(KERNELS_FUSED_GROUP): KERNELS_FUSED_GROUP}.get(n_timed, KERNELS_FUSED)
     per_kernel = {name: [] for name in names[:n_timed]}
     for i in range(K):
-        flush.zero_()
+        flush()
         if use_graph:
             kgraph.replay()
         else:
@@ -448,7 +469,7 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
         pg.barrier()
     torch.cuda.synchronize()
     for i in range(K):
-        flush.zero_()
+        flush()
         e_starts[i].record()
         if use_graph:
             e2e_graph.replay()
@@ -514,7 +535,7 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
                    "global_batch": cfg.T * world, "path": path_used, "parallelism": f"dp{world}",
                    "activations": ("bf16, exact (each value carried into the MMA as two E4M3 terms)"
                                    if args.act == "bf16" else "MXFP8 (E4M3 in 32-value blocks)"),
-                   "l2": "flushed before every step (256 MiB write, outside the step events)",
+                   "l2": L2_TEXT,
                    "timing": "sum of per-step CUDA events on the launching stream; max over ranks",
                    "launch": "CUDA graph replay per step" if use_graph else "host launches per step",
                    "kernel_timing": "separate pass of the same steps with CUDA events around each kernel"},
@@ -554,7 +575,7 @@ def measure_tp(cfg, args, rank, world, local_rank, pg):
     ws = moe.new_workspace(dims, cfg.T)
     part = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device=dev)
     y = torch.empty_like(x_dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def step():
         moe.moe_forward_partial(dims, x_dev, gamma, rw, rb, *W, ws, y_partial=part)
@@ -565,7 +586,7 @@ def measure_tp(cfg, args, rank, world, local_rank, pg):
         return n + moe.last_launch_count()
 
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     if moe.moe_device_status(ws) != moe.MOE_OK:
@@ -579,7 +600,7 @@ def measure_tp(cfg, args, rank, world, local_rank, pg):
     launches = 0
     with ClockSampler(local_rank) as clk:
         for i in range(K):
-            flush.zero_()
+            flush()
             starts[i].record()
             launches += step()
             stops[i].record()
@@ -595,7 +616,7 @@ def measure_tp(cfg, args, rank, world, local_rank, pg):
             "config": {"workload": WORKLOAD_TEXT[cfg.name], "name": cfg.name, "global_batch": cfg.T,
                        "parallelism": f"tp{world}", "slice": [i0, i1], "path": moe.resolved_path(dims, cfg.T),
                        "collective": "NCCL all-reduce (sum) of the fp32 partial outputs [T, d] per step",
-                       "l2": "flushed before every step (256 MiB write, outside the step events)",
+                       "l2": L2_TEXT,
                        "timing": "sum of per-step CUDA events on the launching stream; max over ranks",
                        "launch": "host launches per step"},
             "gpu_launches": launches, "clocks": clk.summary()}
