@@ -185,7 +185,10 @@ moe_status moe_route(const moe_dims* dims, int32_t T, const uint16_t* x, const f
  * per 32 values each: hi = RN(v / 2^s1), lo = RN((v - hi * 2^s1) / 2^s2), s1 and s2 set by
  * the largest |v| and the largest residual of the block.  hi + lo equals v whenever
  * |v| >= 2^-13 * max|block|; smaller values are off by at most 2^-20 * max|block|.  With
- * MOE_ACT_MXFP8 the hi term alone enters (see moe_act_format).
+ * MOE_ACT_MXFP8 the hi term alone enters, with MOE_ACT_MXFP4 E2M1 codes (FP4 x FP4 MMA; see
+ * moe_act_format).  The k routing-weighted expert outputs stay fp32 and are added to the
+ * residual in a fixed order (slot, then reduction-axis split): results do not depend on
+ * scheduling, and repeated calls give identical y.
  * Errors: as moe_route. */
 moe_status moe_forward(const moe_dims* dims, int32_t T, const uint16_t* x, const float* norm_w,
                        const float* router_w, const float* router_b, const uint8_t* w1_codes,
