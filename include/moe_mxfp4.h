@@ -301,7 +301,7 @@ int32_t moe_last_launch_count(void);
  * implicit synchronization once it is running -- use it instead of moe_forward.
  * Scratch: a fixed 16 MiB array in the library's own device memory, present on every GPU
  * that loads the library until the process exits.  T whose moe_workspace_bytes() exceed
- * 16 MiB is rejected with MOE_ERR_WORKSPACE (at d = I = 2880, E = 32, top-4: up to 56
+ * 16 MiB is rejected with MOE_ERR_WORKSPACE (at d = I = 2880, E = 32, top-4: up to 34
  * tokens).
  * The first call in a CUDA context (normally a device's primary context) looks up the
  * array's device address in that context (cudaGetSymbolAddress) and remembers it for that
