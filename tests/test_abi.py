@@ -68,7 +68,12 @@ def _call_forward(L, dims, T, ptr=256, ws_bytes=1 << 40):
 def test_argument_checks_before_device(L):
     ok = moe.make_dims(2880, 2880, 32, 4)
     assert _call_forward(L, moe.make_dims(2880, 2880, 32, 4, block=16), 4) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    # d and I in whole multiples of 64 (the library's rule; the pages' block is 32): odd
+    # multiples of 32 are refused, for either dimension, before anything runs
     assert _call_forward(L, moe.make_dims(2880 + 32, 2880, 32, 4), 4) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert _call_forward(L, moe.make_dims(2880, 2880 + 32, 32, 4), 4) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert _call_forward(L, moe.make_dims(96, 160, 4, 2), 4) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert moe.moe_workspace_bytes(moe.make_dims(96, 128, 4, 2), 4) == 0
     assert _call_forward(L, moe.make_dims(2880, 2880, 32, 33), 4) == moe.MOE_ERR_UNSUPPORTED_SHAPE
     assert _call_forward(L, moe.make_dims(2880, 2880, 300, 4), 4) == moe.MOE_ERR_UNSUPPORTED_SHAPE
     assert _call_forward(L, moe.make_dims(2880, 2880, 4, 5), 4) == moe.MOE_ERR_UNSUPPORTED_SHAPE
