@@ -326,6 +326,20 @@ def cpu_tokens_per_call(cfg):
 # ------------------------------------------------------------------------------ our arm
 
 
+ACT_DTYPE = {"bf16": "mxfp4xbf16", "mxfp8": "mxfp4xmxfp8", "mxfp4": "mxfp4xmxfp4"}
+ACT_NOTE = {
+    "bf16": ("MXFP4 (E2M1 + E8M0) weights x bf16 activations, each carried into the tensor cores as two E4M3 "
+             "terms with their block scales; fp32 accumulation"),
+    "mxfp8": "MXFP4 weights x MXFP8 (E4M3) activations; fp32 accumulation",
+    "mxfp4": "MXFP4 weights x MXFP4 (E2M1) activations (FP4 x FP4 MMA); fp32 accumulation",
+}
+ACT_TEXT = {
+    "bf16": "bf16, exact (each value carried into the MMA as two E4M3 terms)",
+    "mxfp8": "MXFP8 (E4M3 in 32-value blocks)",
+    "mxfp4": "MXFP4 (E2M1 in 32-value blocks, the weights' rule)",
+}
+
+
 class L2Flush:
     """Before every step: write a 256 MiB buffer (twice the L2), then read another one.
     The write evicts everything the previous step left in L2; the read evicts the write's
@@ -495,7 +509,10 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
     layer_ms = total_ms / K
     traffic = ncu_traffic("gate_up", cfg.name, args.act)
     if (P / cfg.E) <= 24:   # few tokens per expert: the weight stream bounds the layer
-        alg = used * w1_bytes + P * d * 2 + P * I * 2   # expert weights streamed once + activations in / out
+        # expert weights streamed once + activations in / out (bf16: two E4M3 bytes per value;
+        # MXFP8: one; MXFP4: half; block scales not counted)
+        act_b = {"bf16": 2.0, "mxfp8": 1.0, "mxfp4": 0.5}[args.act]
+        alg = int(used * w1_bytes + act_b * (P * d + P * I))
         achieved = alg / (gu_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "kernel": "gate_up (mx_expert_kernel<GATE_UP>)", "achieved": round(achieved, 1),
@@ -511,16 +528,22 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
         achieved = alg / (gu_ms * 1e-3) / 1e12
         fp8_peak = round(RATE_VS_BF16["fp8"] * peaks["bf16_tflops"], 1)
         fp4_peak = round(RATE_VS_BF16["fp4"] * peaks["bf16_tflops"], 1)
-        cols = 1 if args.act == "mxfp8" else 2   # E4M3 MMA columns per token
+        cols = 2 if args.act == "bf16" else 1   # MMA columns per token
+        # the MMA's own rate: E2M1 x E4M3 (kind::mxf8f6f4) at the fp8 rate, FP4 x FP4 (kind::mxf4)
+        # at the FP4 rate
+        fp4_mma = args.act == "mxfp4"
+        mma_peak = fp4_peak if fp4_mma else fp8_peak
         roof = {"bound": "tensor", "kernel": "gate_up (mx_expert_kernel<GATE_UP>)", "achieved": round(achieved, 1),
-                "peak": fp8_peak, "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4), "traffic": traffic,
+                "peak": mma_peak, "unit": "TFLOP/s", "frac": round(achieved / mma_peak, 4), "traffic": traffic,
                 "algorithmic_flops_per_launch": alg, "launch_ms": round(gu_ms, 5),
-                "peak_source": f"2 x bf16_tflops burst ({peak_src}): the block-scaled E2M1 x E4M3 MMA "
-                               "(kind::mxf8f6f4) runs at the fp8 rate",
-                "mma_flops_per_launch": cols * alg, "mma_frac": round(cols * achieved / fp8_peak, 4),
+                "peak_source": (f"4 x bf16_tflops burst ({peak_src}): the FP4 x FP4 MMA (kind::mxf4) runs at "
+                                "the FP4 rate" if fp4_mma else
+                                f"2 x bf16_tflops burst ({peak_src}): the block-scaled E2M1 x E4M3 MMA "
+                                "(kind::mxf8f6f4) runs at the fp8 rate"),
+                "mma_flops_per_launch": cols * alg, "mma_frac": round(cols * achieved / mma_peak, 4),
                 "mma_note": ("each bf16 activation enters the MMA as two E4M3 columns (hi and lo terms), so the "
                              "MMA executes 2x the algorithmic flops" if cols == 2 else
-                             "MXFP8 activations: one E4M3 column per token"),
+                             "one MMA column per token"),
                 "frac_of_fp4_peak": round(achieved / fp4_peak, 4),
                 "fp4_peak": fp4_peak, "fp4_peak_source": f"4 x bf16_tflops burst ({peak_src})"}
         layer_flops = 6 * d * I * P
@@ -533,8 +556,7 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
         "ms_per_step": round(total_ms / K, 5),
         "config": {"workload": WORKLOAD_TEXT[cfg.name], "name": cfg.name, "tokens_per_gpu": cfg.T,
                    "global_batch": cfg.T * world, "path": path_used, "parallelism": f"dp{world}",
-                   "activations": ("bf16, exact (each value carried into the MMA as two E4M3 terms)"
-                                   if args.act == "bf16" else "MXFP8 (E4M3 in 32-value blocks)"),
+                   "activations": ACT_TEXT[args.act],
                    "l2": L2_TEXT,
                    "timing": "sum of per-step CUDA events on the launching stream; max over ranks",
                    "launch": "CUDA graph replay per step" if use_graph else "host launches per step",
@@ -637,7 +659,7 @@ def run_ours(args, rank, world, local_rank):
         line = {"metric": METRIC, "value": rec["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": max(3, args.warmup), "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
                 "scaling": "strong", "vs_baseline": None,
-                "dtype": "mxfp4xbf16" if args.act == "bf16" else "mxfp4xmxfp8", "data": "synthetic",
+                "dtype": ACT_DTYPE[args.act], "data": "synthetic",
                 "config": rec["config"], "gpu_launches": rec["gpu_launches"], "clocks": rec["clocks"]}
         if rank == 0:
             print(json.dumps(line), flush=True)
@@ -651,10 +673,8 @@ def run_ours(args, rank, world, local_rank):
     line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "mxfp4xbf16" if args.act == "bf16" else "mxfp4xmxfp8",
-            "dtype_note": ("MXFP4 (E2M1 + E8M0) weights x bf16 activations, each carried into the tensor cores "
-                           "as two E4M3 terms with their block scales; fp32 accumulation"
-                           if args.act == "bf16" else "MXFP4 weights x MXFP8 (E4M3) activations; fp32 accumulation"),
+            "dtype": ACT_DTYPE[args.act],
+            "dtype_note": ACT_NOTE[args.act],
             "data": "synthetic"}
     for key in ("config", "kernel_ms", "roofline", "e2e", "gpu_launches", "clocks", "cpu_baseline"):
         if key in head:
