@@ -82,6 +82,8 @@ def parse(argv=None):
     ap.add_argument("--no-graph", action="store_true", help="launch every step from the host instead of "
                     "replaying a captured CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget per workload")
+    ap.add_argument("--e2e-chunk", type=int, default=0,
+                    help="tokens per chunk of the end-to-end call (0: the library's choice)")
     ap.add_argument("--tp", action="store_true",
                     help="tensor parallelism over the intermediate features: every rank holds a slice of I "
                          "for all experts and runs the whole batch; one all-reduce of the partial outputs")
@@ -459,18 +461,25 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
     kern_ms = {name: statistics.mean(v) for name, v in per_kernel.items()}
     total_ms = max_over_ranks(total_ms, pg)
 
-    # ---- end to end through the public API with host buffers (pinned)
+    # ---- end to end through the public API with host buffers (pinned): moe_forward_host
+    # stages x and y through the device in chunks whose copies, on their own streams,
+    # overlap the layer of the neighbouring chunks
     x_host = torch.empty(inp["x_dev"].shape, dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(inp["x_dev"].cpu())
     y_host = torch.empty_like(x_host, pin_memory=True)
     e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     e_stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     x_dev2 = torch.empty_like(inp["x_dev"])
+    chunk = min(args.e2e_chunk or moe.moe_host_chunk_tokens(dims, cfg.T), cfg.T)
+    n_chunks = (cfg.T + chunk - 1) // chunk
+    last = cfg.T - (n_chunks - 1) * chunk
+    need = max(moe.moe_workspace_bytes(dims, chunk), moe.moe_workspace_bytes(dims, last))
+    ws_e2e = ws if ws.numel() >= need else torch.zeros(need, dtype=torch.uint8, device=ws.device)
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
 
     def e2e_step():
-        x_dev2.copy_(x_host, non_blocking=True)
-        moe.moe_forward(dims, x_dev2, inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws, y=y)
-        y_host.copy_(y, non_blocking=True)
+        moe.moe_forward_host(dims, x_host, inp["gamma_dev"], inp["rw_dev"], inp["rb_dev"], *W, ws_e2e, x_dev2, y,
+                             y_host=y_host, chunk_tokens=chunk, h2d_stream=h2d, d2h_stream=d2h)
 
     e2e_graph = None
     if use_graph:
@@ -495,6 +504,7 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
     e2e_ms = max_over_ranks(e2e_ms, pg)
     del e2e_graph
     assert moe.moe_device_status(ws) == moe.MOE_OK
+    assert moe.moe_device_status(ws_e2e) == moe.MOE_OK
 
     # ---- roofline of the dominant kernel (gate_up) and of the layer
     peaks, peak_src = load_peaks()
@@ -564,11 +574,13 @@ def measure(cfg, args, rank, world, local_rank, pg, want_cpu):
         "kernel_ms": {k_: round(v, 5) for k_, v in kern_ms.items()},
         "roofline": roof,
         "e2e": {"value": round(job_throughput(cfg.T, world, K, e2e_ms), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(inp["x_dev"].numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
+                "h2d_bytes_per_step": int(inp["x_dev"].numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2),
+                "api": "moe_forward_host (pinned host x in, pinned host y out)", "chunks": n_chunks,
+                "chunk_tokens": chunk},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
-    del ws, flush, W, inp["W"]
+    del ws, ws_e2e, flush, W, inp["W"]
     if want_cpu:
         n = cpu_tokens_per_call(cfg)
         v, cores, sample = time_oracle(cfg, oracle_inputs(cfg, inp["x"], np.arange(n)), n,

@@ -28,8 +28,10 @@
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers unless stated otherwise; the caller
- *     owns and allocates every buffer.  The library allocates and frees nothing;
- *     besides a per-host-thread launch counter it keeps no state between calls.
+ *     owns and allocates every buffer.  The library allocates and frees no device
+ *     memory; besides a per-host-thread launch counter, the per-host-thread CUDA
+ *     events of moe_forward_host and the scratch address of moe_forward_no_alloc it
+ *     keeps no state between calls.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous on that stream.  The returned status covers the synchronous
  *     argument checks and launch errors only; errors the kernels detect (a
@@ -256,6 +258,41 @@ moe_status moe_forward_partial(const moe_dims* dims, int32_t T, const uint16_t* 
  * MOE_ERR_UNSUPPORTED_SHAPE (d not a multiple of 64), MOE_ERR_DEVICE, MOE_ERR_CUDA. */
 moe_status moe_residual_norm(int32_t T, int32_t d, const uint16_t* x, const float* s, const float* norm_w,
                              float eps, uint16_t* y, uint16_t* y_norm, void* stream);
+
+/* moe_forward from host memory to host memory, with the copies overlapped with the layer.
+ *   x_host, y_host [T][d] bf16, host memory, page-locked (cudaHostAlloc / cudaHostRegister)
+ *                  for the copies to overlap, and required when `stream` is being captured
+ *   x_dev, y_dev   [T][d] bf16, device buffers the call stages through (distinct)
+ * The other arguments are moe_forward's (device pointers).  The T tokens run as consecutive
+ * chunks of chunk_tokens tokens (the last one shorter; 0 = the library's choice, which
+ * moe_host_chunk_tokens returns).  With one chunk the copy in, the layer and the copy out
+ * run in order on `stream`.  With several, chunk c is copied in on h2d_stream, its layer
+ * runs on `stream` and it is copied out on d2h_stream, so that the copies of the chunks
+ * before and after it overlap its layer (PCIe carries both directions at once); the copies
+ * in first wait for the work enqueued on `stream` before the call, and `stream` waits for
+ * the last copy out at the end.  NULL h2d_stream / d2h_stream: those copies run on
+ * `stream` too.  The call returns once everything is enqueued; y_host is complete when
+ * `stream` has passed the call (the caller synchronizes).  A token's routing and expert
+ * outputs do not depend on the other tokens of its batch, so y_host is moe_forward's y of
+ * each chunk; the down GEMM's split of its reduction axis follows the chunk's tile count,
+ * so y may differ in the last bf16 bit from a single moe_forward over all T tokens (both
+ * follow the layer's definition within the same bound).  ws: moe_workspace_bytes(dims,
+ * chunk) bytes at least (and for the last chunk's size), reused chunk after chunk.
+ * The kernels count as in moe_forward, summed over the chunks.  Everything is enqueued
+ * per chunk on the caller's streams; the call allocates nothing on the device.
+ * Errors: as moe_forward, checked before anything is enqueued; MOE_ERR_INVALID_ARG for
+ * chunk_tokens < 0 or a null / misaligned / aliased x_dev or y_dev; MOE_ERR_WORKSPACE when
+ * ws is smaller than a chunk needs. */
+moe_status moe_forward_host(const moe_dims* dims, int32_t T, const uint16_t* x_host, uint16_t* y_host,
+                            uint16_t* x_dev, uint16_t* y_dev, const float* norm_w, const float* router_w,
+                            const float* router_b, const uint8_t* w1_codes, const uint8_t* w1_scales,
+                            const uint8_t* w2_codes, const uint8_t* w2_scales, void* ws, size_t ws_bytes,
+                            int32_t chunk_tokens, void* stream, void* h2d_stream, void* d2h_stream);
+
+/* Tokens per chunk that moe_forward_host takes for chunk_tokens = 0: all T (one chunk) on
+ * the small-batch path and below 4096 tokens, else ceil(T / n) for n = min(4, T / 2048)
+ * chunks.  Returns -1 for invalid dims. */
+int32_t moe_host_chunk_tokens(const moe_dims* dims, int32_t T);
 
 /* The path moe_forward takes for these dims and T: dims->path, or for MOE_PATH_AUTO the
  * choice it makes (MOE_PATH_GEMV when T*top_k/E <= 24 tokens per expert, else

@@ -136,6 +136,10 @@ def load_library(path: str):
     L.moe_residual_norm.restype = ctypes.c_int
     L.moe_forward_no_alloc.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_forward_no_alloc.restype = ctypes.c_int
+    L.moe_forward_host.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, vp, vp, vp]
+    L.moe_forward_host.restype = ctypes.c_int
+    L.moe_host_chunk_tokens.argtypes = [dp, i32]
+    L.moe_host_chunk_tokens.restype = i32
     L.moe_debug_inject_timeout.argtypes = [i32]
     L.moe_debug_inject_timeout.restype = None
     L.moe_last_launch_count.argtypes = []
@@ -270,6 +274,43 @@ def moe_forward(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scal
                              _ptr(r["counts"]) if r else None, _ptr(ws), ws.numel(), _stream(stream)),
            "moe_forward")
     return (y, r) if want_routing else y
+
+
+def moe_host_chunk_tokens(dims: moe_dims, T: int) -> int:
+    """Tokens per chunk moe_forward_host takes when left to choose (T for one chunk)."""
+    n = lib().moe_host_chunk_tokens(ctypes.byref(dims), T)
+    if n < 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_host_chunk_tokens")
+    return n
+
+
+def _need_host(t: torch.Tensor, name, shape):
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError(f"{name}: a host (CPU) tensor is required")
+    if t.dtype != torch.bfloat16 or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: a contiguous bf16 tensor of shape {tuple(shape)} is required")
+
+
+def moe_forward_host(dims: moe_dims, x_host, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales,
+                     ws, x_dev, y_dev, y_host=None, chunk_tokens=0, h2d_stream=None, d2h_stream=None, stream=None):
+    """y_host [T, d] bf16 (host, page-locked) = x_host + MoE(RMSNorm(x_host)), staged through the
+    device buffers x_dev / y_dev [T, d] in chunks whose copies overlap the layer (h2d_stream and
+    d2h_stream carry the copies; None runs them on `stream`).  Returns y_host once enqueued:
+    synchronize `stream` before reading it."""
+    T, d = x_host.shape
+    _need_host(x_host, "x_host", (T, d))
+    if y_host is None:
+        y_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
+    _need_host(y_host, "y_host", (T, d))
+    _need(x_dev, torch.bfloat16, "x_dev", (T, d))
+    _need(y_dev, torch.bfloat16, "y_dev", (T, d))
+    hs = ctypes.c_void_p(h2d_stream.cuda_stream) if h2d_stream is not None else None
+    ds = ctypes.c_void_p(d2h_stream.cuda_stream) if d2h_stream is not None else None
+    _check(lib().moe_forward_host(ctypes.byref(dims), T, _ptr(x_host), _ptr(y_host), _ptr(x_dev), _ptr(y_dev),
+                                  _ptr(norm_w), _ptr(router_w), _ptr(router_b), _ptr(w1_codes), _ptr(w1_scales),
+                                  _ptr(w2_codes), _ptr(w2_scales), _ptr(ws), ws.numel(), int(chunk_tokens),
+                                  _stream(stream), hs, ds), "moe_forward_host")
+    return y_host
 
 
 def moe_forward_partial(dims: moe_dims, x, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes, w2_scales,

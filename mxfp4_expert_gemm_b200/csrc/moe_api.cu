@@ -1,9 +1,11 @@
 // C-ABI front end: argument checks, workspace carve-up, path choice, launches.
 // Declarations and the contract of every entry point: include/moe_mxfp4.h.
 #include <cuda_runtime.h>
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <vector>
 
 #include "moe_internal.cuh"
 
@@ -190,6 +192,38 @@ moe_status forward_impl(const moe_dims* dims, int32_t T, const uint16_t* x, cons
   return MOE_OK;
 }
 
+// Tokens per chunk of moe_forward_host when the caller leaves the choice to the library.
+// A chunk's copies in and out overlap the layer of its neighbours, but every chunk streams
+// the expert weights once more and fills its token tiles less: one chunk on the small-batch
+// path and below 4096 tokens (copies of a few MB), else two to four chunks of at least 2048
+// tokens.
+int32_t host_chunk(const moe_dims& dm, int32_t T) {
+  if (T < 4096 || resolve_path(dm, T) == MOE_PATH_GEMV) return T;
+  const int32_t n = std::min<int32_t>(4, T / 2048);
+  return (T + n - 1) / n;
+}
+
+// Events for the copy / layer overlap of moe_forward_host, per device and host thread
+// (timing disabled; reused call after call: a wait takes the event's state at the time it
+// is enqueued).
+struct HostEvents {
+  std::vector<cudaEvent_t> ev[64];
+  ~HostEvents() {
+    for (auto& v : ev)
+      for (cudaEvent_t e : v) cudaEventDestroy(e);
+  }
+  cudaEvent_t get(int dev, size_t i) {
+    std::vector<cudaEvent_t>& v = ev[dev & 63];
+    while (v.size() <= i) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+      v.push_back(e);
+    }
+    return v[i];
+  }
+};
+thread_local HostEvents g_host_events;
+
 }  // namespace
 
 namespace moe {
@@ -320,6 +354,79 @@ moe_status moe_residual_norm(int32_t T, int32_t d, const uint16_t* x, const floa
                                 static_cast<cudaStream_t>(stream)) < 0)
     return MOE_ERR_CUDA;
   g_last_launches = 1;
+  return MOE_OK;
+}
+
+int32_t moe_host_chunk_tokens(const moe_dims* dims, int32_t T) {
+  if (check_dims(dims, T) != MOE_OK) return -1;
+  return host_chunk(*dims, T);
+}
+
+moe_status moe_forward_host(const moe_dims* dims, int32_t T, const uint16_t* x_host, uint16_t* y_host,
+                            uint16_t* x_dev, uint16_t* y_dev, const float* norm_w, const float* router_w,
+                            const float* router_b, const uint8_t* w1_codes, const uint8_t* w1_scales,
+                            const uint8_t* w2_codes, const uint8_t* w2_scales, void* ws, size_t ws_bytes,
+                            int32_t chunk_tokens, void* stream, void* h2d_stream, void* d2h_stream) {
+  g_last_launches = 0;
+  moe_status st = check_dims(dims, T);
+  if (st != MOE_OK) return st;
+  if (chunk_tokens < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  // Every argument check of the chunks' forward calls, made before anything is enqueued.
+  if (!x_host || !y_host || !x_dev || !y_dev || !norm_w || !router_w || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_dev) || !aligned16(y_dev) || !aligned16(norm_w) || !aligned16(router_w) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  if ((void*)x_dev == (void*)y_dev || (router_b && !aligned16(router_b))) return MOE_ERR_INVALID_ARG;
+  if (!w1_codes || !w1_scales || !w2_codes || !w2_scales) return MOE_ERR_INVALID_ARG;
+  if (!aligned32(w1_codes) || !aligned16(w1_scales) || !aligned32(w2_codes) || !aligned16(w2_scales))
+    return MOE_ERR_INVALID_ARG;
+  const int32_t chunk = chunk_tokens > 0 ? std::min(chunk_tokens, T) : host_chunk(*dims, T);
+  const int32_t n = (T + chunk - 1) / chunk;
+  const int32_t last = T - (n - 1) * chunk;
+  if (ws_bytes < layout_for(*dims, chunk).total || ws_bytes < layout_for(*dims, last).total)
+    return MOE_ERR_WORKSPACE;
+  if ((st = check_device()) != MOE_OK) return st;
+
+  // One chunk: copy in, layer and copy out in order on `stream`.  Several: the copies in on
+  // h2d_stream, the layers on `stream`, the copies out on d2h_stream, ordered by events.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t sh = (n > 1 && h2d_stream) ? static_cast<cudaStream_t>(h2d_stream) : s;
+  cudaStream_t sd = (n > 1 && d2h_stream) ? static_cast<cudaStream_t>(d2h_stream) : s;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  // events: 0 fork, 1 join, 2 + 2c chunk c copied in, 3 + 2c chunk c's layer done
+  if (!g_host_events.get(dev, 2 * (size_t)n + 1)) return MOE_ERR_CUDA;
+  auto ev = [&](size_t i) { return g_host_events.get(dev, i); };
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  const size_t d = (size_t)dims->d, row_bytes = d * sizeof(uint16_t);
+  auto rows_of = [&](int32_t c) { return c == n - 1 ? last : chunk; };
+
+  // fork: the copies in wait for the work `stream` holds (which may still read x_dev)
+  if (sh != s && !(ok(cudaEventRecord(ev(0), s)) && ok(cudaStreamWaitEvent(sh, ev(0), 0)))) return MOE_ERR_CUDA;
+  for (int32_t c = 0; c < n; ++c) {
+    const size_t off = (size_t)c * chunk * d;
+    if (!ok(cudaMemcpyAsync(x_dev + off, x_host + off, rows_of(c) * row_bytes, cudaMemcpyHostToDevice, sh)))
+      return MOE_ERR_CUDA;
+    if (sh != s && !ok(cudaEventRecord(ev(2 + 2 * (size_t)c), sh))) return MOE_ERR_CUDA;
+  }
+  int32_t launches = 0;
+  for (int32_t c = 0; c < n; ++c) {
+    const size_t off = (size_t)c * chunk * d;
+    if (sh != s && !ok(cudaStreamWaitEvent(s, ev(2 + 2 * (size_t)c), 0))) return MOE_ERR_CUDA;
+    Outputs out;
+    out.y = y_dev + off;
+    st = forward_impl(dims, rows_of(c), x_dev + off, norm_w, router_w, router_b, w1_codes, w1_scales, w2_codes,
+                      w2_scales, out, ws, ws_bytes, stream, nullptr, 0);
+    if (st != MOE_OK) return st;
+    launches += g_last_launches;
+    if (sd != s && !(ok(cudaEventRecord(ev(3 + 2 * (size_t)c), s)) && ok(cudaStreamWaitEvent(sd, ev(3 + 2 * (size_t)c), 0))))
+      return MOE_ERR_CUDA;
+    if (!ok(cudaMemcpyAsync(y_host + off, y_dev + off, rows_of(c) * row_bytes, cudaMemcpyDeviceToHost, sd)))
+      return MOE_ERR_CUDA;
+  }
+  // join: `stream` waits for the last copy out (the copies in were waited for chunk by chunk)
+  if (sd != s && !(ok(cudaEventRecord(ev(1), sd)) && ok(cudaStreamWaitEvent(s, ev(1), 0)))) return MOE_ERR_CUDA;
+  g_last_launches = launches;
   return MOE_OK;
 }
 

@@ -118,3 +118,59 @@ def test_no_alloc_argument_checks_match_moe_forward(L):
         assert call(dims, T) == _call_forward(L, dims, T), (dims.path, dims.act_format, T)
     assert call(None, 4) == moe.MOE_ERR_INVALID_ARG
     assert call(moe.make_dims(2880, 2880, 32, 4), 4096) == moe.MOE_ERR_WORKSPACE   # beyond the 16 MiB scratch
+
+
+def _call_host(L, dims, T, ptr=256, ws_bytes=1 << 40, chunk=0, x_dev=None, y_dev=None, hp=4096):
+    p = ctypes.c_void_p(ptr)
+    xd = ctypes.c_void_p(ptr if x_dev is None else x_dev)
+    yd = ctypes.c_void_p(ptr + 8192 if y_dev is None else y_dev)
+    h = ctypes.c_void_p(hp)
+    return L.moe_forward_host(ctypes.byref(dims) if dims is not None else None, T, h, h, xd, yd, p, p, None,
+                              p, p, p, p, p, ws_bytes, chunk, None, None, None)
+
+
+def test_host_entry_argument_checks_before_device(L):
+    """moe_forward_host refuses bad arguments before it enqueues anything (no GPU needed)."""
+    ok = moe.make_dims(2880, 2880, 32, 4)
+    assert _call_host(L, None, 4) == moe.MOE_ERR_INVALID_ARG
+    assert _call_host(L, ok, -1) == moe.MOE_ERR_INVALID_ARG
+    assert _call_host(L, ok, 0) == moe.MOE_OK                                    # nothing to do
+    assert _call_host(L, ok, 16, chunk=-1) == moe.MOE_ERR_INVALID_ARG
+    assert _call_host(L, ok, 16, hp=0) == moe.MOE_ERR_INVALID_ARG                # null host buffers
+    assert _call_host(L, ok, 16, x_dev=512, y_dev=512) == moe.MOE_ERR_INVALID_ARG  # x_dev aliases y_dev
+    assert _call_host(L, ok, 16, x_dev=520) == moe.MOE_ERR_INVALID_ARG          # misaligned x_dev
+    assert _call_host(L, ok, 16, ptr=16) == moe.MOE_ERR_INVALID_ARG             # codes need 32-byte alignment
+    assert _call_host(L, moe.make_dims(2880 + 32, 2880, 32, 4), 16) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    # the workspace must hold a chunk: the whole batch's is more than enough, a chunk's
+    # exactly enough, a byte less is refused
+    T, c = 8192, moe.moe_host_chunk_tokens(ok, 8192)
+    need = max(moe.moe_workspace_bytes(ok, c), moe.moe_workspace_bytes(ok, T - (T + c - 1) // c * c + c))
+    assert _call_host(L, ok, T, ws_bytes=need - 1) == moe.MOE_ERR_WORKSPACE
+    assert _call_host(L, ok, T, ws_bytes=moe.moe_workspace_bytes(ok, 100), chunk=100) != moe.MOE_ERR_WORKSPACE
+    assert _call_host(L, ok, T, ws_bytes=moe.moe_workspace_bytes(ok, 99), chunk=100) == moe.MOE_ERR_WORKSPACE
+
+
+def test_host_entry_chunk_choice(L):
+    """One chunk on the small-batch path and below 4096 tokens; else two to four chunks of at
+    least 2048 tokens that cover the batch."""
+    d20, d120 = moe.make_dims(2880, 2880, 32, 4), moe.make_dims(2880, 2880, 128, 4)
+    assert moe.moe_host_chunk_tokens(d20, 16) == 16
+    assert moe.moe_host_chunk_tokens(d20, 4095) == 4095
+    assert moe.moe_host_chunk_tokens(d20, 4096) == 2048
+    assert moe.moe_host_chunk_tokens(d120, 16384) == 4096
+    assert moe.moe_host_chunk_tokens(d120, 8192) == 2048
+    assert moe.moe_host_chunk_tokens(d120, 6000) == 3000
+    # few tokens per expert (E = 256, top-1: 16 per expert at 4096 tokens): one chunk
+    assert moe.moe_host_chunk_tokens(moe.make_dims(2880, 2880, 256, 1), 4096) == 4096
+    for T in (4096, 5000, 9999, 16384, 100000):
+        c = moe.moe_host_chunk_tokens(d120, T)
+        n = (T + c - 1) // c
+        assert 2 <= n <= 4 and c >= 2048 and (n - 1) * c < T
+    assert L.moe_host_chunk_tokens(None, 16) == -1
+
+
+def test_no_device_host_entry_is_an_error(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _call_host(L, moe.make_dims(128, 128, 4, 2), 4) in (moe.MOE_ERR_CUDA, moe.MOE_ERR_DEVICE)
