@@ -213,7 +213,8 @@ struct HostEvents {
       for (cudaEvent_t e : v) cudaEventDestroy(e);
   }
   cudaEvent_t get(int dev, size_t i) {
-    std::vector<cudaEvent_t>& v = ev[dev & 63];
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::vector<cudaEvent_t>& v = ev[dev];
     while (v.size() <= i) {
       cudaEvent_t e = nullptr;
       if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
