@@ -13,6 +13,11 @@ half of the metric).  The gpt-oss-20b decode batch (T = 16, E = 32, HBM-bound:
 the "% of HBM bandwidth" half) is measured in the same run and reported under
 ``"decode"`` with its own timing, roofline and end-to-end figures.
 
+The end-to-end figure (``e2e``) times ``moe_forward_host`` per step: x from pinned host
+memory in, y to pinned host memory out, the batch cut into chunks whose copies run on
+their own streams under the neighbouring chunks' layers (``--e2e-chunk`` sets the chunk;
+by default the library picks it).
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--path auto|gemv|gemm]
     python bench.py --impl reference ...   # the CPU oracle on the host cores, same metric
 
